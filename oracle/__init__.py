@@ -1,0 +1,205 @@
+"""fp64 CPU oracle for the DiT attention hot path -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+and reference legs may import this package. The product library
+(``dit_attention_b200``) never does, and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP over rows); this
+module only builds it with gcc on first use and marshals numpy arrays.
+
+Functions (each follows the definition written at its C counterpart):
+
+* ``attention(q, k, v, scale, rows=None)`` -- exact softmax attention and
+  natural-log LSE, inputs bf16 bit arrays [B, H, S, D] (or doubles).
+* ``lse_merge(o_a, lse_a, o_b, lse_b)`` -- two-block (O, LSE) combination.
+* ``rope3d(x, grid, theta)`` -- 3D RoPE, bf16 in/out (rounded to nearest even)
+  or fp64 in/out.
+* ``f64_to_bf16`` / ``bf16_to_f64`` -- the oracle's own rounding and widening.
+
+Parity status: attention and the LSE merge are pinned by the tests against
+brute force, closed forms, invariants and torch's CPU fp64 SDPA. The RoPE
+*pairing convention* (interleaved pairs, axis order t/h/w, 44/42/42 split) is a
+reading of the Wan2.1 architecture the pages name, not something the pages
+print: "parity unpinned" for that convention; the rotation itself is pinned by
+norm preservation, relative-offset invariance, the identity at position 0 and
+reduction to 1D RoPE.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_i64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-ffp-contract=off", "-fopenmp", "-shared", "-fPIC",
+               _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            lib.oracle_attention_f64.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _i64,
+                                                 ctypes.c_double, _i64p, _i64, _dp, _dp]
+            lib.oracle_attention_f64.restype = None
+            lib.oracle_attention_bf16.argtypes = [_u16p, _u16p, _u16p, _i64, _i64, _i64, _i64,
+                                                  ctypes.c_double, _i64p, _i64, _dp, _dp]
+            lib.oracle_attention_bf16.restype = ctypes.c_int
+            lib.oracle_lse_merge_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _dp, _dp]
+            lib.oracle_lse_merge_f64.restype = None
+            lib.oracle_rope3d_f64.argtypes = [_dp, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
+            lib.oracle_rope3d_f64.restype = ctypes.c_int
+            lib.oracle_rope3d_bf16.argtypes = [_u16p, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
+            lib.oracle_rope3d_bf16.restype = ctypes.c_int
+            lib.oracle_f64_to_bf16_array.argtypes = [_dp, _u16p, _i64]
+            lib.oracle_f64_to_bf16_array.restype = None
+            lib.oracle_bf16_to_f64_array.argtypes = [_u16p, _dp, _i64]
+            lib.oracle_bf16_to_f64_array.restype = None
+            lib.oracle_num_threads.argtypes = []
+            lib.oracle_num_threads.restype = ctypes.c_int
+            lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+            lib.oracle_set_num_threads.restype = None
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray, t):
+    return a.ctypes.data_as(t)
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    _load().oracle_set_num_threads(int(n))
+
+
+def f64_to_bf16(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _load().oracle_f64_to_bf16_array(_ptr(x, _dp), _ptr(out, _u16p), x.size)
+    return out
+
+
+def bf16_to_f64(h) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, dtype=np.float64)
+    _load().oracle_bf16_to_f64_array(_ptr(h, _u16p), _ptr(out, _dp), h.size)
+    return out
+
+
+def attention(q, k, v, scale: float, rows=None):
+    """Exact attention. q [..., Sq, D], k/v [..., Skv, D] with equal leading dims.
+
+    Arrays of dtype uint16 are bf16 bit patterns; float64 arrays are used as
+    they are. Returns (out fp64, lse fp64): with rows=None, out has q's shape
+    and lse q's shape without D; with rows (global indices bh*Sq + i) the
+    results are [len(rows), D] and [len(rows)].
+    """
+    lib = _load()
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    Sq, D = q.shape[-2], q.shape[-1]
+    Skv = k.shape[-2]
+    lead = q.shape[:-2]
+    if k.shape[:-2] != lead or v.shape != k.shape or k.shape[-1] != D:
+        raise ValueError("q, k, v shapes do not agree")
+    BH = int(np.prod(lead)) if lead else 1
+    if rows is None:
+        n = BH * Sq
+        rp = None
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        if rows.size and (rows.min() < 0 or rows.max() >= BH * Sq):
+            raise ValueError("row index out of range")
+        n = rows.size
+        rp = _ptr(rows, _i64p)
+    out = np.empty((n, D), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    kinds = {q.dtype, k.dtype, v.dtype}
+    if kinds == {np.dtype(np.uint16)}:
+        rc = lib.oracle_attention_bf16(_ptr(q, _u16p), _ptr(k, _u16p), _ptr(v, _u16p),
+                                       BH, Sq, Skv, D, float(scale), rp, n,
+                                       _ptr(out, _dp), _ptr(lse, _dp))
+        if rc != 0:
+            raise MemoryError("oracle could not allocate its fp64 copies")
+    elif kinds == {np.dtype(np.float64)}:
+        lib.oracle_attention_f64(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp),
+                                 BH, Sq, Skv, D, float(scale), rp, n,
+                                 _ptr(out, _dp), _ptr(lse, _dp))
+    else:
+        raise TypeError("inputs must all be uint16 (bf16 bits) or all float64")
+    if rows is None:
+        return out.reshape(q.shape), lse.reshape(q.shape[:-1])
+    return out, lse
+
+
+def lse_merge(o_a, lse_a, o_b, lse_b):
+    """Two-block merge. o_* [..., D] (bf16 bits or float64), lse_* [...]."""
+    lib = _load()
+
+    def as64(a):
+        a = np.ascontiguousarray(a)
+        return bf16_to_f64(a) if a.dtype == np.uint16 else np.ascontiguousarray(a, dtype=np.float64)
+
+    oa, ob = as64(o_a), as64(o_b)
+    la = np.ascontiguousarray(lse_a, dtype=np.float64)
+    lb = np.ascontiguousarray(lse_b, dtype=np.float64)
+    D = oa.shape[-1]
+    rows = oa.size // D if D else 0
+    if ob.shape != oa.shape or la.size != rows or lb.size != rows:
+        raise ValueError("merge shapes do not agree")
+    out = np.empty(oa.shape, dtype=np.float64)
+    lse = np.empty(la.shape, dtype=np.float64)
+    lib.oracle_lse_merge_f64(_ptr(oa, _dp), _ptr(la, _dp), _ptr(ob, _dp), _ptr(lb, _dp),
+                             rows, D, _ptr(out, _dp), _ptr(lse, _dp))
+    return out, lse
+
+
+def rope3d(x, grid, theta: float = 10000.0):
+    """3D RoPE of x [..., S, D], S = T*Hh*Ww. Returns a new array.
+
+    uint16 input (bf16 bits) -> uint16 output rounded to nearest even;
+    float64 input -> float64 output (no rounding).
+    """
+    lib = _load()
+    T, Hh, Ww = (int(g) for g in grid)
+    x = np.array(x, copy=True, order="C")
+    S, D = x.shape[-2], x.shape[-1]
+    if S != T * Hh * Ww:
+        raise ValueError("sequence length does not match the latent grid")
+    BH = x.size // (S * D) if S * D else 0
+    if x.dtype == np.uint16:
+        rc = lib.oracle_rope3d_bf16(_ptr(x, _u16p), BH, T, Hh, Ww, D, float(theta))
+    elif x.dtype == np.float64:
+        rc = lib.oracle_rope3d_f64(_ptr(x, _dp), BH, T, Hh, Ww, D, float(theta))
+    else:
+        raise TypeError("x must be uint16 (bf16 bits) or float64")
+    if rc != 0:
+        raise ValueError("rope3d needs an even head dim >= 6")
+    return x

@@ -1,0 +1,290 @@
+/*
+ * oracle.c -- plain, slow fp64 CPU reference for the DiT attention hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or
+ * call this file; only the tests, the entry point's smoke check and the
+ * bench's CPU-baseline leg do. It shares no code with the CUDA library.
+ *
+ * What it computes, and where it comes from (ReGenVC, arXiv 2607.28144, as
+ * summarised on the blog.captcha.la page, "Methodology -- deep read" and
+ * "Technical innovations"): the decoder's diffusion transformer runs *exact*
+ * attention, and its sequence parallelism (Ulysses x Ring) preserves that
+ * exactness by streaming KV blocks and combining partial results. There is no
+ * equation on the pages, so each function below writes out the textbook
+ * definition it implements, in fp64, in the order the definition states:
+ *
+ *   oracle_attention_f64   softmax(scale * Q K^T) V per (batch, head, query),
+ *                          with the natural-log LSE of the scaled logits.
+ *   oracle_lse_merge_f64   the two-block combination of (O, LSE) that Ring
+ *                          attention applies between KV blocks.
+ *   oracle_rope3d_f64      3D rotary position embedding of the Wan2.1 DiT
+ *                          that the decoder's architecture matches (page 2,
+ *                          "Methodology -- deep read": the student matches
+ *                          the Wan2.1-Fun-Control teacher). The pages do not
+ *                          print its formula; the reading used is stated at
+ *                          the function. Parity of the pairing convention is
+ *                          unpinned by the pages.
+ *
+ * bf16 inputs are widened exactly to double; bf16 outputs are rounded to
+ * nearest-even directly from the double (no intermediate fp32 rounding).
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC oracle.c -o liboracle.so -lm
+ * (no -ffast-math: the sums run in the plain order written here).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---------------------------------------------------------------- bf16 --- */
+
+double oracle_bf16_to_f64(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to bf16, nearest with ties to even, on its bit pattern. */
+uint16_t oracle_f64_to_bf16(double x)
+{
+    uint64_t b;
+    memcpy(&b, &x, sizeof b);
+    uint16_t sign = (uint16_t)((b >> 48) & 0x8000u);
+    uint64_t mag = b & 0x7FFFFFFFFFFFFFFFull;
+    if (mag > 0x7FF0000000000000ull) return (uint16_t)(sign | 0x7FC0u);  /* NaN */
+    if (mag == 0x7FF0000000000000ull) return (uint16_t)(sign | 0x7F80u); /* inf */
+    if (mag >= 0x3810000000000000ull) {           /* |x| >= 2^-126: normal bf16 */
+        uint64_t keep = mag >> 45;                /* exponent (11) + 7 mantissa bits */
+        uint64_t rem = mag & ((1ull << 45) - 1);
+        uint64_t half = 1ull << 44;
+        if (rem > half || (rem == half && (keep & 1))) keep++;
+        uint64_t r = keep - ((uint64_t)(1023 - 127) << 7);
+        if (r >= 0x7F80u) return (uint16_t)(sign | 0x7F80u);              /* overflow */
+        return (uint16_t)(sign | r);
+    }
+    /* bf16 subnormal range: integer multiples of 2^-133, round the multiple. */
+    double s = ldexp(fabs(x), 133);
+    double fl = floor(s);
+    double fr = s - fl;
+    uint64_t n = (uint64_t)fl;
+    if (fr > 0.5 || (fr == 0.5 && (n & 1))) n++;
+    return (uint16_t)(sign | n);
+}
+
+void oracle_bf16_to_f64_array(const uint16_t *h, double *x, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) x[i] = oracle_bf16_to_f64(h[i]);
+}
+
+void oracle_f64_to_bf16_array(const double *x, uint16_t *h, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) h[i] = oracle_f64_to_bf16(x[i]);
+}
+
+/* ----------------------------------------------------------- attention --- */
+
+/*
+ * One query row of exact softmax attention, by definition:
+ *   s_j   = scale * sum_d q_d k_jd            for j < Skv
+ *   m     = max_j s_j
+ *   p_j   = exp(s_j - m)
+ *   l     = sum_j p_j
+ *   out_d = (sum_j p_j v_jd) / l
+ *   lse   = m + ln l                          (natural log, scaled-logit units)
+ * Skv == 0 gives out = 0 and lse = -inf (the empty softmax).
+ * `p` is caller scratch of Skv doubles.
+ */
+static void attention_row(const double *qi, const double *Kh, const double *Vh,
+                          int64_t Skv, int64_t D, double scale,
+                          double *p, double *out, double *lse)
+{
+    for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
+    if (Skv == 0) {
+        *lse = -INFINITY;
+        return;
+    }
+    double m = -INFINITY;
+    for (int64_t j = 0; j < Skv; ++j) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qi[d] * Kh[j * D + d];
+        p[j] = scale * dot;
+        if (p[j] > m) m = p[j];
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < Skv; ++j) {
+        p[j] = exp(p[j] - m);
+        l += p[j];
+    }
+    for (int64_t j = 0; j < Skv; ++j)
+        for (int64_t d = 0; d < D; ++d) out[d] += p[j] * Vh[j * D + d];
+    for (int64_t d = 0; d < D; ++d) out[d] /= l;
+    *lse = m + log(l);
+}
+
+/*
+ * Attention over BH independent (batch, head) problems laid out [BH][S][D].
+ * rows == NULL: every query row, out [BH*Sq][D], lse [BH*Sq].
+ * rows != NULL: only the nrows global rows rows[r] = bh*Sq + i, out [nrows][D].
+ */
+void oracle_attention_f64(const double *q, const double *k, const double *v,
+                          int64_t BH, int64_t Sq, int64_t Skv, int64_t D, double scale,
+                          const int64_t *rows, int64_t nrows,
+                          double *out, double *lse)
+{
+    int64_t n = rows ? nrows : BH * Sq;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < n; ++r) {
+            int64_t g = rows ? rows[r] : r;
+            int64_t bh = g / Sq;
+            attention_row(q + g * D, k + bh * Skv * D, v + bh * Skv * D, Skv, D, scale,
+                          p, out + r * D, lse + r);
+        }
+        free(p);
+    }
+}
+
+/* Same, on bf16 inputs (widened exactly to double first). */
+int oracle_attention_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          int64_t BH, int64_t Sq, int64_t Skv, int64_t D, double scale,
+                          const int64_t *rows, int64_t nrows,
+                          double *out, double *lse)
+{
+    int64_t nq = BH * Sq * D, nkv = BH * Skv * D;
+    double *qd = (double *)malloc(sizeof(double) * (size_t)(nq > 0 ? nq : 1));
+    double *kd = (double *)malloc(sizeof(double) * (size_t)(nkv > 0 ? nkv : 1));
+    double *vd = (double *)malloc(sizeof(double) * (size_t)(nkv > 0 ? nkv : 1));
+    if (!qd || !kd || !vd) {
+        free(qd); free(kd); free(vd);
+        return -1;
+    }
+    if (rows) {
+        for (int64_t r = 0; r < nrows; ++r)
+            for (int64_t d = 0; d < D; ++d)
+                qd[rows[r] * D + d] = oracle_bf16_to_f64(q[rows[r] * D + d]);
+    } else {
+        oracle_bf16_to_f64_array(q, qd, nq);
+    }
+    oracle_bf16_to_f64_array(k, kd, nkv);
+    oracle_bf16_to_f64_array(v, vd, nkv);
+    oracle_attention_f64(qd, kd, vd, BH, Sq, Skv, D, scale, rows, nrows, out, lse);
+    free(qd); free(kd); free(vd);
+    return 0;
+}
+
+/* ------------------------------------------------------------ LSE merge --- */
+
+/*
+ * Combine two partial attentions of the same queries over disjoint key
+ * blocks a and b (each normalised by its own softmax, with its own LSE):
+ *   m   = max(lse_a, lse_b)
+ *   w_a = exp(lse_a - m),  w_b = exp(lse_b - m)
+ *   out = (w_a o_a + w_b o_b) / (w_a + w_b)
+ *   lse = m + ln(w_a + w_b)
+ * Both LSEs -inf (two empty blocks): out = 0, lse = -inf.
+ */
+void oracle_lse_merge_f64(const double *oa, const double *lsea,
+                          const double *ob, const double *lseb,
+                          int64_t rows, int64_t D, double *out, double *lse)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        double m = lsea[r] > lseb[r] ? lsea[r] : lseb[r];
+        if (m == -INFINITY) {
+            for (int64_t d = 0; d < D; ++d) out[r * D + d] = 0.0;
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double wa = exp(lsea[r] - m);
+        double wb = exp(lseb[r] - m);
+        for (int64_t d = 0; d < D; ++d)
+            out[r * D + d] = (wa * oa[r * D + d] + wb * ob[r * D + d]) / (wa + wb);
+        lse[r] = m + log(wa + wb);
+    }
+}
+
+/* ---------------------------------------------------------------- RoPE --- */
+
+/*
+ * 3D rotary position embedding, in place on x [BH][S][D], S = T*Hh*Ww.
+ *
+ * Reading (the pages give no formula; this is the Wan2.1 DiT's 3D RoPE that
+ * the decoder's architecture matches):
+ *  - token n sits at latent grid position (t, y, x) with n = (t*Hh + y)*Ww + x;
+ *  - the head dimension splits into three axis blocks, in the order t, h, w:
+ *    d_h = d_w = 2*floor(D/6) and d_t = D - 2*d_h (44/42/42 at D = 128);
+ *  - inside an axis block of width d_a, the pair (2j, 2j+1) is rotated by
+ *    angle pos_a * theta^(-2j/d_a), j = 0 .. d_a/2 - 1:
+ *        x'_{2j}   = x_{2j} cos(angle) - x_{2j+1} sin(angle)
+ *        x'_{2j+1} = x_{2j} sin(angle) + x_{2j+1} cos(angle)
+ *    (the product of the pair, read as a complex number, with e^{i angle}).
+ */
+int oracle_rope3d_f64(double *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
+                      int64_t D, double theta)
+{
+    if (D < 6 || (D % 2) != 0) return -1;
+    int64_t dh = 2 * (D / 6);
+    int64_t dt = D - 2 * dh;
+    int64_t S = T * Hh * Ww;
+    int64_t base[3] = {0, dt, dt + dh};
+    int64_t width[3] = {dt, dh, dh};
+#pragma omp parallel for schedule(static)
+    for (int64_t g = 0; g < BH * S; ++g) {
+        int64_t n = g % S;
+        int64_t pos[3];
+        pos[0] = n / (Hh * Ww);
+        pos[1] = (n / Ww) % Hh;
+        pos[2] = n % Ww;
+        double *row = x + g * D;
+        for (int a = 0; a < 3; ++a) {
+            for (int64_t j = 0; j < width[a] / 2; ++j) {
+                double angle = (double)pos[a] * pow(theta, -2.0 * (double)j / (double)width[a]);
+                double c = cos(angle), s = sin(angle);
+                double x0 = row[base[a] + 2 * j];
+                double x1 = row[base[a] + 2 * j + 1];
+                row[base[a] + 2 * j] = x0 * c - x1 * s;
+                row[base[a] + 2 * j + 1] = x0 * s + x1 * c;
+            }
+        }
+    }
+    return 0;
+}
+
+/* In place on bf16: widen, rotate in fp64, round to nearest-even bf16. */
+int oracle_rope3d_bf16(uint16_t *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
+                       int64_t D, double theta)
+{
+    int64_t n = BH * T * Hh * Ww * D;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    if (!xd) return -2;
+    oracle_bf16_to_f64_array(x, xd, n);
+    int rc = oracle_rope3d_f64(xd, BH, T, Hh, Ww, D, theta);
+    if (rc == 0) oracle_f64_to_bf16_array(xd, x, n);
+    free(xd);
+    return rc;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -1,0 +1,327 @@
+"""Pins for the fp64 oracle against facts fixed outside the oracle itself.
+
+Exact attention (ReGenVC blog page, "Technical innovations": the Ulysses x Ring
+sharding keeps attention exact and numerically equivalent) means the oracle
+must equal the textbook softmax attention. It is pinned here by closed forms
+(tests/golden), brute force in Python on tiny inputs, invariants (rows of P
+sum to 1, constant V, joint KV permutation, logit shift, two-block LSE merge)
+and a library cross-check (torch CPU fp64 SDPA). The 3D RoPE reading is pinned
+by closed forms, norm preservation, relative-offset invariance, identity at
+the origin and reduction to 1D RoPE on each axis block.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from dit_attention_b200 import synth
+
+RNG = np.random.default_rng(1234)
+
+
+def _read_golden(path):
+    rows = {}
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        name, rest = line.split(None, 1)
+        rows[name] = rest
+    return rows
+
+
+# ------------------------------------------------------------ attention ---
+
+def test_attention_closed_forms(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "attention_closed_form.txt"))
+    cases = {
+        "A": (1.0, [[1.0]], [[0.0], [1.0]], [[1.0], [0.0]]),
+        "B": (0.5, [[2.0, 0.0]], [[0, 0], [1, 0], [2, 0]], [[1, 0], [0, 1], [1, 1]]),
+        "C": (1.0, [[math.log(3.0)]], [[0.0], [1.0]], [[0.0], [1.0]]),
+    }
+    for name, (scale, q, k, v) in cases.items():
+        vals = [float(t) for t in g[name].split()]
+        out, lse = oracle.attention(np.array(q, float), np.array(k, float), np.array(v, float), scale)
+        np.testing.assert_allclose(out[0], vals[:-1], rtol=1e-14, atol=1e-15)
+        assert abs(lse[0] - vals[-1]) < 1e-14
+
+
+def _brute(q, k, v, scale):
+    """Row-by-row softmax in plain Python floats with math.fsum."""
+    Sq, D = q.shape
+    out = np.zeros((Sq, D))
+    lse = np.zeros(Sq)
+    for i in range(Sq):
+        s = [scale * math.fsum(q[i, d] * k[j, d] for d in range(D)) for j in range(k.shape[0])]
+        z = math.fsum(math.exp(x) for x in s)
+        for d in range(D):
+            out[i, d] = math.fsum(math.exp(s[j]) * v[j, d] for j in range(len(s))) / z
+        lse[i] = math.log(z)
+    return out, lse
+
+
+@pytest.mark.parametrize("Sq,Skv,D", [(1, 1, 1), (3, 5, 2), (8, 8, 4), (5, 7, 3), (2, 8, 8)])
+def test_attention_brute_force(Sq, Skv, D):
+    q = RNG.normal(size=(Sq, D))
+    k = RNG.normal(size=(Skv, D))
+    v = RNG.normal(size=(Skv, D))
+    scale = 0.7
+    out, lse = oracle.attention(q, k, v, scale)
+    ref, rlse = _brute(q, k, v, scale)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, rlse, rtol=1e-13, atol=1e-13)
+
+
+def test_attention_rows_of_p_sum_to_one():
+    # V = identity (Skv == D) makes the output row equal to the softmax row P.
+    D = 16
+    q = RNG.normal(size=(2, 3, 9, D))
+    k = RNG.normal(size=(2, 3, D, D))
+    v = np.broadcast_to(np.eye(D), (2, 3, D, D)).copy()
+    p, lse = oracle.attention(q, k, v, 0.37)
+    assert np.all(p > 0)
+    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=0, atol=1e-12)
+    # P_ij = exp(s_ij - lse_i)
+    s = 0.37 * np.einsum("bhid,bhjd->bhij", q, k)
+    np.testing.assert_allclose(p, np.exp(s - lse[..., None]), rtol=1e-12, atol=1e-14)
+
+
+def test_attention_constant_v():
+    q = RNG.normal(size=(1, 2, 7, 8))
+    k = RNG.normal(size=(1, 2, 11, 8))
+    c = RNG.normal(size=8)
+    v = np.broadcast_to(c, (1, 2, 11, 8)).copy()
+    out, _ = oracle.attention(q, k, v, 0.5)
+    np.testing.assert_allclose(out, np.broadcast_to(c, out.shape), rtol=1e-13, atol=1e-13)
+
+
+def test_attention_kv_permutation_equivariance():
+    q = RNG.normal(size=(1, 2, 6, 8))
+    k = RNG.normal(size=(1, 2, 13, 8))
+    v = RNG.normal(size=(1, 2, 13, 8))
+    perm = RNG.permutation(13)
+    a, la = oracle.attention(q, k, v, 0.4)
+    b, lb = oracle.attention(q, k[:, :, perm], v[:, :, perm], 0.4)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(la, lb, rtol=1e-13, atol=1e-13)
+    # ... and a permutation of the queries permutes the outputs.
+    pq = RNG.permutation(6)
+    c, lc = oracle.attention(q[:, :, pq], k, v, 0.4)
+    np.testing.assert_allclose(c, a[:, :, pq], rtol=1e-13, atol=1e-14)
+
+
+def test_attention_logit_shift():
+    # Append a coordinate: q' = [q, c], k' = [k, 1] adds scale*c to every
+    # logit of the row; out is unchanged and lse moves by scale*c.
+    q = RNG.normal(size=(1, 1, 5, 6))
+    k = RNG.normal(size=(1, 1, 9, 6))
+    v = RNG.normal(size=(1, 1, 9, 6))
+    c = RNG.normal(size=(1, 1, 5, 1)) * 30
+    q2 = np.concatenate([q, c], -1)
+    k2 = np.concatenate([k, np.ones((1, 1, 9, 1))], -1)
+    a, la = oracle.attention(q, k, v, 0.25)
+    b, lb = oracle.attention(q2, k2, np.concatenate([v, np.zeros((1, 1, 9, 1))], -1), 0.25)
+    np.testing.assert_allclose(b[..., :6], a, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(lb, la + 0.25 * c[..., 0], rtol=1e-13, atol=1e-11)
+
+
+def test_attention_scale_zero_and_single_key():
+    q = RNG.normal(size=(1, 2, 4, 8))
+    k = RNG.normal(size=(1, 2, 10, 8))
+    v = RNG.normal(size=(1, 2, 10, 8))
+    out, lse = oracle.attention(q, k, v, 0.0)
+    np.testing.assert_allclose(out, np.broadcast_to(v.mean(2, keepdims=True), out.shape), atol=1e-14)
+    np.testing.assert_allclose(lse, math.log(10), rtol=1e-15)
+    out, lse = oracle.attention(q, k[:, :, :1], v[:, :, :1], 0.3)
+    np.testing.assert_allclose(out, np.broadcast_to(v[:, :, :1], out.shape), atol=1e-15)
+    np.testing.assert_allclose(lse, 0.3 * np.einsum("bhid,bhd->bhi", q, k[:, :, 0]), rtol=1e-13)
+
+
+def test_attention_empty_kv_and_huge_logits():
+    q = RNG.normal(size=(1, 1, 3, 4))
+    out, lse = oracle.attention(q, np.zeros((1, 1, 0, 4)), np.zeros((1, 1, 0, 4)), 1.0)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+    # logits ~1e3 would overflow exp without the max subtraction
+    q = np.array([[[[1.0, 0.0]]]]) * 1000
+    k = np.array([[[[1.0, 0.0], [0.999, 0.0], [-1.0, 0.0]]]])
+    v = np.array([[[[1.0, 2.0], [3.0, 4.0], [5.0, 6.0]]]])
+    out, lse = oracle.attention(q, k, v, 1.0)
+    w = np.array([1.0, math.exp(-1.0), math.exp(-2000.0)])
+    np.testing.assert_allclose(out[0, 0, 0], (w[:, None] * v[0, 0]).sum(0) / w.sum(), rtol=1e-14)
+    assert abs(lse[0, 0, 0] - (1000.0 + math.log(w.sum()))) < 1e-12
+
+
+def test_attention_matches_torch_sdpa_fp64():
+    torch = pytest.importorskip("torch")
+    q = RNG.normal(size=(2, 3, 37, 64))
+    k = RNG.normal(size=(2, 3, 53, 64))
+    v = RNG.normal(size=(2, 3, 53, 64))
+    out, lse = oracle.attention(q, k, v, 0.125)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), scale=0.125).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+    s = torch.from_numpy(q) @ torch.from_numpy(k).transpose(-1, -2) * 0.125
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), rtol=1e-13, atol=1e-12)
+
+
+def test_attention_row_sampling_and_bf16_inputs():
+    q, k, v = (synth.f64_to_bf16_bits(RNG.normal(size=(2, 2, 19, 16))) for _ in range(3))
+    full, lfull = oracle.attention(q, k, v, 0.25)
+    rows = np.array([0, 5, 18, 19, 40, 75])
+    part, lpart = oracle.attention(q, k, v, 0.25, rows=rows)
+    np.testing.assert_array_equal(part, full.reshape(-1, 16)[rows])
+    np.testing.assert_array_equal(lpart, lfull.reshape(-1)[rows])
+    wide = [synth.bf16_bits_to_f64(t) for t in (q, k, v)]
+    f, lf = oracle.attention(*wide, 0.25)
+    np.testing.assert_array_equal(f, full)
+    np.testing.assert_array_equal(lf, lfull)
+
+
+# ------------------------------------------------------------ LSE merge ---
+
+def test_two_block_merge_reproduces_full_attention():
+    q = RNG.normal(size=(2, 2, 9, 16))
+    k = RNG.normal(size=(2, 2, 40, 16)) * 2
+    v = RNG.normal(size=(2, 2, 40, 16))
+    full, lfull = oracle.attention(q, k, v, 0.5)
+    for split in (1, 17, 39):
+        a, la = oracle.attention(q, k[:, :, :split], v[:, :, :split], 0.5)
+        b, lb = oracle.attention(q, k[:, :, split:], v[:, :, split:], 0.5)
+        m, lm = oracle.lse_merge(a, la, b, lb)
+        np.testing.assert_allclose(m, full, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lm, lfull, rtol=1e-13, atol=1e-12)
+
+
+def test_merge_special_cases():
+    o = RNG.normal(size=(5, 8))
+    lse = RNG.normal(size=5) * 10
+    m, lm = oracle.lse_merge(o, lse, o, lse)
+    np.testing.assert_allclose(m, o, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(lm, lse + math.log(2), rtol=1e-15, atol=1e-14)
+    other = RNG.normal(size=(5, 8))
+    m, lm = oracle.lse_merge(o, lse, other, np.full(5, -np.inf))
+    np.testing.assert_array_equal(m, o)
+    np.testing.assert_array_equal(lm, lse)
+    m2, lm2 = oracle.lse_merge(other, np.full(5, -np.inf), o, lse)
+    np.testing.assert_array_equal(m2, o)
+    m, lm = oracle.lse_merge(o, np.full(5, -np.inf), other, np.full(5, -np.inf))
+    assert np.all(m == 0) and np.all(np.isneginf(lm))
+    # weights: lse_b = lse_a + ln 3 gives out = (o_a + 3 o_b) / 4
+    m, lm = oracle.lse_merge(o, lse, other, lse + math.log(3))
+    np.testing.assert_allclose(m, (o + 3 * other) / 4, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lm, lse + math.log(4), rtol=1e-15, atol=1e-13)
+
+
+# ----------------------------------------------------------------- RoPE ---
+
+def test_rope3d_closed_forms(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "rope3d_closed_form.txt"))
+    for name in ("D6", "D12"):
+        head, inp, outp = g[name].split("|")
+        T, Hh, Ww, tok, theta = (float(t) for t in head.split())
+        inp = [float(t) for t in inp.split()]
+        outp = [float(t) for t in outp.split()]
+        D = len(inp)
+        S = int(T * Hh * Ww)
+        x = np.zeros((1, S, D))
+        x[0, int(tok)] = inp
+        y = oracle.rope3d(x, (int(T), int(Hh), int(Ww)), theta)
+        np.testing.assert_allclose(y[0, int(tok)], outp, rtol=0, atol=1e-15)
+
+
+def test_rope3d_norm_and_origin():
+    grid = (3, 4, 5)
+    x = RNG.normal(size=(2, 60, 128))
+    y = oracle.rope3d(x, grid)
+    # rotations preserve each pair's length, hence each row's norm
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-13)
+    pairs_x = np.hypot(x[..., 0::2], x[..., 1::2])
+    pairs_y = np.hypot(y[..., 0::2], y[..., 1::2])
+    np.testing.assert_allclose(pairs_y, pairs_x, rtol=1e-12)
+    np.testing.assert_array_equal(y[:, 0], x[:, 0])   # position (0,0,0) is the identity
+    assert not np.allclose(y[:, 1:], x[:, 1:])
+
+
+def test_rope3d_relative_offsets():
+    grid = (4, 6, 7)
+    Hh, Ww = 6, 7
+
+    def tok(t, yy, xx):
+        return (t * Hh + yy) * Ww + xx
+
+    q = RNG.normal(size=128)
+    k = RNG.normal(size=128)
+    S = 4 * 6 * 7
+
+    def rotated_dot(p1, p2):
+        xq = np.zeros((1, S, 128))
+        xk = np.zeros((1, S, 128))
+        xq[0, tok(*p1)] = q
+        xk[0, tok(*p2)] = k
+        rq = oracle.rope3d(xq, grid)[0, tok(*p1)]
+        rk = oracle.rope3d(xk, grid)[0, tok(*p2)]
+        return float(rq @ rk)
+
+    base = rotated_dot((1, 2, 3), (0, 4, 1))
+    for shift in [(1, 0, 0), (2, 1, 3), (0, -2, 2), (1, 1, -1)]:
+        p1 = tuple(a + b for a, b in zip((1, 2, 3), shift))
+        p2 = tuple(a + b for a, b in zip((0, 4, 1), shift))
+        assert abs(rotated_dot(p1, p2) - base) < 1e-11
+    # and it does depend on the offset in every axis
+    for other in [(2, 2, 3), (1, 3, 3), (1, 2, 4)]:
+        assert abs(rotated_dot(other, (0, 4, 1)) - base) > 1e-3
+
+
+@pytest.mark.parametrize("D", [128, 64, 12])
+def test_rope3d_reduces_to_1d_rope_per_axis(D):
+    dh = 2 * (D // 6)
+    dt = D - 2 * dh
+    grid = (5, 6, 7)
+    blocks = {0: (0, dt), 1: (dt, dh), 2: (dt + dh, dh)}
+    x = RNG.normal(size=(1, 5 * 6 * 7, D))
+    y = oracle.rope3d(x, grid, theta=10000.0)
+    for axis, pos in [(0, 3), (1, 4), (2, 6)]:
+        p = [0, 0, 0]
+        p[axis] = pos
+        n = (p[0] * 6 + p[1]) * 7 + p[2]
+        lo, width = blocks[axis]
+        # independent 1D RoPE on that block via complex multiplication
+        z = x[0, n, lo:lo + width:2] + 1j * x[0, n, lo + 1:lo + width:2]
+        freqs = 10000.0 ** (-np.arange(0, width, 2) / width)
+        r = z * np.exp(1j * pos * freqs)
+        np.testing.assert_allclose(y[0, n, lo:lo + width:2], r.real, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(y[0, n, lo + 1:lo + width:2], r.imag, rtol=1e-12, atol=1e-12)
+        rest = np.ones(D, bool)
+        rest[lo:lo + width] = False
+        np.testing.assert_array_equal(y[0, n, rest], x[0, n, rest])
+
+
+def test_rope3d_bf16_is_rounded_fp64():
+    grid = (2, 3, 4)
+    xb = synth.f64_to_bf16_bits(RNG.normal(size=(3, 24, 128)))
+    yb = oracle.rope3d(xb, grid)
+    y64 = oracle.rope3d(synth.bf16_bits_to_f64(xb), grid)
+    np.testing.assert_array_equal(yb, synth.f64_to_bf16_bits(y64))
+
+
+# ----------------------------------------------------------------- bf16 ---
+
+def test_oracle_bf16_rounding():
+    torch = pytest.importorskip("torch")
+    # doubles that are exact in fp32: torch's fp32 -> bf16 is a correct RNE
+    x = RNG.normal(size=20000).astype(np.float32).astype(np.float64) * 10.0 ** RNG.integers(-30, 30, 20000)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.f64_to_bf16(x), ref)
+    np.testing.assert_array_equal(synth.f64_to_bf16_bits(x), ref)
+    # exact ties round to even; just above a tie rounds up
+    one = 1.0
+    ulp = 2.0 ** -7
+    cases = [(one + ulp / 2, 0x3F80), (one + 1.5 * ulp, 0x3F82), (one + ulp / 2 + 2.0 ** -40, 0x3F81),
+             (-(one + ulp / 2), 0xBF80), (0.0, 0), (-0.0, 0x8000), (np.inf, 0x7F80), (3.5e38, 0x7F80),
+             (2.0 ** -133, 0x0001), (2.0 ** -134, 0x0000), (1.5 * 2.0 ** -133, 0x0002)]
+    for val, bits in cases:
+        assert oracle.f64_to_bf16(np.array([val]))[0] == bits, val
+    np.testing.assert_array_equal(oracle.bf16_to_f64(oracle.f64_to_bf16(x)),
+                                  synth.bf16_bits_to_f64(ref))
