@@ -1,0 +1,436 @@
+"""Benchmark of the DiT attention hot path (one line of JSON on rank 0).
+
+One step = one pass of the whole hot path for one denoising step of the
+77-frame window (B=1, H=40, D=128, latent grid 20 x 30 x 52 -> S = 31200):
+  1. rope3d on Q and K (in place)                       regen_rope3d
+  2. self-attention, 31200 x 31200                      regen_attn_fwd
+  3. cross-attention of the 31200 video tokens to the 1560 reference-frame
+     tokens and, separately, to the 512 conditioning tokens   regen_attn_fwd x2
+  4. the two cross-attention partials merged by LSE     regen_lse_merge
+(3+4 equal one softmax over the 2072 concatenated keys.) Each step rotates
+the Q/K left by the previous step again: the same work on the same shapes.
+
+value = attention FLOPs of the step (4*B*H*Sq*Skv*D, self + cross) / device
+time of the step, summed over ranks (weak scaling: every rank runs its own
+window). Inputs (320 MB per tensor) exceed the 126 MB L2, so no L2 flush is
+used between steps.
+
+--impl reference times the CPU fp64 oracle instead (bounded samples of rows).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s and % of B200 BF16 dense peak at S=31200,H=40,D=128"
+SELF = "win77_s31200"
+CROSS = "cross_s31200_kv2072"
+N_REF = 1560          # reference-frame latent tokens (one 30 x 52 latent frame)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def step_flops():
+    from dit_attention_b200 import synth
+    s = synth.WORKLOADS[SELF]
+    c = synth.WORKLOADS[CROSS]
+    return s.flops, c.flops
+
+
+# ------------------------------------------------------------ clocks ---
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        busy = [x for x in sm if smax and x > 0.3 * smax] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------- native (GPU) ---
+
+def traffic_from_profile():
+    """DRAM bytes per launch of the self-attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "attn_fwd_win77_s31200_traffic.txt")
+    src = os.path.join(ROOT, "dit_attention_b200", "csrc", "attn_fwd.cuh")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if "=" in line and not line.startswith("#"):
+            a, b = line.split("=", 1)
+            kv[a.strip()] = b.strip()
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if kv.get("kernel_source_sha256") != sha:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import dit_attention_b200 as rg
+    from dit_attention_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    rg.load()
+    dev = torch.device("cuda", local_rank)
+    ws = synth.WORKLOADS[SELF]
+    wc = synth.WORKLOADS[CROSS]
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    q, k, v = synth.make_inputs(ws, seed_offset=rank)
+    qc, kc, vc = synth.make_inputs(wc, seed_offset=rank)
+    host = {
+        "q": q, "k": k, "v": v, "qc": qc,
+        "kr": np.ascontiguousarray(kc[:, :, :N_REF]), "vr": np.ascontiguousarray(vc[:, :, :N_REF]),
+        "kx": np.ascontiguousarray(kc[:, :, N_REF:]), "vx": np.ascontiguousarray(vc[:, :, N_REF:]),
+    }
+    d = {name: to_dev(a) for name, a in host.items()}
+    B, H, S, D = ws.B, ws.H, ws.Sq, ws.D
+    out = torch.empty_like(d["q"])
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    oa, ob, oc = (torch.empty_like(d["qc"]) for _ in range(3))
+    la, lb, lc = (torch.empty((B, H, S), dtype=torch.float32, device=dev) for _ in range(3))
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    scale = 1.0 / math.sqrt(D)
+    T, Hh, Ww = ws.grid
+
+    names = ["rope3d", "attn_self", "attn_cross_ref", "attn_cross_ctx", "lse_merge"]
+    LAUNCHES_PER_STEP = len(names)
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        rg.regen_rope3d(d["q"], d["k"], T, Hh, Ww, ws.theta, B, H, D, sh)
+        mark(1)
+        rg.regen_attn_fwd(d["q"], d["k"], d["v"], out, lse, B, H, S, S, D, scale, sh)
+        mark(2)
+        rg.regen_attn_fwd(d["qc"], d["kr"], d["vr"], oa, la, B, H, S, N_REF, D, scale, sh)
+        mark(3)
+        rg.regen_attn_fwd(d["qc"], d["kx"], d["vx"], ob, lb, B, H, S, wc.Skv - N_REF, D, scale, sh)
+        mark(4)
+        rg.regen_lse_merge(oa, la, ob, lb, oc, lc, B * H * S, D, sh)
+        mark(5)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-resident timing: K steps between two events, per-kernel events inside
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    per_kernel = {n: 0.0 for n in names}
+    for i in range(args.steps):
+        for j, n in enumerate(names):
+            per_kernel[n] += evs[i][j].elapsed_time(evs[i][j + 1])
+    per_kernel = {n: t / args.steps for n, t in per_kernel.items()}
+
+    f_self, f_cross = step_flops()
+    flops_step = f_self + f_cross
+    ms_step = ms_total / args.steps
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end: pinned host inputs -> device -> hot path -> outputs to pinned host
+    pin = {n: torch.from_numpy(a.view(np.int16)).pin_memory() for n, a in host.items()}
+    res_host = {"out": torch.empty(out.shape, dtype=torch.int16).pin_memory(),
+                "lse": torch.empty(lse.shape, dtype=torch.float32).pin_memory(),
+                "oc": torch.empty(oc.shape, dtype=torch.int16).pin_memory(),
+                "lc": torch.empty(lc.shape, dtype=torch.float32).pin_memory()}
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in res_host.values())
+
+    def e2e_step():
+        for n, t in pin.items():
+            d[n].view(torch.int16).copy_(t, non_blocking=True)
+        step()
+        res_host["out"].copy_(out.view(torch.int16), non_blocking=True)
+        res_host["lse"].copy_(lse, non_blocking=True)
+        res_host["oc"].copy_(oc.view(torch.int16), non_blocking=True)
+        res_host["lc"].copy_(lc, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
+    e2e_value = world * flops_step / (ms_e2e * 1e-3) / 1e12
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    if rank != 0:
+        return None
+
+    pk, pk_src = peaks()
+    t_self = per_kernel["attn_self"]
+    achieved = f_self / (t_self * 1e-3) / 1e12
+    peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded splitmix64 normals; RMSNormed Q/K; no weights involved)",
+        "config": {
+            "workload": "win77_s31200 self-attention + RoPE, cross-attention to 1560 reference + 512 "
+                        "conditioning tokens merged by LSE (one denoising step of the 77-frame window)",
+            "B": B, "H": H, "S": S, "D": D, "Skv_cross": [N_REF, wc.Skv - N_REF],
+            "latent_grid": [T, Hh, Ww], "scale": scale,
+            "l2": "inputs larger than L2 (320 MB per tensor vs 126 MB); no flush",
+            "parallelism": f"replicas{world}",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "attn_fwd (self-attention, 31200 x 31200, H=40, D=128)",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": f"{pk_src} bf16_tflops_sustained (kernel timed inside a back-to-back loop)",
+            "frac_of_burst_peak": round(achieved / float(pk["bf16_tflops"]), 4),
+            "frac_of_nominal_2250": round(achieved / 2250.0, 4),
+            "traffic": traffic_from_profile(),
+            "algorithmic_flops_per_launch": f_self,
+        },
+        "kernels_ms": {n: round(t, 4) for n, t in per_kernel.items()},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(ms_e2e, 3),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk,
+    }
+    s_merge = per_kernel["lse_merge"]
+    s_rope = per_kernel["rope3d"]
+    line["hbm"] = {
+        "rope3d_gbs": round(4 * B * H * S * D * 2 / (s_rope * 1e-3) / 1e9, 1),
+        "lse_merge_gbs": round((3 * B * H * S * D * 2 + 3 * B * H * S * 4) / (s_merge * 1e-3) / 1e9, 1),
+        "peak_gbs": float(pk["hbm_gbs"]),
+    }
+    return line
+
+
+# ------------------------------------------------------ CPU (oracle) ---
+
+def cpu_sample_rate(target_s: float, seed_rows: int = 0):
+    """Time the fp64 oracle on a bounded sample of query rows of the 77-frame
+    self-attention. RoPE is not applied to the sample's inputs: the values do
+    not change the oracle's cost, and the oracle's RoPE adds no FLOPs counted here."""
+    import oracle
+    from dit_attention_b200 import synth
+    w = synth.WORKLOADS[SELF]
+    q, k, v = synth.make_inputs(w)
+    qr, kr = q, k
+    rng = np.random.default_rng(seed_rows)
+    BH = w.B * w.H
+    # calibrate t(rows) = a + b*rows on two sizes, then size the sample to about target_s
+    def timed(n):
+        rows = rng.choice(BH * w.Sq, size=n, replace=False)
+        t = time.perf_counter()
+        oracle.attention(qr, kr, v, w.scale, rows=rows)
+        return time.perf_counter() - t
+    n1, n2 = 32, 256
+    t1, t2 = timed(n1), timed(n2)
+    per_row = max((t2 - t1) / (n2 - n1), 1e-6)
+    fixed = max(t1 - per_row * n1, 0.0)
+    n_full = int(min(BH * w.Sq, max(64, (target_s - fixed) / per_row)))
+    return dict(q=qr, k=kr, v=v, w=w, rng=rng, rows=n_full, threads=oracle.num_threads())
+
+
+def time_cpu(sample, rows):
+    import oracle
+    w = sample["w"]
+    r = sample["rng"].choice(w.B * w.H * w.Sq, size=rows, replace=False)
+    t = time.perf_counter()
+    oracle.attention(sample["q"], sample["k"], sample["v"], w.scale, rows=r)
+    dt = time.perf_counter() - t
+    flops = 4.0 * rows * w.Skv * w.D
+    return flops / dt / 1e12, dt
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    sample = cpu_sample_rate(min(3.0, args.cpu_seconds))
+    for _ in range(args.warmup):
+        time_cpu(sample, max(16, sample["rows"] // 8))
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        v, dt = time_cpu(sample, sample["rows"])
+        vals.append(v)
+        secs += dt
+    value = statistics.mean(vals)
+    desc = (f"{sample['rows']} random query rows per step of the 77-frame self-attention "
+            f"(all 31200 keys, D=128), fp64")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * secs / args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": "win77_s31200 self-attention rows (CPU oracle)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": sample["threads"], "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    line = run_native(args, rank, world, local_rank)
+    if line is not None and not args.no_cpu_baseline:
+        sample = cpu_sample_rate(args.cpu_seconds)
+        v, dt = time_cpu(sample, sample["rows"])
+        line["cpu_baseline"] = {
+            "value": v, "unit": "TFLOP/s", "cores": sample["threads"], "kind": "oracle",
+            "sample": f"{sample['rows']} random query rows of the 77-frame self-attention (all 31200 keys, "
+                      f"D=128), fp64, {dt:.1f} s",
+        }
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,1 +1,190 @@
-"""DiT attention hot path for B200 (sm_100a)."""
+"""DiT attention hot path for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over ``libregen_attn.so`` (C ABI in include/regen_attn.h).
+Every computation runs in the library's CUDA kernels; this module only
+marshals torch tensors (or raw integer device pointers) into the C calls and
+raises ``RegenError`` on a non-zero status. There is no CPU fallback: if the
+library is missing or fails to load, every entry point raises.
+
+Entry points (same names as the C ABI):
+    regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream=None)
+    regen_rope3d(q, k, T, Hh, Ww, theta, B, H, D, stream=None)
+    regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream=None)
+    regen_last_device_error() -> (status, site)
+    regen_set_wait_limit_ns(ns)
+Convenience wrappers that allocate outputs with torch:
+    attn_fwd(q, k, v, scale=None) -> (out, lse)
+    rope3d_(q, k, grid, theta=10000.0)
+    lse_merge(o_a, lse_a, o_b, lse_b) -> (out, lse)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+__all__ = [
+    "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
+    "regen_status_str", "regen_last_device_error", "regen_set_wait_limit_ns", "regen_version",
+    "attn_fwd", "rope3d_", "lse_merge", "STATUS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libregen_attn.so")
+_lock = threading.Lock()
+_lib = None
+
+STATUS = {0: "REGEN_OK", -1: "REGEN_ERR_INVALID_ARG", -2: "REGEN_ERR_UNSUPPORTED",
+          -3: "REGEN_ERR_MISALIGNED", -4: "REGEN_ERR_CUDA", -5: "REGEN_ERR_TIMEOUT"}
+
+
+class RegenError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({_status_text(status)})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libregen_attn.so (raises if it is not built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is not built; run `python -m dit_attention_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+        L.regen_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
+        L.regen_attn_fwd.restype = i32
+        L.regen_rope3d.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, vp]
+        L.regen_rope3d.restype = i32
+        L.regen_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, vp]
+        L.regen_lse_merge.restype = i32
+        L.regen_status_str.argtypes = [i32]
+        L.regen_status_str.restype = ctypes.c_char_p
+        L.regen_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+        L.regen_last_device_error.restype = i32
+        L.regen_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.regen_set_wait_limit_ns.restype = i32
+        L.regen_version.argtypes = []
+        L.regen_version.restype = i32
+        _lib = L
+        return _lib
+
+
+def _status_text(status: int) -> str:
+    try:
+        return load().regen_status_str(status).decode()
+    except Exception:  # the library itself failed to load
+        return "?"
+
+
+def _ptr(x):
+    """Device address of a tensor (or an integer address, or None -> NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise RegenError(rc, what)
+
+
+# ------------------------------------------------------------- C names ---
+
+def regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream=None) -> None:
+    _check(load().regen_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D,
+                                 float(scale), _stream(stream)), "regen_attn_fwd")
+
+
+def regen_rope3d(q, k, T, Hh, Ww, theta, B, H, D, stream=None) -> None:
+    _check(load().regen_rope3d(_ptr(q), _ptr(k), T, Hh, Ww, float(theta), B, H, D, _stream(stream)),
+           "regen_rope3d")
+
+
+def regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream=None) -> None:
+    _check(load().regen_lse_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out),
+                                  _ptr(lse_out), int(rows), D, _stream(stream)), "regen_lse_merge")
+
+
+def regen_status_str(status: int) -> str:
+    return load().regen_status_str(status).decode()
+
+
+def regen_last_device_error():
+    """(status, site): synchronises the device, reads and clears the kernels' error record."""
+    site = ctypes.c_uint32(0)
+    rc = load().regen_last_device_error(ctypes.byref(site))
+    return rc, site.value
+
+
+def regen_set_wait_limit_ns(ns: int) -> None:
+    _check(load().regen_set_wait_limit_ns(int(ns)), "regen_set_wait_limit_ns")
+
+
+def regen_version() -> int:
+    return load().regen_version()
+
+
+# ------------------------------------------------------- torch helpers ---
+
+def _bhsd(t, name):
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B, H, S, D] tensor")
+    return t.shape
+
+
+def attn_fwd(q, k, v, scale=None, out=None, lse=None, stream=None):
+    """Exact attention on bf16 [B, H, S, D] CUDA tensors -> (out bf16, lse fp32)."""
+    import torch
+    B, H, Sq, D = _bhsd(q, "q")
+    Skv = _bhsd(k, "k")[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream)
+    return out, lse
+
+
+def rope3d_(q, k, grid, theta=10000.0, stream=None):
+    """3D RoPE in place on bf16 [B, H, T*Hh*Ww, D] CUDA tensors (either may be None)."""
+    ref = q if q is not None else k
+    B, H, S, D = _bhsd(ref, "q/k")
+    T, Hh, Ww = grid
+    if S != T * Hh * Ww:
+        raise ValueError("sequence length does not match the latent grid")
+    regen_rope3d(q, k, T, Hh, Ww, theta, B, H, D, stream)
+    return q, k
+
+
+def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None, stream=None):
+    """Merge two partial attentions (bf16 [..., D], fp32 [...]) -> (out, lse)."""
+    import torch
+    D = o_a.shape[-1]
+    rows = o_a.numel() // D
+    if out is None:
+        out = torch.empty_like(o_a)
+    if lse_out is None:
+        lse_out = torch.empty_like(lse_a)
+    regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream)
+    return out, lse_out

@@ -1,0 +1,458 @@
+// attn_fwd.cuh -- exact softmax attention forward for sm_100a.
+//
+// What it computes (ReGenVC, blog.captcha.la page, "Technical innovations":
+// the DiT's attention stays exact under Ulysses x Ring sharding; Ring
+// attention streams KV blocks and combines them by their log-sum-exp):
+//   out_i = sum_j softmax_j(scale * <q_i, k_j>) v_j,  lse_i = ln sum_j exp(scale * <q_i, k_j>)
+// One pass over 128-key blocks with an online softmax, i.e. the same
+// blockwise LSE combination Ring attention applies between GPUs, applied
+// here between key blocks of one GPU.
+//
+// Work unit = one CTA = one (batch*head, 256 query rows) = two 128-row Q tiles;
+// grid = B*H*ceil(Sq/256) CTAs.
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q tiles once, then K/V tiles through NS-stage rings
+//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma and commit
+//   warps 2-3   idle
+//   warps 4-7   softmax + correction + epilogue for Q tile 0 (one thread per row)
+//   warps 8-11  the same for Q tile 1
+// Tensor memory (512 columns, fp32): S0 [0,128), S1 [128,256), O0 and O1 after
+// them (HD columns each). P (bf16) is written over the first 64 columns of
+// its S and fed to the PV MMA straight from TMEM.
+// MMA order, ping-ponging the two tiles so that one tile's softmax overlaps
+// the other tile's MMAs:
+//   S0(0) S1(0) | PV0(0) S0(1) | PV1(0) S1(1) | PV0(1) S0(2) | ...
+// Softmax keeps a per-row running max m (log2 units, scale folded in) and
+// sum l in fp32; O is rescaled only when the max grows by more than 8
+// (log2), which stays exact because P = 2^(s - m) is then at most 2^8 and
+// the final O/l and LSE use the same m.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace regen {
+
+__device__ int g_regen_err;            // first error code recorded by a kernel
+__device__ unsigned int g_regen_err_site;  // which wait gave up
+
+enum WaitSite : uint32_t {
+    SITE_PROD_K_EMPTY = 1,
+    SITE_PROD_V_EMPTY = 2,
+    SITE_MMA_Q = 3,
+    SITE_MMA_K_FULL = 4,
+    SITE_MMA_V_FULL = 5,
+    SITE_MMA_P_FULL = 6,
+    SITE_SM_S_FULL = 7,
+    SITE_SM_O_FULL = 8,
+    SITE_DRAIN = 9,
+};
+
+__device__ __forceinline__ void record_timeout(uint32_t site)
+{
+    if (atomicCAS(&g_regen_err, 0, -5 /* REGEN_ERR_TIMEOUT */) == 0) g_regen_err_site = site;
+}
+
+struct WaitCtl {
+    volatile int *abort;   // CTA-wide flag in shared memory
+    uint64_t limit_ns;
+};
+
+// Bounded wait on an mbarrier phase. Returns false when the CTA is aborting
+// (another role gave up) or when this wait exceeded the limit (then it
+// records the site and raises the abort flag).
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32_t site,
+                                           const WaitCtl &w)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 31) == 0) {
+            if (*w.abort) return false;
+            if (global_timer_ns() - t0 > w.limit_ns) {
+                record_timeout(site);
+                *w.abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+template <int HD>
+struct AttnCfg {
+    static constexpr int BM = 128;                        // query rows per tile
+    static constexpr int BN = 128;                        // keys per block
+    static constexpr int HALVES = HD / 64;                // 128-byte column groups per row
+    static constexpr int TILE_BYTES = 128 * HD * 2;       // one 128-row bf16 tile
+    static constexpr int HALF_BYTES = 128 * 128;          // 128 rows x 128 bytes
+    static constexpr int NS = (HD == 128) ? 2 : 4;        // K ring and V ring depth
+    static constexpr int Q_OFF = 0;
+    static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
+    static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
+    static constexpr int BAR_OFF = V_OFF + NS * TILE_BYTES;
+    // barriers: q, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2],
+    // o_full[2], drain
+    static constexpr int NBARS = 1 + 4 * NS + 6 + 1;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;  // abort flag, TMEM base
+    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int THREADS = 384;
+};
+
+template <int HD, bool NEG_SCALE>
+__global__ void __launch_bounds__(384, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    float *__restrict__ lse, int Sq, int Skv, float scale_log2,
+                    uint64_t wait_limit_ns)
+{
+    using C = AttnCfg<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const uint32_t bar0 = sbase + C::BAR_OFF;
+    const uint32_t bar_q = bar0;
+    auto bar_k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto bar_k_empty = [&](int s) { return bar0 + 8u * (1 + C::NS + s); };
+    auto bar_v_full = [&](int s) { return bar0 + 8u * (1 + 2 * C::NS + s); };
+    auto bar_v_empty = [&](int s) { return bar0 + 8u * (1 + 3 * C::NS + s); };
+    auto bar_s_full = [&](int t) { return bar0 + 8u * (1 + 4 * C::NS + t); };
+    auto bar_p_full = [&](int t) { return bar0 + 8u * (3 + 4 * C::NS + t); };
+    auto bar_o_full = [&](int t) { return bar0 + 8u * (5 + 4 * C::NS + t); };
+    const uint32_t bar_drain = bar0 + 8u * (7 + 4 * C::NS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 8);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(bar_k_full(s), 1);
+            mbar_init(bar_k_empty(s), 1);
+            mbar_init(bar_v_full(s), 1);
+            mbar_init(bar_v_empty(s), 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar_s_full(t), 1);
+            mbar_init(bar_p_full(t), 128);
+            mbar_init(bar_o_full(t), 1);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    const WaitCtl wc{abort_flag, wait_limit_ns};
+    const int nkv = (Skv + C::BN - 1) / C::BN;
+    // 1-D grid, query-tile pairs of one head adjacent so that the CTAs resident
+    // at any time share the K/V of one or two heads in L2.
+    const int npairs = (Sq + 2 * C::BM - 1) / (2 * C::BM);
+    const int bh = static_cast<int>(blockIdx.x / npairs);
+    const int q0 = static_cast<int>(blockIdx.x % npairs) * (2 * C::BM);
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer ---
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const uint64_t keep = l2_policy_evict_last();   // K/V: re-read by every Q tile of the head
+            const uint64_t once = l2_policy_evict_first();  // Q: read once
+            mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+            for (int t = 0; t < 2; ++t)
+                for (int h = 0; h < C::HALVES; ++h)
+                    tma_load_3d(sbase + C::Q_OFF + t * C::TILE_BYTES + h * C::HALF_BYTES, &tm_q, bar_q,
+                                h * 64, q0 + t * C::BM, bh, once);
+            int nk = 0, nv = 0;  // K and V block loads issued so far
+            bool ok = true;
+            for (int j = 0; j < nkv; ++j) {
+                const int s = j % C::NS;
+                const uint32_t ph = (j / C::NS) & 1;
+                ok = wait_phase(bar_k_empty(s), ph ^ 1, SITE_PROD_K_EMPTY, wc);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_k_full(s), C::TILE_BYTES);
+                for (int h = 0; h < C::HALVES; ++h)
+                    tma_load_3d(sbase + C::K_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_k,
+                                bar_k_full(s), h * 64, j * C::BN, bh, keep);
+                ++nk;
+                ok = wait_phase(bar_v_empty(s), ph ^ 1, SITE_PROD_V_EMPTY, wc);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_v_full(s), C::TILE_BYTES);
+                for (int h = 0; h < C::HALVES; ++h)
+                    tma_load_3d(sbase + C::V_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_v,
+                                bar_v_full(s), h * 64, j * C::BN, bh, keep);
+                ++nv;
+            }
+            if (!ok) {
+                // Aborting: wait (bounded) for the copies this warp may still have
+                // in flight -- at most the last NS of each ring and the Q tiles --
+                // so that none lands in shared memory after the CTA has exited.
+                auto drain = [&](uint32_t bar, uint32_t parity) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < wait_limit_ns) {
+                    }
+                };
+                for (int j = (nk > C::NS ? nk - C::NS : 0); j < nk; ++j)
+                    drain(bar_k_full(j % C::NS), (j / C::NS) & 1);
+                for (int j = (nv > C::NS ? nv - C::NS : 0); j < nv; ++j)
+                    drain(bar_v_full(j % C::NS), (j / C::NS) & 1);
+                drain(bar_q, 0);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer ---
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false);  // Q.K^T, both K-major
+            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, true);    // P.V, V is MN-major
+            const uint32_t tm_s[2] = {tmem, tmem + 128u};
+            const uint32_t tm_o[2] = {tmem + 256u, tmem + 256u + HD};
+            // S_t = Q_t K_j^T : M=128, N=128, K=HD in steps of 16 (32 bytes) inside
+            // each 128-byte swizzle row; the second 64-column half starts HALF_BYTES on.
+            auto issue_s = [&](int t, int s) {
+                const uint32_t qa = sbase + C::Q_OFF + t * C::TILE_BYTES;
+                const uint32_t kb = sbase + C::K_OFF + s * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk / 4) * C::HALF_BYTES + (kk % 4) * 32;
+                    mma_ss(tm_s[t], smem_desc_sw128(qa + off, 16, 1024),
+                           smem_desc_sw128(kb + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_t += P_t V_j : M=128, N=HD, K=128 keys in steps of 16. P comes from
+            // TMEM (16 keys = 8 columns); V rows are 128-byte swizzled, 16 keys =
+            // 2048 bytes, the two 64-wide D halves are HALF_BYTES apart (LBO).
+            auto issue_pv = [&](int t, int s, bool acc) {
+                const uint32_t vb = sbase + C::V_OFF + s * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    mma_ts(tm_o[t], tm_s[t] + kk * 8, smem_desc_sw128(vb + kk * 2048, C::HALF_BYTES, 1024),
+                           IDESC_O, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = wait_phase(bar_q, 0, SITE_MMA_Q, wc);
+            if (ok) ok = wait_phase(bar_k_full(0), 0, SITE_MMA_K_FULL, wc);
+            if (ok) {
+                tc_fence_after_sync();
+                issue_s(0, 0);
+                tc_commit(bar_s_full(0));
+                issue_s(1, 0);
+                tc_commit(bar_s_full(1));
+                tc_commit(bar_k_empty(0));
+            }
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int s = j % C::NS;
+                const uint32_t ph = (j / C::NS) & 1;
+                const int s1 = (j + 1) % C::NS;
+                const uint32_t ph1 = ((j + 1) / C::NS) & 1;
+                const bool more = j + 1 < nkv;
+                ok = wait_phase(bar_v_full(s), ph, SITE_MMA_V_FULL, wc);
+                if (!ok) break;
+                ok = wait_phase(bar_p_full(0), j & 1, SITE_MMA_P_FULL, wc);
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_pv(0, s, j > 0);
+                if (more) {
+                    ok = wait_phase(bar_k_full(s1), ph1, SITE_MMA_K_FULL, wc);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    issue_s(0, s1);
+                    tc_commit(bar_s_full(0));
+                } else {
+                    tc_commit(bar_o_full(0));
+                }
+                ok = wait_phase(bar_p_full(1), j & 1, SITE_MMA_P_FULL, wc);
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_pv(1, s, j > 0);
+                tc_commit(bar_v_empty(s));
+                if (more) {
+                    issue_s(1, s1);
+                    tc_commit(bar_s_full(1));
+                    tc_commit(bar_k_empty(s1));
+                } else {
+                    tc_commit(bar_o_full(1));
+                }
+            }
+            // Drain: nothing may still be running on the tensor core when TMEM is freed.
+            tc_commit(bar_drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_drain, 0)) {
+                if (global_timer_ns() - t0 > wait_limit_ns) {
+                    record_timeout(SITE_DRAIN);
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // -------------------------------------------- softmax + epilogue ---
+        const int t = (warp - 4) >> 2;     // Q tile of this warpgroup
+        const int quad = warp & 3;         // TMEM lane quadrant this warp may access
+        const int row = quad * 32 + lane;  // row inside the tile
+        const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t ts = tmem + lane_bits + t * 128u;
+        const uint32_t to = tmem + lane_bits + 256u + t * HD;
+        const int kv_tail = Skv - (nkv - 1) * C::BN;  // valid keys in the last block (1..128)
+        float m = 0.f;   // running max of scaled logits (log2 units); set by block 0
+        float l = 0.f;   // running sum of 2^(s - m)
+        bool ok = true;
+        for (int j = 0; j < nkv; ++j) {
+            // every lane waits; the outcome is made warp-uniform so that the
+            // warp-collective tcgen05 ops below never run on a partial warp
+            ok = __all_sync(0xffffffffu, wait_phase(bar_s_full(t), j & 1, SITE_SM_S_FULL, wc));
+            if (!ok) break;
+            tc_fence_after_sync();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(ts + c * 32, sr[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+            const bool last = (j == nkv - 1);
+            if (last && kv_tail < C::BN) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c * 32 + i >= kv_tail)
+                            sr[c][i] = __float_as_uint(NEG_SCALE ? INFINITY : -INFINITY);
+            }
+            // row extreme of the raw logits -> max of the scaled logits
+            float mx = __uint_as_float(sr[0][0]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    mx = NEG_SCALE ? fminf(mx, __uint_as_float(sr[c][i]))
+                                   : fmaxf(mx, __uint_as_float(sr[c][i]));
+            const float mnew = mx * scale_log2;
+            // Stale-max rule: move m (and rescale O, l) only when the block max
+            // exceeds it by more than 8 in log2 units.
+            bool grow = false;
+            float alpha = 1.0f;
+            if (j == 0) {
+                m = mnew;
+            } else if (mnew > m + 8.0f) {
+                grow = true;
+                alpha = ex2_approx(m - mnew);
+                m = mnew;
+                l *= alpha;
+            }
+            // P = 2^(s*scale_log2 - m), summed in fp32 before rounding to bf16.
+            const float neg_m = -m;
+            float rs = 0.f;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {   // 64 keys -> 32 packed columns per half
+                uint32_t pk[32];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = hv * 2 + cc;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][i]), scale_log2, neg_m));
+                        float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][i + 1]), scale_log2, neg_m));
+                        if (last && kv_tail < C::BN) {
+                            if (c * 32 + i >= kv_tail) p0 = 0.f;
+                            if (c * 32 + i + 1 >= kv_tail) p1 = 0.f;
+                        }
+                        rs += p0 + p1;
+                        pk[cc * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
+                    }
+                }
+                tmem_st_32x32b_x32(ts + hv * 32, pk);
+            }
+            l += rs;
+            // O_t holds exactly PV_t(0..j-1) here: the commit that signalled S_t(j)
+            // follows PV_t(j-1), and PV_t(j) waits for this warpgroup's arrive.
+            if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(to + c * 32, o);
+                    tmem_ld_wait();
+                    reg_fence(o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st_32x32b_x32(to + c * 32, o);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before_sync();
+            mbar_arrive(bar_p_full(t));
+        }
+        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_o_full(t), 0, SITE_SM_O_FULL, wc));
+        if (ok) {
+            tc_fence_after_sync();
+            // Epilogue: O / l -> bf16 into this tile's Q buffer (free now: every
+            // MMA that read it has completed), in the same 128-byte swizzled
+            // layout TMA uses, then one TMA store per 64-column half. Rows past
+            // Sq fall outside the tensor map and are not written.
+            const float inv_l = 1.0f / l;
+            uint8_t *stage = smem + C::Q_OFF + t * C::TILE_BYTES;
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(to + c * 32, o);
+                tmem_ld_wait();
+                reg_fence(o);
+                const int half = c >> 1;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {  // four 16-byte chunks of 8 values
+                    const int chunk = (c & 1) * 4 + g;
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(o[g * 8 + 0]) * inv_l, __uint_as_float(o[g * 8 + 1]) * inv_l);
+                    w.y = pack_bf16x2(__uint_as_float(o[g * 8 + 2]) * inv_l, __uint_as_float(o[g * 8 + 3]) * inv_l);
+                    w.z = pack_bf16x2(__uint_as_float(o[g * 8 + 4]) * inv_l, __uint_as_float(o[g * 8 + 5]) * inv_l);
+                    w.w = pack_bf16x2(__uint_as_float(o[g * 8 + 6]) * inv_l, __uint_as_float(o[g * 8 + 7]) * inv_l);
+                    uint8_t *dst = stage + half * C::HALF_BYTES + row * 128 + ((chunk ^ (row & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(dst) = w;
+                }
+            }
+            const int qrow = q0 + t * C::BM + row;
+            if (lse != nullptr && qrow < Sq)
+                lse[static_cast<int64_t>(bh) * Sq + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+            fence_proxy_async_smem();
+        }
+        // Reached by all 128 threads of the warpgroup on every path.
+        named_bar_sync(1 + t, 128);
+        if (ok && warp == 4 + 4 * t && lane == 0 && q0 + t * C::BM < Sq) {
+            for (int h = 0; h < C::HALVES; ++h)
+                tma_store_3d(&tm_o, sbase + C::Q_OFF + t * C::TILE_BYTES + h * C::HALF_BYTES, h * 64,
+                             q0 + t * C::BM, bh);
+            tma_store_commit();
+            tma_store_wait_all();
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// Skv == 0: the empty softmax. out = 0, lse = -inf.
+__global__ void attn_empty_kernel(uint4 *__restrict__ out, int64_t n16, float *__restrict__ lse,
+                                  int64_t nrows)
+{
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n16; i += stride)
+        out[i] = make_uint4(0, 0, 0, 0);
+    if (lse)
+        for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nrows; i += stride)
+            lse[i] = -INFINITY;
+}
+
+}  // namespace regen

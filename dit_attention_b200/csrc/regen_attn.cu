@@ -1,0 +1,233 @@
+// regen_attn.cu -- C ABI of the DiT attention hot path (declared in
+// include/regen_attn.h): argument checks, TMA descriptor encoding, launches.
+//
+// Every argument check runs before the first CUDA call, so invalid calls are
+// answered on machines without a GPU as well. Launches are asynchronous on
+// the caller's stream; nothing here synchronises except
+// regen_last_device_error().
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "regen_attn.h"
+
+#include "attn_fwd.cuh"
+#include "lse_merge.cuh"
+#include "rope3d.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, int64_t abytes, const void *b, int64_t bbytes)
+{
+    if (!a || !b || abytes <= 0 || bbytes <= 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + static_cast<uintptr_t>(bbytes) && b0 < a0 + static_cast<uintptr_t>(abytes);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// [BH, S, D] bf16 viewed as a 3D tensor (D innermost), boxes of 64 x 128 x 1
+// with the 128-byte swizzle; out-of-range rows read as zero.
+bool make_bhsd_map(CUtensorMap *map, const void *base, int64_t BH, int64_t S, int64_t D)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D * 2), static_cast<cuuint64_t>(S * D * 2)};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int HD, bool NEG>
+int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, regen_bf16 *out,
+                float *lse, int64_t BH, int Sq, int Skv, float scale, cudaStream_t stream)
+{
+    using C = regen::AttnCfg<HD>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(regen::attn_fwd_kernel<HD, NEG>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return REGEN_ERR_CUDA;
+    CUtensorMap tq, tk, tv, to;
+    if (!make_bhsd_map(&tq, q, BH, Sq, HD) || !make_bhsd_map(&tk, k, BH, Skv, HD) ||
+        !make_bhsd_map(&tv, v, BH, Skv, HD) || !make_bhsd_map(&to, out, BH, Sq, HD))
+        return REGEN_ERR_CUDA;
+    const int64_t npairs = (Sq + 2 * C::BM - 1) / (2 * C::BM);
+    const int64_t grid = npairs * BH;
+    if (grid > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    regen::attn_fwd_kernel<HD, NEG><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, to, lse, Sq, Skv, scale_log2, g_wait_limit_ns.load());
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
+int grid_for(int64_t work, int threads)
+{
+    int64_t blocks = (work + threads - 1) / threads;
+    const int64_t cap = 148 * 32;  // grid-stride beyond ~32 resident blocks per SM
+    if (blocks > cap) blocks = cap;
+    return static_cast<int>(blocks < 1 ? 1 : blocks);
+}
+
+}  // namespace
+
+extern "C" {
+
+REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
+                             regen_bf16 *out, float *lse, int B, int H, int Sq, int Skv, int D,
+                             float scale, regen_stream_t stream)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Skv < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0 || Sq == 0) return REGEN_OK;
+    if (BH > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (!q || !out || (Skv > 0 && (!k || !v))) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (Skv > 0 && (!aligned16(k) || !aligned16(v))))
+        return REGEN_ERR_MISALIGNED;
+    const int64_t qbytes = BH * Sq * D * 2, kvbytes = BH * Skv * D * 2, lbytes = BH * Sq * 4;
+    if (overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) ||
+        overlaps(out, qbytes, v, kvbytes) || overlaps(lse, lbytes, q, qbytes) ||
+        overlaps(lse, lbytes, k, kvbytes) || overlaps(lse, lbytes, v, kvbytes) ||
+        overlaps(lse, lbytes, out, qbytes))
+        return REGEN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (Skv == 0) {
+        const int64_t n16 = qbytes / 16;
+        regen::attn_empty_kernel<<<grid_for(n16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(out), n16,
+                                                                      lse, BH * Sq);
+        return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    }
+    const bool neg = scale < 0.0f;
+    if (D == 128)
+        return neg ? launch_attn<128, true>(q, k, v, out, lse, BH, Sq, Skv, scale, st)
+                   : launch_attn<128, false>(q, k, v, out, lse, BH, Sq, Skv, scale, st);
+    return neg ? launch_attn<64, true>(q, k, v, out, lse, BH, Sq, Skv, scale, st)
+               : launch_attn<64, false>(q, k, v, out, lse, BH, Sq, Skv, scale, st);
+}
+
+REGEN_API int regen_rope3d(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta, int B,
+                           int H, int D, regen_stream_t stream)
+{
+    if (T <= 0 || Hh <= 0 || Ww <= 0 || B < 0 || H < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(theta) || !(theta > 0.0f)) return REGEN_ERR_INVALID_ARG;
+    if (D < 8 || D > 512 || (D % 8) != 0) return REGEN_ERR_UNSUPPORTED;
+    const int64_t S = static_cast<int64_t>(T) * Hh * Ww;
+    if (S > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0) return REGEN_OK;
+    if (!q && !k) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k)) return REGEN_ERR_MISALIGNED;
+    const int64_t bytes = BH * S * D * 2;
+    if (overlaps(q, bytes, k, bytes)) return REGEN_ERR_INVALID_ARG;
+    const int64_t work = S * (D / 8);
+    const int threads = 128;
+    const int64_t blocks = (work + threads - 1) / threads;
+    if (blocks > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    regen::rope3d_kernel<<<static_cast<unsigned>(blocks), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        q, k, BH, static_cast<int>(S), Hh, Ww, D, static_cast<double>(theta));
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
+REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a, const regen_bf16 *o_b,
+                              const float *lse_b, regen_bf16 *out, float *lse_out, int64_t rows, int D,
+                              regen_stream_t stream)
+{
+    if (rows < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (D < 8 || D > 512 || (D % 8) != 0) return REGEN_ERR_UNSUPPORTED;
+    if (rows == 0) return REGEN_OK;
+    if (!o_a || !lse_a || !o_b || !lse_b || !out) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(out) || !aligned16(lse_a) || !aligned16(lse_b) ||
+        !aligned16(lse_out))
+        return REGEN_ERR_MISALIGNED;
+    const int64_t obytes = rows * D * 2, lbytes = rows * 4;
+    if (overlaps(lse_out, lbytes, lse_a, lbytes) || overlaps(lse_out, lbytes, lse_b, lbytes) ||
+        overlaps(lse_out, lbytes, o_a, obytes) || overlaps(lse_out, lbytes, o_b, obytes) ||
+        overlaps(lse_out, lbytes, out, obytes) || overlaps(out, obytes, lse_a, lbytes) ||
+        overlaps(out, obytes, lse_b, lbytes))
+        return REGEN_ERR_INVALID_ARG;
+    // out may coincide exactly with o_a or o_b (each chunk is read before it is
+    // written by the same thread); a partial overlap is rejected.
+    if ((overlaps(out, obytes, o_a, obytes) && out != o_a) || (overlaps(out, obytes, o_b, obytes) && out != o_b))
+        return REGEN_ERR_INVALID_ARG;
+    const int64_t work = rows * (D / 8);
+    regen::lse_merge_kernel<<<grid_for(work, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint4 *>(o_a), lse_a, reinterpret_cast<const uint4 *>(o_b), lse_b,
+        reinterpret_cast<uint4 *>(out), lse_out, rows, D);
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
+REGEN_API const char *regen_status_str(int status)
+{
+    switch (status) {
+    case REGEN_OK: return "ok";
+    case REGEN_ERR_INVALID_ARG: return "invalid argument";
+    case REGEN_ERR_UNSUPPORTED: return "unsupported size or head dim";
+    case REGEN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case REGEN_ERR_CUDA: return "CUDA error";
+    case REGEN_ERR_TIMEOUT: return "kernel gave up on a bounded wait";
+    default: return "unknown status";
+    }
+}
+
+REGEN_API int regen_last_device_error(uint32_t *detail)
+{
+    if (detail) *detail = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return REGEN_ERR_CUDA;
+    int code = 0;
+    unsigned int site = 0;
+    if (cudaMemcpyFromSymbol(&code, regen::g_regen_err, sizeof code) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&site, regen::g_regen_err_site, sizeof site) != cudaSuccess)
+        return REGEN_ERR_CUDA;
+    if (code != 0) {
+        const int zero = 0;
+        const unsigned int uzero = 0;
+        if (cudaMemcpyToSymbol(regen::g_regen_err, &zero, sizeof zero) != cudaSuccess ||
+            cudaMemcpyToSymbol(regen::g_regen_err_site, &uzero, sizeof uzero) != cudaSuccess)
+            return REGEN_ERR_CUDA;
+    }
+    if (detail) *detail = site;
+    return code == 0 ? REGEN_OK : code;
+}
+
+REGEN_API int regen_set_wait_limit_ns(uint64_t ns)
+{
+    g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns);
+    return REGEN_OK;
+}
+
+REGEN_API int regen_version(void) { return 100; }
+
+}  // extern "C"

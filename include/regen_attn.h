@@ -1,0 +1,143 @@
+/*
+ * regen_attn.h -- C ABI of the DiT attention hot path on NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of the ReGenVC decoder's diffusion transformer
+ * (arXiv 2607.28144): exact softmax attention over the flattened latent
+ * token sequence (blog.captcha.la page, "Technical innovations": the
+ * Ulysses x Ring sequence parallelism keeps attention exact), its 3D rotary
+ * embedding (the decoder matches the Wan2.1-Fun-Control architecture, blog
+ * page "Methodology -- deep read"), and the log-sum-exp merge of partial
+ * results over key blocks that Ring attention performs while it streams KV
+ * blocks around the GPUs (same section).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major, in [B, H, S, D] order ("BHSD"): element
+ *    (b, h, s, d) sits at ((b*H + h)*S + s)*D + d. No strides.
+ *  - regen_bf16 is the bit pattern of a bfloat16 value; LSE values are fp32
+ *    natural logarithms in units of the scaled logits.
+ *  - Every pointer is a DEVICE pointer owned by the caller; the library keeps
+ *    no reference after the call returns and allocates no device memory per
+ *    call. Pointers must be 16-byte aligned.
+ *  - Calls are asynchronous and stream-ordered on `stream` (NULL = the legacy
+ *    default stream). The return value reports argument and launch errors
+ *    only. A kernel that gives up on a bounded wait records a code that
+ *    regen_last_device_error() reports after the caller synchronises.
+ *  - Inputs and outputs must not overlap, except where "in place" is stated.
+ */
+#ifndef REGEN_ATTN_H
+#define REGEN_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define REGEN_API __declspec(dllexport)
+#else
+#define REGEN_API __attribute__((visibility("default")))
+#endif
+
+typedef uint16_t regen_bf16;
+typedef struct CUstream_st *regen_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    REGEN_OK = 0,
+    REGEN_ERR_INVALID_ARG = -1,  /* NULL pointer, negative size, non-finite scale */
+    REGEN_ERR_UNSUPPORTED = -2,  /* head dim or size outside the supported set */
+    REGEN_ERR_MISALIGNED = -3,   /* a pointer is not 16-byte aligned */
+    REGEN_ERR_CUDA = -4,         /* the CUDA runtime or driver reported an error */
+    REGEN_ERR_TIMEOUT = -5       /* a kernel gave up on a bounded wait */
+} regen_status;
+
+/*
+ * regen_attn_fwd -- exact bidirectional multi-head softmax attention.
+ *
+ * For every (b, h) and query i < Sq, with s_j = scale * <q_i, k_j>, j < Skv:
+ *     out_i = sum_j softmax(s)_j v_j        lse_i = ln sum_j exp(s_j)
+ * (self-attention: Sq == Skv over the same latent tokens; cross-attention:
+ * Skv conditioning / reference-frame tokens). Computed in one pass over key
+ * blocks with an fp32 online softmax; QK^T and PV run on the tensor cores in
+ * bf16 with fp32 accumulation; out is rounded to bf16 (nearest even).
+ *
+ *   q    [B, H, Sq,  D] bf16        k, v [B, H, Skv, D] bf16
+ *   out  [B, H, Sq,  D] bf16        lse  [B, H, Sq] fp32, or NULL to skip it
+ *   D    64 or 128 (else REGEN_ERR_UNSUPPORTED)
+ *   scale  any finite float (1/sqrt(D) is the usual one)
+ * B, H or Sq == 0: nothing to do, REGEN_OK. Skv == 0: out = 0, lse = -inf.
+ * Sizes: B*H < 2^31, Sq and Skv < 2^31 with B*H*S*D < 2^62.
+ */
+REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
+                             regen_bf16 *out, float *lse,
+                             int B, int H, int Sq, int Skv, int D, float scale,
+                             regen_stream_t stream);
+
+/*
+ * regen_rope3d -- 3D rotary position embedding of Q and K, in place.
+ *
+ * The sequence is the flattened latent grid: token n = (t*Hh + y)*Ww + x,
+ * S = T*Hh*Ww. The head dim splits into axis blocks t, h, w of widths
+ * D - 4*floor(D/6), 2*floor(D/6), 2*floor(D/6) (44/42/42 at D = 128); in a
+ * block of width d_a the pair (2j, 2j+1) turns by pos_a * theta^(-2j/d_a):
+ *     x'_{2j} = x_{2j} cos - x_{2j+1} sin,   x'_{2j+1} = x_{2j} sin + x_{2j+1} cos
+ * Angles and the rotation are evaluated in fp64 and the result is rounded
+ * once to bf16 (nearest even).
+ *
+ *   q, k   [B, H, S, D] bf16, rotated in place; either may be NULL (skipped),
+ *          not both. q and k must not overlap.
+ *   T, Hh, Ww > 0 (their product < 2^31); theta > 0 and finite
+ *   D      even, multiple of 8, 8 <= D <= 512
+ * B or H == 0: REGEN_OK, nothing done.
+ */
+REGEN_API int regen_rope3d(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta,
+                           int B, int H, int D, regen_stream_t stream);
+
+/*
+ * regen_lse_merge -- combine two partial attentions of the same queries
+ * over disjoint key blocks a and b:
+ *     m = max(lse_a, lse_b), w_a = exp(lse_a - m), w_b = exp(lse_b - m)
+ *     out = (w_a o_a + w_b o_b) / (w_a + w_b),   lse_out = m + ln(w_a + w_b)
+ * in fp32 per row; out rounded to bf16. Rows whose two LSEs are both -inf
+ * (two empty key blocks) give out = 0 and lse_out = -inf.
+ *
+ *   o_a, o_b, out  [rows, D] bf16;  lse_a, lse_b  [rows] fp32
+ *   lse_out        [rows] fp32 or NULL (skipped); it may alias lse_a or lse_b
+ *   rows = B*H*Sq >= 0;  D multiple of 8, 8 <= D <= 512
+ * out may alias o_a or o_b (element-wise, each element is read before it is
+ * written by the same thread).
+ */
+REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a,
+                              const regen_bf16 *o_b, const float *lse_b,
+                              regen_bf16 *out, float *lse_out,
+                              int64_t rows, int D, regen_stream_t stream);
+
+/* Human-readable text of a status code (static storage). */
+REGEN_API const char *regen_status_str(int status);
+
+/*
+ * regen_last_device_error -- REGEN_OK, or REGEN_ERR_TIMEOUT when a kernel of
+ * this library gave up on a bounded wait since the previous call; clears the
+ * record. It synchronises the device first (cudaDeviceSynchronize) and
+ * returns REGEN_ERR_CUDA if that fails. *detail (may be NULL) receives a code
+ * naming the wait that expired (0 if none).
+ */
+REGEN_API int regen_last_device_error(uint32_t *detail);
+
+/*
+ * regen_set_wait_limit_ns -- upper bound, in nanoseconds, on any single wait
+ * inside the attention kernel (default 2e9 = 2 s; 0 restores the default).
+ * A wait that exceeds it makes the kernel stop, record REGEN_ERR_TIMEOUT and
+ * return; no wait in a correct run comes near the default.
+ */
+REGEN_API int regen_set_wait_limit_ns(uint64_t ns);
+
+/* Version of this ABI (major*10000 + minor*100 + patch). */
+REGEN_API int regen_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* REGEN_ATTN_H */

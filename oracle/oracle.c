@@ -88,6 +88,17 @@ void oracle_f64_to_bf16_array(const double *x, uint16_t *h, int64_t n)
 
 /* ----------------------------------------------------------- attention --- */
 
+/* An input array that is either fp64 or bf16 bit patterns (widened on access). */
+typedef struct {
+    const void *p;
+    int bf16;
+} src_t;
+
+static inline double at(src_t s, int64_t i)
+{
+    return s.bf16 ? oracle_bf16_to_f64(((const uint16_t *)s.p)[i]) : ((const double *)s.p)[i];
+}
+
 /*
  * One query row of exact softmax attention, by definition:
  *   s_j   = scale * sum_d q_d k_jd            for j < Skv
@@ -97,9 +108,10 @@ void oracle_f64_to_bf16_array(const double *x, uint16_t *h, int64_t n)
  *   out_d = (sum_j p_j v_jd) / l
  *   lse   = m + ln l                          (natural log, scaled-logit units)
  * Skv == 0 gives out = 0 and lse = -inf (the empty softmax).
+ * The query row starts at element qo of q, the head's keys/values at ko.
  * `p` is caller scratch of Skv doubles.
  */
-static void attention_row(const double *qi, const double *Kh, const double *Vh,
+static void attention_row(src_t q, int64_t qo, src_t k, src_t v, int64_t ko,
                           int64_t Skv, int64_t D, double scale,
                           double *p, double *out, double *lse)
 {
@@ -111,7 +123,7 @@ static void attention_row(const double *qi, const double *Kh, const double *Vh,
     double m = -INFINITY;
     for (int64_t j = 0; j < Skv; ++j) {
         double dot = 0.0;
-        for (int64_t d = 0; d < D; ++d) dot += qi[d] * Kh[j * D + d];
+        for (int64_t d = 0; d < D; ++d) dot += at(q, qo + d) * at(k, ko + j * D + d);
         p[j] = scale * dot;
         if (p[j] > m) m = p[j];
     }
@@ -121,7 +133,7 @@ static void attention_row(const double *qi, const double *Kh, const double *Vh,
         l += p[j];
     }
     for (int64_t j = 0; j < Skv; ++j)
-        for (int64_t d = 0; d < D; ++d) out[d] += p[j] * Vh[j * D + d];
+        for (int64_t d = 0; d < D; ++d) out[d] += p[j] * at(v, ko + j * D + d);
     for (int64_t d = 0; d < D; ++d) out[d] /= l;
     *lse = m + log(l);
 }
@@ -131,52 +143,48 @@ static void attention_row(const double *qi, const double *Kh, const double *Vh,
  * rows == NULL: every query row, out [BH*Sq][D], lse [BH*Sq].
  * rows != NULL: only the nrows global rows rows[r] = bh*Sq + i, out [nrows][D].
  */
+static int attention_rows(src_t q, src_t k, src_t v, int64_t BH, int64_t Sq, int64_t Skv,
+                          int64_t D, double scale, const int64_t *rows, int64_t nrows,
+                          double *out, double *lse)
+{
+    int64_t n = rows ? nrows : BH * Sq;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+        if (!p) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < n; ++r) {
+            if (!p) continue;
+            int64_t g = rows ? rows[r] : r;
+            int64_t bh = g / Sq;
+            attention_row(q, g * D, k, v, bh * Skv * D, Skv, D, scale, p, out + r * D, lse + r);
+        }
+        free(p);
+    }
+    return failed ? -1 : 0;
+}
+
 void oracle_attention_f64(const double *q, const double *k, const double *v,
                           int64_t BH, int64_t Sq, int64_t Skv, int64_t D, double scale,
                           const int64_t *rows, int64_t nrows,
                           double *out, double *lse)
 {
-    int64_t n = rows ? nrows : BH * Sq;
-#pragma omp parallel
-    {
-        double *p = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
-#pragma omp for schedule(dynamic, 4)
-        for (int64_t r = 0; r < n; ++r) {
-            int64_t g = rows ? rows[r] : r;
-            int64_t bh = g / Sq;
-            attention_row(q + g * D, k + bh * Skv * D, v + bh * Skv * D, Skv, D, scale,
-                          p, out + r * D, lse + r);
-        }
-        free(p);
-    }
+    src_t sq = {q, 0}, sk = {k, 0}, sv = {v, 0};
+    attention_rows(sq, sk, sv, BH, Sq, Skv, D, scale, rows, nrows, out, lse);
 }
 
-/* Same, on bf16 inputs (widened exactly to double first). */
+/* Same, on bf16 inputs (each element widened exactly to double when read). */
 int oracle_attention_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                           int64_t BH, int64_t Sq, int64_t Skv, int64_t D, double scale,
                           const int64_t *rows, int64_t nrows,
                           double *out, double *lse)
 {
-    int64_t nq = BH * Sq * D, nkv = BH * Skv * D;
-    double *qd = (double *)malloc(sizeof(double) * (size_t)(nq > 0 ? nq : 1));
-    double *kd = (double *)malloc(sizeof(double) * (size_t)(nkv > 0 ? nkv : 1));
-    double *vd = (double *)malloc(sizeof(double) * (size_t)(nkv > 0 ? nkv : 1));
-    if (!qd || !kd || !vd) {
-        free(qd); free(kd); free(vd);
-        return -1;
-    }
-    if (rows) {
-        for (int64_t r = 0; r < nrows; ++r)
-            for (int64_t d = 0; d < D; ++d)
-                qd[rows[r] * D + d] = oracle_bf16_to_f64(q[rows[r] * D + d]);
-    } else {
-        oracle_bf16_to_f64_array(q, qd, nq);
-    }
-    oracle_bf16_to_f64_array(k, kd, nkv);
-    oracle_bf16_to_f64_array(v, vd, nkv);
-    oracle_attention_f64(qd, kd, vd, BH, Sq, Skv, D, scale, rows, nrows, out, lse);
-    free(qd); free(kd); free(vd);
-    return 0;
+    src_t sq = {q, 1}, sk = {k, 1}, sv = {v, 1};
+    return attention_rows(sq, sk, sv, BH, Sq, Skv, D, scale, rows, nrows, out, lse);
 }
 
 /* ------------------------------------------------------------ LSE merge --- */

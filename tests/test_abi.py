@@ -1,0 +1,92 @@
+"""The C-ABI library: it builds, loads, exports exactly what include/regen_attn.h
+declares, and answers invalid calls with the documented status before touching
+the GPU (so these run without one)."""
+import os
+import re
+import subprocess
+
+import pytest
+
+import dit_attention_b200 as rg
+from dit_attention_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "regen_attn.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return set(re.findall(r"REGEN_API\s+[\w\s\*]+?\b(regen_\w+)\s*\(", text))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return rg.load()
+
+
+def test_exports_match_header(lib):
+    declared = declared_symbols()
+    assert {"regen_attn_fwd", "regen_rope3d", "regen_lse_merge"} <= declared
+    out = subprocess.run(["nm", "-D", "--defined-only", rg.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.split()[-1].startswith("regen_")}
+    assert exported == declared
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    assert rg.regen_status_str(0) == "ok"
+    assert "bounded wait" in rg.regen_status_str(-5)
+    assert rg.regen_version() == 100
+
+
+FAKE = 0x7F0000000000      # never dereferenced: every call below fails validation first
+MB = 1 << 20
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=96), -2), (dict(D=0), -2), (dict(B=-1), -1), (dict(Sq=-3), -1), (dict(scale=float("inf")), -1),
+    (dict(scale=float("nan")), -1), (dict(q=None), -1), (dict(k=None), -1), (dict(q=FAKE + 8), -3),
+    (dict(lse=FAKE + 40 * MB + 4), -3), (dict(out=FAKE), -1), (dict(lse=FAKE + 1024), -1),
+    (dict(B=0), 0), (dict(Sq=0), 0), (dict(H=0, q=None, out=None), 0),
+])
+def test_attn_fwd_validation(lib, args, status):
+    a = dict(q=FAKE, k=FAKE + 10 * MB, v=FAKE + 20 * MB, out=FAKE + 30 * MB, lse=FAKE + 40 * MB,
+             B=1, H=2, Sq=100, Skv=100, D=128, scale=0.125)
+    a.update(args)
+    rc = lib.regen_attn_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["H"], a["Sq"], a["Skv"],
+                            a["D"], a["scale"], None)
+    assert rc == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(theta=0.0), -1), (dict(theta=float("inf")), -1), (dict(T=0), -1), (dict(D=12), -2),
+    (dict(D=520), -2), (dict(q=None, k=None), -1), (dict(k=FAKE + 2), -3), (dict(k=FAKE + 16), -1),
+    (dict(B=0), 0),
+])
+def test_rope3d_validation(lib, args, status):
+    a = dict(q=FAKE, k=FAKE + 10 * MB, T=2, Hh=3, Ww=4, theta=10000.0, B=1, H=2, D=64)
+    a.update(args)
+    rc = lib.regen_rope3d(a["q"], a["k"], a["T"], a["Hh"], a["Ww"], a["theta"], a["B"], a["H"], a["D"], None)
+    assert rc == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(rows=0), 0), (dict(rows=-1), -1), (dict(D=7), -2), (dict(o_a=None), -1), (dict(lse_b=FAKE + 3), -3),
+    (dict(lse_out=FAKE + 20 * MB), -1), (dict(out=FAKE + 4096), -1),
+])
+def test_lse_merge_validation(lib, args, status):
+    a = dict(o_a=FAKE, lse_a=FAKE + 20 * MB, o_b=FAKE + 10 * MB, lse_b=FAKE + 30 * MB, out=FAKE + 40 * MB,
+             lse_out=FAKE + 50 * MB, rows=1000, D=128)
+    a.update(args)
+    rc = lib.regen_lse_merge(a["o_a"], a["lse_a"], a["o_b"], a["lse_b"], a["out"], a["lse_out"], a["rows"],
+                             a["D"], None)
+    assert rc == status
+
+
+def test_python_binding_raises(lib):
+    with pytest.raises(rg.RegenError) as e:
+        rg.regen_attn_fwd(FAKE, FAKE + MB, FAKE + 2 * MB, FAKE + 3 * MB, None, 1, 1, 8, 8, 96, 0.1, stream=0)
+    assert e.value.status == -2

@@ -1,0 +1,266 @@
+"""GPU parity: rope3d, lse_merge and attention through the C ABI vs the fp64 oracle.
+
+Every expected value comes from ``oracle`` on the same seeded bf16 inputs.
+Accuracy contract (bf16 outputs): |out - ref| <= 1e-2 + 1e-2 |ref|;
+fp32 LSE: |lse - ref| <= 1e-3. RoPE is compared bit for bit (both sides round
+the fp64 rotation once to bf16, nearest-even).
+"""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import dit_attention_b200 as rg  # noqa: E402
+from dit_attention_b200 import synth  # noqa: E402
+from util import bits_to_f64, check_attention, sample_rows, to_bits, to_dev  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+RNG = np.random.default_rng(20261202)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    rg.load()
+    yield
+    rc, site = rg.regen_last_device_error()
+    assert rc == 0, f"a kernel recorded a device error: {rc} at wait site {site}"
+
+
+def rand_bf16(shape, scale=1.0):
+    return synth.f64_to_bf16_bits(RNG.normal(size=shape) * scale)
+
+
+# ------------------------------------------------------------------ RoPE ---
+
+@pytest.mark.parametrize("B,H,grid,D", [
+    (1, 2, (3, 5, 7), 128), (2, 3, (2, 4, 6), 64), (1, 1, (1, 1, 9), 8), (1, 5, (4, 3, 2), 24),
+    (1, 3, (7, 30, 52), 128),
+])
+def test_rope3d_bit_exact(B, H, grid, D):
+    S = grid[0] * grid[1] * grid[2]
+    q = rand_bf16((B, H, S, D))
+    k = rand_bf16((B, H, S, D))
+    dq, dk = to_dev(q), to_dev(k)
+    rg.rope3d_(dq, dk, grid, 10000.0)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_bits(dq), oracle.rope3d(q, grid, 10000.0))
+    np.testing.assert_array_equal(to_bits(dk), oracle.rope3d(k, grid, 10000.0))
+
+
+def test_rope3d_q_only_and_theta():
+    grid = (2, 3, 5)
+    q = rand_bf16((1, 2, 30, 64))
+    dq = to_dev(q)
+    rg.rope3d_(dq, None, grid, 500.0)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_bits(dq), oracle.rope3d(q, grid, 500.0))
+
+
+def test_rope3d_full_77_frame_window_sampled_heads():
+    w = synth.WORKLOADS["win77_s31200"]
+    q, k, _ = synth.make_inputs(w)
+    dq, dk = to_dev(q), to_dev(k)
+    rg.rope3d_(dq, dk, w.grid, w.theta)
+    torch.cuda.synchronize()
+    heads = [0, 17, 39]
+    gq, gk = to_bits(dq), to_bits(dk)
+    for h in heads:
+        np.testing.assert_array_equal(gq[0, h], oracle.rope3d(q[0, h], w.grid, w.theta))
+        np.testing.assert_array_equal(gk[0, h], oracle.rope3d(k[0, h], w.grid, w.theta))
+
+
+# ------------------------------------------------------------- LSE merge ---
+
+@pytest.mark.parametrize("rows,D", [(1, 128), (777, 128), (4096, 64), (33, 8)])
+def test_lse_merge(rows, D):
+    oa, ob = rand_bf16((rows, D)), rand_bf16((rows, D))
+    la = (RNG.normal(size=rows) * 20).astype(np.float32)
+    lb = (RNG.normal(size=rows) * 20).astype(np.float32)
+    la[::7] = -np.inf
+    lb[::11] = -np.inf
+    out, lse = rg.lse_merge(to_dev(oa), torch.from_numpy(la).cuda(), to_dev(ob), torch.from_numpy(lb).cuda())
+    torch.cuda.synchronize()
+    ref, rl = oracle.lse_merge(oa, la.astype(np.float64), ob, lb.astype(np.float64))
+    got = bits_to_f64(to_bits(out))
+    # fp32 weights, one bf16 rounding: within one bf16 ulp of the fp64 value
+    np.testing.assert_array_less(np.abs(got - ref), np.abs(ref) * 2.0 ** -7 + 1e-30)
+    gl = lse.cpu().numpy().astype(np.float64)
+    both = np.isneginf(rl)
+    assert np.array_equal(np.isneginf(gl), both)
+    np.testing.assert_allclose(gl[~both], rl[~both], rtol=0, atol=2e-5 * max(1.0, np.abs(rl[~both]).max()))
+    assert np.all(got[both] == 0)
+
+
+def test_lse_merge_in_place():
+    rows, D = 300, 128
+    oa, ob = rand_bf16((rows, D)), rand_bf16((rows, D))
+    la = RNG.normal(size=rows).astype(np.float32)
+    lb = RNG.normal(size=rows).astype(np.float32)
+    da = to_dev(oa)
+    rg.lse_merge(da, torch.from_numpy(la).cuda(), to_dev(ob), torch.from_numpy(lb).cuda(), out=da)
+    torch.cuda.synchronize()
+    ref, _ = oracle.lse_merge(oa, la.astype(np.float64), ob, lb.astype(np.float64))
+    np.testing.assert_array_less(np.abs(bits_to_f64(to_bits(da)) - ref), np.abs(ref) * 2.0 ** -7 + 1e-30)
+
+
+# ------------------------------------------------------------- attention ---
+
+def run_attention(q, k, v, scale, guard=True):
+    """GPU attention with NaN-filled outputs inside guard regions; checks that
+    nothing outside out/lse was written. Returns (out bits, lse)."""
+    B, H, Sq, D = q.shape
+    Skv = k.shape[2]
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    n_out, n_lse = B * H * Sq * D, B * H * Sq
+    pad = 4096
+    out_buf = torch.full((n_out + 2 * pad,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse_buf = torch.full((n_lse + 2 * pad,), float("nan"), dtype=torch.float32, device="cuda")
+    out = out_buf[pad:pad + n_out].view(B, H, Sq, D)
+    lse = lse_buf[pad:pad + n_lse].view(B, H, Sq)
+    rg.regen_attn_fwd(dq, dk, dv, out, lse, B, H, Sq, Skv, D, scale)
+    torch.cuda.synchronize()
+    if guard:
+        assert torch.isnan(out_buf[:pad].float()).all() and torch.isnan(out_buf[pad + n_out:].float()).all()
+        assert torch.isnan(lse_buf[:pad]).all() and torch.isnan(lse_buf[pad + n_lse:]).all()
+    return to_bits(out), lse.cpu().numpy()
+
+
+@pytest.mark.parametrize("B,H,Sq,Skv,D", [
+    (1, 1, 128, 128, 128), (1, 1, 1, 1, 128), (1, 2, 2, 2, 64), (1, 1, 127, 129, 128),
+    (1, 1, 129, 127, 128), (2, 1, 255, 255, 128), (1, 1, 256, 2072, 128), (1, 1, 300, 1, 64),
+    (1, 2, 257, 384, 64), (3, 1, 100, 1000, 128), (1, 1, 513, 130, 128),
+])
+def test_attention_small_shapes(B, H, Sq, Skv, D):
+    q, k, v = rand_bf16((B, H, Sq, D)), rand_bf16((B, H, Skv, D)), rand_bf16((B, H, Skv, D))
+    scale = 1.0 / math.sqrt(D)
+    out, lse = run_attention(q, k, v, scale)
+    ref, rl = oracle.attention(q, k, v, scale)
+    check_attention(out, lse, ref, rl, f"B{B} H{H} Sq{Sq} Skv{Skv} D{D}")
+
+
+def test_attention_many_heads_more_ctas_than_sms():
+    B, H, S, D = 2, 100, 300, 128        # 400 CTAs over 148 SMs
+    q, k, v = rand_bf16((B, H, S, D)), rand_bf16((B, H, S, D)), rand_bf16((B, H, S, D))
+    out, lse = run_attention(q, k, v, 1 / math.sqrt(D))
+    rows = sample_rows(B * H, S, 4)
+    ref, rl = oracle.attention(q, k, v, 1 / math.sqrt(D), rows=rows)
+    check_attention(out.reshape(-1, D)[rows], lse.reshape(-1)[rows], ref, rl, "many heads")
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.125, 0.5])
+def test_attention_scale_edge_cases(scale):
+    q, k, v = rand_bf16((1, 2, 200, 128)), rand_bf16((1, 2, 333, 128)), rand_bf16((1, 2, 333, 128))
+    out, lse = run_attention(q, k, v, scale)
+    ref, rl = oracle.attention(q, k, v, scale)
+    check_attention(out, lse, ref, rl, f"scale {scale}")
+
+
+def test_attention_spiky_logits_rescale_path():
+    # logits spanning ~100 (log2) units force O rescaling in later key blocks
+    q = rand_bf16((1, 1, 256, 128), 4.0)
+    k = rand_bf16((1, 1, 1024, 128))
+    kk = synth.bf16_bits_to_f64(k)
+    kk[0, 0, 900:910] *= 8.0      # the large logits arrive late
+    k = synth.f64_to_bf16_bits(kk)
+    v = rand_bf16((1, 1, 1024, 128))
+    out, lse = run_attention(q, k, v, 1 / math.sqrt(128))
+    ref, rl = oracle.attention(q, k, v, 1 / math.sqrt(128))
+    check_attention(out, lse, ref, rl, "spiky")
+
+
+def test_attention_empty_kv_and_no_queries():
+    q = rand_bf16((1, 2, 64, 128))
+    dq = to_dev(q)
+    out = torch.full_like(dq, float("nan"))
+    lse = torch.zeros((1, 2, 64), dtype=torch.float32, device="cuda")
+    rg.regen_attn_fwd(dq, None, None, out, lse, 1, 2, 64, 0, 128, 0.1)
+    torch.cuda.synchronize()
+    assert (out.float() == 0).all() and torch.isneginf(lse).all()
+    rg.regen_attn_fwd(dq, dq, dq, out, lse, 1, 2, 0, 64, 128, 0.1)   # Sq = 0: no-op
+
+
+def test_attention_lse_optional():
+    q, k, v = rand_bf16((1, 1, 130, 64)), rand_bf16((1, 1, 130, 64)), rand_bf16((1, 1, 130, 64))
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    out = torch.empty_like(dq)
+    rg.regen_attn_fwd(dq, dk, dv, out, None, 1, 1, 130, 130, 64, 0.125)
+    torch.cuda.synchronize()
+    ref, rl = oracle.attention(q, k, v, 0.125)
+    check_attention(to_bits(out), rl, ref, rl, "lse=NULL")
+
+
+# --------------------------------------------- the five named workloads ---
+
+def _workload(name, per_head, heads=None):
+    """Run RoPE (when the workload has it) and attention on the GPU for the whole
+    workload; compare the given heads (default all) against the oracle, on
+    every row (per_head None) or on sampled rows."""
+    w = synth.WORKLOADS[name]
+    q, k, v = synth.make_inputs(w)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    if w.rope:
+        rg.rope3d_(dq, dk, w.grid, w.theta)
+    out, lse = rg.attn_fwd(dq, dk, dv, w.scale)
+    torch.cuda.synchronize()
+    BH = w.B * w.H
+    heads = list(range(BH)) if heads is None else heads
+    qh = q.reshape(BH, w.Sq, w.D)[heads]
+    kh = k.reshape(BH, w.Skv, w.D)[heads]
+    vh = v.reshape(BH, w.Skv, w.D)[heads]
+    if w.rope:   # the oracle rotates its own copy of the inputs
+        qh = oracle.rope3d(qh, w.grid, w.theta)
+        kh = oracle.rope3d(kh, w.grid, w.theta)
+    gout = to_bits(out).reshape(BH, w.Sq, w.D)[heads].reshape(-1, w.D)
+    glse = lse.cpu().numpy().reshape(BH, w.Sq)[heads].reshape(-1)
+    rows = None if per_head is None else sample_rows(len(heads), w.Sq, per_head)
+    ref, rl = oracle.attention(qh, kh, vh, w.scale, rows=rows)
+    if rows is not None:
+        gout, glse = gout[rows], glse[rows]
+    else:
+        ref, rl = ref.reshape(-1, w.D), rl.reshape(-1)
+    return check_attention(gout, glse, ref, rl, name)
+
+
+SPREAD_HEADS = [0, 5, 11, 17, 23, 29, 35, 39]
+
+
+def test_workload_tiny_full():
+    _workload("tiny_s1024", None)
+
+
+def test_workload_25_frame_window_sampled():
+    _workload("win25_s10920", 48)
+
+
+def test_workload_77_frame_window_sampled():
+    _workload("win77_s31200", 48, heads=SPREAD_HEADS)
+
+
+def test_workload_cross_attention_sampled():
+    _workload("cross_s31200_kv2072", 64, heads=SPREAD_HEADS)
+
+
+def test_workload_softmax_stress_and_two_block_merge():
+    w = synth.WORKLOADS["stress_s10920"]
+    q, k, v = synth.make_inputs(w)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    out, lse = rg.attn_fwd(dq, dk, dv, w.scale)
+    # the same attention as two KV blocks of 5460 keys merged by their LSE
+    s = w.merge_split
+    oa, la = rg.attn_fwd(dq, dk[:, :, :s].contiguous(), dv[:, :, :s].contiguous(), w.scale)
+    ob, lb = rg.attn_fwd(dq, dk[:, :, s:].contiguous(), dv[:, :, s:].contiguous(), w.scale)
+    om, lm = rg.lse_merge(oa, la, ob, lb)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.B * w.H, w.Sq, 24)
+    ref, rl = oracle.attention(q, k, v, w.scale, rows=rows)
+    d1 = check_attention(to_bits(out).reshape(-1, w.D)[rows], lse.cpu().numpy().reshape(-1)[rows], ref, rl,
+                         "stress")
+    d2 = check_attention(to_bits(om).reshape(-1, w.D)[rows], lm.cpu().numpy().reshape(-1)[rows], ref, rl,
+                         "stress two-block merge")
+    assert d1["rms_ref"] > 0.1      # spiky logits: outputs of order one, so the rtol term binds
+    assert d2["max_lse_err"] <= 1e-3
