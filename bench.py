@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--e2e-steps", type=int, default=5)
@@ -60,6 +60,34 @@ def peaks():
         d = json.load(open(path))
         return d, "measured"
     return FALLBACK_PEAKS, "fallback"
+
+
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (the step time every rank reports)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank runs its own replica (weak scaling)."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
+def replica_inputs(workload, rank: int):
+    """The seeded inputs of this rank's replica (seed offset = rank)."""
+    from dit_attention_b200 import synth
+    return synth.make_inputs(workload, seed_offset=rank)
 
 
 def step_flops():
@@ -162,8 +190,8 @@ def run_native(args, rank, world, local_rank):
     def to_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
-    q, k, v = synth.make_inputs(ws, seed_offset=rank)
-    qc, kc, vc = synth.make_inputs(wc, seed_offset=rank)
+    q, k, v = replica_inputs(ws, rank)
+    qc, kc, vc = replica_inputs(wc, rank)
     host = {
         "q": q, "k": k, "v": v, "qc": qc,
         "kr": np.ascontiguousarray(kc[:, :, :N_REF]), "vr": np.ascontiguousarray(vc[:, :, :N_REF]),
@@ -204,14 +232,6 @@ def run_native(args, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -231,7 +251,7 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier()
-    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     per_kernel = {n: 0.0 for n in names}
     for i in range(args.steps):
         for j, n in enumerate(names):
@@ -241,7 +261,7 @@ def run_native(args, rank, world, local_rank):
     f_self, f_cross = step_flops()
     flops_step = f_self + f_cross
     ms_step = ms_total / args.steps
-    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(flops_step, world, ms_step)
 
     # ---- end to end: pinned host inputs -> device -> hot path -> outputs to pinned host
     pin = {n: torch.from_numpy(a.view(np.int16)).pin_memory() for n, a in host.items()}
@@ -272,8 +292,8 @@ def run_native(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
-    e2e_value = world * flops_step / (ms_e2e * 1e-3) / 1e12
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
+    e2e_value = aggregate_tflops(flops_step, world, ms_e2e)
 
     if world > 1:
         import torch.distributed as dist
@@ -401,9 +421,7 @@ def run_reference(args, rank, world):
 
 def main():
     args = parse()
-    rank = int(os.environ.get("RANK", 0))
-    world = int(os.environ.get("WORLD_SIZE", 1))
-    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    rank, world, local_rank = dist_env()
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:

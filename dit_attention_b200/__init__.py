@@ -26,7 +26,7 @@ import threading
 
 __all__ = [
     "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
-    "regen_status_str", "regen_last_device_error", "regen_set_wait_limit_ns", "regen_version",
+    "regen_status_str", "regen_last_device_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
     "attn_fwd", "rope3d_", "lse_merge", "STATUS",
 ]
 
@@ -71,6 +71,10 @@ def load():
         L.regen_last_device_error.restype = i32
         L.regen_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.regen_set_wait_limit_ns.restype = i32
+        L.regen_selftest_exp2.argtypes = [vp, vp, i64, vp]
+        L.regen_selftest_exp2.restype = i32
+        L.regen_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp, vp]
+        L.regen_selftest_bounded_wait.restype = i32
         L.regen_version.argtypes = []
         L.regen_version.restype = i32
         _lib = L
@@ -122,6 +126,15 @@ def regen_rope3d(q, k, T, Hh, Ww, theta, B, H, D, stream=None) -> None:
 def regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream=None) -> None:
     _check(load().regen_lse_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out),
                                   _ptr(lse_out), int(rows), D, _stream(stream)), "regen_lse_merge")
+
+
+def regen_selftest_exp2(x, y, n, stream=None) -> None:
+    _check(load().regen_selftest_exp2(_ptr(x), _ptr(y), int(n), _stream(stream)), "regen_selftest_exp2")
+
+
+def regen_selftest_bounded_wait(limit_ns, done, stream=None) -> None:
+    _check(load().regen_selftest_bounded_wait(int(limit_ns), _ptr(done), _stream(stream)),
+           "regen_selftest_bounded_wait")
 
 
 def regen_status_str(status: int) -> str:

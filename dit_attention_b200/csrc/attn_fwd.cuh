@@ -28,7 +28,13 @@
 // the final O/l and LSE use the same m.
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
+
+#ifndef REGEN_EXP2_EMU_PER8
+#define REGEN_EXP2_EMU_PER8 2
+#endif
 
 namespace regen {
 
@@ -45,12 +51,17 @@ enum WaitSite : uint32_t {
     SITE_SM_S_FULL = 7,
     SITE_SM_O_FULL = 8,
     SITE_DRAIN = 9,
+    SITE_SELFTEST = 10,
 };
 
 __device__ __forceinline__ void record_timeout(uint32_t site)
 {
     if (atomicCAS(&g_regen_err, 0, -5 /* REGEN_ERR_TIMEOUT */) == 0) g_regen_err_site = site;
 }
+
+// Lower bound on the waits that drain a CTA's own copies and MMAs before it
+// exits after an abort (they complete in microseconds; 100 ms).
+constexpr uint64_t kDrainFloorNs = 100000000ull;
 
 struct WaitCtl {
     volatile int *abort;   // CTA-wide flag in shared memory
@@ -97,6 +108,14 @@ struct AttnCfg {
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int THREADS = 384;
+    static constexpr uint32_t REGS_LOW = 64;    // producer / MMA / idle warpgroup
+    static constexpr uint32_t REGS_HIGH = 208;  // the two softmax warpgroups
+    // need (REGS_HIGH - R) * 256 <= (R - REGS_LOW) * 128, i.e. R >= 160
+    static constexpr int MIN_LAUNCH_REGS = 160;
+    // Of every 8 pairs of probabilities, this many are evaluated on the FMA
+    // pipe (exp2_poly_pair) instead of MUFU: ex2 throughput (16/clk/SM) alone
+    // equals the tensor time of a key block, so part of it moves to the FMAs.
+    static constexpr int EMU_PER8 = REGEN_EXP2_EMU_PER8;
 };
 
 template <int HD, bool NEG_SCALE>
@@ -161,6 +180,12 @@ __global__ void __launch_bounds__(384, 1)
     const int bh = static_cast<int>(blockIdx.x / npairs);
     const int q0 = static_cast<int>(blockIdx.x % npairs) * (2 * C::BM);
 
+    // Registers: the producer/MMA warpgroup gives (R - REGS_LOW) per thread back,
+    // the two softmax warpgroups take (REGS_HIGH - R) each; the host launches
+    // only builds with R >= MIN_LAUNCH_REGS, for which the release covers it.
+    // Each register region runs to its own final barrier (no shared tail).
+    if (warp < 4) {
+    setmaxnreg_dec<C::REGS_LOW>();
     if (warp == 0) {
         // ------------------------------------------------------ producer ---
         if (lane == 0) {
@@ -198,9 +223,12 @@ __global__ void __launch_bounds__(384, 1)
                 // Aborting: wait (bounded) for the copies this warp may still have
                 // in flight -- at most the last NS of each ring and the Q tiles --
                 // so that none lands in shared memory after the CTA has exited.
+                // (copies complete in microseconds; the drain never uses less than
+                // kDrainFloorNs even when the caller's wait limit is tiny)
+                const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
                 auto drain = [&](uint32_t bar, uint32_t parity) {
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < wait_limit_ns) {
+                    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
                     }
                 };
                 for (int j = (nk > C::NS ? nk - C::NS : 0); j < nk; ++j)
@@ -215,8 +243,10 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false);  // Q.K^T, both K-major
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, true);    // P.V, V is MN-major
-            const uint32_t tm_s[2] = {tmem, tmem + 128u};
-            const uint32_t tm_o[2] = {tmem + 256u, tmem + 256u + HD};
+            // TMEM columns: S_t at t*128, O_t at 256 + t*HD (computed, not indexed,
+            // so nothing lands in local memory)
+            auto tm_s = [&](int t) { return tmem + static_cast<uint32_t>(t) * 128u; };
+            auto tm_o = [&](int t) { return tmem + 256u + static_cast<uint32_t>(t) * HD; };
             // S_t = Q_t K_j^T : M=128, N=128, K=HD in steps of 16 (32 bytes) inside
             // each 128-byte swizzle row; the second 64-column half starts HALF_BYTES on.
             auto issue_s = [&](int t, int s) {
@@ -225,7 +255,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t off = (kk / 4) * C::HALF_BYTES + (kk % 4) * 32;
-                    mma_ss(tm_s[t], smem_desc_sw128(qa + off, 16, 1024),
+                    mma_ss(tm_s(t), smem_desc_sw128(qa + off, 16, 1024),
                            smem_desc_sw128(kb + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
                 }
             };
@@ -236,7 +266,7 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t vb = sbase + C::V_OFF + s * C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    mma_ts(tm_o[t], tm_s[t] + kk * 8, smem_desc_sw128(vb + kk * 2048, C::HALF_BYTES, 1024),
+                    mma_ts(tm_o(t), tm_s(t) + kk * 8, smem_desc_sw128(vb + kk * 2048, C::HALF_BYTES, 1024),
                            IDESC_O, (acc || kk > 0) ? 1u : 0u);
                 }
             };
@@ -286,16 +316,25 @@ __global__ void __launch_bounds__(384, 1)
             }
             // Drain: nothing may still be running on the tensor core when TMEM is freed.
             tc_commit(bar_drain);
+            const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(bar_drain, 0)) {
-                if (global_timer_ns() - t0 > wait_limit_ns) {
+                if (global_timer_ns() - t0 > drain_ns) {
                     record_timeout(SITE_DRAIN);
                     break;
                 }
             }
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    } else {
+        setmaxnreg_inc<C::REGS_HIGH>();
         // -------------------------------------------- softmax + epilogue ---
         const int t = (warp - 4) >> 2;     // Q tile of this warpgroup
         const int quad = warp & 3;         // TMEM lane quadrant this warp may access
@@ -319,60 +358,84 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-            const bool last = (j == nkv - 1);
-            if (last && kv_tail < C::BN) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c * 32 + i >= kv_tail)
-                            sr[c][i] = __float_as_uint(NEG_SCALE ? INFINITY : -INFINITY);
-            }
-            // row extreme of the raw logits -> max of the scaled logits
-            float mx = __uint_as_float(sr[0][0]);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    mx = NEG_SCALE ? fminf(mx, __uint_as_float(sr[c][i]))
-                                   : fmaxf(mx, __uint_as_float(sr[c][i]));
-            const float mnew = mx * scale_log2;
-            // Stale-max rule: move m (and rescale O, l) only when the block max
-            // exceeds it by more than 8 in log2 units.
+            // One block of the online softmax. MASKED: the last block, whose
+            // columns >= kv_tail lie past Skv (their logits are zero-filled
+            // loads) and get probability 0.
             bool grow = false;
             float alpha = 1.0f;
-            if (j == 0) {
-                m = mnew;
-            } else if (mnew > m + 8.0f) {
-                grow = true;
-                alpha = ex2_approx(m - mnew);
-                m = mnew;
-                l *= alpha;
-            }
-            // P = 2^(s*scale_log2 - m), summed in fp32 before rounding to bf16.
-            const float neg_m = -m;
-            float rs = 0.f;
+            auto block = [&](auto masked_tag) {
+                constexpr bool MASKED = decltype(masked_tag)::value;
+                auto S = [&](int x) { return __uint_as_float(sr[x >> 5][x & 31]); };
+                if constexpr (MASKED) {
 #pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {   // 64 keys -> 32 packed columns per half
-                uint32_t pk[32];
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = hv * 2 + cc;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][i]), scale_log2, neg_m));
-                        float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][i + 1]), scale_log2, neg_m));
-                        if (last && kv_tail < C::BN) {
-                            if (c * 32 + i >= kv_tail) p0 = 0.f;
-                            if (c * 32 + i + 1 >= kv_tail) p1 = 0.f;
-                        }
-                        rs += p0 + p1;
-                        pk[cc * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
-                    }
+                    for (int x = 0; x < 128; ++x)
+                        if (x >= kv_tail) sr[x >> 5][x & 31] = __float_as_uint(NEG_SCALE ? INFINITY : -INFINITY);
                 }
-                tmem_st_32x32b_x32(ts + hv * 32, pk);
-            }
-            l += rs;
+                // Row extreme of the raw logits: 8 independent 3-input chains.
+                float acc[8];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    const int x0 = a * 16;
+                    float r = NEG_SCALE ? fmin3(S(x0), S(x0 + 1), S(x0 + 2)) : fmax3(S(x0), S(x0 + 1), S(x0 + 2));
+#pragma unroll
+                    for (int x = x0 + 3; x + 1 < x0 + 16; x += 2)
+                        r = NEG_SCALE ? fmin3(r, S(x), S(x + 1)) : fmax3(r, S(x), S(x + 1));
+                    r = NEG_SCALE ? fminf(r, S(x0 + 15)) : fmaxf(r, S(x0 + 15));
+                    acc[a] = r;
+                }
+                const float mx = NEG_SCALE
+                    ? fmin3(fmin3(acc[0], acc[1], acc[2]), fmin3(acc[3], acc[4], acc[5]), fminf(acc[6], acc[7]))
+                    : fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
+                const float mnew = mx * scale_log2;
+                // Stale-max rule: move m (and rescale O, l) only when the block
+                // max exceeds it by more than 8 in log2 units.
+                if (j == 0) {
+                    m = mnew;
+                } else if (mnew > m + 8.0f) {
+                    grow = true;
+                    alpha = ex2_approx(m - mnew);
+                    m = mnew;
+                    l *= alpha;
+                }
+                // P = 2^(s*scale_log2 - m): packed FMA for the affine step, MUFU
+                // ex2, fp32 row sum (4 packed accumulators) before rounding to bf16.
+                const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+                const uint64_t nm2 = f2_pack(-m, -m);
+                uint64_t rs2[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int hv = 0; hv < 2; ++hv) {   // 64 keys -> 32 packed columns per half
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 64; i += 2) {
+                        const int x = hv * 64 + i;
+                        float y0, y1;
+                        f2_unpack(f2_fma(f2_pack(S(x), S(x + 1)), c2, nm2), y0, y1);
+                        float p0, p1;
+                        if ((i >> 1) % 8 < C::EMU_PER8) {
+                            exp2_poly_pair(y0, y1, p0, p1);     // FMA pipe
+                        } else {
+                            p0 = ex2_approx(y0);                // MUFU
+                            p1 = ex2_approx(y1);
+                        }
+                        if constexpr (MASKED) {
+                            if (x >= kv_tail) p0 = 0.f;
+                            if (x + 1 >= kv_tail) p1 = 0.f;
+                        }
+                        rs2[(i >> 1) & 3] = f2_add(rs2[(i >> 1) & 3], f2_pack(p0, p1));
+                        pk[i >> 1] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st_32x32b_x32(ts + hv * 32, pk);
+                }
+                float r0, r1, r2, r3;
+                f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), r0, r1);
+                (void)r2;
+                (void)r3;
+                l += r0 + r1;
+            };
+            if (j == nkv - 1 && kv_tail < C::BN)
+                block(std::true_type{});
+            else
+                block(std::false_type{});
             // O_t holds exactly PV_t(0..j-1) here: the commit that signalled S_t(j)
             // follows PV_t(j-1), and PV_t(j) waits for this warpgroup's arrive.
             if (__any_sync(0xffffffffu, grow)) {
@@ -433,13 +496,39 @@ __global__ void __launch_bounds__(384, 1)
             tma_store_commit();
             tma_store_wait_all();
         }
+        tc_fence_before_sync();
+        __syncthreads();
     }
+}
 
-    tc_fence_before_sync();
+// Self-test of the bounded wait: one warp waits on an mbarrier that nothing
+// arrives on; after limit_ns it records REGEN_ERR_TIMEOUT (site SITE_SELFTEST)
+// and returns. *done is set to 1 when the kernel has returned from the wait.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int *done)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+    }
     __syncthreads();
-    if (warp == 1) {
-        tc_fence_after_sync();
-        tmem_dealloc(tmem, C::TMEM_COLS);
+    const WaitCtl wc{&abort_flag, limit_ns};
+    const bool ok = __all_sync(0xffffffffu, wait_phase(smem_u32(&bar), 0, SITE_SELFTEST, wc));
+    __syncthreads();
+    if (threadIdx.x == 0) *done = ok ? 2 : 1;
+}
+
+// Self-test of the kernel's FMA-pipe exp2 (n even): y[i] = 2^x[i].
+__global__ void exp2_poly_selftest_kernel(const float *__restrict__ x, float *__restrict__ y, int64_t npairs)
+{
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < npairs; i += stride) {
+        float a, b;
+        exp2_poly_pair(x[2 * i], x[2 * i + 1], a, b);
+        y[2 * i] = a;
+        y[2 * i + 1] = b;
     }
 }
 

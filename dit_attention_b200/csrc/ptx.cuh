@@ -268,6 +268,97 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// Per-warpgroup register re-allocation. Every warp of a warpgroup must execute
+// the same one. The increase waits for registers released by decreases in the
+// same CTA, so the shares must add up within the launch's allocation.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Three-input max / min (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c)
+{
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): lo in the low 32 bits.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^y for a pair of floats on the FMA pipe (no MUFU). Range reduction after
+// Cody & Waite: y clamped to >= -127, j = round-to-nearest(y) through the
+// 1.5 * 2^23 shifter, f = y - j in [-1/2, 1/2]; 2^f by a degree-4 polynomial
+// whose coefficients were fitted for minimum relative error on [-1/2, 1/2]
+// by dit_attention_b200/csrc/fit_exp2.py (max relative error 2.9e-6 in fp32);
+// 2^j is applied by adding j to the exponent field. y = -127 gives exactly 0.
+__device__ __forceinline__ void exp2_poly_pair(float y0, float y1, float &p0, float &p1)
+{
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c1 = 6.931242347e-01f, c2 = 2.402409911e-01f, c3 = 5.590614304e-02f,
+                    c4 = 9.582744911e-03f;
+    const uint64_t y2 = f2_pack(fmaxf(y0, -127.0f), fmaxf(y1, -127.0f));
+    const uint64_t sh2 = f2_pack(kShift, kShift);
+    const uint64_t t2 = f2_add(y2, sh2);          // shifter + j (j in the low mantissa bits)
+    const uint64_t f2 = f2_sub(y2, f2_sub(t2, sh2));
+    uint64_t p2 = f2_fma(f2_pack(c4, c4), f2, f2_pack(c3, c3));
+    p2 = f2_fma(p2, f2, f2_pack(c2, c2));
+    p2 = f2_fma(p2, f2, f2_pack(c1, c1));
+    p2 = f2_fma(p2, f2, f2_pack(1.0f, 1.0f));
+    float a, b, ta, tb;
+    f2_unpack(p2, a, b);
+    f2_unpack(t2, ta, tb);
+    // bits(t) << 23 == j << 23 (mod 2^32): the shifter's own bits vanish
+    p0 = __uint_as_float(__float_as_uint(ta) * 8388608u + __float_as_uint(a));
+    p1 = __uint_as_float(__float_as_uint(tb) * 8388608u + __float_as_uint(b));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     uint32_t r;

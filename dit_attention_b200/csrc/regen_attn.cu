@@ -73,12 +73,18 @@ int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, r
 {
     using C = regen::AttnCfg<HD>;
     static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
+    static int attr_status = REGEN_OK;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(regen::attn_fwd_kernel<HD, NEG>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        cudaFuncAttributes fa;
+        if (cudaFuncSetAttribute(regen::attn_fwd_kernel<HD, NEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, regen::attn_fwd_kernel<HD, NEG>) != cudaSuccess)
+            attr_status = REGEN_ERR_CUDA;
+        else if (fa.numRegs < C::MIN_LAUNCH_REGS)
+            // the in-kernel register re-allocation would not fit: refuse to launch
+            attr_status = REGEN_ERR_UNSUPPORTED;
     });
-    if (attr_err != cudaSuccess) return REGEN_ERR_CUDA;
+    if (attr_status != REGEN_OK) return attr_status;
     CUtensorMap tq, tk, tv, to;
     if (!make_bhsd_map(&tq, q, BH, Sq, HD) || !make_bhsd_map(&tk, k, BH, Skv, HD) ||
         !make_bhsd_map(&tv, v, BH, Skv, HD) || !make_bhsd_map(&to, out, BH, Sq, HD))
@@ -186,6 +192,25 @@ REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a, const r
     regen::lse_merge_kernel<<<grid_for(work, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const uint4 *>(o_a), lse_a, reinterpret_cast<const uint4 *>(o_b), lse_b,
         reinterpret_cast<uint4 *>(out), lse_out, rows, D);
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
+REGEN_API int regen_selftest_exp2(const float *x, float *y, int64_t n, regen_stream_t stream)
+{
+    if (n < 0 || (n & 1)) return REGEN_ERR_INVALID_ARG;
+    if (n == 0) return REGEN_OK;
+    if (!x || !y) return REGEN_ERR_INVALID_ARG;
+    const int64_t npairs = n / 2;
+    regen::exp2_poly_selftest_kernel<<<grid_for(npairs, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        x, y, npairs);
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
+REGEN_API int regen_selftest_bounded_wait(uint64_t limit_ns, int *done, regen_stream_t stream)
+{
+    if (!done) return REGEN_ERR_INVALID_ARG;
+    if (limit_ns == 0 || limit_ns > 5000000000ull) return REGEN_ERR_INVALID_ARG;
+    regen::bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, done);
     return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
 }
 

@@ -103,15 +103,35 @@ REGEN_API int regen_rope3d(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, 
  * (two empty key blocks) give out = 0 and lse_out = -inf.
  *
  *   o_a, o_b, out  [rows, D] bf16;  lse_a, lse_b  [rows] fp32
- *   lse_out        [rows] fp32 or NULL (skipped); it may alias lse_a or lse_b
+ *   lse_out        [rows] fp32 or NULL (skipped); must not overlap any other array
  *   rows = B*H*Sq >= 0;  D multiple of 8, 8 <= D <= 512
- * out may alias o_a or o_b (element-wise, each element is read before it is
- * written by the same thread).
+ * out may be exactly o_a or o_b (each element is read before the same thread
+ * writes it); any other overlap is REGEN_ERR_INVALID_ARG.
  */
 REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a,
                               const regen_bf16 *o_b, const float *lse_b,
                               regen_bf16 *out, float *lse_out,
                               int64_t rows, int D, regen_stream_t stream);
+
+/*
+ * regen_selftest_exp2 -- diagnostic: evaluates, for each x[i], the FMA-pipe
+ * 2^x that the attention kernel uses for part of its softmax probabilities
+ * (degree-4 polynomial after Cody-Waite range reduction; inputs below -127
+ * are clamped to -127, whose result is 0). x, y: device fp32 arrays of n
+ * elements, n even. No counterpart on the pages: it exists so that tests can
+ * check the kernel's exponential against CUDA's exp2f and its error bound.
+ */
+REGEN_API int regen_selftest_exp2(const float *x, float *y, int64_t n, regen_stream_t stream);
+
+/*
+ * regen_selftest_bounded_wait -- diagnostic of the failure-detection path: a
+ * single-warp kernel waits, with the same bounded wait the attention kernel
+ * uses, on a barrier that nothing ever completes. After limit_ns (1 ns .. 5 s)
+ * it records REGEN_ERR_TIMEOUT with site code 10, writes 1 to *done (device
+ * int; 2 would mean the wait unexpectedly succeeded) and returns, leaving the
+ * context usable. No counterpart on the pages.
+ */
+REGEN_API int regen_selftest_bounded_wait(uint64_t limit_ns, int *done, regen_stream_t stream);
 
 /* Human-readable text of a status code (static storage). */
 REGEN_API const char *regen_status_str(int status);

@@ -265,3 +265,28 @@ def test_workload_softmax_stress_and_two_block_merge():
                          "stress two-block merge")
     assert d1["rms_ref"] > 0.1      # spiky logits: outputs of order one, so the rtol term binds
     assert d2["max_lse_err"] <= 1e-3
+
+
+# ------------------------------------------------ the kernel's FMA exp2 ---
+
+def test_selftest_exp2_against_cuda_exp2f_and_fp64():
+    # 2^x over the range the softmax feeds it (x <= 8 with the stale-max rule),
+    # compared with CUDA's exp2f (torch.exp2 on the GPU) and with fp64.
+    x = torch.cat([torch.linspace(-126.0, 8.5, 1 << 20), torch.tensor([-127.0, -200.0, -1e30, 0.0, -0.5, 0.5]),
+                   torch.rand(1 << 16) * -30.0]).float().cuda()
+    if x.numel() % 2:
+        x = torch.cat([x, torch.zeros(1, device="cuda")])
+    y = torch.empty_like(x)
+    rg.regen_selftest_exp2(x, y, x.numel())
+    torch.cuda.synchronize()
+    ref64 = torch.exp2(x.double())
+    cuda32 = torch.exp2(x)
+    normal = x >= -125.5
+    rel = ((y.double() - ref64) / ref64)[normal].abs().max().item()
+    rel_cuda = ((y.double() - cuda32.double()) / ref64)[normal].abs().max().item()
+    assert rel < 4e-6, rel            # fitted bound 2.9e-6 plus fp32 rounding of the reduction
+    assert rel_cuda < 4e-6, rel_cuda
+    low = x <= -127.0                 # clamped: exactly zero, never negative or NaN
+    assert (y[low] == 0).all()
+    tiny = (~normal) & (~low)
+    assert (y[tiny] >= 0).all() and (y[tiny] < 2.0 ** -124).all()
