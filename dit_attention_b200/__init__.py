@@ -9,11 +9,15 @@ library is missing or fails to load, every entry point raises.
 Entry points (same names as the C ABI):
     regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream=None)
     regen_rope3d(q, k, T, Hh, Ww, theta, B, H, D, stream=None)
+    regen_attn_fwd_rope3d(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream, T, Hh, Ww, theta,
+                          workspace, workspace_bytes)
+    regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
     regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream=None)
     regen_last_device_error() -> (status, site)
     regen_set_wait_limit_ns(ns)
 Convenience wrappers that allocate outputs with torch:
     attn_fwd(q, k, v, scale=None) -> (out, lse)
+    attn_fwd_rope3d(q, k, v, grid, theta=10000.0) -> (out, lse)
     rope3d_(q, k, grid, theta=10000.0)
     lse_merge(o_a, lse_a, o_b, lse_b) -> (out, lse)
 """
@@ -27,7 +31,8 @@ import threading
 __all__ = [
     "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
     "regen_status_str", "regen_last_device_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
-    "attn_fwd", "rope3d_", "lse_merge", "STATUS",
+    "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes",
+    "attn_fwd", "attn_fwd_rope3d", "rope3d_", "lse_merge", "STATUS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -61,6 +66,11 @@ def load():
         vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
         L.regen_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
         L.regen_attn_fwd.restype = i32
+        L.regen_attn_fwd_rope3d.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp,
+                                            i32, i32, i32, f32, vp, i64]
+        L.regen_attn_fwd_rope3d.restype = i32
+        L.regen_attn_fwd_rope3d_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.regen_attn_fwd_rope3d_workspace_bytes.restype = i64
         L.regen_rope3d.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, vp]
         L.regen_rope3d.restype = i32
         L.regen_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, vp]
@@ -116,6 +126,20 @@ def _check(rc: int, what: str) -> None:
 def regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream=None) -> None:
     _check(load().regen_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D,
                                  float(scale), _stream(stream)), "regen_attn_fwd")
+
+
+def regen_attn_fwd_rope3d(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream, T, Hh, Ww, theta,
+                          workspace, workspace_bytes) -> None:
+    _check(load().regen_attn_fwd_rope3d(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D,
+                                        float(scale), _stream(stream), T, Hh, Ww, float(theta), _ptr(workspace),
+                                        int(workspace_bytes)), "regen_attn_fwd_rope3d")
+
+
+def regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D) -> int:
+    n = load().regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
+    if n < 0:
+        raise RegenError(int(n), "regen_attn_fwd_rope3d_workspace_bytes")
+    return int(n)
 
 
 def regen_rope3d(q, k, T, Hh, Ww, theta, B, H, D, stream=None) -> None:
@@ -176,6 +200,25 @@ def attn_fwd(q, k, v, scale=None, out=None, lse=None, stream=None):
     if lse is None:
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
     regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream)
+    return out, lse
+
+
+def attn_fwd_rope3d(q, k, v, grid, theta=10000.0, scale=None, out=None, lse=None, workspace=None, stream=None):
+    """Self-attention with 3D RoPE on Q and K (q, k not modified) -> (out, lse)."""
+    import torch
+    B, H, S, D = _bhsd(q, "q")
+    T, Hh, Ww = grid
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    need = regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    regen_attn_fwd_rope3d(q, k, v, out, lse, B, H, S, S, D, scale, stream, T, Hh, Ww, theta, workspace,
+                          workspace.numel() * workspace.element_size())
     return out, lse
 
 

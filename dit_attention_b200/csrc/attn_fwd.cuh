@@ -31,6 +31,7 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "rope3d.cuh"
 
 #ifndef REGEN_EXP2_EMU_PER8
 #define REGEN_EXP2_EMU_PER8 2
@@ -51,6 +52,7 @@ enum WaitSite : uint32_t {
     SITE_SM_S_FULL = 7,
     SITE_SM_O_FULL = 8,
     SITE_DRAIN = 9,
+    SITE_SM_Q = 11,
     SITE_SELFTEST = 10,
 };
 
@@ -102,8 +104,8 @@ struct AttnCfg {
     static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
     static constexpr int BAR_OFF = V_OFF + NS * TILE_BYTES;
     // barriers: q, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2],
-    // o_full[2], drain
-    static constexpr int NBARS = 1 + 4 * NS + 6 + 1;
+    // o_full[2], drain, q_rotated
+    static constexpr int NBARS = 1 + 4 * NS + 6 + 1 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;  // abort flag, TMEM base
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -118,12 +120,17 @@ struct AttnCfg {
     static constexpr int EMU_PER8 = REGEN_EXP2_EMU_PER8;
 };
 
-template <int HD, bool NEG_SCALE>
+// ROPE_Q: the Q tiles are rotated by the 3D RoPE in shared memory right after
+// their TMA load (each softmax thread rotates its own row, from the (cos, sin)
+// table `rope_tab`), before the first S MMA reads them; the rotation is the
+// same fp64 arithmetic and rounding as rope3d_kernel, so the result equals
+// rotating Q in HBM first.
+template <int HD, bool NEG_SCALE, bool ROPE_Q>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     float *__restrict__ lse, int Sq, int Skv, float scale_log2,
-                    uint64_t wait_limit_ns)
+                    uint64_t wait_limit_ns, const double *__restrict__ rope_tab, RopeGeom rope_geom)
 {
     using C = AttnCfg<HD>;
     extern __shared__ uint8_t smem_raw[];
@@ -143,6 +150,7 @@ __global__ void __launch_bounds__(384, 1)
     auto bar_p_full = [&](int t) { return bar0 + 8u * (3 + 4 * C::NS + t); };
     auto bar_o_full = [&](int t) { return bar0 + 8u * (5 + 4 * C::NS + t); };
     const uint32_t bar_drain = bar0 + 8u * (7 + 4 * C::NS);
+    const uint32_t bar_qrot = bar0 + 8u * (8 + 4 * C::NS);  // Q tiles rotated (ROPE_Q)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 8);
 
@@ -160,6 +168,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(bar_o_full(t), 1);
         }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_qrot, 256);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -270,7 +279,7 @@ __global__ void __launch_bounds__(384, 1)
                            IDESC_O, (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            bool ok = wait_phase(bar_q, 0, SITE_MMA_Q, wc);
+            bool ok = wait_phase(ROPE_Q ? bar_qrot : bar_q, 0, SITE_MMA_Q, wc);
             if (ok) ok = wait_phase(bar_k_full(0), 0, SITE_MMA_K_FULL, wc);
             if (ok) {
                 tc_fence_after_sync();
@@ -346,7 +355,24 @@ __global__ void __launch_bounds__(384, 1)
         float m = 0.f;   // running max of scaled logits (log2 units); set by block 0
         float l = 0.f;   // running sum of 2^(s - m)
         bool ok = true;
-        for (int j = 0; j < nkv; ++j) {
+        if constexpr (ROPE_Q) {
+            // Rotate this thread's row of its Q tile in place in shared memory
+            // (128-byte swizzled rows: 16-byte chunk cw of row r sits at chunk
+            // cw ^ (r & 7)), then hand the tile to the MMA issuer.
+            ok = __all_sync(0xffffffffu, wait_phase(bar_q, 0, SITE_SM_Q, wc));
+            const int n = q0 + t * C::BM + row;
+            if (ok && n < Sq) {
+                uint8_t *rowp = smem + C::Q_OFF + t * C::TILE_BYTES + row * 128;
+#pragma unroll 4
+                for (int c = 0; c < HD / 8; ++c) {
+                    uint4 *p = reinterpret_cast<uint4 *>(rowp + (c >> 3) * C::HALF_BYTES + (((c & 7) ^ (row & 7)) << 4));
+                    *p = rotate_chunk(*p, c, n, rope_geom, rope_tab);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar_qrot);
+        }
+        for (int j = 0; ok && j < nkv; ++j) {
             // every lane waits; the outcome is made warp-uniform so that the
             // warp-collective tcgen05 ops below never run on a partial warp
             ok = __all_sync(0xffffffffu, wait_phase(bar_s_full(t), j & 1, SITE_SM_S_FULL, wc));

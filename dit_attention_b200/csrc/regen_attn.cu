@@ -67,18 +67,19 @@ bool make_bhsd_map(CUtensorMap *map, const void *base, int64_t BH, int64_t S, in
     return r == CUDA_SUCCESS;
 }
 
-template <int HD, bool NEG>
+template <int HD, bool NEG, bool ROPE_Q = false>
 int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, regen_bf16 *out,
-                float *lse, int64_t BH, int Sq, int Skv, float scale, cudaStream_t stream)
+                float *lse, int64_t BH, int Sq, int Skv, float scale, cudaStream_t stream,
+                const double *rope_tab = nullptr, regen::RopeGeom geom = regen::RopeGeom{})
 {
     using C = regen::AttnCfg<HD>;
     static std::once_flag once;
     static int attr_status = REGEN_OK;
     std::call_once(once, [] {
         cudaFuncAttributes fa;
-        if (cudaFuncSetAttribute(regen::attn_fwd_kernel<HD, NEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncGetAttributes(&fa, regen::attn_fwd_kernel<HD, NEG>) != cudaSuccess)
+        if (cudaFuncSetAttribute(regen::attn_fwd_kernel<HD, NEG, ROPE_Q>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, regen::attn_fwd_kernel<HD, NEG, ROPE_Q>) != cudaSuccess)
             attr_status = REGEN_ERR_CUDA;
         else if (fa.numRegs < C::MIN_LAUNCH_REGS)
             // the in-kernel register re-allocation would not fit: refuse to launch
@@ -93,8 +94,8 @@ int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, r
     const int64_t grid = npairs * BH;
     if (grid > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
     const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    regen::attn_fwd_kernel<HD, NEG><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, to, lse, Sq, Skv, scale_log2, g_wait_limit_ns.load());
+    regen::attn_fwd_kernel<HD, NEG, ROPE_Q><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, to, lse, Sq, Skv, scale_log2, g_wait_limit_ns.load(), rope_tab, geom);
     return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
 }
 
@@ -104,6 +105,38 @@ int grid_for(int64_t work, int threads)
     const int64_t cap = 148 * 32;  // grid-stride beyond ~32 resident blocks per SM
     if (blocks > cap) blocks = cap;
     return static_cast<int>(blocks < 1 ? 1 : blocks);
+}
+
+// Scratch of the RoPE-fused attention: the fp64 (cos, sin) table, then the
+// rotated K ([B*H, S, D] bf16), each starting on a 256-byte boundary.
+int64_t rope_table_bytes(const regen::RopeGeom &g) { return (g.entries() * 16 + 255) / 256 * 256; }
+
+int64_t rope_workspace_bytes(int64_t BH, int64_t S, const regen::RopeGeom &g, int D)
+{
+    return rope_table_bytes(g) + BH * S * D * 2;
+}
+
+// Table -> rotated K -> attention with Q rotated in shared memory; every
+// argument has been checked by the caller. `scratch` holds at least
+// rope_workspace_bytes(...) bytes of device memory.
+int attn_rope3d_with_scratch(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, regen_bf16 *out,
+                             float *lse, int64_t BH, int S, int D, float scale, float theta,
+                             const regen::RopeGeom &geom, uint8_t *scratch, cudaStream_t st)
+{
+    double *tab = reinterpret_cast<double *>(scratch);
+    regen_bf16 *k_rot = reinterpret_cast<regen_bf16 *>(scratch + rope_table_bytes(geom));
+    regen::rope_table_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
+    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    const int64_t chunks = BH * S * (D / 8);
+    regen::rope_apply_kernel<<<grid_for(chunks, 256), 256, 0, st>>>(
+        reinterpret_cast<const uint4 *>(k), reinterpret_cast<uint4 *>(k_rot), BH, S, D, geom, tab);
+    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    const bool neg = scale < 0.0f;
+    if (D == 128)
+        return neg ? launch_attn<128, true, true>(q, k_rot, v, out, lse, BH, S, S, scale, st, tab, geom)
+                   : launch_attn<128, false, true>(q, k_rot, v, out, lse, BH, S, S, scale, st, tab, geom);
+    return neg ? launch_attn<64, true, true>(q, k_rot, v, out, lse, BH, S, S, scale, st, tab, geom)
+               : launch_attn<64, false, true>(q, k_rot, v, out, lse, BH, S, S, scale, st, tab, geom);
 }
 
 }  // namespace
@@ -142,6 +175,50 @@ REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const reg
                    : launch_attn<128, false>(q, k, v, out, lse, BH, Sq, Skv, scale, st);
     return neg ? launch_attn<64, true>(q, k, v, out, lse, BH, Sq, Skv, scale, st)
                : launch_attn<64, false>(q, k, v, out, lse, BH, Sq, Skv, scale, st);
+}
+
+REGEN_API int64_t regen_attn_fwd_rope3d_workspace_bytes(int B, int H, int T, int Hh, int Ww, int D)
+{
+    if (B < 0 || H < 0 || T <= 0 || Hh <= 0 || Ww <= 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
+    const int64_t S = static_cast<int64_t>(T) * Hh * Ww;
+    if (S > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    return rope_workspace_bytes(static_cast<int64_t>(B) * H, S, regen::RopeGeom::make(T, Hh, Ww, D), D);
+}
+
+REGEN_API int regen_attn_fwd_rope3d(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
+                                    regen_bf16 *out, float *lse, int B, int H, int Sq, int Skv, int D,
+                                    float scale, regen_stream_t stream, int T, int Hh, int Ww, float theta,
+                                    void *workspace, int64_t workspace_bytes)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Skv < 0 || D < 0 || T <= 0 || Hh <= 0 || Ww <= 0 || workspace_bytes < 0)
+        return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !std::isfinite(theta) || !(theta > 0.0f)) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
+    const int64_t S = static_cast<int64_t>(T) * Hh * Ww;
+    if (S > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (Sq != S || Skv != S) return REGEN_ERR_INVALID_ARG;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0) return REGEN_OK;
+    if (BH > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !out || !workspace) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return REGEN_ERR_MISALIGNED;
+    const regen::RopeGeom geom = regen::RopeGeom::make(T, Hh, Ww, D);
+    const int64_t need = rope_workspace_bytes(BH, S, geom, D);
+    if (workspace_bytes < need) return REGEN_ERR_INVALID_ARG;
+    const int64_t tbytes = BH * S * D * 2, lbytes = BH * S * 4;
+    const void *ins[3] = {q, k, v};
+    for (const void *in : ins)
+        if (overlaps(out, tbytes, in, tbytes) || overlaps(lse, lbytes, in, tbytes) ||
+            overlaps(workspace, need, in, tbytes))
+            return REGEN_ERR_INVALID_ARG;
+    if (overlaps(lse, lbytes, out, tbytes) || overlaps(workspace, need, out, tbytes) ||
+        overlaps(workspace, need, lse, lbytes))
+        return REGEN_ERR_INVALID_ARG;
+    return attn_rope3d_with_scratch(q, k, v, out, lse, BH, static_cast<int>(S), D, scale, theta, geom,
+                                    static_cast<uint8_t *>(workspace), reinterpret_cast<cudaStream_t>(stream));
 }
 
 REGEN_API int regen_rope3d(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta, int B,

@@ -37,13 +37,107 @@ __device__ __forceinline__ uint32_t double_to_bf16_bits(double x)
     return b >> 16;
 }
 
+// Rotate one (even, odd) pair packed as two bf16 by the angle with cosine c
+// and sine s, in fp64 with one explicit rounding order (so every kernel that
+// rotates gives the same bits), then round each result once to bf16.
 __device__ __forceinline__ uint32_t rotate_pair(uint32_t packed, double c, double s)
 {
     const double x0 = bf16_bits_to_double(packed & 0xFFFFu);
     const double x1 = bf16_bits_to_double(packed >> 16);
-    const double y0 = x0 * c - x1 * s;
-    const double y1 = x0 * s + x1 * c;
+    const double y0 = __fma_rn(x0, c, -__dmul_rn(x1, s));
+    const double y1 = __fma_rn(x0, s, __dmul_rn(x1, c));
     return double_to_bf16_bits(y0) | (double_to_bf16_bits(y1) << 16);
+}
+
+// cos and sin of pos * theta^(-local/width) for the pair starting at
+// dimension `local` of an axis block of `width` dimensions (fp64).
+__device__ __forceinline__ void rope_angle(int pos, int local, int width, double theta, double &c, double &s)
+{
+    const double freq = pow(theta, -static_cast<double>(local) / static_cast<double>(width));
+    sincos(static_cast<double>(pos) * freq, &s, &c);
+}
+
+// Geometry of the 3D RoPE for a latent grid and head dim: axis blocks t, h, w
+// of widths dt, dh, dh; table of (cos, sin) per (axis, position, pair) laid
+// out as [T][dt/2] then [Hh][dh/2] then [Ww][dh/2] entries of two doubles.
+struct RopeGeom {
+    int T, Hh, Ww, dt, dh;
+    __host__ __device__ static RopeGeom make(int T, int Hh, int Ww, int D)
+    {
+        RopeGeom g;
+        g.T = T; g.Hh = Hh; g.Ww = Ww;
+        g.dh = 2 * (D / 6);
+        g.dt = D - 2 * g.dh;
+        return g;
+    }
+    __host__ __device__ int64_t entries() const
+    {
+        return static_cast<int64_t>(T) * (dt / 2) + static_cast<int64_t>(Hh) * (dh / 2) +
+               static_cast<int64_t>(Ww) * (dh / 2);
+    }
+    // table entry of the pair whose first dimension is d, for token n
+    __device__ __forceinline__ int64_t entry(int n, int d) const
+    {
+        if (d < dt) return static_cast<int64_t>(n / (Hh * Ww)) * (dt / 2) + d / 2;
+        const int64_t base_h = static_cast<int64_t>(T) * (dt / 2);
+        if (d < dt + dh) return base_h + static_cast<int64_t>((n / Ww) % Hh) * (dh / 2) + (d - dt) / 2;
+        const int64_t base_w = base_h + static_cast<int64_t>(Hh) * (dh / 2);
+        return base_w + static_cast<int64_t>(n % Ww) * (dh / 2) + (d - dt - dh) / 2;
+    }
+};
+
+// tab[2e], tab[2e+1] = cos, sin of every table entry e (grid-stride).
+__global__ void rope_table_kernel(double *__restrict__ tab, RopeGeom g, double theta)
+{
+    const int64_t n = g.entries();
+    const int64_t base_h = static_cast<int64_t>(g.T) * (g.dt / 2);
+    const int64_t base_w = base_h + static_cast<int64_t>(g.Hh) * (g.dh / 2);
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n; e += stride) {
+        int pos, j, width;
+        if (e < base_h) {
+            pos = static_cast<int>(e / (g.dt / 2)); j = static_cast<int>(e % (g.dt / 2)); width = g.dt;
+        } else if (e < base_w) {
+            pos = static_cast<int>((e - base_h) / (g.dh / 2)); j = static_cast<int>((e - base_h) % (g.dh / 2));
+            width = g.dh;
+        } else {
+            pos = static_cast<int>((e - base_w) / (g.dh / 2)); j = static_cast<int>((e - base_w) % (g.dh / 2));
+            width = g.dh;
+        }
+        double c, s;
+        rope_angle(pos, 2 * j, width, theta, c, s);
+        tab[2 * e] = c;
+        tab[2 * e + 1] = s;
+    }
+}
+
+// Rotate the 16-byte chunk holding dimensions [8c, 8c + 8) of token n's row.
+__device__ __forceinline__ uint4 rotate_chunk(uint4 v, int c, int n, const RopeGeom &g,
+                                              const double *__restrict__ tab)
+{
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int64_t e = g.entry(n, c * 8 + 2 * p);
+        w[p] = rotate_pair(w[p], __ldg(tab + 2 * e), __ldg(tab + 2 * e + 1));
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// dst = RoPE(src) for `rows` rows of S x D (out of place), from the table.
+__global__ void rope_apply_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int64_t rows, int S,
+                                  int D, RopeGeom g, const double *__restrict__ tab)
+{
+    const int chunks = D >> 3;
+    const int64_t per_row = static_cast<int64_t>(S) * chunks;
+    const int64_t total = rows * per_row;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total; i += stride) {
+        const int64_t in_row = i % per_row;
+        const int n = static_cast<int>(in_row / chunks);
+        const int c = static_cast<int>(in_row % chunks);
+        dst[i] = rotate_chunk(src[i], c, n, g, tab);
+    }
 }
 
 // grid: ceil(S * D/8 / blockDim) blocks; x (q then k) has `rows` rows of S x D.
@@ -70,8 +164,7 @@ __global__ void rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k
         } else {
             axis = 2; local = d - dt - dh; width = dh;
         }
-        const double freq = pow(theta, -static_cast<double>(local) / static_cast<double>(width));
-        sincos(static_cast<double>(pos[axis]) * freq, &sn[p], &cs[p]);
+        rope_angle(pos[axis], local, width, theta, cs[p], sn[p]);
     }
     const int64_t row_stride = static_cast<int64_t>(S) * D;
     const int64_t off = static_cast<int64_t>(n) * D + c * 8;

@@ -75,6 +75,41 @@ REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const reg
                              regen_stream_t stream);
 
 /*
+ * regen_attn_fwd_rope3d -- self-attention with the 3D RoPE applied on the
+ * way in: the same result, bit for bit, as regen_rope3d(q, k, ...) followed
+ * by regen_attn_fwd(...), but q and k are left unmodified.
+ *  - Q is rotated inside the attention kernel, on its 128-row tiles in
+ *    shared memory right after they are loaded (fused into the Q load).
+ *  - K is rotated once into the workspace: every query tile of a head reads
+ *    every key tile, so rotating K per load would repeat the work for each of
+ *    the ceil(S/256) query-tile pairs.
+ *  - The (cos, sin) of every (axis, position, pair) are computed once, in fp64,
+ *    into a small table at the start of the workspace.
+ *
+ *   q, k, v, out, lse, B, H, D, scale, stream: as regen_attn_fwd
+ *   Sq == Skv == T*Hh*Ww (else REGEN_ERR_INVALID_ARG); T, Hh, Ww, theta: as regen_rope3d
+ *   workspace        device scratch owned by the caller, 256-byte aligned, at least
+ *                    regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D) bytes;
+ *                    it must not overlap any other argument; its contents are
+ *                    overwritten and need not be initialised
+ *   workspace_bytes  its size (a smaller size is REGEN_ERR_INVALID_ARG)
+ * Three launches on `stream`: the table, the rotated K, the attention.
+ */
+REGEN_API int regen_attn_fwd_rope3d(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
+                                    regen_bf16 *out, float *lse,
+                                    int B, int H, int Sq, int Skv, int D, float scale,
+                                    regen_stream_t stream,
+                                    int T, int Hh, int Ww, float theta,
+                                    void *workspace, int64_t workspace_bytes);
+
+/*
+ * Bytes of workspace regen_attn_fwd_rope3d needs: a 256-byte-rounded table of
+ * 16 * (T*(D - 4*floor(D/6))/2 + (Hh + Ww)*floor(D/6)) bytes plus B*H*S*D*2
+ * bytes of rotated K. Negative (a regen_status) for invalid sizes.
+ */
+REGEN_API int64_t regen_attn_fwd_rope3d_workspace_bytes(int B, int H, int T, int Hh, int Ww, int D);
+
+/*
  * regen_rope3d -- 3D rotary position embedding of Q and K, in place.
  *
  * The sequence is the flattened latent grid: token n = (t*Hh + y)*Ww + x,

@@ -90,3 +90,28 @@ def test_python_binding_raises(lib):
     with pytest.raises(rg.RegenError) as e:
         rg.regen_attn_fwd(FAKE, FAKE + MB, FAKE + 2 * MB, FAKE + 3 * MB, None, 1, 1, 8, 8, 96, 0.1, stream=0)
     assert e.value.status == -2
+
+
+def test_rope3d_fused_workspace_bytes(lib):
+    # table: 16 * (T*dt/2 + (Hh + Ww)*dh/2), rounded up to 256; plus B*H*S*D*2 of rotated K
+    T, Hh, Ww, D = 20, 30, 52, 128
+    table = (16 * (T * 22 + (Hh + Ww) * 21) + 255) // 256 * 256
+    assert rg.regen_attn_fwd_rope3d_workspace_bytes(1, 40, T, Hh, Ww, D) == table + 40 * T * Hh * Ww * D * 2
+    assert lib.regen_attn_fwd_rope3d_workspace_bytes(1, 1, 0, 1, 1, 128) == -1
+    assert lib.regen_attn_fwd_rope3d_workspace_bytes(1, 1, 1, 1, 1, 96) == -2
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(Sq=99), -1), (dict(Skv=99), -1), (dict(D=96), -2), (dict(theta=0.0), -1), (dict(scale=float("nan")), -1),
+    (dict(workspace=None), -1), (dict(workspace=FAKE + 100 * MB + 16), -3), (dict(workspace_bytes=1000), -1),
+    (dict(workspace=FAKE), -1), (dict(B=0), 0),
+])
+def test_rope3d_fused_validation(lib, args, status):
+    a = dict(q=FAKE, k=FAKE + 10 * MB, v=FAKE + 20 * MB, out=FAKE + 30 * MB, lse=FAKE + 40 * MB, B=1, H=2, Sq=60,
+             Skv=60, D=128, scale=0.1, T=3, Hh=4, Ww=5, theta=1e4, workspace=FAKE + 100 * MB,
+             workspace_bytes=64 * MB)
+    a.update(args)
+    rc = lib.regen_attn_fwd_rope3d(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["H"], a["Sq"], a["Skv"],
+                                   a["D"], a["scale"], None, a["T"], a["Hh"], a["Ww"], a["theta"], a["workspace"],
+                                   a["workspace_bytes"])
+    assert rc == status

@@ -290,3 +290,53 @@ def test_selftest_exp2_against_cuda_exp2f_and_fp64():
     assert (y[low] == 0).all()
     tiny = (~normal) & (~low)
     assert (y[tiny] >= 0).all() and (y[tiny] < 2.0 ** -124).all()
+
+
+# ------------------------------------------------- RoPE fused into Q load ---
+
+@pytest.mark.parametrize("B,H,grid,D", [
+    (1, 2, (2, 5, 13), 128), (2, 1, (3, 7, 11), 64), (1, 3, (1, 16, 16), 128), (1, 1, (4, 30, 52), 128),
+])
+def test_rope3d_fused_equals_unfused(B, H, grid, D):
+    S = grid[0] * grid[1] * grid[2]
+    q, k, v = rand_bf16((B, H, S, D)), rand_bf16((B, H, S, D)), rand_bf16((B, H, S, D))
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    out, lse = rg.attn_fwd_rope3d(dq, dk, dv, grid)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_bits(dq), q)            # inputs untouched
+    np.testing.assert_array_equal(to_bits(dk), k)
+    uq, uk = dq.clone(), dk.clone()
+    rg.rope3d_(uq, uk, grid)
+    ref_out, ref_lse = rg.attn_fwd(uq, uk, dv)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_bits(out), to_bits(ref_out))
+    np.testing.assert_array_equal(lse.cpu().numpy(), ref_lse.cpu().numpy())
+
+
+def test_rope3d_fused_25_frame_window_vs_oracle():
+    w = synth.WORKLOADS["win25_s10920"]
+    q, k, v = synth.make_inputs(w)
+    out, lse = rg.attn_fwd_rope3d(to_dev(q), to_dev(k), to_dev(v), w.grid, w.theta)
+    torch.cuda.synchronize()
+    heads = [0, 5, 11]
+    qh = oracle.rope3d(q.reshape(12, w.Sq, w.D)[heads], w.grid, w.theta)
+    kh = oracle.rope3d(k.reshape(12, w.Skv, w.D)[heads], w.grid, w.theta)
+    rows = sample_rows(len(heads), w.Sq, 64)
+    ref, rl = oracle.attention(qh, kh, v.reshape(12, w.Skv, w.D)[heads], w.scale, rows=rows)
+    gout = to_bits(out).reshape(12, w.Sq, w.D)[heads].reshape(-1, w.D)[rows]
+    glse = lse.cpu().numpy().reshape(12, w.Sq)[heads].reshape(-1)[rows]
+    check_attention(gout, glse, ref, rl, "fused rope, 25-frame window")
+
+
+def test_rope3d_fused_workspace_errors():
+    grid = (2, 3, 4)
+    q = to_dev(rand_bf16((1, 1, 24, 128)))
+    need = rg.regen_attn_fwd_rope3d_workspace_bytes(1, 1, *grid, 128)
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(rg.RegenError) as e:
+        rg.attn_fwd_rope3d(q, q.clone(), q.clone(), grid, workspace=small)
+    assert e.value.status == -1
+    ws = torch.empty(need + 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(rg.RegenError) as e:
+        rg.attn_fwd_rope3d(q, q.clone(), q.clone(), grid, workspace=ws[16:])
+    assert e.value.status == -3
