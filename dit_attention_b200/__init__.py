@@ -31,7 +31,7 @@ import threading
 __all__ = [
     "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
     "regen_status_str", "regen_last_device_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
-    "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes",
+    "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes", "regen_attn_fwd_rope3d_noalloc",
     "attn_fwd", "attn_fwd_rope3d", "rope3d_", "lse_merge", "STATUS",
 ]
 
@@ -69,6 +69,9 @@ def load():
         L.regen_attn_fwd_rope3d.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp,
                                             i32, i32, i32, f32, vp, i64]
         L.regen_attn_fwd_rope3d.restype = i32
+        L.regen_attn_fwd_rope3d_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp,
+                                                    i32, i32, i32, f32]
+        L.regen_attn_fwd_rope3d_noalloc.restype = i32
         L.regen_attn_fwd_rope3d_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
         L.regen_attn_fwd_rope3d_workspace_bytes.restype = i64
         L.regen_rope3d.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, vp]
@@ -133,6 +136,22 @@ def regen_attn_fwd_rope3d(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream, T,
     _check(load().regen_attn_fwd_rope3d(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D,
                                         float(scale), _stream(stream), T, Hh, Ww, float(theta), _ptr(workspace),
                                         int(workspace_bytes)), "regen_attn_fwd_rope3d")
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20   # REGEN_NOALLOC_SCRATCH_BYTES
+
+
+def regen_attn_fwd_rope3d_noalloc(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream, T, Hh, Ww, theta) -> None:
+    """The RoPE-fused attention with the library's fixed scratch instead of a
+    caller workspace: for callers that may not allocate device memory."""
+    rc = load().regen_attn_fwd_rope3d_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D,
+                                              float(scale), _stream(stream), T, Hh, Ww, float(theta))
+    if rc == -2 and D in (64, 128) and T > 0 and Hh > 0 and Ww > 0:
+        need = load().regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
+        if need > NOALLOC_SCRATCH_BYTES:
+            raise RegenError(rc, f"regen_attn_fwd_rope3d_noalloc: needs {need} bytes of scratch, "
+                                 f"the fixed array holds {NOALLOC_SCRATCH_BYTES}")
+    _check(rc, "regen_attn_fwd_rope3d_noalloc")
 
 
 def regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D) -> int:

@@ -139,6 +139,34 @@ int attn_rope3d_with_scratch(const regen_bf16 *q, const regen_bf16 *k, const reg
                : launch_attn<64, false, true>(q, k_rot, v, out, lse, BH, S, S, scale, st, tab, geom);
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for regen_attn_fwd_rope3d_noalloc (declared in regen_attn.h).
+// The array belongs to this library: every device that loads the library
+// holds it until the process exits. In host code `g_noalloc_scratch` names
+// only a host-side stand-in; the device address comes from
+// cudaGetSymbolAddress, resolved once per device (with that device current)
+// on the first call made on that device, and cached.
+constexpr int64_t kNoAllocScratchBytes = REGEN_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+uint8_t *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the fixed scratch on the current device (nullptr on error).
+uint8_t *noalloc_scratch_on_current_device()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
+    }
+    return g_noalloc_ptr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -219,6 +247,40 @@ REGEN_API int regen_attn_fwd_rope3d(const regen_bf16 *q, const regen_bf16 *k, co
         return REGEN_ERR_INVALID_ARG;
     return attn_rope3d_with_scratch(q, k, v, out, lse, BH, static_cast<int>(S), D, scale, theta, geom,
                                     static_cast<uint8_t *>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+REGEN_API int regen_attn_fwd_rope3d_noalloc(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
+                                            regen_bf16 *out, float *lse, int B, int H, int Sq, int Skv, int D,
+                                            float scale, regen_stream_t stream, int T, int Hh, int Ww,
+                                            float theta)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Skv < 0 || D < 0 || T <= 0 || Hh <= 0 || Ww <= 0)
+        return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !std::isfinite(theta) || !(theta > 0.0f)) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
+    const int64_t S = static_cast<int64_t>(T) * Hh * Ww;
+    if (S > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (Sq != S || Skv != S) return REGEN_ERR_INVALID_ARG;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0) return REGEN_OK;
+    if (BH > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const regen::RopeGeom geom = regen::RopeGeom::make(T, Hh, Ww, D);
+    // the whole scratch (table + rotated K) must fit the fixed array
+    if (rope_workspace_bytes(BH, S, geom, D) > kNoAllocScratchBytes) return REGEN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !out) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+        return REGEN_ERR_MISALIGNED;
+    const int64_t tbytes = BH * S * D * 2, lbytes = BH * S * 4;
+    const void *ins[3] = {q, k, v};
+    for (const void *in : ins)
+        if (overlaps(out, tbytes, in, tbytes) || overlaps(lse, lbytes, in, tbytes)) return REGEN_ERR_INVALID_ARG;
+    if (overlaps(lse, lbytes, out, tbytes)) return REGEN_ERR_INVALID_ARG;
+    uint8_t *scratch = noalloc_scratch_on_current_device();
+    if (!scratch) return REGEN_ERR_CUDA;
+    // Every scratch byte this call reads is written earlier in the same call
+    // (table, then rotated K), so nothing left by a previous call matters.
+    return attn_rope3d_with_scratch(q, k, v, out, lse, BH, static_cast<int>(S), D, scale, theta, geom, scratch,
+                                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 REGEN_API int regen_rope3d(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta, int B,

@@ -110,6 +110,37 @@ REGEN_API int regen_attn_fwd_rope3d(const regen_bf16 *q, const regen_bf16 *k, co
 REGEN_API int64_t regen_attn_fwd_rope3d_workspace_bytes(int B, int H, int T, int Hh, int Ww, int D);
 
 /*
+ * regen_attn_fwd_rope3d_noalloc -- regen_attn_fwd_rope3d without a workspace
+ * argument, for callers that cannot allocate device memory: for example a
+ * plug-in running inside a host application that owns every device
+ * allocation, or a serving loop in which cudaMalloc/cudaFree (which may
+ * synchronise the device and stall other work) are not permitted. It takes
+ * the same arguments and gives the same results, but calls no allocator at
+ * all (no cudaMalloc, no cudaFree, no allocating library routine).
+ * The pages have no counterpart: this is a deployment convenience.
+ *
+ *  - Scratch: a fixed array of REGEN_NOALLOC_SCRATCH_BYTES (64 MiB) inside
+ *    this library, kept by every device that loads the library until the
+ *    process exits. A call whose scratch -- the same size
+ *    regen_attn_fwd_rope3d_workspace_bytes reports -- exceeds it is rejected
+ *    with REGEN_ERR_UNSUPPORTED before anything is launched (that admits e.g.
+ *    12 heads of 10920 tokens at D = 128, not 40 heads of 31200).
+ *  - Set-up: the first call made on a device, with that device current, looks
+ *    up the array's device address (cudaGetSymbolAddress) and caches it;
+ *    make that first call before any stream capture on that device.
+ *  - Sharing: all calls use the same array, which keeps whatever the last
+ *    call left in it. Nothing there needs clearing, since each call writes
+ *    every byte it later reads. Calls whose work overlaps on the GPU (for
+ *    example on two unordered streams) race on the array: order them.
+ */
+#define REGEN_NOALLOC_SCRATCH_BYTES (64LL << 20)
+REGEN_API int regen_attn_fwd_rope3d_noalloc(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
+                                            regen_bf16 *out, float *lse,
+                                            int B, int H, int Sq, int Skv, int D, float scale,
+                                            regen_stream_t stream,
+                                            int T, int Hh, int Ww, float theta);
+
+/*
  * regen_rope3d -- 3D rotary position embedding of Q and K, in place.
  *
  * The sequence is the flattened latent grid: token n = (t*Hh + y)*Ww + x,
