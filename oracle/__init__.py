@@ -36,6 +36,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+# Tests that check the pins against deliberately broken copies of oracle.c
+# point this at such a copy (tests/test_oracle_mutants.py); nothing else sets it.
+_LIB_OVERRIDE = os.environ.get("ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
@@ -45,14 +48,19 @@ _i64p = ctypes.POINTER(ctypes.c_int64)
 _i64 = ctypes.c_int64
 
 
+def compile_library(src: str, out: str) -> str:
+    """gcc -O2 -ffp-contract=off -fopenmp -shared: the oracle's one build recipe."""
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-ffp-contract=off", "-fopenmp", "-shared", "-fPIC", src, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
     """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-O2", "-ffp-contract=off", "-fopenmp", "-shared", "-fPIC",
-               _SRC, "-o", tmp, "-lm"]
-        subprocess.run(cmd, check=True)
-        os.replace(tmp, _LIB)
+        compile_library(_SRC, _LIB)
     return _LIB
 
 
@@ -60,8 +68,11 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB)
+            if _LIB_OVERRIDE:
+                lib = ctypes.CDLL(_LIB_OVERRIDE)
+            else:
+                build()
+                lib = ctypes.CDLL(_LIB)
             lib.oracle_attention_f64.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _i64,
                                                  ctypes.c_double, _i64p, _i64, _dp, _dp]
             lib.oracle_attention_f64.restype = None

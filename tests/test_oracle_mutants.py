@@ -1,0 +1,64 @@
+"""The pins catch plausible mistakes in the oracle.
+
+Each case below plants one mistake in a copy of oracle/oracle.c (a transposed
+operand, a wrong sign, a dropped term, a wrong index or exponent), builds it
+with the oracle's own recipe, and runs tests/test_oracle_pins.py against it in
+a subprocess: at least one pin must fail. The unmodified source, built the
+same way, must pass them all. Everything runs on the CPU.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+MUTANTS = {
+    "K transposed in QK^T": ("dot += at(q, qo + d) * at(k, ko + j * D + d);",
+                             "dot += at(q, qo + d) * at(k, ko + d * Skv + j);"),
+    "V transposed in PV": ("out[d] += p[j] * at(v, ko + j * D + d);",
+                           "out[d] += p[j] * at(v, ko + d * Skv + j);"),
+    "scale applied twice": ("p[j] = scale * dot;", "p[j] = scale * scale * dot;"),
+    "max not subtracted": ("p[j] = exp(p[j] - m);", "p[j] = exp(p[j]);"),
+    "normalisation dropped": ("for (int64_t d = 0; d < D; ++d) out[d] /= l;", ""),
+    "lse without the max": ("*lse = m + log(l);", "*lse = log(l);"),
+    "merge weights swapped": ("(wa * oa[r * D + d] + wb * ob[r * D + d])",
+                              "(wb * oa[r * D + d] + wa * ob[r * D + d])"),
+    "rope rotation sign": ("row[base[a] + 2 * j] = x0 * c - x1 * s;", "row[base[a] + 2 * j] = x0 * c + x1 * s;"),
+    "rope h and w swapped": ("pos[1] = (n / Ww) % Hh;\n        pos[2] = n % Ww;",
+                             "pos[1] = n % Ww;\n        pos[2] = (n / Ww) % Hh;"),
+    "rope frequency exponent": ("-2.0 * (double)j / (double)width[a]", "-1.0 * (double)j / (double)width[a]"),
+    "rope pair partner index": ("double x1 = row[base[a] + 2 * j + 1];", "double x1 = row[base[a] + j + 1];"),
+}
+
+
+def _run_pins(lib_path):
+    env = dict(os.environ, ORACLE_LIB=lib_path)
+    res = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                          "-x", "-q", "-p", "no:cacheprovider"], cwd=ROOT, env=env, capture_output=True, text=True,
+                         timeout=600)
+    return res.returncode, res.stdout[-2000:]
+
+
+def _build(tmp_path, name, text):
+    src = tmp_path / f"{name}.c"
+    src.write_text(text)
+    return oracle.compile_library(str(src), str(tmp_path / f"lib{name}.so"))
+
+
+def test_unmodified_oracle_passes_its_pins(tmp_path):
+    rc, out = _run_pins(_build(tmp_path, "clean", open(SRC).read()))
+    assert rc == 0, out
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(tmp_path, name):
+    old, new = MUTANTS[name]
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation target not found once: {old!r}"
+    rc, out = _run_pins(_build(tmp_path, "mutant", text.replace(old, new)))
+    assert rc != 0, f"no pin caught the planted mistake '{name}'"
