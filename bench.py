@@ -48,7 +48,7 @@ def parse():
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
-    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--e2e-steps", type=int, default=12)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     return p.parse_args()
@@ -211,20 +211,25 @@ def run_native(args, rank, world, local_rank):
     names = ["rope3d", "attn_self", "attn_cross_ref", "attn_cross_ctx", "lse_merge"]
     LAUNCHES_PER_STEP = len(names)
 
-    def step(ev=None):
+    outs0 = dict(out=out, lse=lse, oa=oa, la=la, ob=ob, lb=lb, oc=oc, lc=lc)
+
+    def step(ev=None, inp=None, o=None):
+        inp = d if inp is None else inp
+        o = outs0 if o is None else o
+
         def mark(i):
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        rg.regen_rope3d(d["q"], d["k"], T, Hh, Ww, ws.theta, B, H, D, sh)
+        rg.regen_rope3d(inp["q"], inp["k"], T, Hh, Ww, ws.theta, B, H, D, sh)
         mark(1)
-        rg.regen_attn_fwd(d["q"], d["k"], d["v"], out, lse, B, H, S, S, D, scale, sh)
+        rg.regen_attn_fwd(inp["q"], inp["k"], inp["v"], o["out"], o["lse"], B, H, S, S, D, scale, sh)
         mark(2)
-        rg.regen_attn_fwd(d["qc"], d["kr"], d["vr"], oa, la, B, H, S, N_REF, D, scale, sh)
+        rg.regen_attn_fwd(inp["qc"], inp["kr"], inp["vr"], o["oa"], o["la"], B, H, S, N_REF, D, scale, sh)
         mark(3)
-        rg.regen_attn_fwd(d["qc"], d["kx"], d["vx"], ob, lb, B, H, S, wc.Skv - N_REF, D, scale, sh)
+        rg.regen_attn_fwd(inp["qc"], inp["kx"], inp["vx"], o["ob"], o["lb"], B, H, S, wc.Skv - N_REF, D, scale, sh)
         mark(4)
-        rg.regen_lse_merge(oa, la, ob, lb, oc, lc, B * H * S, D, sh)
+        rg.regen_lse_merge(o["oa"], o["la"], o["ob"], o["lb"], o["oc"], o["lc"], B * H * S, D, sh)
         mark(5)
 
     def barrier():
@@ -263,6 +268,35 @@ def run_native(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     value = aggregate_tflops(flops_step, world, ms_step)
 
+    # ---- the same step with the RoPE fused into the Q load (regen_attn_fwd_rope3d):
+    # Q rotated on its tiles in shared memory, K rotated once into the workspace;
+    # q and k are not modified, so every step starts from the unrotated inputs.
+    rope_ws_bytes = rg.regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
+    rope_ws = torch.empty(rope_ws_bytes, dtype=torch.uint8, device=dev)
+
+    def step_fused():
+        rg.regen_attn_fwd_rope3d(d["q"], d["k"], d["v"], out, lse, B, H, S, S, D, scale, sh, T, Hh, Ww,
+                                 ws.theta, rope_ws, rope_ws_bytes)
+        rg.regen_attn_fwd(d["qc"], d["kr"], d["vr"], oa, la, B, H, S, N_REF, D, scale, sh)
+        rg.regen_attn_fwd(d["qc"], d["kx"], d["vx"], ob, lb, B, H, S, wc.Skv - N_REF, D, scale, sh)
+        rg.regen_lse_merge(oa, la, ob, lb, oc, lc, B * H * S, D, sh)
+
+    n_alt = max(3, min(args.steps, 20))
+    for _ in range(args.warmup):
+        step_fused()
+    torch.cuda.synchronize()
+    barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(n_alt):
+        step_fused()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_fused = max_over_ranks(f0.elapsed_time(f1), world, dev) / n_alt
+    del rope_ws
+
     # ---- end to end: pinned host inputs -> device -> hot path -> outputs to pinned host
     pin = {n: torch.from_numpy(a.view(np.int16)).pin_memory() for n, a in host.items()}
     res_host = {"out": torch.empty(out.shape, dtype=torch.int16).pin_memory(),
@@ -272,28 +306,80 @@ def run_native(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = sum(t.numel() * t.element_size() for t in res_host.values())
 
-    def e2e_step():
+    def read_back(o):
+        res_host["out"].copy_(o["out"].view(torch.int16), non_blocking=True)
+        res_host["lse"].copy_(o["lse"], non_blocking=True)
+        res_host["oc"].copy_(o["oc"].view(torch.int16), non_blocking=True)
+        res_host["lc"].copy_(o["lc"], non_blocking=True)
+
+    # (a) serial: copy in, compute, copy out, one step after the other on one stream
+    def e2e_serial_step():
         for n, t in pin.items():
             d[n].view(torch.int16).copy_(t, non_blocking=True)
         step()
-        res_host["out"].copy_(out.view(torch.int16), non_blocking=True)
-        res_host["lse"].copy_(lse, non_blocking=True)
-        res_host["oc"].copy_(oc.view(torch.int16), non_blocking=True)
-        res_host["lc"].copy_(lc, non_blocking=True)
+        read_back(outs0)
 
-    e2e_step()
+    e2e_serial_step()
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
+    n_serial = max(2, min(args.e2e_steps, 5))
+    for _ in range(n_serial):
+        e2e_serial_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e_serial = max_over_ranks(e0.elapsed_time(e1), world, dev) / n_serial
+
+    # (b) pipelined: step i's host->device copies (stream h2d) and step i-1's
+    # device->host read-back (stream d2h) overlap step i-1's / i's kernels
+    # (compute stream); two device buffer sets alternate, ordered by events.
+    # Every step still moves all its inputs in and all its results out.
+    d_alt = {n: torch.empty_like(t) for n, t in d.items()}
+    outs_alt = {n: torch.empty_like(t) for n, t in outs0.items()}
+    in_sets, out_sets = [d, d_alt], [outs0, outs_alt]
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+    for bset in range(2):
+        comp_done[bset].record(stream)
+        d2h_done[bset].record(s_d2h)
+
+    def e2e_pipelined_step(i):
+        bset = i % 2
+        with torch.cuda.stream(s_h2d):
+            s_h2d.wait_event(comp_done[bset])            # step i-2 is done reading this input set
+            for n, t in pin.items():
+                in_sets[bset][n].view(torch.int16).copy_(t, non_blocking=True)
+            h2d_done[bset].record(s_h2d)
+        stream.wait_event(h2d_done[bset])
+        stream.wait_event(d2h_done[bset])                # step i-2's results have been read back
+        step(inp=in_sets[bset], o=out_sets[bset])
+        comp_done[bset].record(stream)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(comp_done[bset])
+            read_back(out_sets[bset])
+            d2h_done[bset].record(s_d2h)
+
+    e2e_pipelined_step(0)
+    e2e_pipelined_step(1)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_h2d)
+    for i in range(args.e2e_steps):
+        e2e_pipelined_step(i)
+    stream.wait_event(d2h_done[(args.e2e_steps - 1) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
     e2e_value = aggregate_tflops(flops_step, world, ms_e2e)
+    del d_alt, outs_alt
 
     if world > 1:
         import torch.distributed as dist
@@ -342,8 +428,19 @@ def run_native(args, rank, world, local_rank):
         "kernels_ms": {n: round(t, 4) for n, t in per_kernel.items()},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(ms_e2e, 3),
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                "how": "pinned host inputs -> device -> the five launches -> outputs and LSEs to pinned host "
+                       "every step; copies on their own streams overlap the neighbouring steps' kernels "
+                       "(two device buffer sets); timed from the first copy to the last read-back",
+                "serial_ms_per_step": round(ms_e2e_serial, 3),
+                "serial_value": round(aggregate_tflops(flops_step, world, ms_e2e_serial), 2)},
         "clocks": clk,
+    }
+    line["rope_fused_step"] = {
+        "what": "the same step with regen_attn_fwd_rope3d (RoPE fused into the Q tile load, K rotated into "
+                "workspace) in place of regen_rope3d + regen_attn_fwd; 7 launches per step",
+        "steps": n_alt, "ms_per_step": round(ms_fused, 4),
+        "value": round(aggregate_tflops(flops_step, world, ms_fused), 2), "unit": "TFLOP/s",
     }
     s_merge = per_kernel["lse_merge"]
     s_rope = per_kernel["rope3d"]
