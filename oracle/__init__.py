@@ -11,6 +11,7 @@ Functions (each follows the definition written at its C counterpart):
 
 * ``attention(q, k, v, scale, rows=None)`` -- exact softmax attention and
   natural-log LSE, inputs bf16 bit arrays [B, H, S, D] (or doubles).
+* ``attention_bwd(q, k, v, dout, scale)`` -- dQ, dK, dV of exact attention.
 * ``lse_merge(o_a, lse_a, o_b, lse_b)`` -- two-block (O, LSE) combination.
 * ``rope3d(x, grid, theta)`` -- 3D RoPE, bf16 in/out (rounded to nearest even)
   or fp64 in/out.
@@ -79,6 +80,12 @@ def _load():
             lib.oracle_attention_bf16.argtypes = [_u16p, _u16p, _u16p, _i64, _i64, _i64, _i64,
                                                   ctypes.c_double, _i64p, _i64, _dp, _dp]
             lib.oracle_attention_bf16.restype = ctypes.c_int
+            lib.oracle_attention_bwd_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64,
+                                                     ctypes.c_double, _dp, _dp, _dp]
+            lib.oracle_attention_bwd_f64.restype = ctypes.c_int
+            lib.oracle_attention_bwd_bf16.argtypes = [_u16p, _u16p, _u16p, _u16p, _i64, _i64, _i64, _i64,
+                                                      ctypes.c_double, _dp, _dp, _dp]
+            lib.oracle_attention_bwd_bf16.restype = ctypes.c_int
             lib.oracle_lse_merge_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _dp, _dp]
             lib.oracle_lse_merge_f64.restype = None
             lib.oracle_rope3d_f64.argtypes = [_dp, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
@@ -168,6 +175,36 @@ def attention(q, k, v, scale: float, rows=None):
     if rows is None:
         return out.reshape(q.shape), lse.reshape(q.shape[:-1])
     return out, lse
+
+
+def attention_bwd(q, k, v, dout, scale: float):
+    """Gradients (dq, dk, dv) in fp64 of exact attention for upstream dout.
+
+    q, dout [..., Sq, D]; k, v [..., Skv, D]; all uint16 (bf16 bits) or all float64.
+    """
+    lib = _load()
+    q, k, v, dout = (np.ascontiguousarray(a) for a in (q, k, v, dout))
+    Sq, D = q.shape[-2], q.shape[-1]
+    Skv = k.shape[-2]
+    lead = q.shape[:-2]
+    if k.shape[:-2] != lead or v.shape != k.shape or dout.shape != q.shape or k.shape[-1] != D:
+        raise ValueError("q, k, v, dout shapes do not agree")
+    BH = int(np.prod(lead)) if lead else 1
+    dq = np.empty(q.shape, dtype=np.float64)
+    dk = np.empty(k.shape, dtype=np.float64)
+    dv = np.empty(k.shape, dtype=np.float64)
+    kinds = {a.dtype for a in (q, k, v, dout)}
+    if kinds == {np.dtype(np.uint16)}:
+        rc = lib.oracle_attention_bwd_bf16(*(_ptr(a, _u16p) for a in (q, k, v, dout)), BH, Sq, Skv, D,
+                                           float(scale), _ptr(dq, _dp), _ptr(dk, _dp), _ptr(dv, _dp))
+    elif kinds == {np.dtype(np.float64)}:
+        rc = lib.oracle_attention_bwd_f64(*(_ptr(a, _dp) for a in (q, k, v, dout)), BH, Sq, Skv, D,
+                                          float(scale), _ptr(dq, _dp), _ptr(dk, _dp), _ptr(dv, _dp))
+    else:
+        raise TypeError("inputs must all be uint16 (bf16 bits) or all float64")
+    if rc != 0:
+        raise MemoryError("oracle could not allocate its per-head P and dS")
+    return dq, dk, dv
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b):

@@ -15,6 +15,8 @@
  *
  *   oracle_attention_f64   softmax(scale * Q K^T) V per (batch, head, query),
  *                          with the natural-log LSE of the scaled logits.
+ *   oracle_attention_bwd_f64  the gradients dQ, dK, dV of that attention for an
+ *                          upstream dO (chain rule through the softmax).
  *   oracle_lse_merge_f64   the two-block combination of (O, LSE) that Ring
  *                          attention applies between KV blocks.
  *   oracle_rope3d_f64      3D rotary position embedding of the Wan2.1 DiT
@@ -185,6 +187,97 @@ int oracle_attention_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *
 {
     src_t sq = {q, 1}, sk = {k, 1}, sv = {v, 1};
     return attention_rows(sq, sk, sv, BH, Sq, Skv, D, scale, rows, nrows, out, lse);
+}
+
+/* ------------------------------------------------------------ backward --- */
+
+/*
+ * Gradients of exact attention for one (batch, head), by the chain rule
+ * applied to the definition above (no page prints them; the distillation
+ * step that trains the decoder needs them). With s_ij = scale <q_i, k_j>,
+ * P = softmax_j(s), O = P V and an upstream gradient dO:
+ *   dV_j   = sum_i P_ij dO_i
+ *   dP_ij  = <dO_i, v_j>
+ *   delta_i = sum_j P_ij dP_ij            (= <dO_i, O_i>)
+ *   dS_ij  = P_ij (dP_ij - delta_i)        (softmax Jacobian)
+ *   dQ_i   = scale sum_j dS_ij k_j
+ *   dK_j   = scale sum_i dS_ij q_i
+ * Everything in fp64 from q, k, v, dO; P is recomputed exactly per row.
+ * Inputs [Sq][D] / [Skv][D] of one head; outputs dq [Sq][D], dk, dv [Skv][D].
+ */
+static void attention_bwd_head(src_t q, int64_t qo, src_t k, src_t v, int64_t ko, src_t dout, int64_t doo,
+                               int64_t Sq, int64_t Skv, int64_t D, double scale,
+                               double *P, double *dS, double *dq, double *dk, double *dv)
+{
+    for (int64_t i = 0; i < Sq; ++i) {
+        double m = -INFINITY;
+        for (int64_t j = 0; j < Skv; ++j) {
+            double dot = 0.0;
+            for (int64_t d = 0; d < D; ++d) dot += at(q, qo + i * D + d) * at(k, ko + j * D + d);
+            P[i * Skv + j] = scale * dot;
+            if (P[i * Skv + j] > m) m = P[i * Skv + j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < Skv; ++j) {
+            P[i * Skv + j] = exp(P[i * Skv + j] - m);
+            l += P[i * Skv + j];
+        }
+        for (int64_t j = 0; j < Skv; ++j) P[i * Skv + j] /= l;
+        double delta = 0.0;
+        for (int64_t j = 0; j < Skv; ++j) {
+            double dp = 0.0;
+            for (int64_t d = 0; d < D; ++d) dp += at(dout, doo + i * D + d) * at(v, ko + j * D + d);
+            dS[i * Skv + j] = dp;
+            delta += P[i * Skv + j] * dp;
+        }
+        for (int64_t j = 0; j < Skv; ++j) dS[i * Skv + j] = P[i * Skv + j] * (dS[i * Skv + j] - delta);
+    }
+    for (int64_t x = 0; x < Sq * D; ++x) dq[x] = 0.0;
+    for (int64_t x = 0; x < Skv * D; ++x) { dk[x] = 0.0; dv[x] = 0.0; }
+    for (int64_t i = 0; i < Sq; ++i)
+        for (int64_t j = 0; j < Skv; ++j)
+            for (int64_t d = 0; d < D; ++d) {
+                dv[j * D + d] += P[i * Skv + j] * at(dout, doo + i * D + d);
+                dq[i * D + d] += scale * dS[i * Skv + j] * at(k, ko + j * D + d);
+                dk[j * D + d] += scale * dS[i * Skv + j] * at(q, qo + i * D + d);
+            }
+}
+
+static int attention_bwd(src_t q, src_t k, src_t v, src_t dout, int64_t BH, int64_t Sq, int64_t Skv, int64_t D,
+                         double scale, double *dq, double *dk, double *dv)
+{
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        double *P = (double *)malloc(sizeof(double) * (size_t)(Sq * Skv > 0 ? Sq * Skv : 1));
+        double *dS = (double *)malloc(sizeof(double) * (size_t)(Sq * Skv > 0 ? Sq * Skv : 1));
+        if (!P || !dS) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            attention_bwd_head(q, bh * Sq * D, k, v, bh * Skv * D, dout, bh * Sq * D, Sq, Skv, D, scale, P, dS,
+                               dq + bh * Sq * D, dk + bh * Skv * D, dv + bh * Skv * D);
+        }
+        free(P);
+        free(dS);
+    }
+    return failed ? -1 : 0;
+}
+
+int oracle_attention_bwd_f64(const double *q, const double *k, const double *v, const double *dout,
+                             int64_t BH, int64_t Sq, int64_t Skv, int64_t D, double scale,
+                             double *dq, double *dk, double *dv)
+{
+    src_t sq = {q, 0}, sk = {k, 0}, sv = {v, 0}, sd = {dout, 0};
+    return attention_bwd(sq, sk, sv, sd, BH, Sq, Skv, D, scale, dq, dk, dv);
+}
+
+int oracle_attention_bwd_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                              int64_t BH, int64_t Sq, int64_t Skv, int64_t D, double scale,
+                              double *dq, double *dk, double *dv)
+{
+    src_t sq = {q, 1}, sk = {k, 1}, sv = {v, 1}, sd = {dout, 1};
+    return attention_bwd(sq, sk, sv, sd, BH, Sq, Skv, D, scale, dq, dk, dv);
 }
 
 /* ------------------------------------------------------------ LSE merge --- */

@@ -32,6 +32,12 @@ MUTANTS = {
     "rope h and w swapped": ("pos[1] = (n / Ww) % Hh;\n        pos[2] = n % Ww;",
                              "pos[1] = n % Ww;\n        pos[2] = (n / Ww) % Hh;"),
     "rope frequency exponent": ("-2.0 * (double)j / (double)width[a]", "-1.0 * (double)j / (double)width[a]"),
+    "bwd: delta dropped": ("dS[i * Skv + j] = P[i * Skv + j] * (dS[i * Skv + j] - delta);",
+                           "dS[i * Skv + j] = P[i * Skv + j] * dS[i * Skv + j];"),
+    "bwd: dK without scale": ("dk[j * D + d] += scale * dS[i * Skv + j] * at(q, qo + i * D + d);",
+                              "dk[j * D + d] += dS[i * Skv + j] * at(q, qo + i * D + d);"),
+    "bwd: dV uses dS": ("dv[j * D + d] += P[i * Skv + j] * at(dout, doo + i * D + d);",
+                        "dv[j * D + d] += dS[i * Skv + j] * at(dout, doo + i * D + d);"),
     "rope pair partner index": ("double x1 = row[base[a] + 2 * j + 1];", "double x1 = row[base[a] + j + 1];"),
 }
 

@@ -325,3 +325,69 @@ def test_oracle_bf16_rounding():
         assert oracle.f64_to_bf16(np.array([val]))[0] == bits, val
     np.testing.assert_array_equal(oracle.bf16_to_f64(oracle.f64_to_bf16(x)),
                                   synth.bf16_bits_to_f64(ref))
+
+
+# ------------------------------------------------------------- backward ---
+
+def _loss(q, k, v, g, scale):
+    out, _ = oracle.attention(q, k, v, scale)
+    return float(np.sum(out * g))
+
+
+@pytest.mark.parametrize("Sq,Skv,D", [(3, 4, 3), (2, 5, 4)])
+def test_attention_bwd_finite_differences(Sq, Skv, D):
+    # L = sum(out * G): dL/dq etc. by central differences of the forward oracle
+    q = RNG.normal(size=(1, 1, Sq, D))
+    k = RNG.normal(size=(1, 1, Skv, D))
+    v = RNG.normal(size=(1, 1, Skv, D))
+    g = RNG.normal(size=(1, 1, Sq, D))
+    scale = 0.6
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, scale)
+    eps = 1e-6
+    for x, grad in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            x[idx] += eps
+            lp = _loss(q, k, v, g, scale)
+            x[idx] -= 2 * eps
+            lm = _loss(q, k, v, g, scale)
+            x[idx] += eps
+            num[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
+
+
+def test_attention_bwd_matches_torch_autograd_fp64():
+    torch = pytest.importorskip("torch")
+    q = RNG.normal(size=(2, 2, 17, 32))
+    k = RNG.normal(size=(2, 2, 23, 32))
+    v = RNG.normal(size=(2, 2, 23, 32))
+    g = RNG.normal(size=(2, 2, 17, 32))
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=0.2)
+    out.backward(torch.from_numpy(g))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, 0.2)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_bwd_invariants():
+    q = RNG.normal(size=(1, 2, 9, 8))
+    k = RNG.normal(size=(1, 2, 13, 8))
+    v = RNG.normal(size=(1, 2, 13, 8))
+    g = RNG.normal(size=(1, 2, 9, 8))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, 0.5)
+    # shifting every key by one vector leaves the logits' softmax unchanged
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+    # dO = 1 on one coordinate: dV_j on it = column sums of P
+    ones = np.zeros_like(g)
+    ones[..., 0] = 1.0
+    _, _, dv1 = oracle.attention_bwd(q, k, v, ones, 0.5)
+    s = 0.5 * np.einsum("bhid,bhjd->bhij", q, k)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    np.testing.assert_allclose(dv1[..., 0], p.sum(axis=2), rtol=1e-12, atol=1e-13)
+    # all keys equal: P is uniform and dQ vanishes
+    kc = np.broadcast_to(k[:, :, :1], k.shape).copy()
+    dq0, _, _ = oracle.attention_bwd(q, kc, v, g, 0.5)
+    np.testing.assert_allclose(dq0, 0.0, atol=1e-12)
