@@ -14,7 +14,7 @@ Functions (each follows the definition written at its C counterpart):
 * ``attention_bwd(q, k, v, dout, scale)`` -- dQ, dK, dV of exact attention.
 * ``lse_merge(o_a, lse_a, o_b, lse_b)`` -- two-block (O, LSE) combination.
 * ``rope3d(x, grid, theta)`` -- 3D RoPE, bf16 in/out (rounded to nearest even)
-  or fp64 in/out.
+  or fp64 in/out; ``rope3d_bwd`` -- its gradient (the transposed rotation).
 * ``f64_to_bf16`` / ``bf16_to_f64`` -- the oracle's own rounding and widening.
 
 Parity status: attention and the LSE merge are pinned by the tests against
@@ -92,6 +92,10 @@ def _load():
             lib.oracle_rope3d_f64.restype = ctypes.c_int
             lib.oracle_rope3d_bf16.argtypes = [_u16p, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
             lib.oracle_rope3d_bf16.restype = ctypes.c_int
+            lib.oracle_rope3d_bwd_f64.argtypes = [_dp, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
+            lib.oracle_rope3d_bwd_f64.restype = ctypes.c_int
+            lib.oracle_rope3d_bwd_bf16.argtypes = [_u16p, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
+            lib.oracle_rope3d_bwd_bf16.restype = ctypes.c_int
             lib.oracle_f64_to_bf16_array.argtypes = [_dp, _u16p, _i64]
             lib.oracle_f64_to_bf16_array.restype = None
             lib.oracle_bf16_to_f64_array.argtypes = [_u16p, _dp, _i64]
@@ -235,6 +239,18 @@ def rope3d(x, grid, theta: float = 10000.0):
     uint16 input (bf16 bits) -> uint16 output rounded to nearest even;
     float64 input -> float64 output (no rounding).
     """
+    return _rope3d(x, grid, theta, False)
+
+
+def rope3d_bwd(g, grid, theta: float = 10000.0):
+    """Gradient of rope3d: R^T g, every pair turned back by its angle.
+
+    Same dtypes and rounding as ``rope3d``.
+    """
+    return _rope3d(g, grid, theta, True)
+
+
+def _rope3d(x, grid, theta, transpose):
     lib = _load()
     T, Hh, Ww = (int(g) for g in grid)
     x = np.array(x, copy=True, order="C")
@@ -243,9 +259,11 @@ def rope3d(x, grid, theta: float = 10000.0):
         raise ValueError("sequence length does not match the latent grid")
     BH = x.size // (S * D) if S * D else 0
     if x.dtype == np.uint16:
-        rc = lib.oracle_rope3d_bf16(_ptr(x, _u16p), BH, T, Hh, Ww, D, float(theta))
+        fn = lib.oracle_rope3d_bwd_bf16 if transpose else lib.oracle_rope3d_bf16
+        rc = fn(_ptr(x, _u16p), BH, T, Hh, Ww, D, float(theta))
     elif x.dtype == np.float64:
-        rc = lib.oracle_rope3d_f64(_ptr(x, _dp), BH, T, Hh, Ww, D, float(theta))
+        fn = lib.oracle_rope3d_bwd_f64 if transpose else lib.oracle_rope3d_f64
+        rc = fn(_ptr(x, _dp), BH, T, Hh, Ww, D, float(theta))
     else:
         raise TypeError("x must be uint16 (bf16 bits) or float64")
     if rc != 0:

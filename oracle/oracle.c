@@ -327,8 +327,8 @@ void oracle_lse_merge_f64(const double *oa, const double *lsea,
  *        x'_{2j+1} = x_{2j} sin(angle) + x_{2j+1} cos(angle)
  *    (the product of the pair, read as a complex number, with e^{i angle}).
  */
-int oracle_rope3d_f64(double *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
-                      int64_t D, double theta)
+static int rope3d_apply(double *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
+                        int64_t D, double theta, int transpose)
 {
     if (D < 6 || (D % 2) != 0) return -1;
     int64_t dh = 2 * (D / 6);
@@ -350,26 +350,61 @@ int oracle_rope3d_f64(double *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
                 double c = cos(angle), s = sin(angle);
                 double x0 = row[base[a] + 2 * j];
                 double x1 = row[base[a] + 2 * j + 1];
-                row[base[a] + 2 * j] = x0 * c - x1 * s;
-                row[base[a] + 2 * j + 1] = x0 * s + x1 * c;
+                if (!transpose) {
+                    row[base[a] + 2 * j] = x0 * c - x1 * s;
+                    row[base[a] + 2 * j + 1] = x0 * s + x1 * c;
+                } else {
+                    /* R^T: the same rotation matrix, transposed */
+                    row[base[a] + 2 * j] = c * x0 + s * x1;
+                    row[base[a] + 2 * j + 1] = c * x1 - s * x0;
+                }
             }
         }
     }
     return 0;
 }
 
-/* In place on bf16: widen, rotate in fp64, round to nearest-even bf16. */
-int oracle_rope3d_bf16(uint16_t *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
-                       int64_t D, double theta)
+int oracle_rope3d_f64(double *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
+                      int64_t D, double theta)
+{
+    return rope3d_apply(x, BH, T, Hh, Ww, D, theta, 0);
+}
+
+/*
+ * Gradient of the 3D RoPE: x' = R x with R orthogonal and block-diagonal
+ * (one 2x2 rotation per pair), so dL/dx = R^T dL/dx' -- every pair turned
+ * back by its angle. In place on g [BH][S][D].
+ */
+int oracle_rope3d_bwd_f64(double *g, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
+                          int64_t D, double theta)
+{
+    return rope3d_apply(g, BH, T, Hh, Ww, D, theta, 1);
+}
+
+static int rope3d_bf16(uint16_t *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
+                       int64_t D, double theta, int transpose)
 {
     int64_t n = BH * T * Hh * Ww * D;
     double *xd = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
     if (!xd) return -2;
     oracle_bf16_to_f64_array(x, xd, n);
-    int rc = oracle_rope3d_f64(xd, BH, T, Hh, Ww, D, theta);
+    int rc = rope3d_apply(xd, BH, T, Hh, Ww, D, theta, transpose);
     if (rc == 0) oracle_f64_to_bf16_array(xd, x, n);
     free(xd);
     return rc;
+}
+
+/* In place on bf16: widen, rotate in fp64, round to nearest-even bf16. */
+int oracle_rope3d_bf16(uint16_t *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
+                       int64_t D, double theta)
+{
+    return rope3d_bf16(x, BH, T, Hh, Ww, D, theta, 0);
+}
+
+int oracle_rope3d_bwd_bf16(uint16_t *g, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
+                           int64_t D, double theta)
+{
+    return rope3d_bf16(g, BH, T, Hh, Ww, D, theta, 1);
 }
 
 int oracle_num_threads(void)

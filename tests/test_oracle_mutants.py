@@ -38,6 +38,8 @@ MUTANTS = {
                               "dk[j * D + d] += dS[i * Skv + j] * at(q, qo + i * D + d);"),
     "bwd: dV uses dS": ("dv[j * D + d] += P[i * Skv + j] * at(dout, doo + i * D + d);",
                         "dv[j * D + d] += dS[i * Skv + j] * at(dout, doo + i * D + d);"),
+    "rope bwd: forward rotation used": ("row[base[a] + 2 * j + 1] = c * x1 - s * x0;",
+                                        "row[base[a] + 2 * j + 1] = c * x1 + s * x0;"),
     "rope pair partner index": ("double x1 = row[base[a] + 2 * j + 1];", "double x1 = row[base[a] + j + 1];"),
 }
 

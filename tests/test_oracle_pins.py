@@ -391,3 +391,18 @@ def test_attention_bwd_invariants():
     kc = np.broadcast_to(k[:, :, :1], k.shape).copy()
     dq0, _, _ = oracle.attention_bwd(q, kc, v, g, 0.5)
     np.testing.assert_allclose(dq0, 0.0, atol=1e-12)
+
+
+def test_rope3d_bwd_is_the_adjoint():
+    # <R x, g> = <x, R^T g> for every x, g: fixes the transpose, not just the inverse
+    grid = (3, 4, 5)
+    x = RNG.normal(size=(2, 60, 128))
+    g = RNG.normal(size=(2, 60, 128))
+    lhs = np.sum(oracle.rope3d(x, grid, 10000.0) * g)
+    rhs = np.sum(x * oracle.rope3d_bwd(g, grid, 10000.0))
+    assert abs(lhs - rhs) <= 1e-12 * np.sum(np.abs(x * g)) * 10
+    # and R^T R = I
+    np.testing.assert_allclose(oracle.rope3d_bwd(oracle.rope3d(x, grid, 500.0), grid, 500.0), x,
+                               rtol=0, atol=1e-12)
+    # position 0 is the identity for the transpose as well
+    np.testing.assert_array_equal(oracle.rope3d_bwd(x[:, :1], (1, 1, 1), 10000.0), x[:, :1])
