@@ -13,6 +13,10 @@ Entry points (same names as the C ABI):
                           workspace, workspace_bytes)
     regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
     regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream=None)
+    regen_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Sq, Skv, D, scale, stream,
+                   workspace, workspace_bytes, accumulate_dq)
+    regen_attn_bwd_workspace_bytes(B, H, Sq, D)
+    regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream=None)
     regen_last_device_error() -> (status, site)
     regen_set_wait_limit_ns(ns)
 Convenience wrappers that allocate outputs with torch:
@@ -20,6 +24,8 @@ Convenience wrappers that allocate outputs with torch:
     attn_fwd_rope3d(q, k, v, grid, theta=10000.0) -> (out, lse)
     rope3d_(q, k, grid, theta=10000.0)
     lse_merge(o_a, lse_a, o_b, lse_b) -> (out, lse)
+    attn_bwd(q, k, v, out, lse, dout, scale=None) -> (dq, dk, dv)
+    rope3d_bwd_(dq, dk, grid, theta=10000.0)
 """
 from __future__ import annotations
 
@@ -32,7 +38,8 @@ __all__ = [
     "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
     "regen_status_str", "regen_last_device_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
     "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes", "regen_attn_fwd_rope3d_noalloc",
-    "attn_fwd", "attn_fwd_rope3d", "rope3d_", "lse_merge", "STATUS",
+    "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd",
+    "attn_fwd", "attn_fwd_rope3d", "rope3d_", "lse_merge", "attn_bwd", "rope3d_bwd_", "STATUS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +85,13 @@ def load():
         L.regen_rope3d.restype = i32
         L.regen_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, vp]
         L.regen_lse_merge.restype = i32
+        L.regen_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp,
+                                     vp, i64, i32]
+        L.regen_attn_bwd.restype = i32
+        L.regen_attn_bwd_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.regen_attn_bwd_workspace_bytes.restype = i64
+        L.regen_rope3d_bwd.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, vp]
+        L.regen_rope3d_bwd.restype = i32
         L.regen_status_str.argtypes = [i32]
         L.regen_status_str.restype = ctypes.c_char_p
         L.regen_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
@@ -169,6 +183,25 @@ def regen_rope3d(q, k, T, Hh, Ww, theta, B, H, D, stream=None) -> None:
 def regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream=None) -> None:
     _check(load().regen_lse_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out),
                                   _ptr(lse_out), int(rows), D, _stream(stream)), "regen_lse_merge")
+
+
+def regen_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Sq, Skv, D, scale, stream, workspace,
+                   workspace_bytes, accumulate_dq=0) -> None:
+    _check(load().regen_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), B, H, Sq, Skv, D, float(scale), _stream(stream), _ptr(workspace),
+                                 int(workspace_bytes), int(accumulate_dq)), "regen_attn_bwd")
+
+
+def regen_attn_bwd_workspace_bytes(B, H, Sq, D) -> int:
+    n = load().regen_attn_bwd_workspace_bytes(B, H, Sq, D)
+    if n < 0:
+        raise RegenError(int(n), "regen_attn_bwd_workspace_bytes")
+    return int(n)
+
+
+def regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream=None) -> None:
+    _check(load().regen_rope3d_bwd(_ptr(dq), _ptr(dk), T, Hh, Ww, float(theta), B, H, D, _stream(stream)),
+           "regen_rope3d_bwd")
 
 
 def regen_selftest_exp2(x, y, n, stream=None) -> None:
@@ -263,3 +296,38 @@ def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None, stream=None):
         lse_out = torch.empty_like(lse_a)
     regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream)
     return out, lse_out
+
+
+def attn_bwd(q, k, v, out, lse, dout, scale=None, dq=None, dk=None, dv=None, accumulate_dq=False,
+             workspace=None, stream=None):
+    """Gradients of attn_fwd -> (dq, dk, dv), bf16 like the inputs.
+
+    out and lse are the forward's (or, for one key block of a merged
+    attention, the merged ones). accumulate_dq adds into the given dq."""
+    import torch
+    B, H, Sq, D = _bhsd(q, "q")
+    Skv = _bhsd(k, "k")[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if accumulate_dq and dq is None:
+        raise ValueError("accumulate_dq needs the dq to add into")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = regen_attn_bwd_workspace_bytes(B, H, Sq, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    regen_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Sq, Skv, D, scale, stream, workspace,
+                   workspace.numel() * workspace.element_size(), 1 if accumulate_dq else 0)
+    return dq, dk, dv
+
+
+def rope3d_bwd_(dq, dk, grid, theta=10000.0, stream=None):
+    """Gradient of rope3d_, in place on the gradients (either may be None)."""
+    ref = dq if dq is not None else dk
+    B, H, S, D = _bhsd(ref, "dq/dk")
+    T, Hh, Ww = grid
+    if S != T * Hh * Ww:
+        raise ValueError("sequence length does not match the latent grid")
+    regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream)
+    return dq, dk

@@ -17,6 +17,7 @@
 
 #include "regen_attn.h"
 
+#include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "lse_merge.cuh"
 #include "rope3d.cuh"
@@ -99,6 +100,12 @@ int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, r
     return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
 }
 
+// Gradient launches: prep (delta, lse2) -> dK/dV -> dQ, all on `stream`.
+template <int HD>
+int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, const regen_bf16 *out,
+               const float *lse, const regen_bf16 *dout, regen_bf16 *dq, regen_bf16 *dk, regen_bf16 *dv,
+               int64_t BH, int Sq, int Skv, float scale, float *ws, bool accumulate, cudaStream_t stream);
+
 int grid_for(int64_t work, int threads)
 {
     int64_t blocks = (work + threads - 1) / threads;
@@ -106,6 +113,61 @@ int grid_for(int64_t work, int threads)
     if (blocks > cap) blocks = cap;
     return static_cast<int>(blocks < 1 ? 1 : blocks);
 }
+
+template <int HD>
+int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, const regen_bf16 *out,
+               const float *lse, const regen_bf16 *dout, regen_bf16 *dq, regen_bf16 *dk, regen_bf16 *dv,
+               int64_t BH, int Sq, int Skv, float scale, float *ws, bool accumulate, cudaStream_t stream)
+{
+    using C = regen::BwdCfg<HD>;
+    static std::once_flag once;
+    static int attr_status = REGEN_OK;
+    std::call_once(once, [] {
+        auto setup = [](const void *fn, int smem) {
+            cudaFuncAttributes fa;
+            if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+                cudaFuncGetAttributes(&fa, fn) != cudaSuccess)
+                return static_cast<int>(REGEN_ERR_CUDA);
+            // the in-kernel register re-allocation would not fit: refuse to launch
+            return fa.numRegs < C::MIN_LAUNCH_REGS ? static_cast<int>(REGEN_ERR_UNSUPPORTED)
+                                                   : static_cast<int>(REGEN_OK);
+        };
+        int st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dkdv_kernel<HD>), C::A_SMEM_BYTES);
+        if (st == REGEN_OK)
+            st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, false>), C::B_SMEM_BYTES);
+        if (st == REGEN_OK)
+            st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, true>), C::B_SMEM_BYTES);
+        attr_status = st;
+    });
+    if (attr_status != REGEN_OK) return attr_status;
+    CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
+    if (!make_bhsd_map(&tq, q, BH, Sq, HD) || !make_bhsd_map(&tk, k, BH, Skv, HD) ||
+        !make_bhsd_map(&tv, v, BH, Skv, HD) || !make_bhsd_map(&tdo, dout, BH, Sq, HD) ||
+        !make_bhsd_map(&tdq, dq, BH, Sq, HD) || !make_bhsd_map(&tdk, dk, BH, Skv, HD) ||
+        !make_bhsd_map(&tdv, dv, BH, Skv, HD))
+        return REGEN_ERR_CUDA;
+    const int nq = (Sq + C::BM - 1) / C::BM;
+    const int nkv = (Skv + C::BN - 1) / C::BN;
+    if (BH * nq > 0x7FFFFFFF || BH * nkv > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const int64_t prep_work = BH * nq * 128 * (HD / 8);
+    regen::attn_bwd_prep_kernel<<<grid_for(prep_work, 256), 256, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(out), reinterpret_cast<const uint4 *>(dout), lse, ws, BH, Sq, HD, nq);
+    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    const uint64_t limit = g_wait_limit_ns.load();
+    regen::attn_bwd_dkdv_kernel<HD><<<static_cast<unsigned>(BH * nkv), C::THREADS, C::A_SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, tdk, tdv, ws, Sq, Skv, scale, scale_log2, limit);
+    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    if (accumulate)
+        regen::attn_bwd_dq_kernel<HD, true><<<static_cast<unsigned>(BH * nq), C::THREADS, C::B_SMEM_BYTES, stream>>>(
+            tq, tk, tv, tdo, tdq, dq, ws, Sq, Skv, scale, scale_log2, limit);
+    else
+        regen::attn_bwd_dq_kernel<HD, false><<<static_cast<unsigned>(BH * nq), C::THREADS, C::B_SMEM_BYTES, stream>>>(
+            tq, tk, tv, tdo, tdq, dq, ws, Sq, Skv, scale, scale_log2, limit);
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
+int64_t bwd_workspace_bytes(int64_t BH, int64_t Sq) { return BH * ((Sq + 127) / 128) * 1024; }
 
 // Scratch of the RoPE-fused attention: the fp64 (cos, sin) table, then the
 // rotated K ([B*H, S, D] bf16), each starting on a 256-byte boundary.
@@ -166,6 +228,30 @@ uint8_t *noalloc_scratch_on_current_device()
     }
     return g_noalloc_ptr[dev];
 }
+
+int rope3d_common(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta, int B, int H, int D,
+                  regen_stream_t stream, bool inverse)
+{
+    if (T <= 0 || Hh <= 0 || Ww <= 0 || B < 0 || H < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(theta) || !(theta > 0.0f)) return REGEN_ERR_INVALID_ARG;
+    if (D < 8 || D > 512 || (D % 8) != 0) return REGEN_ERR_UNSUPPORTED;
+    const int64_t S = static_cast<int64_t>(T) * Hh * Ww;
+    if (S > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0) return REGEN_OK;
+    if (!q && !k) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k)) return REGEN_ERR_MISALIGNED;
+    const int64_t bytes = BH * S * D * 2;
+    if (overlaps(q, bytes, k, bytes)) return REGEN_ERR_INVALID_ARG;
+    const int64_t work = S * (D / 8);
+    const int threads = 128;
+    const int64_t blocks = (work + threads - 1) / threads;
+    if (blocks > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    regen::rope3d_kernel<<<static_cast<unsigned>(blocks), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        q, k, BH, static_cast<int>(S), Hh, Ww, D, static_cast<double>(theta), inverse);
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
 
 }  // namespace
 
@@ -283,27 +369,79 @@ REGEN_API int regen_attn_fwd_rope3d_noalloc(const regen_bf16 *q, const regen_bf1
                                     reinterpret_cast<cudaStream_t>(stream));
 }
 
+
 REGEN_API int regen_rope3d(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta, int B,
                            int H, int D, regen_stream_t stream)
 {
-    if (T <= 0 || Hh <= 0 || Ww <= 0 || B < 0 || H < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
-    if (!std::isfinite(theta) || !(theta > 0.0f)) return REGEN_ERR_INVALID_ARG;
-    if (D < 8 || D > 512 || (D % 8) != 0) return REGEN_ERR_UNSUPPORTED;
-    const int64_t S = static_cast<int64_t>(T) * Hh * Ww;
-    if (S > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    return rope3d_common(q, k, T, Hh, Ww, theta, B, H, D, stream, false);
+}
+
+REGEN_API int regen_rope3d_bwd(regen_bf16 *dq, regen_bf16 *dk, int T, int Hh, int Ww, float theta, int B,
+                               int H, int D, regen_stream_t stream)
+{
+    return rope3d_common(dq, dk, T, Hh, Ww, theta, B, H, D, stream, true);
+}
+
+REGEN_API int64_t regen_attn_bwd_workspace_bytes(int B, int H, int Sq, int D)
+{
+    if (B < 0 || H < 0 || Sq < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
+    return bwd_workspace_bytes(static_cast<int64_t>(B) * H, Sq);
+}
+
+REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
+                             const regen_bf16 *out, const float *lse, const regen_bf16 *dout, regen_bf16 *dq,
+                             regen_bf16 *dk, regen_bf16 *dv, int B, int H, int Sq, int Skv, int D, float scale,
+                             regen_stream_t stream, void *workspace, int64_t workspace_bytes, int accumulate_dq)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Skv < 0 || D < 0 || workspace_bytes < 0) return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return REGEN_ERR_INVALID_ARG;
+    if (accumulate_dq != 0 && accumulate_dq != 1) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
     const int64_t BH = static_cast<int64_t>(B) * H;
-    if (BH == 0) return REGEN_OK;
-    if (!q && !k) return REGEN_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k)) return REGEN_ERR_MISALIGNED;
-    const int64_t bytes = BH * S * D * 2;
-    if (overlaps(q, bytes, k, bytes)) return REGEN_ERR_INVALID_ARG;
-    const int64_t work = S * (D / 8);
-    const int threads = 128;
-    const int64_t blocks = (work + threads - 1) / threads;
-    if (blocks > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
-    regen::rope3d_kernel<<<static_cast<unsigned>(blocks), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        q, k, BH, static_cast<int>(S), Hh, Ww, D, static_cast<double>(theta));
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    if (BH == 0 || (Sq == 0 && Skv == 0)) return REGEN_OK;
+    if (BH > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const int64_t qbytes = BH * Sq * D * 2, kvbytes = BH * Skv * D * 2, lbytes = BH * Sq * 4;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (Sq == 0) {  // no query: dk = dv = 0
+        if (!dk || !dv) return REGEN_ERR_INVALID_ARG;
+        if (!aligned16(dk) || !aligned16(dv)) return REGEN_ERR_MISALIGNED;
+        if (overlaps(dk, kvbytes, dv, kvbytes)) return REGEN_ERR_INVALID_ARG;
+        for (regen_bf16 *z : {dk, dv}) {
+            regen::attn_empty_kernel<<<grid_for(kvbytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(z),
+                                                                                 kvbytes / 16, nullptr, 0);
+            if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+        }
+        return REGEN_OK;
+    }
+    if (Skv == 0) {  // no key: dq = 0 (unchanged when accumulating)
+        if (!dq) return REGEN_ERR_INVALID_ARG;
+        if (!aligned16(dq)) return REGEN_ERR_MISALIGNED;
+        if (accumulate_dq) return REGEN_OK;
+        regen::attn_empty_kernel<<<grid_for(qbytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(dq),
+                                                                            qbytes / 16, nullptr, 0);
+        return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    }
+    if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return REGEN_ERR_MISALIGNED;
+    const int64_t need = bwd_workspace_bytes(BH, Sq);
+    if (workspace_bytes < need) return REGEN_ERR_INVALID_ARG;
+    struct Span { const void *p; int64_t n; };
+    const Span ins[6] = {{q, qbytes}, {k, kvbytes}, {v, kvbytes}, {out, qbytes}, {lse, lbytes}, {dout, qbytes}};
+    const Span outs[4] = {{dq, qbytes}, {dk, kvbytes}, {dv, kvbytes}, {workspace, need}};
+    for (int a = 0; a < 4; ++a) {
+        for (const Span &in : ins)
+            if (overlaps(outs[a].p, outs[a].n, in.p, in.n)) return REGEN_ERR_INVALID_ARG;
+        for (int b = a + 1; b < 4; ++b)
+            if (overlaps(outs[a].p, outs[a].n, outs[b].p, outs[b].n)) return REGEN_ERR_INVALID_ARG;
+    }
+    float *ws = static_cast<float *>(workspace);
+    if (D == 128)
+        return launch_bwd<128>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, accumulate_dq != 0, st);
+    return launch_bwd<64>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, accumulate_dq != 0, st);
 }
 
 REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a, const regen_bf16 *o_b,

@@ -141,8 +141,10 @@ __global__ void rope_apply_kernel(const uint4 *__restrict__ src, uint4 *__restri
 }
 
 // grid: ceil(S * D/8 / blockDim) blocks; x (q then k) has `rows` rows of S x D.
+// inverse: turn every pair back by its angle (sine negated), the transposed
+// rotation that carries gradients through the RoPE.
 __global__ void rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k, int64_t rows,
-                              int S, int Hh, int Ww, int D, double theta)
+                              int S, int Hh, int Ww, int D, double theta, bool inverse)
 {
     const int chunks = D >> 3;
     const int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
@@ -165,6 +167,7 @@ __global__ void rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k
             axis = 2; local = d - dt - dh; width = dh;
         }
         rope_angle(pos[axis], local, width, theta, cs[p], sn[p]);
+        if (inverse) sn[p] = -sn[p];
     }
     const int64_t row_stride = static_cast<int64_t>(S) * D;
     const int64_t off = static_cast<int64_t>(n) * D + c * 8;

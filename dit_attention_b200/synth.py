@@ -21,7 +21,7 @@ Random stream (defined here, independent of torch's and numpy's RNGs):
 * Normal pairs by Box-Muller: for pair p with u1 = U(2p), u2 = U(2p+1),
   z(2p) = sqrt(-2 ln u1) cos(2 pi u2), z(2p+1) = sqrt(-2 ln u1) sin(2 pi u2).
 
-Streams: q = 0, k = 1, v = 2, spike-row choice = 3.
+Streams: q = 0, k = 1, v = 2, spike-row choice = 3, upstream gradient dO = 4.
 
 The workloads are the latent-token shapes of the ReGenVC decoder's DiT
 (Wan2.1-class, head dim 128, latent grid 30 x 52 per latent frame): a 25-frame
@@ -42,7 +42,7 @@ GAMMA = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
-STREAM_Q, STREAM_K, STREAM_V, STREAM_SPIKE = 0, 1, 2, 3
+STREAM_Q, STREAM_K, STREAM_V, STREAM_SPIKE, STREAM_DOUT = 0, 1, 2, 3, 4
 
 _CHUNK = 1 << 16  # normal pairs per chunk (cache-sized temporaries)
 
@@ -280,3 +280,9 @@ def make_inputs(w: Workload, seed_offset: int = 0):
             rows = spike_rows(seed, bh, w.Skv, w.spike_count)
             kk[bh, rows] = f64_to_bf16_bits(bf16_bits_to_f64(kk[bh, rows]) * w.spike_mult)
     return q, k, v
+
+
+def make_dout(w: Workload, seed_offset: int = 0):
+    """Upstream gradient dO [B,H,Sq,D] for the backward pass: N(0,1) rounded
+    to bf16 (a synthetic stand-in for the loss gradient; no dataset here)."""
+    return _normal_bf16(w.seed + seed_offset, STREAM_DOUT, (w.B, w.H, w.Sq, w.D), False)

@@ -180,6 +180,53 @@ REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a,
                               int64_t rows, int D, regen_stream_t stream);
 
 /*
+ * regen_attn_bwd -- gradients of regen_attn_fwd (the decoder's student DiT is
+ * trained by distillation: arXiv 2607.28144, blog page "Technical
+ * innovations"). With s_ij = scale <q_i, k_j>, the forward's out and lse,
+ * and an upstream gradient dout:
+ *     P_ij = exp(s_ij - lse_i),  dP_ij = <dout_i, v_j>,  delta_i = <dout_i, out_i>
+ *     dS_ij = P_ij (dP_ij - delta_i)
+ *     dv_j = sum_i P_ij dout_i,  dk_j = scale sum_i dS_ij q_i,  dq_i = scale sum_j dS_ij k_j
+ * Products of bf16 tiles on the tensor cores with fp32 accumulation; P and dS
+ * are rounded to bf16 before their products; results rounded once to bf16.
+ * No atomics: the same inputs give the same bits on every run.
+ *
+ * Key blocks: when the keys were split into blocks whose partial results were
+ * combined by regen_lse_merge, passing the MERGED out and lse with one
+ * block's k, v gives that block's exact dk, dv and its share of dq; call once
+ * per block with accumulate_dq = 1 after the first to sum the dq shares.
+ *
+ *   q, out, dout, dq  [B, H, Sq, D] bf16;  k, v, dk, dv  [B, H, Skv, D] bf16
+ *   lse       [B, H, Sq] fp32 (the forward's, natural log)
+ *   D         64 or 128 (else REGEN_ERR_UNSUPPORTED); scale finite
+ *   workspace device scratch of at least regen_attn_bwd_workspace_bytes(B, H, Sq, D)
+ *             bytes, 256-byte aligned, owned by the caller; overwritten.
+ *   accumulate_dq  0: dq = result;  1: dq = bf16(dq + result) (dq read first)
+ * dq, dk, dv must not overlap each other, an input or the workspace.
+ * Sq == 0: dk = dv = 0. Skv == 0: dq = 0 (unchanged when accumulating).
+ * B or H == 0: REGEN_OK, nothing done.
+ */
+REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
+                             const regen_bf16 *out, const float *lse, const regen_bf16 *dout,
+                             regen_bf16 *dq, regen_bf16 *dk, regen_bf16 *dv,
+                             int B, int H, int Sq, int Skv, int D, float scale,
+                             regen_stream_t stream, void *workspace, int64_t workspace_bytes,
+                             int accumulate_dq);
+
+/* Bytes of workspace regen_attn_bwd needs (B*H*ceil(Sq/128)*1024), or a
+ * negative status for invalid sizes. */
+REGEN_API int64_t regen_attn_bwd_workspace_bytes(int B, int H, int Sq, int D);
+
+/*
+ * regen_rope3d_bwd -- gradient of regen_rope3d, in place: every pair of the
+ * gradients dq, dk is turned back by its angle (the transposed rotation),
+ *     g'_{2j} = g_{2j} cos + g_{2j+1} sin,   g'_{2j+1} = g_{2j+1} cos - g_{2j} sin
+ * with the same angles, fp64 arithmetic, rounding and arguments as regen_rope3d.
+ */
+REGEN_API int regen_rope3d_bwd(regen_bf16 *dq, regen_bf16 *dk, int T, int Hh, int Ww, float theta,
+                               int B, int H, int D, regen_stream_t stream);
+
+/*
  * regen_selftest_exp2 -- diagnostic: evaluates, for each x[i], the FMA-pipe
  * 2^x that the attention kernel uses for part of its softmax probabilities
  * (degree-4 polynomial after Cody-Waite range reduction; inputs below -127

@@ -11,7 +11,8 @@ Functions (each follows the definition written at its C counterpart):
 
 * ``attention(q, k, v, scale, rows=None)`` -- exact softmax attention and
   natural-log LSE, inputs bf16 bit arrays [B, H, S, D] (or doubles).
-* ``attention_bwd(q, k, v, dout, scale)`` -- dQ, dK, dV of exact attention.
+* ``attention_bwd(q, k, v, dout, scale)`` -- dQ, dK, dV of exact attention;
+  ``attention_bwd_rows`` -- the same for chosen query / key rows only.
 * ``lse_merge(o_a, lse_a, o_b, lse_b)`` -- two-block (O, LSE) combination.
 * ``rope3d(x, grid, theta)`` -- 3D RoPE, bf16 in/out (rounded to nearest even)
   or fp64 in/out; ``rope3d_bwd`` -- its gradient (the transposed rotation).
@@ -86,6 +87,10 @@ def _load():
             lib.oracle_attention_bwd_bf16.argtypes = [_u16p, _u16p, _u16p, _u16p, _i64, _i64, _i64, _i64,
                                                       ctypes.c_double, _dp, _dp, _dp]
             lib.oracle_attention_bwd_bf16.restype = ctypes.c_int
+            lib.oracle_attention_bwd_rows_bf16.argtypes = [_u16p, _u16p, _u16p, _u16p, _i64, _i64, _i64, _i64,
+                                                           ctypes.c_double, _i64p, _i64, _i64p, _i64, _dp, _dp,
+                                                           _dp]
+            lib.oracle_attention_bwd_rows_bf16.restype = ctypes.c_int
             lib.oracle_lse_merge_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _dp, _dp]
             lib.oracle_lse_merge_f64.restype = None
             lib.oracle_rope3d_f64.argtypes = [_dp, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
@@ -208,6 +213,39 @@ def attention_bwd(q, k, v, dout, scale: float):
         raise TypeError("inputs must all be uint16 (bf16 bits) or all float64")
     if rc != 0:
         raise MemoryError("oracle could not allocate its per-head P and dS")
+    return dq, dk, dv
+
+
+def attention_bwd_rows(q, k, v, dout, scale: float, qrows, krows):
+    """The gradients for chosen rows of every head: dq[..., len(qrows), D] for
+    those query rows, dk, dv[..., len(krows), D] for those key rows (fp64).
+
+    Inputs as ``attention_bwd`` but bf16 bits only; for sizes where the full
+    gradient would take too long (every query row's statistics are still
+    computed, once per head).
+    """
+    lib = _load()
+    q, k, v, dout = (np.ascontiguousarray(a) for a in (q, k, v, dout))
+    if {a.dtype for a in (q, k, v, dout)} != {np.dtype(np.uint16)}:
+        raise TypeError("inputs must be uint16 (bf16 bits)")
+    Sq, D = q.shape[-2], q.shape[-1]
+    Skv = k.shape[-2]
+    lead = q.shape[:-2]
+    if k.shape[:-2] != lead or v.shape != k.shape or dout.shape != q.shape or k.shape[-1] != D:
+        raise ValueError("q, k, v, dout shapes do not agree")
+    BH = int(np.prod(lead)) if lead else 1
+    qr = np.ascontiguousarray(qrows, dtype=np.int64)
+    kr = np.ascontiguousarray(krows, dtype=np.int64)
+    if qr.size and (qr.min() < 0 or qr.max() >= Sq) or kr.size and (kr.min() < 0 or kr.max() >= Skv):
+        raise IndexError("row index out of range")
+    dq = np.empty(lead + (qr.size, D), dtype=np.float64)
+    dk = np.empty(lead + (kr.size, D), dtype=np.float64)
+    dv = np.empty(lead + (kr.size, D), dtype=np.float64)
+    rc = lib.oracle_attention_bwd_rows_bf16(*(_ptr(a, _u16p) for a in (q, k, v, dout)), BH, Sq, Skv, D,
+                                            float(scale), _ptr(qr, _i64p), qr.size, _ptr(kr, _i64p), kr.size,
+                                            _ptr(dq, _dp), _ptr(dk, _dp), _ptr(dv, _dp))
+    if rc != 0:
+        raise MemoryError("oracle could not allocate its row statistics")
     return dq, dk, dv
 
 

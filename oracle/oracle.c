@@ -280,6 +280,99 @@ int oracle_attention_bwd_bf16(const uint16_t *q, const uint16_t *k, const uint16
     return attention_bwd(sq, sk, sv, sd, BH, Sq, Skv, D, scale, dq, dk, dv);
 }
 
+/*
+ * The same gradients for chosen rows only, at sizes where the full Sq x Skv
+ * matrices do not fit: dq for the query rows qrows[0..nqr), dk and dv for the
+ * key rows krows[0..nkr), of every (b, h). dk_j and dv_j sum over every query
+ * row, so each query row's max m_i, sum l_i and delta_i are computed first
+ * (one pass over its logits), then P_ij = exp(s_ij - m_i) / l_i is recomputed
+ * where it is needed. Outputs dq [BH][nqr][D], dk, dv [BH][nkr][D].
+ */
+static double dot_f64(const double *a, const double *b, int64_t D)
+{
+    double acc = 0.0;
+    for (int64_t d = 0; d < D; ++d) acc += a[d] * b[d];
+    return acc;
+}
+
+int oracle_attention_bwd_rows_bf16(const uint16_t *q16, const uint16_t *k16, const uint16_t *v16,
+                                   const uint16_t *do16, int64_t BH, int64_t Sq, int64_t Skv, int64_t D,
+                                   double scale, const int64_t *qrows, int64_t nqr, const int64_t *krows,
+                                   int64_t nkr, double *dq, double *dk, double *dv)
+{
+    /* one head at a time, widened to fp64 (exact) */
+    size_t nq = (size_t)(Sq * D > 0 ? Sq * D : 1), nk = (size_t)(Skv * D > 0 ? Skv * D : 1);
+    size_t ns = (size_t)(Sq > 0 ? Sq : 1);
+    double *q = (double *)malloc(sizeof(double) * nq), *g = (double *)malloc(sizeof(double) * nq);
+    double *k = (double *)malloc(sizeof(double) * nk), *v = (double *)malloc(sizeof(double) * nk);
+    double *m = (double *)malloc(sizeof(double) * ns), *l = (double *)malloc(sizeof(double) * ns);
+    double *delta = (double *)malloc(sizeof(double) * ns);
+    int rc = (q && g && k && v && m && l && delta) ? 0 : -1;
+    for (int64_t bh = 0; rc == 0 && bh < BH; ++bh) {
+        oracle_bf16_to_f64_array(q16 + bh * Sq * D, q, Sq * D);
+        oracle_bf16_to_f64_array(do16 + bh * Sq * D, g, Sq * D);
+        oracle_bf16_to_f64_array(k16 + bh * Skv * D, k, Skv * D);
+        oracle_bf16_to_f64_array(v16 + bh * Skv * D, v, Skv * D);
+        /* per query row: m_i, l_i, then delta_i = sum_j P_ij dP_ij */
+#pragma omp parallel
+        {
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t i = 0; i < Sq; ++i) {
+                if (!srow) continue;
+                double mi = -INFINITY;
+                for (int64_t j = 0; j < Skv; ++j) {
+                    srow[j] = scale * dot_f64(q + i * D, k + j * D, D);
+                    if (srow[j] > mi) mi = srow[j];
+                }
+                double li = 0.0, di = 0.0;
+                for (int64_t j = 0; j < Skv; ++j) {
+                    double e = exp(srow[j] - mi);
+                    li += e;
+                    di += e * dot_f64(g + i * D, v + j * D, D);
+                }
+                m[i] = mi;
+                l[i] = li;
+                delta[i] = di / li;
+            }
+            if (!srow) {
+#pragma omp atomic write
+                rc = -1;
+            }
+            free(srow);
+        }
+        /* dq_i = scale sum_j dS_ij k_j */
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nqr; ++r) {
+            int64_t i = qrows[r];
+            double *o = dq + (bh * nqr + r) * D;
+            for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+            for (int64_t j = 0; j < Skv; ++j) {
+                double p = exp(scale * dot_f64(q + i * D, k + j * D, D) - m[i]) / l[i];
+                double ds = p * (dot_f64(g + i * D, v + j * D, D) - delta[i]);
+                for (int64_t d = 0; d < D; ++d) o[d] += scale * ds * k[j * D + d];
+            }
+        }
+        /* dv_j = sum_i P_ij dO_i,  dk_j = scale sum_i dS_ij q_i */
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nkr; ++r) {
+            int64_t j = krows[r];
+            double *ov = dv + (bh * nkr + r) * D, *ok = dk + (bh * nkr + r) * D;
+            for (int64_t d = 0; d < D; ++d) { ov[d] = 0.0; ok[d] = 0.0; }
+            for (int64_t i = 0; i < Sq; ++i) {
+                double p = exp(scale * dot_f64(q + i * D, k + j * D, D) - m[i]) / l[i];
+                double ds = p * (dot_f64(g + i * D, v + j * D, D) - delta[i]);
+                for (int64_t d = 0; d < D; ++d) {
+                    ov[d] += p * g[i * D + d];
+                    ok[d] += scale * ds * q[i * D + d];
+                }
+            }
+        }
+    }
+    free(q); free(g); free(k); free(v); free(m); free(l); free(delta);
+    return rc;
+}
+
 /* ------------------------------------------------------------ LSE merge --- */
 
 /*

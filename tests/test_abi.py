@@ -115,3 +115,49 @@ def test_rope3d_fused_validation(lib, args, status):
                                    a["D"], a["scale"], None, a["T"], a["Hh"], a["Ww"], a["theta"], a["workspace"],
                                    a["workspace_bytes"])
     assert rc == status
+
+
+def test_attn_bwd_workspace_bytes(lib):
+    # [B*H][ceil(Sq/128)][2][128] floats
+    assert rg.regen_attn_bwd_workspace_bytes(1, 40, 31200, 128) == 40 * 244 * 1024
+    assert rg.regen_attn_bwd_workspace_bytes(2, 3, 1, 64) == 6 * 1024
+    assert rg.regen_attn_bwd_workspace_bytes(1, 1, 0, 128) == 0
+    assert lib.regen_attn_bwd_workspace_bytes(1, 1, 128, 96) == -2
+    assert lib.regen_attn_bwd_workspace_bytes(-1, 1, 128, 128) == -1
+
+
+# inputs q, out, dout (Sq rows), k, v (Skv rows), lse; outputs dq, dk, dv; workspace
+_BWD = dict(q=FAKE, k=FAKE + 10 * MB, v=FAKE + 20 * MB, out=FAKE + 30 * MB, lse=FAKE + 40 * MB,
+            dout=FAKE + 50 * MB, dq=FAKE + 60 * MB, dk=FAKE + 70 * MB, dv=FAKE + 80 * MB, ws=FAKE + 90 * MB,
+            B=1, H=2, Sq=100, Skv=100, D=128, scale=0.125, wsb=2048, acc=0)
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=96), -2), (dict(B=-1), -1), (dict(Skv=-1), -1), (dict(scale=float("nan")), -1), (dict(acc=2), -1),
+    (dict(wsb=-1), -1), (dict(wsb=2047), -1), (dict(ws=None), -1), (dict(lse=None), -1), (dict(dout=None), -1),
+    (dict(dk=None), -1), (dict(ws=FAKE + 90 * MB + 16), -3), (dict(dq=FAKE + 60 * MB + 2), -3),
+    (dict(dq=FAKE + 4096), -1),            # dq overlaps q
+    (dict(dk=FAKE + 60 * MB + 4096), -1),  # dk overlaps dq
+    (dict(ws=FAKE + 50 * MB), -1),         # workspace overlaps dout
+    (dict(dv=FAKE + 40 * MB), -1),         # dv overlaps lse
+    (dict(B=0), 0), (dict(H=0, q=None), 0), (dict(Sq=0, Skv=0), 0),
+    (dict(Sq=0, dk=None), -1), (dict(Skv=0, dq=FAKE + 60 * MB + 8), -3),
+    (dict(Skv=0, acc=1, dq=FAKE + 60 * MB), 0),   # accumulating nothing: dq unchanged, no launch
+])
+def test_attn_bwd_validation(lib, args, status):
+    a = dict(_BWD)
+    a.update(args)
+    rc = lib.regen_attn_bwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["dout"], a["dq"], a["dk"], a["dv"],
+                            a["B"], a["H"], a["Sq"], a["Skv"], a["D"], a["scale"], None, a["ws"], a["wsb"], a["acc"])
+    assert rc == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(T=0), -1), (dict(theta=0.0), -1), (dict(D=12), -2), (dict(q=FAKE + 2), -3), (dict(q=None, k=None), -1),
+    (dict(B=0), 0),
+])
+def test_rope3d_bwd_validation(lib, args, status):
+    a = dict(q=FAKE, k=FAKE + 10 * MB, T=2, Hh=3, Ww=4, theta=1e4, B=1, H=2, D=128)
+    a.update(args)
+    rc = lib.regen_rope3d_bwd(a["q"], a["k"], a["T"], a["Hh"], a["Ww"], a["theta"], a["B"], a["H"], a["D"], None)
+    assert rc == status

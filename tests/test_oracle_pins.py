@@ -406,3 +406,16 @@ def test_rope3d_bwd_is_the_adjoint():
                                rtol=0, atol=1e-12)
     # position 0 is the identity for the transpose as well
     np.testing.assert_array_equal(oracle.rope3d_bwd(x[:, :1], (1, 1, 1), 10000.0), x[:, :1])
+
+
+def test_attention_bwd_rows_equals_full():
+    # the row-sampled gradients agree with the full ones (ragged sizes, both dims)
+    rng = np.random.default_rng(5)
+    q, k, v, g = (oracle.f64_to_bf16(rng.normal(size=s)) for s in
+                  ((2, 1, 37, 16), (2, 1, 53, 16), (2, 1, 53, 16), (2, 1, 37, 16)))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, 0.3)
+    qr, kr = [0, 5, 36], [52, 0, 17, 3]
+    sq, sk, sv = oracle.attention_bwd_rows(q, k, v, g, 0.3, qr, kr)
+    np.testing.assert_allclose(sq, dq[:, :, qr], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(sk, dk[:, :, kr], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(sv, dv[:, :, kr], rtol=1e-12, atol=1e-14)

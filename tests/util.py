@@ -52,3 +52,32 @@ def check_attention(out_bits, lse_gpu, ref_out, ref_lse, label=""):
     assert np.all(np.isfinite(lse_err)) and lse_err.max() <= LSE_ATOL, f"{label}: lse {diag}"
     assert diag["max_err_over_rms"] < 0.05, f"{label}: error budget {diag}"
     return diag
+
+
+# Gradient contract. dV sums P rounded to bf16; dK and dQ sum dS rounded to
+# bf16, whose delta term uses the forward's bf16 output; each result is
+# rounded once more. That is a handful of independent roundings of unit
+# roundoff u = 2^-9 per summand, so the error of one element behaves like a
+# few u times the RMS of the gradient, and its maximum over ~1e6 elements stays
+# below ~20u = 0.04 of the RMS; a relative term of 10u = 0.02 covers the large
+# elements. The mean error is the sharper signal: a few u, bounded by 0.01.
+GRAD_ATOL_RMS, GRAD_RTOL, GRAD_MEAN_RMS = 4e-2, 2e-2, 1e-2
+
+
+def check_grad(got, ref, label=""):
+    """Assert |got - ref| <= 0.04 rms(ref) + 0.02 |ref| elementwise and
+    mean |got - ref| <= 0.01 rms(ref); got is bf16 bits or float64."""
+    g = bits_to_f64(got) if np.asarray(got).dtype == np.uint16 else np.asarray(got, dtype=np.float64)
+    g = g.reshape(ref.shape)
+    err = np.abs(g - ref)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    diag = {"max_err_over_rms": float(err.max() / rms) if rms else float(err.max()),
+            "mean_err_over_rms": float(err.mean() / rms) if rms else float(err.mean()), "rms_ref": rms}
+    assert np.all(np.isfinite(g)), f"{label}: non-finite gradient"
+    if rms == 0.0:
+        assert err.max() == 0.0, f"{label}: expected exact zeros; {diag}"
+        return diag
+    bad = err > GRAD_ATOL_RMS * rms + GRAD_RTOL * np.abs(ref)
+    assert not bad.any(), f"{label}: {int(bad.sum())} of {bad.size} gradients out of tolerance; {diag}"
+    assert diag["mean_err_over_rms"] <= GRAD_MEAN_RMS, f"{label}: mean error {diag}"
+    return diag
