@@ -64,20 +64,69 @@ def check_attention(out_bits, lse_gpu, ref_out, ref_lse, label=""):
 GRAD_ATOL_RMS, GRAD_RTOL, GRAD_MEAN_RMS = 4e-2, 2e-2, 1e-2
 
 
-def check_grad(got, ref, label=""):
-    """Assert |got - ref| <= 0.04 rms(ref) + 0.02 |ref| elementwise and
-    mean |got - ref| <= 0.01 rms(ref); got is bf16 bits or float64."""
+def check_grad(got, ref, label="", extra=0.0):
+    """Assert |got - ref| <= 0.04 rms(ref) + 0.02 |ref| + extra elementwise and
+    mean |got - ref| <= 0.01 rms(ref) + mean(extra); got is bf16 bits or float64.
+
+    extra (scalar or per element): the error inherited through delta, see
+    delta_bounds; where the exact gradient is identically zero it is the
+    whole allowance."""
     g = bits_to_f64(got) if np.asarray(got).dtype == np.uint16 else np.asarray(got, dtype=np.float64)
     g = g.reshape(ref.shape)
+    extra = np.broadcast_to(np.asarray(extra, dtype=np.float64), ref.shape)
     err = np.abs(g - ref)
     rms = float(np.sqrt(np.mean(ref ** 2)))
     diag = {"max_err_over_rms": float(err.max() / rms) if rms else float(err.max()),
-            "mean_err_over_rms": float(err.mean() / rms) if rms else float(err.mean()), "rms_ref": rms}
+            "mean_err_over_rms": float(err.mean() / rms) if rms else float(err.mean()), "rms_ref": rms,
+            "max_err_over_bound": float((err / (GRAD_ATOL_RMS * rms + GRAD_RTOL * np.abs(ref) + extra + 1e-300)).max())}
     assert np.all(np.isfinite(g)), f"{label}: non-finite gradient"
     if rms == 0.0:
-        assert err.max() == 0.0, f"{label}: expected exact zeros; {diag}"
+        assert np.all(err <= extra), f"{label}: expected zeros up to the delta bound; {diag}"
         return diag
-    bad = err > GRAD_ATOL_RMS * rms + GRAD_RTOL * np.abs(ref)
+    bad = err > GRAD_ATOL_RMS * rms + GRAD_RTOL * np.abs(ref) + extra
     assert not bad.any(), f"{label}: {int(bad.sum())} of {bad.size} gradients out of tolerance; {diag}"
-    assert diag["mean_err_over_rms"] <= GRAD_MEAN_RMS, f"{label}: mean error {diag}"
+    assert err.mean() <= GRAD_MEAN_RMS * rms + extra.mean(), f"{label}: mean error {diag}"
     return diag
+
+
+U_BF16 = 2.0 ** -9
+
+
+def delta_bounds(q, k, v, g, scale, qrows=None, krows=None):
+    """Per-element bounds (bq for dq, bk for dk) on the error a backward
+    inherits from delta_i = <dO_i, O_i> evaluated with the forward's bf16
+    output, as every FlashAttention-style backward does. |O_bf16 - O| is at
+    most ~2u sum_j P_ij |v_j| (the forward's rounding of P and of O), and the
+    fp32 sums of delta and dP add 2 D 2^-24 of the same magnitude; so with
+    A_i = sum_j P_ij |v_j| and c_i = 3u sum_d |dO_id| A_id:
+        |d dS_ij| <= P_ij c_i
+        |d dq_id| <= |scale| c_i sum_j P_ij |k_jd|,  |d dk_jd| <= |scale| sum_i P_ij c_i |q_id|
+    It is small where softmax rows are diffuse and dominates where they are
+    nearly one-hot (dP_ij* ~ delta_i: cancellation). Every sum of P above is
+    the oracle's own attention (values |v|, |k|) or the dv leg of its backward
+    (upstream gradient c_i |q_i|). qrows / krows: the query rows for bq and
+    the key rows for bk, the same in every head (all if None)."""
+    import oracle
+    from dit_attention_b200 import synth
+    absbits = lambda x: np.asarray(x, dtype=np.uint16) & np.uint16(0x7FFF)  # noqa: E731  |bf16| exactly
+    A, _ = oracle.attention(q, k, absbits(v), scale)
+    G = bits_to_f64(g).reshape(A.shape)
+    D = A.shape[-1]
+    c = (3 * U_BF16 + 2 * D * 2.0 ** -24) * np.sum(np.abs(G) * A, axis=-1)
+    if qrows is None:
+        Kabs, _ = oracle.attention(q, k, absbits(k), scale)
+        bq = abs(scale) * c[..., None] * Kabs
+    else:
+        Sq = A.shape[-2]
+        heads = int(np.prod(A.shape[:-2]))
+        qrows = np.asarray(qrows, dtype=np.int64)
+        glob = (np.arange(heads, dtype=np.int64)[:, None] * Sq + qrows[None, :]).reshape(-1)
+        Kabs, _ = oracle.attention(q, k, absbits(k), scale, rows=glob)
+        bq = abs(scale) * c.reshape(heads, Sq)[:, qrows].reshape(A.shape[:-2] + (qrows.size, 1)) * \
+            Kabs.reshape(A.shape[:-2] + (qrows.size, D))
+    X = synth.f64_to_bf16_bits(c[..., None] * bits_to_f64(absbits(q)).reshape(A.shape) * (1 + 2.0 ** -7))
+    if krows is None:
+        bk = oracle.attention_bwd(q, k, v, X, scale)[2]
+    else:
+        bk = oracle.attention_bwd_rows(q, k, v, X, scale, [], krows)[2]
+    return bq, abs(scale) * bk
