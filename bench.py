@@ -268,6 +268,15 @@ def run_native(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     value = aggregate_tflops(flops_step, world, ms_step)
 
+    # ---- backward: the gradient step of the same window (the decoder is trained by
+    # distillation). dO synthetic; the forward's out/lse of the last timed step
+    # (taken before anything else overwrites them).
+    # Self: regen_attn_bwd then regen_rope3d_bwd on dq, dk (gradients w.r.t. the
+    # unrotated Q, K). Cross: one regen_attn_bwd per key block with the MERGED
+    # out/lse, the second accumulating dq. Each regen_attn_bwd is 3 launches
+    # (prep, dK/dV, dQ).
+    bwd = run_backward(args, rg, synth, d, outs0, ws, wc, rank, dev, stream, world, barrier, to_dev)
+
     # ---- the same step with the RoPE fused into the Q load (regen_attn_fwd_rope3d):
     # Q rotated on its tiles in shared memory, K rotated once into the workspace;
     # q and k are not modified, so every step starts from the unrotated inputs.
@@ -436,6 +445,7 @@ def run_native(args, rank, world, local_rank):
                 "serial_value": round(aggregate_tflops(flops_step, world, ms_e2e_serial), 2)},
         "clocks": clk,
     }
+    line["backward"] = bwd
     line["rope_fused_step"] = {
         "what": "the same step with regen_attn_fwd_rope3d (RoPE fused into the Q tile load, K rotated into "
                 "workspace) in place of regen_rope3d + regen_attn_fwd; 7 launches per step",
@@ -450,6 +460,77 @@ def run_native(args, rank, world, local_rank):
         "peak_gbs": float(pk["hbm_gbs"]),
     }
     return line
+
+
+def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, barrier, to_dev):
+    """Times the gradient step; returns its JSON object (rank 0 uses it)."""
+    import torch
+    B, H, S, D = ws.B, ws.H, ws.Sq, ws.D
+    T, Hh, Ww = ws.grid
+    scale = 1.0 / math.sqrt(D)
+    sh = stream.cuda_stream
+    g_self = to_dev(synth.make_dout(ws, seed_offset=rank))
+    g_cross = to_dev(synth.make_dout(wc, seed_offset=rank))
+    n_ref, n_ctx = N_REF, wc.Skv - N_REF
+    dq, dk, dv = (torch.empty_like(d[n]) for n in ("q", "k", "v"))
+    dqc = torch.empty_like(d["qc"])
+    dkr, dvr = torch.empty_like(d["kr"]), torch.empty_like(d["vr"])
+    dkx, dvx = torch.empty_like(d["kx"]), torch.empty_like(d["vx"])
+    wsb = rg.regen_attn_bwd_workspace_bytes(B, H, S, D)
+    work = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    names = ["attn_bwd_self", "rope3d_bwd", "attn_bwd_cross_ref", "attn_bwd_cross_ctx"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        rg.regen_attn_bwd(d["q"], d["k"], d["v"], outs["out"], outs["lse"], g_self, dq, dk, dv, B, H, S, S, D,
+                          scale, sh, work, wsb, 0)
+        mark(1)
+        rg.regen_rope3d_bwd(dq, dk, T, Hh, Ww, ws.theta, B, H, D, sh)
+        mark(2)
+        rg.regen_attn_bwd(d["qc"], d["kr"], d["vr"], outs["oc"], outs["lc"], g_cross, dqc, dkr, dvr, B, H, S,
+                          n_ref, D, scale, sh, work, wsb, 0)
+        mark(3)
+        rg.regen_attn_bwd(d["qc"], d["kx"], d["vx"], outs["oc"], outs["lc"], g_cross, dqc, dkx, dvx, B, H, S,
+                          n_ctx, D, scale, sh, work, wsb, 1)
+        mark(4)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 10))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(n):
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(evs[0][0].elapsed_time(evs[n - 1][4]), world, dev) / n
+    per = {nm: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n)) / n for j, nm in enumerate(names)}
+    f_self, f_cross = step_flops()
+    flops = 2.5 * (f_self + f_cross)      # S, dP, dV, dK, dQ: five products of the forward's two sizes
+    pk, pk_src = peaks()
+    peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
+    achieved = 2.5 * f_self / (per["attn_bwd_self"] * 1e-3) / 1e12
+    del work
+    return {
+        "what": "gradient step of the same window: regen_attn_bwd (self) + regen_rope3d_bwd + regen_attn_bwd per "
+                "cross-attention key block with the merged out/LSE (dq of the second accumulated); synthetic dO",
+        "steps": n, "ms_per_step": round(ms, 4),
+        "value": round(aggregate_tflops(flops, world, ms), 2), "unit": "TFLOP/s",
+        "flops_note": "algorithmic: 2.5x the forward's (QK^T, dO V^T, P^T dO, dS^T Q, dS K); the kernels also "
+                      "recompute QK^T and dO V^T once more (7 products in all, no atomics)",
+        "kernels_ms": {nm: round(t, 4) for nm, t in per.items()},
+        "launches_per_step": 3 + 1 + 3 + 3,
+        "roofline": {"bound": "tensor", "kernel": "regen_attn_bwd self-attention (prep + dK/dV + dQ launches)",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4),
+                     "peak_source": f"{pk_src} bf16_tflops_sustained",
+                     "issued_tensor_flops_frac": round(achieved * 7 / 5 / peak, 4)},
+    }
 
 
 # ------------------------------------------------------ CPU (oracle) ---
