@@ -17,6 +17,8 @@ Functions (each follows the definition written at its C counterpart):
 * ``rope3d(x, grid, theta)`` -- 3D RoPE, bf16 in/out (rounded to nearest even)
   or fp64 in/out; ``rope3d_bwd`` -- its gradient (the transposed rotation).
 * ``f64_to_bf16`` / ``bf16_to_f64`` -- the oracle's own rounding and widening.
+* ``f64_to_e4m3`` / ``e4m3_to_f64`` / ``quantize_e4m3`` / ``dequantize_e4m3`` --
+  OCP E4M3 rounding and the FP8 variant's blockwise quantisation.
 
 Parity status: attention and the LSE merge are pinned by the tests against
 brute force, closed forms, invariants and torch's CPU fp64 SDPA. The RoPE
@@ -91,6 +93,13 @@ def _load():
                                                            ctypes.c_double, _i64p, _i64, _i64p, _i64, _dp, _dp,
                                                            _dp]
             lib.oracle_attention_bwd_rows_bf16.restype = ctypes.c_int
+            lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+            lib.oracle_f64_to_e4m3_array.argtypes = [_dp, ctypes.POINTER(ctypes.c_uint8), _i64]
+            lib.oracle_f64_to_e4m3_array.restype = None
+            lib.oracle_quantize_e4m3.argtypes = [_u16p, _i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_uint8),
+                                                 ctypes.POINTER(ctypes.c_float)]
+            lib.oracle_quantize_e4m3.restype = ctypes.c_int
             lib.oracle_lse_merge_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _dp, _dp]
             lib.oracle_lse_merge_f64.restype = None
             lib.oracle_rope3d_f64.argtypes = [_dp, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
@@ -247,6 +256,49 @@ def attention_bwd_rows(q, k, v, dout, scale: float, qrows, krows):
     if rc != 0:
         raise MemoryError("oracle could not allocate its row statistics")
     return dq, dk, dv
+
+
+def e4m3_to_f64(codes):
+    """Decode OCP E4M3 codes (uint8 array) to doubles (exact)."""
+    lib = _load()
+    table = np.array([lib.oracle_e4m3_to_f64(c) for c in range(256)], dtype=np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def f64_to_e4m3(x):
+    """Round doubles to E4M3 codes: nearest, ties to even, saturating at +-448."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint8)
+    lib.oracle_f64_to_e4m3_array(_ptr(x, _dp), out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), x.size)
+    return out
+
+
+def quantize_e4m3(x, block_rows: int = 128):
+    """Blockwise E4M3 quantisation of bf16 bits x [..., S, D] (see oracle.c):
+    returns (codes uint8 [..., S, D], scales float32 [..., ceil(S/block_rows)])."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    S, D = x.shape[-2], x.shape[-1]
+    lead = x.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+    nb = -(-S // block_rows)
+    codes = np.empty(x.shape, dtype=np.uint8)
+    scales = np.empty(lead + (nb,), dtype=np.float32)
+    rc = lib.oracle_quantize_e4m3(_ptr(x, _u16p), BH, S, D, block_rows,
+                                  codes.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                  scales.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    if rc != 0:
+        raise ValueError("block_rows must be positive")
+    return codes, scales
+
+
+def dequantize_e4m3(codes, scales, block_rows: int = 128):
+    """code * scale of its block, in fp64 (exact): the values the FP8 path represents."""
+    v = e4m3_to_f64(codes)
+    S = v.shape[-2]
+    rep = np.repeat(np.asarray(scales, dtype=np.float64), block_rows, axis=-1)[..., :S]
+    return v * rep[..., None]
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b):

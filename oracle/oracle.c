@@ -404,6 +404,98 @@ void oracle_lse_merge_f64(const double *oa, const double *lsea,
     }
 }
 
+/* ------------------------------------------------------ FP8 (e4m3) --- */
+
+/*
+ * OCP FP8 E4M3 ("fn": no infinities): 1 sign bit, 4 exponent bits with bias
+ * 7, 3 mantissa bits. Exponent field 1..15 encodes 2^(e-7) (1 + m/8), except
+ * field 15 with m = 7 which is NaN, so the largest finite value is 448;
+ * field 0 encodes subnormals 2^-6 (m/8). Rounding here: to nearest, ties to
+ * even, then saturation of finite values to +-448 (the "satfinite" rounding
+ * of the FP8 variant). The FP8 attention variant is not on the pages; its
+ * quantisation is defined here (see oracle_quantize_e4m3).
+ */
+double oracle_e4m3_to_f64(uint8_t c)
+{
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);               /* 2^-6 * m/8 */
+    else
+        v = ldexp(8.0 + m, e - 7 - 3);          /* 2^(e-7) * (8+m)/8 */
+    return sgn ? -v : v;
+}
+
+uint8_t oracle_f64_to_e4m3(double x)
+{
+    if (x != x) return 0x7F;
+    uint8_t sgn = (x < 0) ? 0x80 : 0;
+    double a = fabs(x);
+    if (a >= 448.0) return sgn | 0x7E;           /* saturate */
+    int e2;
+    frexp(a, &e2);                               /* a = f 2^e2, f in [0.5, 1) */
+    int e = e2 - 1;                              /* a in [2^e, 2^(e+1)) */
+    if (e < -6) e = -6;                          /* subnormal spacing 2^-9 */
+    double ulp = ldexp(1.0, e - 3);
+    double n = nearbyint(a / ulp);               /* exact quotient, ties to even */
+    double r = n * ulp;
+    if (r >= 448.0) return sgn | 0x7E;
+    if (r == 0.0) return sgn;
+    int re2;
+    frexp(r, &re2);
+    int re = re2 - 1;
+    if (re < -6) return sgn | (uint8_t)(r / ldexp(1.0, -9));     /* subnormal: m = r / 2^-9 */
+    int mant = (int)(r / ldexp(1.0, re - 3)) - 8;                 /* 0..7 */
+    return sgn | (uint8_t)(((re + 7) << 3) | mant);
+}
+
+void oracle_f64_to_e4m3_array(const double *x, uint8_t *c, int64_t n)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) c[i] = oracle_f64_to_e4m3(x[i]);
+}
+
+/*
+ * Blockwise quantisation of x [BH][S][D] (bf16) for the FP8 attention: each
+ * block of `block_rows` consecutive rows of one (b, h) -- the last one
+ * ragged -- gets amax = max |x| over the block, scale = amax / 448 and
+ * inv = 448 / amax, both rounded to fp32; every element is multiplied by inv
+ * in fp32 and rounded to e4m3 as above; x is represented by code * scale. An
+ * all-zero block gets scale = inv = 1. Outputs codes [BH][S][D] and scales
+ * [BH][ceil(S / block_rows)].
+ */
+int oracle_quantize_e4m3(const uint16_t *x, int64_t BH, int64_t S, int64_t D, int64_t block_rows,
+                         uint8_t *codes, float *scales)
+{
+    if (block_rows <= 0) return -1;
+    int64_t nb = (S + block_rows - 1) / block_rows;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < BH * nb; ++t) {
+        int64_t bh = t / nb, b = t % nb;
+        int64_t r0 = b * block_rows, r1 = r0 + block_rows < S ? r0 + block_rows : S;
+        const uint16_t *xb = x + (bh * S + r0) * D;
+        uint8_t *cb = codes + (bh * S + r0) * D;
+        int64_t n = (r1 - r0) * D;
+        float amax = 0.0f;
+        for (int64_t i = 0; i < n; ++i) {
+            float a = fabsf((float)oracle_bf16_to_f64(xb[i]));
+            if (a > amax) amax = a;
+        }
+        volatile float scale = 1.0f, inv = 1.0f;   /* volatile: each op rounded to fp32 */
+        if (amax > 0.0f) {
+            scale = amax / 448.0f;
+            inv = 448.0f / amax;
+        }
+        scales[t] = scale;
+        for (int64_t i = 0; i < n; ++i) {
+            volatile float y = (float)oracle_bf16_to_f64(xb[i]) * inv;
+            cb[i] = oracle_f64_to_e4m3((double)y);
+        }
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------- RoPE --- */
 
 /*

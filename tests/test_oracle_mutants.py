@@ -40,6 +40,8 @@ MUTANTS = {
                         "dv[j * D + d] += dS[i * Skv + j] * at(dout, doo + i * D + d);"),
     "rope bwd: forward rotation used": ("row[base[a] + 2 * j + 1] = c * x1 - s * x0;",
                                         "row[base[a] + 2 * j + 1] = c * x1 + s * x0;"),
+    "e4m3 mantissa width": ("double ulp = ldexp(1.0, e - 3);", "double ulp = ldexp(1.0, e - 2);"),
+    "e4m3 quantiser scale not inverted": ("inv = 448.0f / amax;", "inv = amax / 448.0f;"),
     "rope pair partner index": ("double x1 = row[base[a] + 2 * j + 1];", "double x1 = row[base[a] + j + 1];"),
 }
 

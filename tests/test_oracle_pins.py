@@ -419,3 +419,60 @@ def test_attention_bwd_rows_equals_full():
     np.testing.assert_allclose(sq, dq[:, :, qr], rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(sk, dk[:, :, kr], rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(sv, dv[:, :, kr], rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------------------- FP8 e4m3 ---
+
+def test_e4m3_decode_table():
+    # the OCP E4M3 values: +-0, subnormals k 2^-9, normals up to 448, NaN at 0x7F / 0xFF
+    v = oracle.e4m3_to_f64(np.arange(256))
+    assert v[0] == 0.0 and v[1] == 2.0 ** -9 and v[7] == 7 * 2.0 ** -9 and v[8] == 2.0 ** -6
+    assert v[0x38] == 1.0 and v[0x7E] == 448.0 and np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    assert v[0x80 | 0x38] == -1.0
+    finite = v[np.isfinite(v)]
+    assert len(finite) == 254 and len(np.unique(finite[finite > 0])) == 126
+
+
+def test_e4m3_round_trip_and_ties():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF, 0x80)], dtype=np.uint8)
+    vals = oracle.e4m3_to_f64(codes)
+    np.testing.assert_array_equal(oracle.f64_to_e4m3(vals), codes)
+    pos = np.sort(oracle.e4m3_to_f64(np.arange(0, 0x7F)))
+    mid = (pos[:-1] + pos[1:]) / 2
+    got = oracle.e4m3_to_f64(oracle.f64_to_e4m3(mid))
+    lo_even = (oracle.f64_to_e4m3(pos[:-1]) & 1) == 0
+    np.testing.assert_array_equal(got, np.where(lo_even, pos[:-1], pos[1:]))   # ties to the even code
+    assert oracle.e4m3_to_f64(oracle.f64_to_e4m3(np.array([460.0, 1e6, -1e6]))).tolist() == [448, 448, -448]
+
+
+def test_e4m3_matches_torch_cast():
+    torch = pytest.importorskip("torch")
+    if not hasattr(torch, "float8_e4m3fn"):
+        pytest.skip("torch without float8")
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.uniform(-463.9, 463.9, 20000), rng.normal(size=20000) * 2.0 ** -7,
+                        rng.normal(size=20000)]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.f64_to_e4m3(x.astype(np.float64)), ref)
+
+
+def test_quantize_e4m3_properties():
+    rng = np.random.default_rng(4)
+    x = oracle.f64_to_bf16(rng.normal(size=(2, 3, 300, 128)) * np.array([1.0, 1e-3, 50.0])[None, :, None, None])
+    x[1, 2, 128:256] = 0                                 # an all-zero block
+    codes, scales = oracle.quantize_e4m3(x, 128)
+    assert codes.shape == x.shape and scales.shape == (2, 3, 3)
+    xf = oracle.bf16_to_f64(x)
+    blocks = [(0, 128), (128, 256), (256, 300)]
+    for b, (r0, r1) in enumerate(blocks):
+        amax = np.abs(xf[:, :, r0:r1]).max(axis=(2, 3)).astype(np.float32)
+        want = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0))
+        np.testing.assert_array_equal(scales[:, :, b], want)
+    deq = oracle.dequantize_e4m3(codes, scales, 128)
+    # each value within half an e4m3 step: relative 2^-4 of itself (normals) or
+    # 2^-10 * scale absolute (subnormals), plus the fp32 rounding of inv
+    sc = np.repeat(scales.astype(np.float64), 128, axis=-1)[..., :300, None]
+    assert np.all(np.abs(deq - xf) <= 2.0 ** -4 * np.abs(xf) * (1 + 1e-6) + 2.0 ** -10 * sc)
+    # the block's largest element lands on +-448 (within fp32 rounding of 448/amax)
+    assert np.abs(oracle.e4m3_to_f64(codes[0, 0, :128])).max() == 448.0
+    assert not codes[1, 2, 128:256].any() and scales[1, 2, 1] == 1.0
