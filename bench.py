@@ -277,6 +277,10 @@ def run_native(args, rank, world, local_rank):
     # (prep, dK/dV, dQ).
     bwd = run_backward(args, rg, synth, d, outs0, ws, wc, rank, dev, stream, world, barrier, to_dev)
 
+    # ---- the FP8 variant of the self-attention (after the same RoPE): blockwise
+    # E4M3 quantisation of Q, K, V (3 launches) and the E4M3 attention.
+    fp8 = run_fp8(args, rg, d, ws, dev, stream, world, barrier)
+
     # ---- the same step with the RoPE fused into the Q load (regen_attn_fwd_rope3d):
     # Q rotated on its tiles in shared memory, K rotated once into the workspace;
     # q and k are not modified, so every step starts from the unrotated inputs.
@@ -446,6 +450,7 @@ def run_native(args, rank, world, local_rank):
         "clocks": clk,
     }
     line["backward"] = bwd
+    line["fp8"] = fp8
     line["rope_fused_step"] = {
         "what": "the same step with regen_attn_fwd_rope3d (RoPE fused into the Q tile load, K rotated into "
                 "workspace) in place of regen_rope3d + regen_attn_fwd; 7 launches per step",
@@ -530,6 +535,64 @@ def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, bar
                      "frac": round(achieved / peak, 4),
                      "peak_source": f"{pk_src} bf16_tflops_sustained",
                      "issued_tensor_flops_frac": round(achieved * 7 / 5 / peak, 4)},
+    }
+
+
+def run_fp8(args, rg, d, ws, dev, stream, world, barrier):
+    """Times quantise + FP8 self-attention on the 77-frame window; returns its JSON object."""
+    import torch
+    B, H, S, D = ws.B, ws.H, ws.Sq, ws.D
+    scale = 1.0 / math.sqrt(D)
+    sh = stream.cuda_stream
+    nb = -(-S // 128)
+    codes = {n: torch.empty((B, H, S, D), dtype=torch.uint8, device=dev) for n in ("q", "k", "v")}
+    scales = {n: torch.empty((B, H, nb), dtype=torch.float32, device=dev) for n in ("q", "k", "v")}
+    out = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        for n in ("q", "k", "v"):
+            rg.regen_quant_e4m3(d[n], codes[n], scales[n], B, H, S, D, sh)
+        if ev is not None:
+            ev[1].record(stream)
+        rg.regen_attn_fwd_fp8(codes["q"], scales["q"], codes["k"], scales["k"], codes["v"], scales["v"], out, lse,
+                              B, H, S, S, D, scale, sh)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 20))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(n):
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(evs[0][0].elapsed_time(evs[n - 1][2]), world, dev) / n
+    t_q = sum(e[0].elapsed_time(e[1]) for e in evs) / n
+    t_a = sum(e[1].elapsed_time(e[2]) for e in evs) / n
+    f_self = step_flops()[0]
+    pk, pk_src = peaks()
+    peak8 = 2.0 * float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
+    achieved = f_self / (t_a * 1e-3) / 1e12
+    qbytes = 3 * B * H * S * D * 3 + 3 * B * H * nb * 4    # read bf16, write codes, write scales
+    return {
+        "what": "FP8 (E4M3) variant of the 77-frame self-attention after its RoPE: blockwise quantisation of Q, K, V "
+                "(regen_quant_e4m3 x3) + regen_attn_fwd_fp8; accuracy contract in the tests (E4M3 rounding of P)",
+        "steps": n, "ms_per_step": round(ms, 4),
+        "value": round(aggregate_tflops(f_self, world, ms), 2), "unit": "TFLOP/s",
+        "kernels_ms": {"quant_e4m3_x3": round(t_q, 4), "attn_fwd_fp8": round(t_a, 4)},
+        "quant_gbs": round(qbytes / (t_q * 1e-3) / 1e9, 1),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_fp8 (31200 x 31200, H=40, D=128)",
+                     "achieved": round(achieved, 2), "peak": peak8, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak8, 4),
+                     "peak_source": f"{pk_src} bf16_tflops_sustained x 2 (dense E4M3 : BF16 nominal ratio)"},
+        "launches_per_step": 4,
     }
 
 

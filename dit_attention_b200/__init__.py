@@ -17,6 +17,8 @@ Entry points (same names as the C ABI):
                    workspace, workspace_bytes, accumulate_dq)
     regen_attn_bwd_workspace_bytes(B, H, Sq, D)
     regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream=None)
+    regen_quant_e4m3(x, codes, scales, B, H, S, D, stream=None)
+    regen_attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, B, H, Sq, Skv, D, scale, stream=None)
     regen_last_device_error() -> (status, site)
     regen_set_wait_limit_ns(ns)
 Convenience wrappers that allocate outputs with torch:
@@ -26,6 +28,7 @@ Convenience wrappers that allocate outputs with torch:
     lse_merge(o_a, lse_a, o_b, lse_b) -> (out, lse)
     attn_bwd(q, k, v, out, lse, dout, scale=None) -> (dq, dk, dv)
     rope3d_bwd_(dq, dk, grid, theta=10000.0)
+    quant_e4m3(x) -> (codes, scales);  attn_fwd_fp8(q8, qs, k8, ks, v8, vs, scale=None) -> (out, lse)
 """
 from __future__ import annotations
 
@@ -38,7 +41,8 @@ __all__ = [
     "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
     "regen_status_str", "regen_last_device_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
     "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes", "regen_attn_fwd_rope3d_noalloc",
-    "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd",
+    "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd", "regen_quant_e4m3",
+    "regen_attn_fwd_fp8", "quant_e4m3", "attn_fwd_fp8",
     "attn_fwd", "attn_fwd_rope3d", "rope3d_", "lse_merge", "attn_bwd", "rope3d_bwd_", "STATUS",
 ]
 
@@ -92,6 +96,10 @@ def load():
         L.regen_attn_bwd_workspace_bytes.restype = i64
         L.regen_rope3d_bwd.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, vp]
         L.regen_rope3d_bwd.restype = i32
+        L.regen_quant_e4m3.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+        L.regen_quant_e4m3.restype = i32
+        L.regen_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
+        L.regen_attn_fwd_fp8.restype = i32
         L.regen_status_str.argtypes = [i32]
         L.regen_status_str.restype = ctypes.c_char_p
         L.regen_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
@@ -202,6 +210,18 @@ def regen_attn_bwd_workspace_bytes(B, H, Sq, D) -> int:
 def regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream=None) -> None:
     _check(load().regen_rope3d_bwd(_ptr(dq), _ptr(dk), T, Hh, Ww, float(theta), B, H, D, _stream(stream)),
            "regen_rope3d_bwd")
+
+
+def regen_quant_e4m3(x, codes, scales, B, H, S, D, stream=None) -> None:
+    _check(load().regen_quant_e4m3(_ptr(x), _ptr(codes), _ptr(scales), B, H, S, D, _stream(stream)),
+           "regen_quant_e4m3")
+
+
+def regen_attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, B, H, Sq, Skv, D, scale,
+                       stream=None) -> None:
+    _check(load().regen_attn_fwd_fp8(_ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v8), _ptr(v_scale),
+                                     _ptr(out), _ptr(lse), B, H, Sq, Skv, D, float(scale), _stream(stream)),
+           "regen_attn_fwd_fp8")
 
 
 def regen_selftest_exp2(x, y, n, stream=None) -> None:
@@ -331,3 +351,31 @@ def rope3d_bwd_(dq, dk, grid, theta=10000.0, stream=None):
         raise ValueError("sequence length does not match the latent grid")
     regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream)
     return dq, dk
+
+
+def quant_e4m3(x, codes=None, scales=None, stream=None):
+    """Blockwise E4M3 codes (uint8, same shape) and fp32 scales [B, H, ceil(S/128)]
+    of a bf16 [B, H, S, D] CUDA tensor."""
+    import torch
+    B, H, S, D = _bhsd(x, "x")
+    if codes is None:
+        codes = torch.empty((B, H, S, D), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, H, -(-S // 128)), dtype=torch.float32, device=x.device)
+    regen_quant_e4m3(x, codes, scales, B, H, S, D, stream)
+    return codes, scales
+
+
+def attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, scale=None, out=None, lse=None, stream=None):
+    """FP8 attention from quant_e4m3 outputs -> (out bf16, lse fp32)."""
+    import torch
+    B, H, Sq, D = _bhsd(q8, "q8")
+    Skv = _bhsd(k8, "k8")[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, H, Sq, D), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q8.device)
+    regen_attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, B, H, Sq, Skv, D, scale, stream)
+    return out, lse

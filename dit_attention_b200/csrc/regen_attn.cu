@@ -18,6 +18,7 @@
 #include "regen_attn.h"
 
 #include "attn_bwd.cuh"
+#include "attn_fp8.cuh"
 #include "attn_fwd.cuh"
 #include "lse_merge.cuh"
 #include "rope3d.cuh"
@@ -66,6 +67,52 @@ bool make_bhsd_map(CUtensorMap *map, const void *base, int64_t BH, int64_t S, in
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// [BH, S, 128] E4M3 codes as a 3D tensor (128 codes innermost), boxes of
+// 128 x 128 x 1 with the 128-byte swizzle; out-of-range rows read as zero.
+bool make_u8_map(CUtensorMap *map, const void *base, int64_t BH, int64_t S)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(S * 128)};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool NEG>
+int launch_attn_fp8(const uint8_t *q8, const float *qs, const uint8_t *k8, const float *ks, const uint8_t *v8,
+                    const float *vs, regen_bf16 *out, float *lse, int64_t BH, int Sq, int Skv, float scale,
+                    cudaStream_t stream)
+{
+    using C = regen::Fp8Cfg;
+    static std::once_flag once;
+    static int attr_status = REGEN_OK;
+    std::call_once(once, [] {
+        cudaFuncAttributes fa;
+        if (cudaFuncSetAttribute(regen::attn_fwd_fp8_kernel<NEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, regen::attn_fwd_fp8_kernel<NEG>) != cudaSuccess)
+            attr_status = REGEN_ERR_CUDA;
+        else if (fa.numRegs < C::MIN_LAUNCH_REGS)
+            attr_status = REGEN_ERR_UNSUPPORTED;
+    });
+    if (attr_status != REGEN_OK) return attr_status;
+    CUtensorMap tq, tk, tv, to;
+    if (!make_u8_map(&tq, q8, BH, Sq) || !make_u8_map(&tk, k8, BH, Skv) || !make_u8_map(&tv, v8, BH, Skv) ||
+        !make_bhsd_map(&to, out, BH, Sq, 128))
+        return REGEN_ERR_CUDA;
+    const int64_t grid = (Sq + 2 * C::BM - 1) / (2 * C::BM) * BH;
+    if (grid > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    regen::attn_fwd_fp8_kernel<NEG><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, to, qs, ks, vs, lse, Sq, Skv, scale_log2, g_wait_limit_ns.load());
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
 }
 
 template <int HD, bool NEG, bool ROPE_Q = false>
@@ -470,6 +517,67 @@ REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a, const r
         reinterpret_cast<const uint4 *>(o_a), lse_a, reinterpret_cast<const uint4 *>(o_b), lse_b,
         reinterpret_cast<uint4 *>(out), lse_out, rows, D);
     return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
+REGEN_API int regen_quant_e4m3(const regen_bf16 *x, uint8_t *codes, float *scales, int B, int H, int S, int D,
+                               regen_stream_t stream)
+{
+    if (B < 0 || H < 0 || S < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0 || S == 0) return REGEN_OK;
+    if (!x || !codes || !scales) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return REGEN_ERR_MISALIGNED;
+    const int64_t nb = (S + 127) / 128;
+    if (BH * nb > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const int64_t xbytes = BH * S * D * 2, cbytes = BH * S * D, sbytes = BH * nb * 4;
+    if (overlaps(codes, cbytes, x, xbytes) || overlaps(scales, sbytes, x, xbytes) ||
+        overlaps(scales, sbytes, codes, cbytes))
+        return REGEN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned grid = static_cast<unsigned>(BH * nb);
+    if (D == 128)
+        regen::quant_e4m3_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(x),
+                                                            reinterpret_cast<uint2 *>(codes), scales, S,
+                                                            static_cast<int>(nb));
+    else
+        regen::quant_e4m3_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(x),
+                                                           reinterpret_cast<uint2 *>(codes), scales, S,
+                                                           static_cast<int>(nb));
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+}
+
+REGEN_API int regen_attn_fwd_fp8(const uint8_t *q8, const float *q_scale, const uint8_t *k8, const float *k_scale,
+                                 const uint8_t *v8, const float *v_scale, regen_bf16 *out, float *lse, int B, int H,
+                                 int Sq, int Skv, int D, float scale, regen_stream_t stream)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Skv < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return REGEN_ERR_INVALID_ARG;
+    if (D != 128) return REGEN_ERR_UNSUPPORTED;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0 || Sq == 0) return REGEN_OK;
+    if (BH > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (!q8 || !q_scale || !out || (Skv > 0 && (!k8 || !k_scale || !v8 || !v_scale))) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q8) || !aligned16(out) || !aligned16(lse) || (Skv > 0 && (!aligned16(k8) || !aligned16(v8))) ||
+        (reinterpret_cast<uintptr_t>(q_scale) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+        return REGEN_ERR_MISALIGNED;
+    const int64_t obytes = BH * Sq * D * 2, lbytes = BH * Sq * 4;
+    const int64_t qb = BH * Sq * D, kvb = BH * Skv * D;
+    const int64_t qsb = BH * ((Sq + 127) / 128) * 4, kvsb = BH * ((Skv + 127) / 128) * 4;
+    struct Span { const void *p; int64_t n; };
+    const Span ins[6] = {{q8, qb}, {k8, kvb}, {v8, kvb}, {q_scale, qsb}, {k_scale, kvsb}, {v_scale, kvsb}};
+    for (const Span &in : ins)
+        if (overlaps(out, obytes, in.p, in.n) || overlaps(lse, lbytes, in.p, in.n)) return REGEN_ERR_INVALID_ARG;
+    if (overlaps(lse, lbytes, out, obytes)) return REGEN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (Skv == 0) {
+        regen::attn_empty_kernel<<<grid_for(obytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(out),
+                                                                            obytes / 16, lse, BH * Sq);
+        return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    }
+    return scale < 0.0f ? launch_attn_fp8<true>(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, BH, Sq, Skv, scale, st)
+                        : launch_attn_fp8<false>(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, BH, Sq, Skv, scale, st);
 }
 
 REGEN_API int regen_selftest_exp2(const float *x, float *y, int64_t n, regen_stream_t stream)

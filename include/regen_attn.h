@@ -227,6 +227,39 @@ REGEN_API int regen_rope3d_bwd(regen_bf16 *dq, regen_bf16 *dk, int T, int Hh, in
                                int B, int H, int D, regen_stream_t stream);
 
 /*
+ * regen_quant_e4m3 -- blockwise FP8 quantisation for regen_attn_fwd_fp8 (a
+ * speed/accuracy variant of the attention; the pages do not describe one).
+ * For each (b, h) and each block of 128 consecutive rows (the last ragged):
+ *     amax = max |x|,  scale = amax / 448,  inv = 448 / amax   (fp32; 1 and 1 if amax == 0)
+ *     codes = E4M3(x * inv)   (OCP E4M3, round to nearest even, saturating at +-448)
+ * so that x ~ codes * scale.
+ *
+ *   x       [B, H, S, D] bf16;  D = 64 or 128 (else REGEN_ERR_UNSUPPORTED)
+ *   codes   [B, H, S, D] bytes, 16-byte aligned
+ *   scales  [B, H, ceil(S/128)] fp32, 4-byte aligned
+ * No overlaps. B, H or S == 0: REGEN_OK, nothing done.
+ */
+REGEN_API int regen_quant_e4m3(const regen_bf16 *x, uint8_t *codes, float *scales, int B, int H, int S, int D,
+                               regen_stream_t stream);
+
+/*
+ * regen_attn_fwd_fp8 -- attention of the dequantised inputs (codes * block
+ * scale, from regen_quant_e4m3) with E4M3 tensor-core products:
+ *     S = Q8 K8^T (fp32 accumulate) times scale * sq * sk,  online softmax in fp32,
+ *     O = sum_j P_j V_j with P rounded to E4M3 (in units of 2^-4 of the running
+ *     row max, so at most 2^8) and V's block scales folded into P's exponent,
+ *     out = O / l in bf16,  lse = m + ln l (fp32)
+ * The row sum l uses P before rounding. Arguments and edge cases as
+ * regen_attn_fwd, with the codes and scales in place of bf16 q, k, v:
+ *   q8 [B,H,Sq,128], k8, v8 [B,H,Skv,128] bytes (16-byte aligned);
+ *   q_scale [B,H,ceil(Sq/128)], k_scale, v_scale [B,H,ceil(Skv/128)] fp32.
+ *   D must be 128 (else REGEN_ERR_UNSUPPORTED).
+ */
+REGEN_API int regen_attn_fwd_fp8(const uint8_t *q8, const float *q_scale, const uint8_t *k8, const float *k_scale,
+                                 const uint8_t *v8, const float *v_scale, regen_bf16 *out, float *lse,
+                                 int B, int H, int Sq, int Skv, int D, float scale, regen_stream_t stream);
+
+/*
  * regen_selftest_exp2 -- diagnostic: evaluates, for each x[i], the FMA-pipe
  * 2^x that the attention kernel uses for part of its softmax probabilities
  * (degree-4 polynomial after Cody-Waite range reduction; inputs below -127

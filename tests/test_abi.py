@@ -161,3 +161,27 @@ def test_rope3d_bwd_validation(lib, args, status):
     a.update(args)
     rc = lib.regen_rope3d_bwd(a["q"], a["k"], a["T"], a["Hh"], a["Ww"], a["theta"], a["B"], a["H"], a["D"], None)
     assert rc == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=96), -2), (dict(B=-1), -1), (dict(x=None), -1), (dict(codes=FAKE + 20 * MB + 8), -3),
+    (dict(scales=FAKE + 30 * MB + 2), -3), (dict(codes=FAKE + 4096), -1), (dict(S=0), 0), (dict(H=0, x=None), 0),
+])
+def test_quant_e4m3_validation(lib, args, status):
+    a = dict(x=FAKE, codes=FAKE + 20 * MB, scales=FAKE + 30 * MB, B=1, H=2, S=300, D=128)
+    a.update(args)
+    assert lib.regen_quant_e4m3(a["x"], a["codes"], a["scales"], a["B"], a["H"], a["S"], a["D"], None) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=64), -2), (dict(Sq=-1), -1), (dict(scale=float("inf")), -1), (dict(q8=None), -1), (dict(vs=None), -1),
+    (dict(q8=FAKE + 4), -3), (dict(ks=FAKE + 50 * MB + 1), -3), (dict(out=FAKE + 1024), -1),
+    (dict(lse=FAKE + 60 * MB + 16), -1), (dict(B=0), 0), (dict(Sq=0), 0),
+])
+def test_attn_fwd_fp8_validation(lib, args, status):
+    a = dict(q8=FAKE, qs=FAKE + 10 * MB, k8=FAKE + 20 * MB, ks=FAKE + 30 * MB, v8=FAKE + 40 * MB, vs=FAKE + 50 * MB,
+             out=FAKE + 60 * MB, lse=FAKE + 70 * MB, B=1, H=2, Sq=300, Skv=200, D=128, scale=0.1)
+    a.update(args)
+    rc = lib.regen_attn_fwd_fp8(a["q8"], a["qs"], a["k8"], a["ks"], a["v8"], a["vs"], a["out"], a["lse"], a["B"],
+                                a["H"], a["Sq"], a["Skv"], a["D"], a["scale"], None)
+    assert rc == status

@@ -130,3 +130,38 @@ def delta_bounds(q, k, v, g, scale, qrows=None, krows=None):
     else:
         bk = oracle.attention_bwd_rows(q, k, v, X, scale, [], krows)[2]
     return bq, abs(scale) * bk
+
+
+def check_fp8_attention(out_bits, lse_gpu, qd, kd, vd, scale, rows=None, label=""):
+    """FP8 attention contract, against the oracle's exact attention of the
+    DEQUANTISED inputs qd, kd, vd (fp64, code * block scale).
+
+    The kernel rounds P to E4M3 before P V: p_j (1 + e_j) with |e_j| <= 2^-4,
+    errors of different keys independent, so out_d carries an error of standard
+    deviation at most sigma_d = 2^-4 / sqrt(3) * sqrt(sum_j p_j^2 v_jd^2), and
+    sum_j p_j^2 v_jd^2 = exp(lse2 - 2 lse) out2_d with (out2, lse2) the
+    oracle's attention of values v^2 at twice the scale. Asserted: |err| <=
+    6 sigma + 2^-8 |ref| (bf16 output) + 1e-5 (keys whose P lands in E4M3's
+    subnormals) elementwise, mean |err| <= mean sigma + 2^-8 mean |ref|, and
+    |lse - ref| <= 1e-3 (the row sum uses P before rounding)."""
+    import oracle
+    ref, rl = oracle.attention(qd, kd, vd, scale, rows=rows)
+    out2, rl2 = oracle.attention(qd, kd, vd * vd, 2.0 * scale, rows=rows)
+    D = ref.shape[-1]
+    ref, rl = ref.reshape(-1, D), rl.reshape(-1)
+    out2, rl2 = out2.reshape(-1, D), rl2.reshape(-1)
+    sigma = 2.0 ** -4 / np.sqrt(3.0) * np.sqrt(np.maximum(out2, 0.0) * np.exp(rl2 - 2.0 * rl)[:, None])
+    got = bits_to_f64(out_bits).reshape(-1, D)
+    err = np.abs(got - ref)
+    allow = 6.0 * sigma + 2.0 ** -8 * np.abs(ref) + 1e-5
+    lse_err = np.abs(np.asarray(lse_gpu, dtype=np.float64).reshape(-1) - rl)
+    diag = {"max_err_over_sigma": float((err / (sigma + 1e-30)).max()),
+            "mean_err_over_mean_sigma": float(err.mean() / max(sigma.mean(), 1e-30)),
+            "max_abs_err": float(err.max()), "max_lse_err": float(lse_err.max()),
+            "rms_ref": float(np.sqrt(np.mean(ref ** 2)))}
+    assert np.all(np.isfinite(got)), f"{label}: non-finite output"
+    bad = err > allow
+    assert not bad.any(), f"{label}: {int(bad.sum())} of {bad.size} outputs outside 6 sigma; {diag}"
+    assert err.mean() <= sigma.mean() + 2.0 ** -8 * np.abs(ref).mean(), f"{label}: mean error {diag}"
+    assert lse_err.max() <= LSE_ATOL, f"{label}: lse {diag}"
+    return diag
