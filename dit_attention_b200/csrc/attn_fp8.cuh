@@ -20,8 +20,10 @@
 #include "attn_fwd.cuh"
 #include "ptx.cuh"
 
+// Pairs of every 8 whose 2^x runs on the FMA pipe; 2 and 3 measured equal on the
+// 77-frame window, 4 and 5 slower (the softmax is issue-bound, not MUFU-bound).
 #ifndef REGEN_FP8_EXP2_EMU_PER8
-#define REGEN_FP8_EXP2_EMU_PER8 3
+#define REGEN_FP8_EXP2_EMU_PER8 2
 #endif
 
 namespace regen {

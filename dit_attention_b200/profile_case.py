@@ -6,7 +6,8 @@ No timing is done here (use bench.py); this only gives ncu a small, bounded
 launch sequence of one kernel: --kernel attn (self-attention with the 77-frame
 window's sequence length, or --kv for cross-attention), rope (3D RoPE on the
 latent grid of that sequence length), merge (two-block LSE merge) or bwd (one
-forward, then --iters gradient calls: prep, dK/dV and dQ launches each).
+forward, then --iters gradient calls: prep, dK/dV and dQ launches each) or
+fp8 (quantisation of Q, K, V once, then --iters FP8 attention calls).
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ GRIDS = {31200: (20, 30, 52), 10920: (7, 30, 52), 1024: (1, 32, 32)}
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("--kernel", choices=["attn", "rope", "merge", "bwd"], default="attn")
+    p.add_argument("--kernel", choices=["attn", "rope", "merge", "bwd", "fp8"], default="attn")
     p.add_argument("--heads", type=int, default=8)
     p.add_argument("--seq", type=int, default=31200)
     p.add_argument("--kv", type=int, default=0, help="key count (default: --seq)")
@@ -44,8 +45,12 @@ def main():
         scale = 1.0 / math.sqrt(a.dim)
         out, lse = rg.attn_fwd(dq, dk, dv, scale)
         g = dev(synth.make_dout(w))
+    if a.kernel == "fp8":
+        quant = [rg.quant_e4m3(x) for x in (dq, dk, dv)]
     for _ in range(a.iters):
-        if a.kernel == "attn":
+        if a.kernel == "fp8":
+            rg.attn_fwd_fp8(*quant[0], *quant[1], *quant[2], 1.0 / math.sqrt(a.dim))
+        elif a.kernel == "attn":
             rg.attn_fwd(dq, dk, dv, 1.0 / math.sqrt(a.dim))
         elif a.kernel == "bwd":
             rg.attn_bwd(dq, dk, dv, out, lse, g, scale)
