@@ -17,6 +17,8 @@ Functions (each follows the definition written at its C counterpart):
 * ``rope3d(x, grid, theta)`` -- 3D RoPE, bf16 in/out (rounded to nearest even)
   or fp64 in/out; ``rope3d_bwd`` -- its gradient (the transposed rotation).
 * ``f64_to_bf16`` / ``bf16_to_f64`` -- the oracle's own rounding and widening.
+* ``qkv_proj`` / ``out_proj`` -- the DiT block's projections around the
+  attention (linear layer, per-head RMSNorm and 3D RoPE on q and k).
 * ``f64_to_e4m3`` / ``e4m3_to_f64`` / ``quantize_e4m3`` / ``dequantize_e4m3`` --
   OCP E4M3 rounding and the FP8 variant's blockwise quantisation.
 
@@ -100,6 +102,11 @@ def _load():
             lib.oracle_quantize_e4m3.argtypes = [_u16p, _i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_uint8),
                                                  ctypes.POINTER(ctypes.c_float)]
             lib.oracle_quantize_e4m3.restype = ctypes.c_int
+            lib.oracle_qkv_proj_rows.argtypes = [_u16p, _u16p, _dp, _dp, _dp] + [_i64] * 8 + [
+                ctypes.c_double, ctypes.c_double, _i64p, _i64, _dp, _dp, _dp]
+            lib.oracle_qkv_proj_rows.restype = ctypes.c_int
+            lib.oracle_out_proj_rows.argtypes = [_u16p, _u16p, _dp] + [_i64] * 5 + [_i64p, _i64, _dp]
+            lib.oracle_out_proj_rows.restype = ctypes.c_int
             lib.oracle_lse_merge_f64.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _dp, _dp]
             lib.oracle_lse_merge_f64.restype = None
             lib.oracle_rope3d_f64.argtypes = [_dp, _i64, _i64, _i64, _i64, _i64, ctypes.c_double]
@@ -299,6 +306,60 @@ def dequantize_e4m3(codes, scales, block_rows: int = 128):
     S = v.shape[-2]
     rep = np.repeat(np.asarray(scales, dtype=np.float64), block_rows, axis=-1)[..., :S]
     return v * rep[..., None]
+
+
+def _opt_f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def qkv_proj(x, w, bias, gamma_q, gamma_k, heads: int, grid, theta: float = 10000.0, eps: float = 1e-6,
+             rows=None):
+    """QKV projection of the DiT block for token rows of x [B, S, C] (bf16 bits):
+    y = x W^T + b, split into q | k | v of `heads` heads; per-head RMSNorm
+    (weights gamma_q / gamma_k [H*D], None = 1) and 3D RoPE on q and k.
+    w [3*H*D, C] bf16 bits; bias [3*H*D] float or None. rows: global token ids
+    b*S + s (all if None). Returns q, k, v [len(rows), H, D] in fp64."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    B, S, C = x.shape
+    N = w.shape[0]
+    H = int(heads)
+    D = N // (3 * H)
+    if w.shape != (3 * H * D, C) or 3 * H * D != N:
+        raise ValueError("w must be [3*H*D, C]")
+    T, Hh, Ww = (int(g) for g in grid)
+    r = np.arange(B * S, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    q = np.empty((r.size, H, D)); k = np.empty_like(q); v = np.empty_like(q)
+    b, gq, gk = _opt_f64(bias), _opt_f64(gamma_q), _opt_f64(gamma_k)
+    rc = lib.oracle_qkv_proj_rows(_ptr(x, _u16p), _ptr(w, _u16p), _ptr(b, _dp) if b is not None else None,
+                                  _ptr(gq, _dp) if gq is not None else None, _ptr(gk, _dp) if gk is not None else None,
+                                  B, S, C, H, D, T, Hh, Ww, float(theta), float(eps), _ptr(r, _i64p), r.size,
+                                  _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp))
+    if rc != 0:
+        raise ValueError("bad sizes or row ids")
+    return q, k, v
+
+
+def out_proj(o, w, bias, rows=None):
+    """Output projection y = o W^T + b for token rows, o the attention output
+    [B, H, S, D] (bf16 bits) with heads concatenated per token; w [N, H*D].
+    Returns y [len(rows), N] in fp64 (rows: global token ids, all if None)."""
+    lib = _load()
+    o = np.ascontiguousarray(o, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    B, H, S, D = o.shape
+    N = w.shape[0]
+    if w.shape[1] != H * D:
+        raise ValueError("w must be [N, H*D]")
+    r = np.arange(B * S, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    y = np.empty((r.size, N))
+    b = _opt_f64(bias)
+    rc = lib.oracle_out_proj_rows(_ptr(o, _u16p), _ptr(w, _u16p), _ptr(b, _dp) if b is not None else None,
+                                  B, S, H, D, N, _ptr(r, _i64p), r.size, _ptr(y, _dp))
+    if rc != 0:
+        raise ValueError("bad row ids")
+    return y
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b):

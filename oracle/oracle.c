@@ -404,6 +404,105 @@ void oracle_lse_merge_f64(const double *oa, const double *lsea,
     }
 }
 
+/* --------------------------------------------------------- projections --- */
+
+static void rope_row(double *row, int64_t n, int64_t Hh, int64_t Ww, int64_t D, double theta, int transpose);
+
+/*
+ * The projections around the attention in a DiT block (the decoder's DiT
+ * matches the Wan2.1 architecture: blog page, "Methodology -- deep read"):
+ *   y = x W^T + b,  x one token's row of C model features, W [N][C] (the
+ *   usual linear-layer layout), b [N] or none.
+ * QKV (N = 3 H D): y = [q | k | v], head h of q at columns h D .. h D + D - 1.
+ * q and k then get, per head, RMSNorm over its D values with a weight g
+ * (x / sqrt(mean x^2 + eps) * g; g = 1 when none) and the 3D RoPE of the
+ * token's latent grid position (rope_row above); v is left as is. Reading:
+ * the norm is per head, as in the input preparation of every workload.
+ * Tokens: x [B][S][C] bf16, S = T Hh Ww; rows[] are global token ids b S + s.
+ * Outputs q, k, v [nrows][H][D] in fp64.
+ */
+int oracle_qkv_proj_rows(const uint16_t *x, const uint16_t *w, const double *bias, const double *gq,
+                         const double *gk, int64_t B, int64_t S, int64_t C, int64_t H, int64_t D, int64_t T,
+                         int64_t Hh, int64_t Ww, double theta, double eps, const int64_t *rows, int64_t nrows,
+                         double *q, double *k, double *v)
+{
+    if (T * Hh * Ww != S || D < 6 || (D % 2) != 0) return -1;
+    int64_t N = 3 * H * D;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t tok = rows[r];
+        if (tok < 0 || tok >= B * S) {
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        double *y = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!y) {
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < C; ++c)
+                acc += oracle_bf16_to_f64(x[tok * C + c]) * oracle_bf16_to_f64(w[n * C + c]);
+            y[n] = acc + (bias ? bias[n] : 0.0);
+        }
+        for (int64_t which = 0; which < 3; ++which) {
+            double *dst = which == 0 ? q : which == 1 ? k : v;
+            const double *g = which == 0 ? gq : gk;
+            for (int64_t h = 0; h < H; ++h) {
+                double *src = y + which * H * D + h * D;
+                double *o = dst + (r * H + h) * D;
+                if (which < 2) {
+                    double ms = 0.0;
+                    for (int64_t d = 0; d < D; ++d) ms += src[d] * src[d];
+                    ms /= (double)D;
+                    double inv = 1.0 / sqrt(ms + eps);
+                    for (int64_t d = 0; d < D; ++d) o[d] = src[d] * inv * (g ? g[h * D + d] : 1.0);
+                    rope_row(o, tok % S, Hh, Ww, D, theta, 0);
+                } else {
+                    for (int64_t d = 0; d < D; ++d) o[d] = src[d];
+                }
+            }
+        }
+        free(y);
+    }
+    return failed ? -1 : 0;
+}
+
+/*
+ * Output projection: y = o W^T + b for token rows o of H D values, the
+ * attention output of that token with its heads concatenated:
+ * o[h D + d] = O[b][h][s][d] for O [B][H][S][D]. W [N][H D], b [N] or none.
+ * Output y [nrows][N] in fp64.
+ */
+int oracle_out_proj_rows(const uint16_t *O, const uint16_t *w, const double *bias, int64_t B, int64_t S,
+                         int64_t H, int64_t D, int64_t N, const int64_t *rows, int64_t nrows, double *y)
+{
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t tok = rows[r];
+        if (tok < 0 || tok >= B * S) {
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        int64_t b = tok / S, s = tok % S;
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t h = 0; h < H; ++h)
+                for (int64_t d = 0; d < D; ++d)
+                    acc += oracle_bf16_to_f64(O[((b * H + h) * S + s) * D + d]) *
+                           oracle_bf16_to_f64(w[n * H * D + h * D + d]);
+            y[r * N + n] = acc + (bias ? bias[n] : 0.0);
+        }
+    }
+    return failed ? -1 : 0;
+}
+
 /* ------------------------------------------------------ FP8 (e4m3) --- */
 
 /*
@@ -512,40 +611,42 @@ int oracle_quantize_e4m3(const uint16_t *x, int64_t BH, int64_t S, int64_t D, in
  *        x'_{2j+1} = x_{2j} sin(angle) + x_{2j+1} cos(angle)
  *    (the product of the pair, read as a complex number, with e^{i angle}).
  */
+/* Rotate one row of D values of token n in place (R, or R^T with transpose). */
+static void rope_row(double *row, int64_t n, int64_t Hh, int64_t Ww, int64_t D, double theta, int transpose)
+{
+    int64_t dh = 2 * (D / 6);
+    int64_t dt = D - 2 * dh;
+    int64_t base[3] = {0, dt, dt + dh};
+    int64_t width[3] = {dt, dh, dh};
+    int64_t pos[3];
+    pos[0] = n / (Hh * Ww);
+    pos[1] = (n / Ww) % Hh;
+    pos[2] = n % Ww;
+    for (int a = 0; a < 3; ++a) {
+        for (int64_t j = 0; j < width[a] / 2; ++j) {
+            double angle = (double)pos[a] * pow(theta, -2.0 * (double)j / (double)width[a]);
+            double c = cos(angle), s = sin(angle);
+            double x0 = row[base[a] + 2 * j];
+            double x1 = row[base[a] + 2 * j + 1];
+            if (!transpose) {
+                row[base[a] + 2 * j] = x0 * c - x1 * s;
+                row[base[a] + 2 * j + 1] = x0 * s + x1 * c;
+            } else {
+                /* R^T: the same rotation matrix, transposed */
+                row[base[a] + 2 * j] = c * x0 + s * x1;
+                row[base[a] + 2 * j + 1] = c * x1 - s * x0;
+            }
+        }
+    }
+}
+
 static int rope3d_apply(double *x, int64_t BH, int64_t T, int64_t Hh, int64_t Ww,
                         int64_t D, double theta, int transpose)
 {
     if (D < 6 || (D % 2) != 0) return -1;
-    int64_t dh = 2 * (D / 6);
-    int64_t dt = D - 2 * dh;
     int64_t S = T * Hh * Ww;
-    int64_t base[3] = {0, dt, dt + dh};
-    int64_t width[3] = {dt, dh, dh};
 #pragma omp parallel for schedule(static)
-    for (int64_t g = 0; g < BH * S; ++g) {
-        int64_t n = g % S;
-        int64_t pos[3];
-        pos[0] = n / (Hh * Ww);
-        pos[1] = (n / Ww) % Hh;
-        pos[2] = n % Ww;
-        double *row = x + g * D;
-        for (int a = 0; a < 3; ++a) {
-            for (int64_t j = 0; j < width[a] / 2; ++j) {
-                double angle = (double)pos[a] * pow(theta, -2.0 * (double)j / (double)width[a]);
-                double c = cos(angle), s = sin(angle);
-                double x0 = row[base[a] + 2 * j];
-                double x1 = row[base[a] + 2 * j + 1];
-                if (!transpose) {
-                    row[base[a] + 2 * j] = x0 * c - x1 * s;
-                    row[base[a] + 2 * j + 1] = x0 * s + x1 * c;
-                } else {
-                    /* R^T: the same rotation matrix, transposed */
-                    row[base[a] + 2 * j] = c * x0 + s * x1;
-                    row[base[a] + 2 * j + 1] = c * x1 - s * x0;
-                }
-            }
-        }
-    }
+    for (int64_t g = 0; g < BH * S; ++g) rope_row(x + g * D, g % S, Hh, Ww, D, theta, transpose);
     return 0;
 }
 

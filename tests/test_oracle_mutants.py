@@ -29,8 +29,8 @@ MUTANTS = {
     "merge weights swapped": ("(wa * oa[r * D + d] + wb * ob[r * D + d])",
                               "(wb * oa[r * D + d] + wa * ob[r * D + d])"),
     "rope rotation sign": ("row[base[a] + 2 * j] = x0 * c - x1 * s;", "row[base[a] + 2 * j] = x0 * c + x1 * s;"),
-    "rope h and w swapped": ("pos[1] = (n / Ww) % Hh;\n        pos[2] = n % Ww;",
-                             "pos[1] = n % Ww;\n        pos[2] = (n / Ww) % Hh;"),
+    "rope h and w swapped": ("pos[1] = (n / Ww) % Hh;\n    pos[2] = n % Ww;",
+                             "pos[1] = n % Ww;\n    pos[2] = (n / Ww) % Hh;"),
     "rope frequency exponent": ("-2.0 * (double)j / (double)width[a]", "-1.0 * (double)j / (double)width[a]"),
     "bwd: delta dropped": ("dS[i * Skv + j] = P[i * Skv + j] * (dS[i * Skv + j] - delta);",
                            "dS[i * Skv + j] = P[i * Skv + j] * dS[i * Skv + j];"),
@@ -42,6 +42,11 @@ MUTANTS = {
                                         "row[base[a] + 2 * j + 1] = c * x1 + s * x0;"),
     "e4m3 mantissa width": ("double ulp = ldexp(1.0, e - 3);", "double ulp = ldexp(1.0, e - 2);"),
     "e4m3 quantiser scale not inverted": ("inv = 448.0f / amax;", "inv = amax / 448.0f;"),
+    "proj: norm over the sum, not the mean": ("ms /= (double)D;", ""),
+    "proj: out-proj head and position swapped": ("acc += oracle_bf16_to_f64(O[((b * H + h) * S + s) * D + d]) *",
+                                                 "acc += oracle_bf16_to_f64(O[((b * S + s) * H + h) * D + d]) *"),
+    "proj: rope on v too": ("                } else {\n                    for (int64_t d = 0; d < D; ++d) o[d] = src[d];",
+                            "                } else {\n                    for (int64_t d = 0; d < D; ++d) o[d] = src[d];\n                    rope_row(o, tok % S, Hh, Ww, D, theta, 0);"),
     "rope pair partner index": ("double x1 = row[base[a] + 2 * j + 1];", "double x1 = row[base[a] + j + 1];"),
 }
 

@@ -476,3 +476,67 @@ def test_quantize_e4m3_properties():
     # the block's largest element lands on +-448 (within fp32 rounding of 448/amax)
     assert np.abs(oracle.e4m3_to_f64(codes[0, 0, :128])).max() == 448.0
     assert not codes[1, 2, 128:256].any() and scales[1, 2, 1] == 1.0
+
+
+# ---------------------------------------------------------- projections ---
+
+def _proj_inputs(rng, B=2, S=30, C=48, H=2, D=12):
+    x = oracle.f64_to_bf16(rng.normal(size=(B, S, C)))
+    w = oracle.f64_to_bf16(rng.normal(size=(3 * H * D, C)) / np.sqrt(C))
+    bias = rng.normal(size=3 * H * D) * 0.1
+    gq, gk = 1 + 0.1 * rng.normal(size=H * D), 1 + 0.1 * rng.normal(size=H * D)
+    return x, w, bias, gq, gk
+
+
+def test_qkv_proj_matches_torch_linear_rmsnorm_and_rope():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(11)
+    B, S, C, H, D, grid = 2, 30, 48, 2, 12, (2, 3, 5)
+    x, w, bias, gq, gk = _proj_inputs(rng, B, S, C, H, D)
+    q, k, v = oracle.qkv_proj(x, w, bias, gq, gk, H, grid, 500.0, 1e-6)
+    y = torch.nn.functional.linear(torch.from_numpy(oracle.bf16_to_f64(x)), torch.from_numpy(oracle.bf16_to_f64(w)),
+                                   torch.from_numpy(bias)).view(B, S, 3, H, D)
+    for i, (got, g) in enumerate(((q, gq), (k, gk))):
+        n = torch.nn.functional.rms_norm(y[:, :, i], (D,), eps=1e-6) * torch.from_numpy(g.reshape(H, D))
+        want = oracle.rope3d(n.permute(0, 2, 1, 3).numpy().copy(), grid, 500.0)     # [B, H, S, D]
+        np.testing.assert_allclose(got.reshape(B, S, H, D), want.transpose(0, 2, 1, 3), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(v.reshape(B, S, H, D), y[:, :, 2].numpy(), rtol=1e-12, atol=1e-12)
+    # sampled rows equal the full computation
+    rows = [0, 7, 59, 31]
+    q2, k2, v2 = oracle.qkv_proj(x, w, bias, gq, gk, H, grid, 500.0, 1e-6, rows=rows)
+    np.testing.assert_array_equal(q2, q[rows])
+    np.testing.assert_array_equal(v2, v[rows])
+
+
+def test_qkv_proj_closed_forms():
+    rng = np.random.default_rng(12)
+    B, S, H, D, grid = 1, 6, 2, 12, (1, 2, 3)
+    C = H * D
+    x = oracle.f64_to_bf16(rng.normal(size=(B, S, C)))
+    eye = oracle.f64_to_bf16(np.tile(np.eye(C), (3, 1)))          # W = [I; I; I]
+    q, k, v = oracle.qkv_proj(x, eye, None, None, None, H, grid, 10000.0, 0.0)
+    xf = oracle.bf16_to_f64(x).reshape(S, H, D)
+    np.testing.assert_array_equal(v, xf)                              # v = x
+    np.testing.assert_allclose(q, k, rtol=0, atol=0)
+    # unit RMS per head, then a rotation (norm-preserving): sum of squares = D
+    np.testing.assert_allclose((q ** 2).sum(-1), D, rtol=1e-12)
+    # scale invariance of the normed q (eps = 0), x -> 4 x exactly
+    x4 = oracle.f64_to_bf16(oracle.bf16_to_f64(x) * 4.0)
+    q4, _, v4 = oracle.qkv_proj(x4, eye, None, None, None, H, grid, 10000.0, 0.0)
+    np.testing.assert_allclose(q4, q, rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(v4, 4.0 * v)
+
+
+def test_out_proj_matches_torch_linear():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(13)
+    B, H, S, D, N = 2, 3, 17, 8, 20
+    o = oracle.f64_to_bf16(rng.normal(size=(B, H, S, D)))
+    w = oracle.f64_to_bf16(rng.normal(size=(N, H * D)))
+    bias = rng.normal(size=N)
+    y = oracle.out_proj(o, w, bias)
+    of = torch.from_numpy(oracle.bf16_to_f64(o)).permute(0, 2, 1, 3).reshape(B * S, H * D)
+    want = torch.nn.functional.linear(of, torch.from_numpy(oracle.bf16_to_f64(w)), torch.from_numpy(bias))
+    np.testing.assert_allclose(y, want.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(oracle.out_proj(o, w, None, rows=[5, 33])[1] + bias,
+                                  y[33])
