@@ -277,6 +277,10 @@ def run_native(args, rank, world, local_rank):
     # (prep, dK/dV, dQ).
     bwd = run_backward(args, rg, synth, d, outs0, ws, wc, rank, dev, stream, world, barrier, to_dev)
 
+    # ---- the projections around the attention of a 14B-class DiT block on the same
+    # window: fused QKV projection (+ RMSNorm + RoPE) and the output projection.
+    proj = run_proj(args, rg, synth, ws, dev, stream, world, barrier, to_dev, rank)
+
     # ---- the FP8 variant of the self-attention (after the same RoPE): blockwise
     # E4M3 quantisation of Q, K, V (3 launches) and the E4M3 attention.
     fp8 = run_fp8(args, rg, d, ws, dev, stream, world, barrier)
@@ -451,6 +455,7 @@ def run_native(args, rank, world, local_rank):
     }
     line["backward"] = bwd
     line["fp8"] = fp8
+    line["projections"] = proj
     line["rope_fused_step"] = {
         "what": "the same step with regen_attn_fwd_rope3d (RoPE fused into the Q tile load, K rotated into "
                 "workspace) in place of regen_rope3d + regen_attn_fwd; 7 launches per step",
@@ -535,6 +540,87 @@ def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, bar
                      "frac": round(achieved / peak, 4),
                      "peak_source": f"{pk_src} bf16_tflops_sustained",
                      "issued_tensor_flops_frac": round(achieved * 7 / 5 / peak, 4)},
+    }
+
+
+C_MODEL = 5120   # model width of the 14B-class DiT (40 heads x 128)
+
+
+def run_proj(args, rg, synth, ws, dev, stream, world, barrier, to_dev, rank):
+    """Times regen_qkv_proj and regen_out_proj on the 77-frame window of a 14B-class
+    DiT block (C = 5120, 40 heads); a cuBLAS GEMM of the same shapes is timed beside
+    them for comparison only. Returns the JSON object."""
+    import torch
+    B, H, S, D = ws.B, ws.H, ws.Sq, ws.D
+    T, Hh, Ww = ws.grid
+    C = C_MODEL
+    sh = stream.cuda_stream
+    seed = 100 + rank
+    x = to_dev(synth._normal_bf16(seed, 0, (B, S, C), False))
+    w = to_dev(synth.f64_to_bf16_bits(synth.normal(seed, 1, 3 * H * D * C).reshape(3 * H * D, C) / math.sqrt(C)))
+    wo = to_dev(synth.f64_to_bf16_bits(synth.normal(seed, 2, C * H * D).reshape(C, H * D) / math.sqrt(H * D)))
+    bias = torch.from_numpy((synth.normal(seed, 3, 3 * H * D) * 0.1).astype(np.float32)).to(dev)
+    bo = torch.from_numpy((synth.normal(seed, 4, C) * 0.1).astype(np.float32)).to(dev)
+    q, k, v = (torch.empty((B, H, S, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    y = torch.empty((B, S, C), dtype=torch.bfloat16, device=dev)
+    o = to_dev(synth._normal_bf16(seed, 5, (B, H, S, D), False))
+    wsb = rg.regen_qkv_proj_workspace_bytes(T, Hh, Ww, D)
+    work = torch.empty(wsb, dtype=torch.uint8, device=dev)
+
+    def qkv():
+        rg.regen_qkv_proj(x, w, bias, None, None, q, k, v, B, S, C, H, D, T, Hh, Ww, ws.theta, 1e-6, sh, work, wsb)
+
+    def outp():
+        rg.regen_out_proj(o, wo, bo, y, B, S, H, D, C, sh)
+
+    xm = x.view(B * S, C)
+    om = o.permute(0, 2, 1, 3).reshape(B * S, H * D).contiguous()
+    res = torch.empty((B * S, 3 * H * D), dtype=torch.bfloat16, device=dev)
+    reso = torch.empty((B * S, C), dtype=torch.bfloat16, device=dev)
+
+    def cublas_qkv():
+        torch.matmul(xm, w.t(), out=res)
+
+    def cublas_out():
+        torch.matmul(om, wo.t(), out=reso)
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev) / n
+
+    n = max(5, min(args.steps, 40))
+    t_qkv, t_out = timed(qkv, n), timed(outp, n)
+    t_cq, t_co = timed(cublas_qkv, n), timed(cublas_out, n)
+    f_qkv = 2.0 * B * S * C * 3 * H * D
+    f_out = 2.0 * B * S * H * D * C
+    pk, pk_src = peaks()
+    peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
+    tf = lambda f, ms: f / (ms * 1e-3) / 1e12  # noqa: E731
+    del work, x, w, wo, o, q, k, v, y, res, reso, om
+    return {
+        "what": "DiT block projections on the 77-frame window, 14B-class (C = 5120, 40 heads x 128): regen_qkv_proj "
+                "(x W^T + b, per-head RMSNorm + 3D RoPE on q and k, q/k/v written as [B,H,S,128]) and regen_out_proj "
+                "(attention output read in place as token rows); a plain cuBLAS GEMM of each shape (torch.matmul, "
+                "no epilogue) timed beside them for comparison only",
+        "steps": n,
+        "qkv_proj": {"ms": round(t_qkv, 4), "tflops": round(tf(f_qkv, t_qkv), 2), "M": B * S, "N": 3 * H * D, "K": C,
+                     "cublas_gemm_ms": round(t_cq, 4), "cublas_tflops": round(tf(f_qkv, t_cq), 2)},
+        "out_proj": {"ms": round(t_out, 4), "tflops": round(tf(f_out, t_out), 2), "M": B * S, "N": C, "K": H * D,
+                     "cublas_gemm_ms": round(t_co, 4), "cublas_tflops": round(tf(f_out, t_co), 2)},
+        "roofline": {"bound": "tensor", "kernel": "proj_gemm_kernel<QKV> (31200 x 15360 x 5120)",
+                     "achieved": round(tf(f_qkv, t_qkv), 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(tf(f_qkv, t_qkv) / peak, 4), "peak_source": f"{pk_src} bf16_tflops_sustained"},
+        "launches_per_step": 3,
     }
 
 

@@ -19,6 +19,9 @@ Entry points (same names as the C ABI):
     regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream=None)
     regen_quant_e4m3(x, codes, scales, B, H, S, D, stream=None)
     regen_attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, B, H, Sq, Skv, D, scale, stream=None)
+    regen_qkv_proj(x, w, bias, gamma_q, gamma_k, q, k, v, B, S, C, H, D, T, Hh, Ww, theta, eps, stream,
+                   workspace, workspace_bytes);  regen_qkv_proj_workspace_bytes(T, Hh, Ww, D)
+    regen_out_proj(o, w, bias, y, B, S, H, D, N, stream=None)
     regen_last_device_error() -> (status, site)
     regen_set_wait_limit_ns(ns)
 Convenience wrappers that allocate outputs with torch:
@@ -29,6 +32,8 @@ Convenience wrappers that allocate outputs with torch:
     attn_bwd(q, k, v, out, lse, dout, scale=None) -> (dq, dk, dv)
     rope3d_bwd_(dq, dk, grid, theta=10000.0)
     quant_e4m3(x) -> (codes, scales);  attn_fwd_fp8(q8, qs, k8, ks, v8, vs, scale=None) -> (out, lse)
+    qkv_proj(x, w, heads, grid, bias=None, gamma_q=None, gamma_k=None) -> (q, k, v)
+    out_proj(o, w, bias=None) -> y
 """
 from __future__ import annotations
 
@@ -42,7 +47,8 @@ __all__ = [
     "regen_status_str", "regen_last_device_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
     "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes", "regen_attn_fwd_rope3d_noalloc",
     "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd", "regen_quant_e4m3",
-    "regen_attn_fwd_fp8", "quant_e4m3", "attn_fwd_fp8",
+    "regen_attn_fwd_fp8", "quant_e4m3", "attn_fwd_fp8", "regen_qkv_proj", "regen_qkv_proj_workspace_bytes",
+    "regen_out_proj", "qkv_proj", "out_proj",
     "attn_fwd", "attn_fwd_rope3d", "rope3d_", "lse_merge", "attn_bwd", "rope3d_bwd_", "STATUS",
 ]
 
@@ -100,6 +106,12 @@ def load():
         L.regen_quant_e4m3.restype = i32
         L.regen_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
         L.regen_attn_fwd_fp8.restype = i32
+        L.regen_qkv_proj.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp] + [i32] * 8 + [f32, f32, vp, vp, i64]
+        L.regen_qkv_proj.restype = i32
+        L.regen_qkv_proj_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.regen_qkv_proj_workspace_bytes.restype = i64
+        L.regen_out_proj.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
+        L.regen_out_proj.restype = i32
         L.regen_status_str.argtypes = [i32]
         L.regen_status_str.restype = ctypes.c_char_p
         L.regen_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
@@ -222,6 +234,25 @@ def regen_attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, B, H, Sq
     _check(load().regen_attn_fwd_fp8(_ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v8), _ptr(v_scale),
                                      _ptr(out), _ptr(lse), B, H, Sq, Skv, D, float(scale), _stream(stream)),
            "regen_attn_fwd_fp8")
+
+
+def regen_qkv_proj(x, w, bias, gamma_q, gamma_k, q, k, v, B, S, C, H, D, T, Hh, Ww, theta, eps, stream,
+                   workspace, workspace_bytes) -> None:
+    _check(load().regen_qkv_proj(_ptr(x), _ptr(w), _ptr(bias), _ptr(gamma_q), _ptr(gamma_k), _ptr(q), _ptr(k),
+                                 _ptr(v), B, S, C, H, D, T, Hh, Ww, float(theta), float(eps), _stream(stream),
+                                 _ptr(workspace), int(workspace_bytes)), "regen_qkv_proj")
+
+
+def regen_qkv_proj_workspace_bytes(T, Hh, Ww, D) -> int:
+    n = load().regen_qkv_proj_workspace_bytes(T, Hh, Ww, D)
+    if n < 0:
+        raise RegenError(int(n), "regen_qkv_proj_workspace_bytes")
+    return int(n)
+
+
+def regen_out_proj(o, w, bias, y, B, S, H, D, N, stream=None) -> None:
+    _check(load().regen_out_proj(_ptr(o), _ptr(w), _ptr(bias), _ptr(y), B, S, H, D, N, _stream(stream)),
+           "regen_out_proj")
 
 
 def regen_selftest_exp2(x, y, n, stream=None) -> None:
@@ -379,3 +410,36 @@ def attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, scale=None, out=None, ls
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q8.device)
     regen_attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, B, H, Sq, Skv, D, scale, stream)
     return out, lse
+
+
+def qkv_proj(x, w, heads, grid, bias=None, gamma_q=None, gamma_k=None, theta=10000.0, eps=1e-6, q=None, k=None,
+             v=None, workspace=None, stream=None):
+    """Fused QKV projection of bf16 token features x [B, S, C] with w [3*heads*128, C]
+    -> q, k, v [B, heads, S, 128] (RMSNorm + 3D RoPE on q and k)."""
+    import torch
+    if x.dim() != 3 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous [B, S, C] tensor")
+    B, S, C = x.shape
+    T, Hh, Ww = grid
+    H, D = int(heads), 128
+    shape = (B, H, S, D)
+    q = torch.empty(shape, dtype=torch.bfloat16, device=x.device) if q is None else q
+    k = torch.empty(shape, dtype=torch.bfloat16, device=x.device) if k is None else k
+    v = torch.empty(shape, dtype=torch.bfloat16, device=x.device) if v is None else v
+    need = regen_qkv_proj_workspace_bytes(T, Hh, Ww, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    regen_qkv_proj(x, w, bias, gamma_q, gamma_k, q, k, v, B, S, C, H, D, T, Hh, Ww, theta, eps, stream, workspace,
+                   workspace.numel() * workspace.element_size())
+    return q, k, v
+
+
+def out_proj(o, w, bias=None, y=None, stream=None):
+    """Output projection of the attention output o [B, H, S, 128] with w [N, H*128]
+    -> y [B, S, N] bf16."""
+    import torch
+    B, H, S, D = _bhsd(o, "o")
+    N = w.shape[0]
+    y = torch.empty((B, S, N), dtype=torch.bfloat16, device=o.device) if y is None else y
+    regen_out_proj(o, w, bias, y, B, S, H, D, N, stream)
+    return y

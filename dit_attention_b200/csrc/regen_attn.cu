@@ -21,6 +21,7 @@
 #include "attn_fp8.cuh"
 #include "attn_fwd.cuh"
 #include "lse_merge.cuh"
+#include "proj_gemm.cuh"
 #include "rope3d.cuh"
 
 namespace {
@@ -83,6 +84,56 @@ bool make_u8_map(CUtensorMap *map, const void *base, int64_t BH, int64_t S)
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// bf16 [d2][d1][d0] (d0 innermost) as a 3D tensor with boxes of box0 x box1 x 1
+// and the 128-byte swizzle (box0 = 64: one 128-byte row); out-of-range reads zero.
+bool make_bf16_map3(CUtensorMap *map, const void *base, int64_t d0, int64_t d1, int64_t d2, uint32_t box0,
+                    uint32_t box1)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1), static_cast<cuuint64_t>(d2)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d0 * 2), static_cast<cuuint64_t>(d0 * d1 * 2)};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+template <int MODE>
+int launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const regen::ProjShape &shape,
+                const regen::ProjEpi &ep, cudaStream_t stream)
+{
+    using C = regen::ProjCfg;
+    static std::once_flag once;
+    static int attr_status = REGEN_OK;
+    std::call_once(once, [] {
+        cudaFuncAttributes fa;
+        if (cudaFuncSetAttribute(regen::proj_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, regen::proj_gemm_kernel<MODE>) != cudaSuccess)
+            attr_status = REGEN_ERR_CUDA;
+        else if (fa.numRegs < C::MIN_LAUNCH_REGS)
+            attr_status = REGEN_ERR_UNSUPPORTED;
+    });
+    if (attr_status != REGEN_OK) return attr_status;
+    const int64_t total = static_cast<int64_t>(shape.num_mt) * shape.num_nt;
+    const int sms = num_sms();
+    if (sms <= 0) return REGEN_ERR_CUDA;
+    const int grid = static_cast<int>(total < sms ? total : sms);
+    regen::proj_gemm_kernel<MODE><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, shape, ep, g_wait_limit_ns.load());
+    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
 }
 
 template <bool NEG>
@@ -578,6 +629,80 @@ REGEN_API int regen_attn_fwd_fp8(const uint8_t *q8, const float *q_scale, const 
     }
     return scale < 0.0f ? launch_attn_fp8<true>(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, BH, Sq, Skv, scale, st)
                         : launch_attn_fp8<false>(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, BH, Sq, Skv, scale, st);
+}
+
+REGEN_API int64_t regen_qkv_proj_workspace_bytes(int T, int Hh, int Ww, int D)
+{
+    if (T <= 0 || Hh <= 0 || Ww <= 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (D != 128) return REGEN_ERR_UNSUPPORTED;
+    return (regen::RopeGeom::make(T, Hh, Ww, D).entries() * 8 + 255) / 256 * 256;
+}
+
+REGEN_API int regen_qkv_proj(const regen_bf16 *x, const regen_bf16 *w, const float *bias, const float *gamma_q,
+                             const float *gamma_k, regen_bf16 *q, regen_bf16 *k, regen_bf16 *v, int B, int S, int C,
+                             int H, int D, int T, int Hh, int Ww, float theta, float eps, regen_stream_t stream,
+                             void *workspace, int64_t workspace_bytes)
+{
+    if (B < 0 || S < 0 || C < 0 || H < 0 || D < 0 || T <= 0 || Hh <= 0 || Ww <= 0 || workspace_bytes < 0)
+        return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(theta) || !(theta > 0.0f) || !std::isfinite(eps) || eps < 0.0f) return REGEN_ERR_INVALID_ARG;
+    if (D != 128 || (C % 8) != 0) return REGEN_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(T) * Hh * Ww != S) return REGEN_ERR_INVALID_ARG;
+    if (B == 0 || S == 0 || H == 0) return REGEN_OK;
+    const int64_t N = 3LL * H * 128;
+    if (C == 0 || N > 0x7FFFFFFF || static_cast<int64_t>(B) * H > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (!x || !w || !q || !k || !v || !workspace) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(bias) ||
+        !aligned16(gamma_q) || !aligned16(gamma_k) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return REGEN_ERR_MISALIGNED;
+    const regen::RopeGeom geom = regen::RopeGeom::make(T, Hh, Ww, D);
+    const int64_t tab_bytes = geom.entries() * 8;
+    if (workspace_bytes < tab_bytes) return REGEN_ERR_INVALID_ARG;
+    const int64_t xb = static_cast<int64_t>(B) * S * C * 2, wb = N * C * 2, ob = static_cast<int64_t>(B) * H * S * 256;
+    struct Span { const void *p; int64_t n; };
+    const Span ins[6] = {{x, xb}, {w, wb}, {bias, N * 4}, {gamma_q, H * 512LL}, {gamma_k, H * 512LL}, {workspace, tab_bytes}};
+    const Span outs[3] = {{q, ob}, {k, ob}, {v, ob}};
+    for (int a = 0; a < 3; ++a) {
+        for (const Span &in : ins)
+            if (overlaps(outs[a].p, outs[a].n, in.p, in.n)) return REGEN_ERR_INVALID_ARG;
+        for (int b2 = a + 1; b2 < 3; ++b2)
+            if (overlaps(outs[a].p, outs[a].n, outs[b2].p, outs[b2].n)) return REGEN_ERR_INVALID_ARG;
+    }
+    for (int a = 0; a < 5; ++a)
+        if (overlaps(workspace, tab_bytes, ins[a].p, ins[a].n)) return REGEN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float2 *tab = static_cast<float2 *>(workspace);
+    regen::rope_table_f32_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
+    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    CUtensorMap ta, tb;
+    if (!make_bf16_map3(&ta, x, C, S, B, 64, 128) || !make_bf16_map3(&tb, w, C, N, 1, 64, 256)) return REGEN_ERR_CUDA;
+    regen::ProjShape shape{B, S, C, static_cast<int>(N), H, B * ((S + 127) / 128), static_cast<int>((N + 255) / 256)};
+    regen::ProjEpi ep{bias, gamma_q, gamma_k, q, k, v, tab, geom, eps};
+    return launch_proj<regen::PROJ_QKV>(ta, tb, shape, ep, st);
+}
+
+REGEN_API int regen_out_proj(const regen_bf16 *o, const regen_bf16 *w, const float *bias, regen_bf16 *y, int B,
+                             int S, int H, int D, int N, regen_stream_t stream)
+{
+    if (B < 0 || S < 0 || H < 0 || D < 0 || N < 0) return REGEN_ERR_INVALID_ARG;
+    if (D != 128 || (N % 8) != 0) return REGEN_ERR_UNSUPPORTED;
+    if (B == 0 || S == 0 || N == 0) return REGEN_OK;
+    if (H == 0) return REGEN_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * H > 0x7FFFFFFF || static_cast<int64_t>(H) * 128 > 0x7FFFFFFF)
+        return REGEN_ERR_UNSUPPORTED;
+    if (!o || !w || !y) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(o) || !aligned16(w) || !aligned16(y) || !aligned16(bias)) return REGEN_ERR_MISALIGNED;
+    const int64_t K = static_cast<int64_t>(H) * 128;
+    const int64_t obytes = static_cast<int64_t>(B) * H * S * 256, wbytes = N * K * 2,
+                  ybytes = static_cast<int64_t>(B) * S * N * 2;
+    if (overlaps(y, ybytes, o, obytes) || overlaps(y, ybytes, w, wbytes) || overlaps(y, ybytes, bias, N * 4LL))
+        return REGEN_ERR_INVALID_ARG;
+    CUtensorMap ta, tb;
+    if (!make_bhsd_map(&ta, o, static_cast<int64_t>(B) * H, S, 128) || !make_bf16_map3(&tb, w, K, N, 1, 64, 256))
+        return REGEN_ERR_CUDA;
+    regen::ProjShape shape{B, S, static_cast<int>(K), N, H, B * ((S + 127) / 128), (N + 255) / 256};
+    regen::ProjEpi ep{bias, nullptr, nullptr, y, nullptr, nullptr, nullptr, regen::RopeGeom{}, 0.0f};
+    return launch_proj<regen::PROJ_OUT>(ta, tb, shape, ep, reinterpret_cast<cudaStream_t>(stream));
 }
 
 REGEN_API int regen_selftest_exp2(const float *x, float *y, int64_t n, regen_stream_t stream)

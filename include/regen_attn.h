@@ -260,6 +260,47 @@ REGEN_API int regen_attn_fwd_fp8(const uint8_t *q8, const float *q_scale, const 
                                  int B, int H, int Sq, int Skv, int D, float scale, regen_stream_t stream);
 
 /*
+ * regen_qkv_proj -- the QKV projection that feeds the self-attention of a DiT
+ * block (the decoder's DiT matches the Wan2.1 architecture: blog page,
+ * "Methodology -- deep read"), fused with the per-head QK RMSNorm and the 3D
+ * RoPE, writing q, k, v in the attention's [B, H, S, 128] layout:
+ *     y = x W^T + b                     (bf16 tensor-core products, fp32 accumulate)
+ *     [q | k | v] = y, head h of q at features h*128 .. h*128+127
+ *     q_h <- RoPE( q_h / sqrt(mean(q_h^2) + eps) * gamma_q[h*128 ..] ), likewise k; v as is
+ * with RoPE as in regen_rope3d (here in fp32 from an fp64-computed table) and
+ * one rounding of each result to bf16.
+ *
+ *   x        [B, S, C] bf16 token features, S = T*Hh*Ww (else REGEN_ERR_INVALID_ARG)
+ *   w        [3*H*128, C] bf16 (row n = output feature n);  C multiple of 8
+ *   bias     [3*H*128] fp32 or NULL;  gamma_q, gamma_k  [H*128] fp32 or NULL (= 1)
+ *   q, k, v  [B, H, S, 128] bf16 outputs (must not overlap anything else)
+ *   D        must be 128 (else REGEN_ERR_UNSUPPORTED);  eps >= 0;  theta > 0
+ *   workspace  >= regen_qkv_proj_workspace_bytes(T, Hh, Ww, D) bytes, 256-byte
+ *            aligned, caller-owned (the RoPE table); overwritten
+ * All pointers 16-byte aligned. B, S or H == 0: REGEN_OK, nothing done.
+ */
+REGEN_API int regen_qkv_proj(const regen_bf16 *x, const regen_bf16 *w, const float *bias, const float *gamma_q,
+                             const float *gamma_k, regen_bf16 *q, regen_bf16 *k, regen_bf16 *v,
+                             int B, int S, int C, int H, int D, int T, int Hh, int Ww, float theta, float eps,
+                             regen_stream_t stream, void *workspace, int64_t workspace_bytes);
+
+/* Bytes of workspace regen_qkv_proj needs, or a negative status. */
+REGEN_API int64_t regen_qkv_proj_workspace_bytes(int T, int Hh, int Ww, int D);
+
+/*
+ * regen_out_proj -- the output projection after the attention, reading its
+ * output in place: y[b, s, :] = o_tok W^T + b where o_tok[h*128 + d] =
+ * o[b, h, s, d] (the heads of one token concatenated).
+ *
+ *   o     [B, H, S, 128] bf16 (the attention output);  D must be 128
+ *   w     [N, H*128] bf16;  bias [N] fp32 or NULL;  N multiple of 8
+ *   y     [B, S, N] bf16 output (must not overlap o, w, bias)
+ * All pointers 16-byte aligned. B, S or N == 0: REGEN_OK, nothing done.
+ */
+REGEN_API int regen_out_proj(const regen_bf16 *o, const regen_bf16 *w, const float *bias, regen_bf16 *y,
+                             int B, int S, int H, int D, int N, regen_stream_t stream);
+
+/*
  * regen_selftest_exp2 -- diagnostic: evaluates, for each x[i], the FMA-pipe
  * 2^x that the attention kernel uses for part of its softmax probabilities
  * (degree-4 polynomial after Cody-Waite range reduction; inputs below -127

@@ -185,3 +185,38 @@ def test_attn_fwd_fp8_validation(lib, args, status):
     rc = lib.regen_attn_fwd_fp8(a["q8"], a["qs"], a["k8"], a["ks"], a["v8"], a["vs"], a["out"], a["lse"], a["B"],
                                 a["H"], a["Sq"], a["Skv"], a["D"], a["scale"], None)
     assert rc == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=64), -2), (dict(C=100), -2), (dict(S=61), -1), (dict(theta=0.0), -1), (dict(eps=-1.0), -1),
+    (dict(x=None), -1), (dict(ws=None), -1), (dict(wsb=16), -1), (dict(bias=FAKE + 40 * MB + 4), -3),
+    (dict(ws=FAKE + 90 * MB + 64), -3), (dict(q=FAKE + 4096), -1), (dict(k=FAKE + 50 * MB + 1024), -1),
+    (dict(ws=FAKE + 10 * MB), -1), (dict(B=0), 0), (dict(H=0, x=None), 0),
+])
+def test_qkv_proj_validation(lib, args, status):
+    # x [1, 60, 256]; w [3*2*128, 256]; grid 3x4x5
+    a = dict(x=FAKE, w=FAKE + 10 * MB, bias=FAKE + 40 * MB, gq=None, gk=None, q=FAKE + 50 * MB, k=FAKE + 60 * MB,
+             v=FAKE + 70 * MB, B=1, S=60, C=256, H=2, D=128, T=3, Hh=4, Ww=5, theta=1e4, eps=1e-6,
+             ws=FAKE + 90 * MB, wsb=4096)
+    a.update(args)
+    rc = lib.regen_qkv_proj(a["x"], a["w"], a["bias"], a["gq"], a["gk"], a["q"], a["k"], a["v"], a["B"], a["S"],
+                            a["C"], a["H"], a["D"], a["T"], a["Hh"], a["Ww"], a["theta"], a["eps"], None, a["ws"],
+                            a["wsb"])
+    assert rc == status
+
+
+def test_qkv_proj_workspace_bytes(lib):
+    # (20*22 + 30*21 + 52*21) entries of (cos, sin) fp32, rounded up to 256 bytes
+    assert rg.regen_qkv_proj_workspace_bytes(20, 30, 52, 128) == -(-(440 + 630 + 1092) * 8 // 256) * 256
+    assert lib.regen_qkv_proj_workspace_bytes(2, 3, 4, 64) == -2
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=64), -2), (dict(N=100), -2), (dict(H=0), -1), (dict(o=None), -1), (dict(y=FAKE + 8), -3),
+    (dict(y=FAKE + 4096), -1), (dict(y=FAKE + 10 * MB), -1), (dict(B=0), 0), (dict(N=0), 0),
+])
+def test_out_proj_validation(lib, args, status):
+    a = dict(o=FAKE, w=FAKE + 10 * MB, bias=None, y=FAKE + 30 * MB, B=1, S=60, H=2, D=128, N=256)
+    a.update(args)
+    rc = lib.regen_out_proj(a["o"], a["w"], a["bias"], a["y"], a["B"], a["S"], a["H"], a["D"], a["N"], None)
+    assert rc == status

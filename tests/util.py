@@ -165,3 +165,17 @@ def check_fp8_attention(out_bits, lse_gpu, qd, kd, vd, scale, rows=None, label="
     assert err.mean() <= sigma.mean() + 2.0 ** -8 * np.abs(ref).mean(), f"{label}: mean error {diag}"
     assert lse_err.max() <= LSE_ATOL, f"{label}: lse {diag}"
     return diag
+
+
+def check_proj(got_bits, ref, label=""):
+    """Projection contract: bf16 x bf16 products are exact in fp32, sums in fp32
+    (relative ~1e-6 of the sum of |products|), one rounding of the result to
+    bf16 (2^-9 relative): |got - ref| <= 2^-8 |ref| + 2e-3 rms(ref)."""
+    got = bits_to_f64(got_bits).reshape(ref.shape)
+    err = np.abs(got - ref)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    diag = {"max_err_over_rms": float(err.max() / rms), "mean_err_over_rms": float(err.mean() / rms), "rms_ref": rms}
+    bad = err > 2.0 ** -8 * np.abs(ref) + 2e-3 * rms
+    assert np.all(np.isfinite(got)), f"{label}: non-finite"
+    assert not bad.any(), f"{label}: {int(bad.sum())} of {bad.size} out of tolerance; {diag}"
+    return diag
