@@ -13,14 +13,21 @@
 //         token rows of H*128 features (one TMA box per (head, 64 values)), W
 //         [N][H 128]; y [B][S][N].
 //
-// One persistent CTA per SM walks 128-token x 256-feature tiles in groups of
-// 8 token tiles (so the CTAs in flight share A and W in L2). Warp 0 is the
-// TMA producer (A 128 x 64 and B 256 x 64 bf16 per stage, 4 stages), warp 1
-// owns TMEM and issues the M128 N256 K16 MMAs into one of two 256-column
-// accumulators, and two epilogue warpgroups (warps 4-7, 8-11) each drain one
-// accumulator, so a tile's epilogue overlaps the next tile's main loop. In the
-// epilogue a thread owns one token row: the RMSNorm of a 128-value head needs
-// no reduction across threads, and each thread stores its rows directly.
+// Pairs of SMs (clusters of 2 CTAs, tcgen05 cta_group::2) walk persistently
+// over 256-token x 256-feature tiles, in groups of 8 token tiles (so the pairs
+// in flight share A and W in L2). Each CTA holds its own 128 token rows of A
+// and one 128-feature half of B per stage (6 stages, 32 KB each), loaded by
+// its warp 0 with the pair form of the TMA load, all completing on the even
+// CTA's stage barrier; the even CTA's warp 1 issues M256 N256 K16 MMAs over
+// both CTAs' shared memory into one of two 256-column accumulators per CTA
+// (each CTA's TMEM holds its own 128 rows), and releases stages and
+// accumulators to both CTAs with multicast commits. Two epilogue warpgroups
+// per CTA (warps 4-7, 8-11) each drain one accumulator, so a tile's epilogue
+// overlaps the next tile's main loop; the odd CTA's epilogue reports to the
+// even CTA's barrier. Per SM this halves the B operand bytes a 128 x 256 tile
+// of one CTA would read. In the epilogue a thread owns one token row: the
+// RMSNorm of a 128-value head needs no reduction across threads, and each
+// thread stores its rows directly. No load multicasts.
 #pragma once
 
 #include "attn_fwd.cuh"
@@ -34,14 +41,15 @@ enum ProjMode : int { PROJ_QKV = 0, PROJ_OUT = 1 };
 struct ProjShape {
     int B, S, K, N;     // tokens per batch S, input features K, output features N
     int H;              // heads: of q/k/v (QKV) or of the attention output read as A (OUT)
-    int num_mt, num_nt; // tiles along tokens (per batch, ceil(S/128) each) and features (ceil(N/256))
+    int num_mt, num_nt; // pair tiles along tokens (per batch, ceil(S/256) each) and features (ceil(N/256))
 };
 
 struct ProjCfg {
-    static constexpr int BM = 128, BN = 256, BK = 64;
-    static constexpr int NS = 4;
-    static constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-    static constexpr int B_BYTES = BN * BK * 2;   // 32 KB
+    static constexpr int BM = 128, BN = 256, BK = 64;   // per CTA: 128 tokens; per pair: 256 x 256
+    static constexpr int PAIR_M = 2 * BM;
+    static constexpr int NS = 6;
+    static constexpr int A_BYTES = BM * BK * 2;         // 16 KB: this CTA's 128 token rows
+    static constexpr int B_BYTES = (BN / 2) * BK * 2;   // 16 KB: this CTA's 128-feature half
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = NS * A_BYTES;
     static constexpr int BAR_OFF = B_OFF + NS * B_BYTES;
@@ -127,78 +135,83 @@ __global__ void __launch_bounds__(384, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 8);
 
+    const uint32_t rank = cluster_ctarank();   // 0: the pair's MMA issuer
+    const bool leader = rank == 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NS; ++s) {
-            mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 1);
+            mbar_init(bar_full(s), 1);         // the leader's: both CTAs' loads complete on it
+            mbar_init(bar_empty(s), 1);        // each CTA's: the leader's multicast commit
         }
         for (int e = 0; e < 2; ++e) {
-            mbar_init(bar_acc_full(e), 1);
-            mbar_init(bar_acc_empty(e), 128);
+            mbar_init(bar_acc_full(e), 1);     // each CTA's: multicast commit
+            mbar_init(bar_acc_empty(e), 256);  // the leader's: both CTAs' epilogue threads
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before_sync();
     __syncthreads();
+    cluster_sync_all();    // both CTAs' barriers exist before any remote use
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
     const WaitCtl wc{abort_flag, wait_limit_ns};
     const int total = p.num_mt * p.num_nt;
     const int kblocks = (p.K + C::BK - 1) / C::BK;
-    const int mpb = (p.S + C::BM - 1) / C::BM;   // token tiles per batch
+    const int mpb = (p.S + C::PAIR_M - 1) / C::PAIR_M;   // pair tiles per batch along tokens
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (warp < 4) {
     setmaxnreg_dec<C::REGS_LOW>();
     if (warp == 0) {
         // ------------------------------------------------------ producer ---
+        // Each CTA loads its own A rows and B half; both complete on the
+        // leader's stage barrier, where the leader posts both CTAs' bytes.
         if (lane == 0) {
             tma_prefetch_desc(&tm_a);
             tma_prefetch_desc(&tm_b);
             const uint64_t keep = l2_policy_evict_last();
-            int it = 0, issued = 0;
+            int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+            for (int t = pair; ok && t < total; t += npairs) {
                 int mt, nt;
                 proj_tile(t, p, mt, nt);
-                const int b = mt / mpb, s0 = (mt % mpb) * C::BM, n0 = nt * C::BN;
+                const int b = mt / mpb, s0 = (mt % mpb) * C::PAIR_M + static_cast<int>(rank) * C::BM;
+                const int nb0 = nt * C::BN + static_cast<int>(rank) * (C::BN / 2);
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const int s = it % C::NS;
                     ok = wait_phase(bar_empty(s), ((it / C::NS) & 1) ^ 1, SITE_PROJ_PROD, wc);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(bar_full(s), C::A_BYTES + C::B_BYTES);
+                    const uint32_t full_leader = mapa_shared(bar_full(s), 0);
+                    if (leader) mbar_arrive_expect_tx(bar_full(s), 2 * (C::A_BYTES + C::B_BYTES));
                     if constexpr (MODE == PROJ_QKV)
-                        tma_load_3d(sbase + C::A_OFF + s * C::A_BYTES, &tm_a, bar_full(s), kb * C::BK, s0, b, keep);
+                        tma_load_3d_pair(sbase + C::A_OFF + s * C::A_BYTES, &tm_a, full_leader, kb * C::BK, s0, b, keep);
                     else  // the attention output: k block kb = (head kb/2, values 64 (kb%2) ..)
-                        tma_load_3d(sbase + C::A_OFF + s * C::A_BYTES, &tm_a, bar_full(s), (kb & 1) * 64, s0,
-                                    b * p.H + (kb >> 1), keep);
-                    tma_load_3d(sbase + C::B_OFF + s * C::B_BYTES, &tm_b, bar_full(s), kb * C::BK, n0, 0, keep);
-                    ++issued;
+                        tma_load_3d_pair(sbase + C::A_OFF + s * C::A_BYTES, &tm_a, full_leader, (kb & 1) * 64, s0,
+                                         b * p.H + (kb >> 1), keep);
+                    tma_load_3d_pair(sbase + C::B_OFF + s * C::B_BYTES, &tm_b, full_leader, kb * C::BK, nb0, 0, keep);
                 }
             }
             if (!ok) {
-                const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
-                for (int i = (issued > C::NS ? issued - C::NS : 0); i < issued; ++i) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar_full(i % C::NS), (i / C::NS) & 1) &&
-                           global_timer_ns() - t0 < drain_ns) {
-                    }
+                // Aborting: the copies in flight land in this CTA's memory within
+                // microseconds; give them a bounded moment before the CTA leaves.
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 1000000ull) {
                 }
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------- MMA issuer ---
-        if (lane == 0) {
-            constexpr uint32_t IDESC = idesc_bf16_f32(128, 256, false);   // both K-major
+        // ------------------------------------------ MMA issuer (leader only) ---
+        if (lane == 0 && leader) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(256, 256, false);   // M over the pair; both K-major
             int it = 0, local = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < total; t += gridDim.x, ++local) {
+            for (int t = pair; ok && t < total; t += npairs, ++local) {
                 const int e = local & 1;
                 ok = wait_phase(bar_acc_empty(e), ((local >> 1) & 1) ^ 1, SITE_PROJ_MMA, wc);
                 if (!ok) break;
@@ -213,13 +226,13 @@ __global__ void __launch_bounds__(384, 1)
                     const uint32_t bb = sbase + C::B_OFF + s * C::B_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < C::BK / 16; ++kk)
-                        mma_ss(acc, smem_desc_sw128(a + kk * 32, 16, 1024), smem_desc_sw128(bb + kk * 32, 16, 1024),
-                               IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(bar_empty(s));
+                        mma_ss_pair(acc, smem_desc_sw128(a + kk * 32, 16, 1024), smem_desc_sw128(bb + kk * 32, 16, 1024),
+                                    IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit_pair(bar_empty(s), 0x3);
                 }
-                if (ok) tc_commit(bar_acc_full(e));
+                if (ok) tc_commit_pair(bar_acc_full(e), 0x3);
             }
-            tc_commit(bar_drain);
+            tc_commit_pair(bar_drain, 0x1);
             const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(bar_drain, 0)) {
@@ -233,9 +246,10 @@ __global__ void __launch_bounds__(384, 1)
     }
     tc_fence_before_sync();
     __syncthreads();
+    cluster_sync_all();    // the pair's MMAs, commits and remote arrivals are over
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, C::TMEM_COLS);
+        tmem_dealloc_pair(tmem, C::TMEM_COLS);
     }
     } else {
         setmaxnreg_inc<C::REGS_HIGH>();
@@ -245,13 +259,15 @@ __global__ void __launch_bounds__(384, 1)
         const int row = quad * 32 + lane;   // token row inside the tile
         const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
         const uint32_t acc = tmem + lane_bits + 256u * e;
+        const uint32_t acc_empty_leader = mapa_shared(bar_acc_empty(e), 0);
         bool ok = true;
         int local = 0;
-        for (int t = blockIdx.x; ok && t < total; t += gridDim.x, ++local) {
+        for (int t = pair; ok && t < total; t += npairs, ++local) {
             if ((local & 1) != e) continue;
             int mt, nt;
             proj_tile(t, p, mt, nt);
-            const int b = mt / mpb, s = (mt % mpb) * C::BM + row, n0 = nt * C::BN;
+            const int b = mt / mpb, n0 = nt * C::BN;
+            const int s = (mt % mpb) * C::PAIR_M + static_cast<int>(rank) * C::BM + row;
             ok = __all_sync(0xffffffffu, wait_phase(bar_acc_full(e), (local >> 1) & 1, SITE_PROJ_EPI, wc));
             if (!ok) break;
             tc_fence_after_sync();
@@ -347,10 +363,14 @@ __global__ void __launch_bounds__(384, 1)
             }
             // every TMEM read of this accumulator is complete (waited above)
             tc_fence_before_sync();
-            mbar_arrive(bar_acc_empty(e));
+            if (leader)
+                mbar_arrive(bar_acc_empty(e));
+            else
+                mbar_arrive_remote(acc_empty_leader);
         }
         tc_fence_before_sync();
         __syncthreads();
+        cluster_sync_all();
     }
 }
 

@@ -128,11 +128,25 @@ int launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const regen::ProjS
             attr_status = REGEN_ERR_UNSUPPORTED;
     });
     if (attr_status != REGEN_OK) return attr_status;
-    const int64_t total = static_cast<int64_t>(shape.num_mt) * shape.num_nt;
+    const int64_t total = static_cast<int64_t>(shape.num_mt) * shape.num_nt;   // pair tiles
     const int sms = num_sms();
-    if (sms <= 0) return REGEN_ERR_CUDA;
-    const int grid = static_cast<int>(total < sms ? total : sms);
-    regen::proj_gemm_kernel<MODE><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, shape, ep, g_wait_limit_ns.load());
+    if (sms < 2) return REGEN_ERR_CUDA;
+    const int pairs = static_cast<int>(total < sms / 2 ? total : sms / 2);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const uint64_t limit = g_wait_limit_ns.load();
+    if (cudaLaunchKernelEx(&cfg, regen::proj_gemm_kernel<MODE>, ta, tb, shape, ep, limit) != cudaSuccess)
+        return REGEN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
 }
 
@@ -675,8 +689,8 @@ REGEN_API int regen_qkv_proj(const regen_bf16 *x, const regen_bf16 *w, const flo
     regen::rope_table_f32_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
     if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
     CUtensorMap ta, tb;
-    if (!make_bf16_map3(&ta, x, C, S, B, 64, 128) || !make_bf16_map3(&tb, w, C, N, 1, 64, 256)) return REGEN_ERR_CUDA;
-    regen::ProjShape shape{B, S, C, static_cast<int>(N), H, B * ((S + 127) / 128), static_cast<int>((N + 255) / 256)};
+    if (!make_bf16_map3(&ta, x, C, S, B, 64, 128) || !make_bf16_map3(&tb, w, C, N, 1, 64, 128)) return REGEN_ERR_CUDA;
+    regen::ProjShape shape{B, S, C, static_cast<int>(N), H, B * ((S + 255) / 256), static_cast<int>((N + 255) / 256)};
     regen::ProjEpi ep{bias, gamma_q, gamma_k, q, k, v, tab, geom, eps};
     return launch_proj<regen::PROJ_QKV>(ta, tb, shape, ep, st);
 }
@@ -698,9 +712,9 @@ REGEN_API int regen_out_proj(const regen_bf16 *o, const regen_bf16 *w, const flo
     if (overlaps(y, ybytes, o, obytes) || overlaps(y, ybytes, w, wbytes) || overlaps(y, ybytes, bias, N * 4LL))
         return REGEN_ERR_INVALID_ARG;
     CUtensorMap ta, tb;
-    if (!make_bhsd_map(&ta, o, static_cast<int64_t>(B) * H, S, 128) || !make_bf16_map3(&tb, w, K, N, 1, 64, 256))
+    if (!make_bhsd_map(&ta, o, static_cast<int64_t>(B) * H, S, 128) || !make_bf16_map3(&tb, w, K, N, 1, 64, 128))
         return REGEN_ERR_CUDA;
-    regen::ProjShape shape{B, S, static_cast<int>(K), N, H, B * ((S + 127) / 128), (N + 255) / 256};
+    regen::ProjShape shape{B, S, static_cast<int>(K), N, H, B * ((S + 255) / 256), (N + 255) / 256};
     regen::ProjEpi ep{bias, nullptr, nullptr, y, nullptr, nullptr, nullptr, regen::RopeGeom{}, 0.0f};
     return launch_proj<regen::PROJ_OUT>(ta, tb, shape, ep, reinterpret_cast<cudaStream_t>(stream));
 }
