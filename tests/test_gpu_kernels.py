@@ -340,3 +340,14 @@ def test_rope3d_fused_workspace_errors():
     with pytest.raises(rg.RegenError) as e:
         rg.attn_fwd_rope3d(q, q.clone(), q.clone(), grid, workspace=ws[16:])
     assert e.value.status == -3
+
+
+@pytest.mark.parametrize("B,H,Sq,Skv", [(1, 2, 257, 300), (1, 3, 513, 129), (2, 2, 700, 1000), (1, 1, 1024, 77),
+                                        (1, 2, 1500, 2072)])
+def test_attention_ragged_multi_tile(B, H, Sq, Skv):
+    q, k, v = rand_bf16((B, H, Sq, 128)), rand_bf16((B, H, Skv, 128)), rand_bf16((B, H, Skv, 128))
+    out, lse = rg.attn_fwd(to_dev(q), to_dev(k), to_dev(v), 1 / math.sqrt(128))
+    torch.cuda.synchronize()
+    ref, rl = oracle.attention(q, k, v, 1 / math.sqrt(128))
+    check_attention(to_bits(out).reshape(-1, 128), lse.cpu().numpy().reshape(-1), ref.reshape(-1, 128),
+                    rl.reshape(-1), f"{B}x{H}x{Sq}x{Skv}")
