@@ -17,6 +17,7 @@ Entry points (same names as the C ABI):
                    workspace, workspace_bytes, accumulate_dq)
     regen_attn_bwd_workspace_bytes(B, H, Sq, D)
     regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream=None)
+    regen_rope3d_shard(q, k, T, Hh, Ww, theta, B, H, D, n0, S_local, inverse=0, stream=None)
     regen_quant_e4m3(x, codes, scales, B, H, S, D, stream=None)
     regen_attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, B, H, Sq, Skv, D, scale, stream=None)
     regen_qkv_proj(x, w, bias, gamma_q, gamma_k, q, k, v, B, S, C, H, D, T, Hh, Ww, theta, eps, stream,
@@ -46,7 +47,7 @@ __all__ = [
     "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
     "regen_status_str", "regen_last_device_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
     "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes", "regen_attn_fwd_rope3d_noalloc",
-    "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd", "regen_quant_e4m3",
+    "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd", "regen_rope3d_shard", "regen_quant_e4m3",
     "regen_attn_fwd_fp8", "quant_e4m3", "attn_fwd_fp8", "regen_qkv_proj", "regen_qkv_proj_workspace_bytes",
     "regen_out_proj", "qkv_proj", "out_proj",
     "attn_fwd", "attn_fwd_rope3d", "rope3d_", "lse_merge", "attn_bwd", "rope3d_bwd_", "STATUS",
@@ -102,6 +103,8 @@ def load():
         L.regen_attn_bwd_workspace_bytes.restype = i64
         L.regen_rope3d_bwd.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, vp]
         L.regen_rope3d_bwd.restype = i32
+        L.regen_rope3d_shard.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, i32, i32, i32, vp]
+        L.regen_rope3d_shard.restype = i32
         L.regen_quant_e4m3.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
         L.regen_quant_e4m3.restype = i32
         L.regen_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
@@ -253,6 +256,11 @@ def regen_qkv_proj_workspace_bytes(T, Hh, Ww, D) -> int:
 def regen_out_proj(o, w, bias, y, B, S, H, D, N, stream=None) -> None:
     _check(load().regen_out_proj(_ptr(o), _ptr(w), _ptr(bias), _ptr(y), B, S, H, D, N, _stream(stream)),
            "regen_out_proj")
+
+
+def regen_rope3d_shard(q, k, T, Hh, Ww, theta, B, H, D, n0, S_local, inverse=0, stream=None) -> None:
+    _check(load().regen_rope3d_shard(_ptr(q), _ptr(k), T, Hh, Ww, float(theta), B, H, D, int(n0), int(S_local),
+                                     int(inverse), _stream(stream)), "regen_rope3d_shard")
 
 
 def regen_selftest_exp2(x, y, n, stream=None) -> None:

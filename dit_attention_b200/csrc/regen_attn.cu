@@ -341,14 +341,18 @@ uint8_t *noalloc_scratch_on_current_device()
     return g_noalloc_ptr[dev];
 }
 
+// S_local < 0: the whole grid (n0 = 0, S = T*Hh*Ww).
 int rope3d_common(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta, int B, int H, int D,
-                  regen_stream_t stream, bool inverse)
+                  regen_stream_t stream, bool inverse, int n0 = 0, int S_local = -1)
 {
     if (T <= 0 || Hh <= 0 || Ww <= 0 || B < 0 || H < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
     if (!std::isfinite(theta) || !(theta > 0.0f)) return REGEN_ERR_INVALID_ARG;
     if (D < 8 || D > 512 || (D % 8) != 0) return REGEN_ERR_UNSUPPORTED;
-    const int64_t S = static_cast<int64_t>(T) * Hh * Ww;
-    if (S > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const int64_t grid_tokens = static_cast<int64_t>(T) * Hh * Ww;
+    if (grid_tokens > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (S_local >= 0 && (n0 < 0 || static_cast<int64_t>(n0) + S_local > grid_tokens)) return REGEN_ERR_INVALID_ARG;
+    const int64_t S = S_local >= 0 ? S_local : grid_tokens;
+    if (S == 0) return REGEN_OK;
     const int64_t BH = static_cast<int64_t>(B) * H;
     if (BH == 0) return REGEN_OK;
     if (!q && !k) return REGEN_ERR_INVALID_ARG;
@@ -360,7 +364,7 @@ int rope3d_common(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float the
     const int64_t blocks = (work + threads - 1) / threads;
     if (blocks > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
     regen::rope3d_kernel<<<static_cast<unsigned>(blocks), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        q, k, BH, static_cast<int>(S), Hh, Ww, D, static_cast<double>(theta), inverse);
+        q, k, BH, static_cast<int>(S), Hh, Ww, D, static_cast<double>(theta), inverse, S_local >= 0 ? n0 : 0);
     return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
 }
 
@@ -492,6 +496,13 @@ REGEN_API int regen_rope3d_bwd(regen_bf16 *dq, regen_bf16 *dk, int T, int Hh, in
                                int H, int D, regen_stream_t stream)
 {
     return rope3d_common(dq, dk, T, Hh, Ww, theta, B, H, D, stream, true);
+}
+
+REGEN_API int regen_rope3d_shard(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta, int B, int H,
+                                 int D, int n0, int S_local, int inverse, regen_stream_t stream)
+{
+    if (S_local < 0 || (inverse != 0 && inverse != 1)) return REGEN_ERR_INVALID_ARG;
+    return rope3d_common(q, k, T, Hh, Ww, theta, B, H, D, stream, inverse != 0, n0, S_local);
 }
 
 REGEN_API int64_t regen_attn_bwd_workspace_bytes(int B, int H, int Sq, int D)

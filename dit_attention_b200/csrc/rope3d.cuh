@@ -140,18 +140,20 @@ __global__ void rope_apply_kernel(const uint4 *__restrict__ src, uint4 *__restri
     }
 }
 
-// grid: ceil(S * D/8 / blockDim) blocks; x (q then k) has `rows` rows of S x D.
+// grid: ceil(S * D/8 / blockDim) blocks; x (q then k) has `rows` rows of S x D
+// holding the latent tokens n0 .. n0 + S - 1 (a sequence shard when n0 > 0).
 // inverse: turn every pair back by its angle (sine negated), the transposed
 // rotation that carries gradients through the RoPE.
 __global__ void rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k, int64_t rows,
-                              int S, int Hh, int Ww, int D, double theta, bool inverse)
+                              int S, int Hh, int Ww, int D, double theta, bool inverse, int n0)
 {
     const int chunks = D >> 3;
     const int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
     if (gid >= static_cast<int64_t>(S) * chunks) return;
     const int n = static_cast<int>(gid / chunks);
     const int c = static_cast<int>(gid % chunks);
-    const int pos[3] = {n / (Hh * Ww), (n / Ww) % Hh, n % Ww};
+    const int tok = n0 + n;   // position on the latent grid
+    const int pos[3] = {tok / (Hh * Ww), (tok / Ww) % Hh, tok % Ww};
     const int dh = 2 * (D / 6);
     const int dt = D - 2 * dh;
     double cs[4], sn[4];

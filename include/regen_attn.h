@@ -161,6 +161,18 @@ REGEN_API int regen_rope3d(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, 
                            int B, int H, int D, regen_stream_t stream);
 
 /*
+ * regen_rope3d_shard -- regen_rope3d (inverse = 0) or regen_rope3d_bwd
+ * (inverse = 1) on a sequence shard: q, k [B, H, S_local, D] hold the latent
+ * tokens n0 .. n0 + S_local - 1 of the T x Hh x Ww grid, which set their
+ * positions. Needs 0 <= n0 and n0 + S_local <= T*Hh*Ww (else
+ * REGEN_ERR_INVALID_ARG); S_local == 0: REGEN_OK, nothing done. Same
+ * arithmetic, rounding and other arguments as regen_rope3d, so a sharded
+ * rotation equals the matching rows of the whole-grid one bit for bit.
+ */
+REGEN_API int regen_rope3d_shard(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta,
+                                 int B, int H, int D, int n0, int S_local, int inverse, regen_stream_t stream);
+
+/*
  * regen_lse_merge -- combine two partial attentions of the same queries
  * over disjoint key blocks a and b:
  *     m = max(lse_a, lse_b), w_a = exp(lse_a - m), w_b = exp(lse_b - m)

@@ -220,3 +220,16 @@ def test_out_proj_validation(lib, args, status):
     a.update(args)
     rc = lib.regen_out_proj(a["o"], a["w"], a["bias"], a["y"], a["B"], a["S"], a["H"], a["D"], a["N"], None)
     assert rc == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(n0=-1), -1), (dict(n0=50, S=11), -1), (dict(S=-1), -1), (dict(inv=2), -1), (dict(D=12), -2),
+    (dict(S=0), 0), (dict(q=FAKE + 2), -3), (dict(B=0), 0),
+])
+def test_rope3d_shard_validation(lib, args, status):
+    # grid 3 x 4 x 5 = 60 tokens; the shard holds tokens n0 .. n0 + S - 1
+    a = dict(q=FAKE, k=FAKE + 10 * MB, T=3, Hh=4, Ww=5, theta=1e4, B=1, H=2, D=128, n0=20, S=30, inv=0)
+    a.update(args)
+    rc = lib.regen_rope3d_shard(a["q"], a["k"], a["T"], a["Hh"], a["Ww"], a["theta"], a["B"], a["H"], a["D"], a["n0"],
+                                a["S"], a["inv"], None)
+    assert rc == status

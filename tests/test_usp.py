@@ -1,0 +1,169 @@
+"""Sequence parallelism (dit_attention_b200.usp): Ring and Ulysses exchanges on
+2 and 4 ranks.
+
+CPU tests: gloo ranks run the exchange logic with the oracle as the per-rank
+attention and merge (fp64), and every rank's result must equal the oracle's
+attention over the whole window -- the exactness the sharding promises. The GPU
+test runs two ranks on one GPU with the library's kernels as the per-rank
+compute; the shards travel through gloo (host memory), since two ranks cannot
+share one GPU under NCCL.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from dit_attention_b200 import synth, usp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _oracle_attn(q, k, v, scale):
+    out, lse = oracle.attention(q.numpy(), k.numpy(), v.numpy(), scale)
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+def _oracle_merge(oa, la, ob, lb):
+    out, lse = oracle.lse_merge(oa.numpy(), la.numpy(), ob.numpy(), lb.numpy())
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+def _window(B=1, H=4, S=96, D=16, seed=5):
+    rng = np.random.default_rng(seed)
+    return [rng.normal(size=(B, H, S, D)) * f for f in (1.5, 1.5, 1.0)]
+
+
+def _run(world, fn, *args):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_worker, args=(world, port, out, fn, args), nprocs=world, start_method="spawn", join=True)
+        return dict(out)
+
+
+def _worker(rank, world, port, out, fn, args):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        out[rank] = fn(rank, world, *args)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def _ring_case(rank, world, S):
+    q, k, v = _window(S=S)
+    scale = 0.25
+    a, b = usp.shard_range(S, rank, world)
+    o, l = usp.ring_attention(torch.from_numpy(q[:, :, a:b].copy()), torch.from_numpy(k[:, :, a:b].copy()),
+                              torch.from_numpy(v[:, :, a:b].copy()), None, scale, _oracle_attn, _oracle_merge)
+    ref, rl = oracle.attention(q, k, v, scale)
+    return float(np.abs(o.numpy() - ref[:, :, a:b]).max()), float(np.abs(l.numpy() - rl[:, :, a:b]).max())
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ring_attention_is_exact(world):
+    res = _run(world, _ring_case, 96)
+    assert sorted(res) == list(range(world))
+    for r, (eo, el) in res.items():
+        assert eo < 1e-12 and el < 1e-12, (r, eo, el)
+
+
+def _ulysses_case(rank, world):
+    x = _window(H=4, S=64)[0]
+    a, b = usp.shard_range(64, rank, world)
+    mine = torch.from_numpy(x[:, :, a:b].copy())
+    heads = usp.seq_to_heads(mine, None)
+    hq = 4 // world
+    # this rank's heads, every token
+    ok_fwd = np.array_equal(heads.numpy(), x[:, rank * hq:(rank + 1) * hq])
+    back = usp.heads_to_seq(heads, None)
+    lse_like = torch.from_numpy(x[..., 0][:, :, a:b].copy())           # [B, H, S_local]: 3-dim tensors too
+    lse_back = usp.heads_to_seq(usp.seq_to_heads(lse_like, None), None)
+    return ok_fwd, bool(torch.equal(back, mine)), bool(torch.equal(lse_back, lse_like))
+
+
+def test_ulysses_all_to_all_round_trip():
+    res = _run(2, _ulysses_case)
+    for r, (f, b, lse_ok) in res.items():
+        assert f and b and lse_ok, r
+
+
+def _usp_case(rank, world, U, R):
+    ug, rg_ = usp.usp_groups(U, R)
+    q, k, v = _window(H=4, S=96)
+    scale = 0.25
+    a, b = usp.shard_range(96, rank, world)
+    args = [torch.from_numpy(t[:, :, a:b].copy()) for t in (q, k, v)]
+    o, l = usp.usp_attention(*args, ug, rg_, scale, _oracle_attn, _oracle_merge)
+    ref, rl = oracle.attention(q, k, v, scale)
+    return float(np.abs(o.numpy() - ref[:, :, a:b]).max()), float(np.abs(l.numpy() - rl[:, :, a:b]).max())
+
+
+def test_unified_sequence_parallel_ulysses2_ring2():
+    # the pages' layout scaled down: 2 (Ulysses) x 2 (Ring) ranks
+    res = _run(4, _usp_case, 2, 2)
+    for r, (eo, el) in res.items():
+        assert eo < 1e-12 and el < 1e-12, (r, eo, el)
+
+
+def test_shard_range():
+    assert usp.shard_range(31200, 3, 8) == (11700, 15600)
+    with pytest.raises(ValueError):
+        usp.shard_range(10, 1, 3)
+
+
+# ------------------------------------------------- with the GPU kernels ---
+
+def _gpu_ring_case(rank, world):
+    import dit_attention_b200 as rg
+    torch.cuda.set_device(0)
+    w = synth.Workload("usp", B=1, H=4, D=128, Sq=1040, Skv=1040, seed=9, grid=(2, 20, 26), rope=True, rmsnorm=True)
+    q, k, v = synth.make_inputs(w)
+    a, b = usp.shard_range(w.Sq, rank, world)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
+    tq, tk, tv = dev(q[:, :, a:b]), dev(k[:, :, a:b]), dev(v[:, :, a:b])
+    T, Hh, Ww = w.grid
+    rg.regen_rope3d_shard(tq, tk, T, Hh, Ww, w.theta, w.B, w.H, w.D, a, b - a, 0)   # RoPE at global positions
+
+    # per-rank compute in the library's kernels; the shards travel as host tensors
+    def attn(qh, kh, vh, scale):
+        o, l = rg.attn_fwd(qh.cuda(), kh.cuda(), vh.cuda(), scale)
+        return o.cpu(), l.cpu()
+
+    def merge(oa, la, ob, lb):
+        o, l = rg.lse_merge(oa.cuda(), la.cuda(), ob.cuda(), lb.cuda())
+        return o.cpu(), l.cpu()
+
+    o, l = usp.ring_attention(tq.cpu(), tk.cpu(), tv.cpu(), None, w.scale, attn, merge)
+    torch.cuda.synchronize()
+    return (o.contiguous().view(torch.int16).numpy().view(np.uint16), l.numpy(), a, b,
+            tq.cpu().contiguous().view(torch.int16).numpy().view(np.uint16),
+            tk.cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+@pytest.mark.gpu
+def test_ring_attention_with_kernels_two_ranks_one_gpu():
+    from util import check_attention
+    assert torch.cuda.is_available()
+    res = _run(2, _gpu_ring_case)
+    w = synth.Workload("usp", B=1, H=4, D=128, Sq=1040, Skv=1040, seed=9, grid=(2, 20, 26), rope=True, rmsnorm=True)
+    q, k, v = synth.make_inputs(w)
+    qr, kr = oracle.rope3d(q, w.grid, w.theta), oracle.rope3d(k, w.grid, w.theta)
+    ref, rl = oracle.attention(qr, kr, v, w.scale)
+    for r, (o, l, a, b, gq, gk) in res.items():
+        # the sharded RoPE equals the whole-grid one on these rows, bit for bit
+        np.testing.assert_array_equal(gq, qr[:, :, a:b])
+        np.testing.assert_array_equal(gk, kr[:, :, a:b])
+        check_attention(o.reshape(-1, 128), l.reshape(-1), ref[:, :, a:b].reshape(-1, 128), rl[:, :, a:b].reshape(-1),
+                        f"ring rank {r}")
