@@ -13,28 +13,28 @@
 // of Q and then of K, so the trigonometry is amortised over 2*B*H rows.
 // Adjacent threads own adjacent chunks of a row: each warp access is two
 // contiguous 256-byte rows. The rotation is done in fp64 and rounded once to
-// bf16 (round to odd into fp32, then nearest-even into bf16, which equals one
-// correct rounding).
+// bf16 (one direct fp64 -> bf16 conversion, nearest-even).
 #pragma once
 
 #include <stdint.h>
 
 namespace regen {
 
+// bf16 -> double, exact (every bf16 is a double).
 __device__ __forceinline__ double bf16_bits_to_double(uint32_t h16)
 {
-    return static_cast<double>(__uint_as_float(h16 << 16));
+    double d;
+    asm("cvt.f64.bf16 %0, %1;" : "=d"(d) : "h"(static_cast<unsigned short>(h16)));
+    return d;
 }
 
-// Correctly rounded double -> bf16 (nearest, ties to even).
+// Correctly rounded double -> bf16 (nearest, ties to even) in one conversion,
+// no intermediate fp32 rounding; NaN becomes the canonical 0x7FC0.
 __device__ __forceinline__ uint32_t double_to_bf16_bits(double x)
 {
-    if (x != x) return 0x7FC0u;
-    const float f = __double2float_rz(x);
-    uint32_t b = __float_as_uint(f);
-    if (static_cast<double>(f) != x) b |= 1u;  // sticky: round to odd
-    b += 0x7FFFu + ((b >> 16) & 1u);
-    return b >> 16;
+    unsigned short h;
+    asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(h) : "d"(x));
+    return x != x ? 0x7FC0u : static_cast<uint32_t>(h);
 }
 
 // Rotate one (even, odd) pair packed as two bf16 by the angle with cosine c
