@@ -100,57 +100,94 @@ def step_flops():
 # ------------------------------------------------------------ clocks ---
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, board power and clock-event reasons of this process's GPU,
+    sampled every 20 ms during the timed region by read-only NVML queries
+    (nvidia-smi on the same GPU if NVML cannot be loaded). The GPU is found by
+    its UUID: NVML numbers every GPU of the machine and ignores
+    CUDA_VISIBLE_DEVICES, so an index could name another process's GPU."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.hw_power_brake_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device):
+        import torch
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        self.uuid = u if u.startswith("GPU-") else "GPU-" + u
+        self.samples = []          # (sm_mhz, power_w, set of reason names)
+        self.sm_max = None
+        self.source = None
+        self._stop = threading.Event()
+        self._first = threading.Event()
+        self.proc = self.t = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            masks = [(n, getattr(pynvml, c)) for n, c in self.REASONS if hasattr(pynvml, c)]
+            self.source = "nvml"
+            self.t = threading.Thread(target=self._poll_nvml, args=(pynvml, h, masks), daemon=True)
+        except Exception:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.SMI_FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                return
+            self.source = "nvidia-smi"
+            self.t = threading.Thread(target=self._read_smi, daemon=True)
+        self.t.start()
+        self._first.wait(timeout=10.0)   # the first sample precedes the timed region
 
-    def _read(self):
+    def _poll_nvml(self, pynvml, h, masks):
+        while not self._stop.is_set():
+            try:
+                sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, pw, {n for n, m in masks if bits & m}))
+            except Exception:
+                pass
+            self._first.set()
+            self._stop.wait(0.02)
+
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            f = [x.strip() for x in line.split(",")]
+            try:
+                sm, self.sm_max, pw = float(f[0]), float(f[1]), float(f[2])
+            except (ValueError, IndexError):
+                continue
+            self.samples.append((sm, pw, {n for n, v in zip(names, f[3:8]) if v.lower() == "active"}))
+            self._first.set()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.t.join(timeout=5)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
+        if self.t is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, f[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        busy = [x for x in sm if smax and x > 0.3 * smax] or sm
-        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.t.join(timeout=5)
+        smax = self.sm_max
+        busy = [x for x in self.samples if smax and x[0] > 0.3 * smax] or self.samples
+        reasons = set().union(*(x[2] for x in self.samples)) if self.samples else set()
+        return {"sm_mhz": statistics.median(x[0] for x in busy) if busy else None,
+                "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(self.samples),
+                "power_w": statistics.median(x[1] for x in busy) if busy else None,
+                "source": self.source}
 
 
 # ------------------------------------------------------- native (GPU) ---
@@ -243,7 +280,7 @@ def run_native(args, rank, world, local_rank):
 
     # ---- device-resident timing: K steps between two events, per-kernel events inside
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(dev)
     barrier()
     torch.cuda.synchronize()
     clocks.start()
