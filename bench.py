@@ -124,6 +124,7 @@ class ClockSampler:
         self._stop = threading.Event()
         self._first = threading.Event()
         self.proc = self.t = None
+        self.power_kind = "1 s average"
 
     def start(self):
         try:
@@ -133,6 +134,7 @@ class ClockSampler:
             self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
             masks = [(n, getattr(pynvml, c)) for n, c in self.REASONS if hasattr(pynvml, c)]
             self.source = "nvml"
+            self.power_kind = "instant" if self._instant_power(pynvml, h) is not None else "1 s average"
             self.t = threading.Thread(target=self._poll_nvml, args=(pynvml, h, masks), daemon=True)
         except Exception:
             try:
@@ -147,11 +149,26 @@ class ClockSampler:
         self.t.start()
         self._first.wait(timeout=10.0)   # the first sample precedes the timed region
 
+    @staticmethod
+    def _instant_power(pynvml, h):
+        """Board power now, in W (the plain power query averages over a second,
+        longer than a short timed region); None where the field is missing."""
+        try:
+            v = pynvml.nvmlDeviceGetFieldValues(h, [pynvml.NVML_FI_DEV_POWER_INSTANT])[0]
+            if v.nvmlReturn != 0:
+                return None
+            raw = {0: "dVal", 1: "uiVal", 2: "ulVal", 3: "ullVal", 4: "sllVal"}.get(v.valueType)
+            return float(getattr(v.value, raw)) / 1000.0 if raw else None
+        except Exception:
+            return None
+
     def _poll_nvml(self, pynvml, h, masks):
         while not self._stop.is_set():
             try:
                 sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
-                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                pw = self._instant_power(pynvml, h) if self.power_kind == "instant" else None
+                if pw is None:
+                    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
                 bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
                 self.samples.append((sm, pw, {n for n, m in masks if bits & m}))
             except Exception:
@@ -187,7 +204,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(x[0] for x in busy) if busy else None,
                 "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(self.samples),
                 "power_w": statistics.median(x[1] for x in busy) if busy else None,
-                "source": self.source}
+                "power_kind": self.power_kind, "source": self.source}
 
 
 # ------------------------------------------------------- native (GPU) ---
