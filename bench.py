@@ -51,6 +51,8 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=12)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
+    p.add_argument("--configs", action="store_true",
+                   help="instead of the step: CUDA-event medians of every workload's kernels (1 GPU)")
     return p.parse_args()
 
 
@@ -774,6 +776,88 @@ def time_cpu(sample, rows):
     return flops / dt / 1e12, dt
 
 
+def run_configs(args):
+    """CUDA-event medians (20 launches after 5 warm-ups, L2 flushed between
+    launches) of the kernels of every workload, through the C ABI:
+    tiny (D = 64, no RoPE), the 25- and 77-frame windows (RoPE, then the
+    self-attention; for the 77-frame one also four back-to-back calls, one per
+    denoising step), the cross-attention over the 2072 concatenated reference
+    + conditioning keys in one call, and the stress workload whole, as two
+    5460-key halves, and their merge. Prints one JSON object."""
+    import torch
+    import dit_attention_b200 as rg
+    from dit_attention_b200 import synth
+
+    torch.cuda.set_device(0)
+    rg.load()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2 (126 MB)
+    REPS, WARM = 20, 5
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    def median_ms(fn, reps=REPS, warm=WARM):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    def tflops(w, skv, ms):
+        return 4.0 * w.B * w.H * w.Sq * skv * w.D / (ms * 1e-3) / 1e12
+
+    rows = []
+    for name, w in synth.WORKLOADS.items():
+        q, k, v = (to_dev(x) for x in synth.make_inputs(w))
+        B, H, Sq, Skv, D = w.B, w.H, w.Sq, w.Skv, w.D
+        scale = w.scale
+        out = torch.empty((B, H, Sq, D), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+        rec = {"workload": name, "B": B, "H": H, "Sq": Sq, "Skv": Skv, "D": D}
+        if w.rope:
+            T, Hh, Ww = w.grid
+            qr, kr = q.clone(), k.clone()
+            ms = median_ms(lambda: rg.regen_rope3d(qr, kr, T, Hh, Ww, w.theta, B, H, D, sh))
+            rec["rope3d_ms"] = round(ms, 4)
+            rec["rope3d_gbs"] = round(2 * 2 * B * H * Sq * D * 2 / (ms * 1e-3) / 1e9, 1)
+            rg.regen_rope3d(q, k, T, Hh, Ww, w.theta, B, H, D, sh)   # attention on the rotated inputs
+        ms = median_ms(lambda: rg.regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, sh))
+        rec["attn_ms"] = round(ms, 4)
+        rec["attn_tflops"] = round(tflops(w, Skv, ms), 1)
+        if name == SELF:
+            def four():
+                for _ in range(4):
+                    rg.regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, sh)
+            rec["attn_four_calls_ms"] = round(median_ms(four, reps=5, warm=1), 3)
+        if w.merge_split:
+            h = w.merge_split
+            ka, va = k[:, :, :h].contiguous(), v[:, :, :h].contiguous()
+            kb, vb = k[:, :, h:].contiguous(), v[:, :, h:].contiguous()
+            oa, ob, om = (torch.empty_like(out) for _ in range(3))
+            la, lb, lm = (torch.empty_like(lse) for _ in range(3))
+            ma = median_ms(lambda: rg.regen_attn_fwd(q, ka, va, oa, la, B, H, Sq, h, D, scale, sh))
+            mb = median_ms(lambda: rg.regen_attn_fwd(q, kb, vb, ob, lb, B, H, Sq, Skv - h, D, scale, sh))
+            mm = median_ms(lambda: rg.regen_lse_merge(oa, la, ob, lb, om, lm, B * H * Sq, D, sh))
+            rec.update(half_a_ms=round(ma, 4), half_b_ms=round(mb, 4), merge_ms=round(mm, 4),
+                       merge_gbs=round(B * H * Sq * (3 * D * 2 + 3 * 4) / (mm * 1e-3) / 1e9, 1),
+                       split_path_ms=round(ma + mb + mm, 4))
+        rows.append(rec)
+        del q, k, v, out, lse
+        torch.cuda.empty_cache()
+    return {"what": "CUDA-event medians per workload (20 launches after 5 warm-ups, 256 MB L2 flush "
+                    "between launches); TFLOP/s = 4 B H Sq Skv D / time", "configs": rows}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -808,6 +892,10 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
+    if args.configs:
+        if rank == 0:
+            print(json.dumps(run_configs(args)), flush=True)
+        return
     if world > 1:
         import datetime
         import torch
@@ -817,12 +905,23 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     line = run_native(args, rank, world, local_rank)
     if line is not None and not args.no_cpu_baseline:
+        import oracle
         sample = cpu_sample_rate(args.cpu_seconds)
         v, dt = time_cpu(sample, sample["rows"])
+        # the same oracle once more on one thread, on a smaller sample (~1/3 of the time above)
+        threads = sample["threads"]
+        rows1 = max(16, sample["rows"] // max(1, 3 * threads))
+        oracle.set_num_threads(1)
+        try:
+            v1, dt1 = time_cpu(sample, rows1)
+        finally:
+            oracle.set_num_threads(threads)
         line["cpu_baseline"] = {
-            "value": v, "unit": "TFLOP/s", "cores": sample["threads"], "kind": "oracle",
+            "value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": f"{sample['rows']} random query rows of the 77-frame self-attention (all 31200 keys, "
                       f"D=128), fp64, {dt:.1f} s",
+            "single_thread": {"value": v1, "unit": "TFLOP/s", "cores": 1,
+                              "sample": f"{rows1} random query rows, same workload, {dt1:.1f} s"},
         }
     if line is not None:
         print(json.dumps(line), flush=True)
