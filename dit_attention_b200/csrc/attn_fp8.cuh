@@ -20,10 +20,10 @@
 #include "attn_fwd.cuh"
 #include "ptx.cuh"
 
-// Pairs of every 8 whose 2^x runs on the FMA pipe; 2 and 3 measured equal on the
-// 77-frame window, 4 and 5 slower (the softmax is issue-bound, not MUFU-bound).
+// Pairs of every 8 whose 2^x runs on the FMA pipe. On the 77-frame window 1 is
+// the fastest, by about 0.5 % over 2; 2 and 3 measured equal, and 0, 4 and 5 slower.
 #ifndef REGEN_FP8_EXP2_EMU_PER8
-#define REGEN_FP8_EXP2_EMU_PER8 2
+#define REGEN_FP8_EXP2_EMU_PER8 1
 #endif
 
 namespace regen {
