@@ -33,8 +33,12 @@
 #include "ptx.cuh"
 #include "rope3d.cuh"
 
+// Pairs of every 8 probabilities whose 2^x runs on the FMA pipe (exp2_poly_pair)
+// instead of MUFU, in the forward and the gradient kernels. On the 77-frame
+// window 1 measured equal to 2 for the forward and ~2 % faster for the
+// gradient; 3 is slower for both.
 #ifndef REGEN_EXP2_EMU_PER8
-#define REGEN_EXP2_EMU_PER8 2
+#define REGEN_EXP2_EMU_PER8 1
 #endif
 
 namespace regen {
