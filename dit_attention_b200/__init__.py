@@ -35,6 +35,8 @@ Convenience wrappers that allocate outputs with torch:
     quant_e4m3(x) -> (codes, scales);  attn_fwd_fp8(q8, qs, k8, ks, v8, vs, scale=None) -> (out, lse)
     qkv_proj(x, w, heads, grid, bias=None, gamma_q=None, gamma_k=None) -> (q, k, v)
     out_proj(o, w, bias=None) -> y
+Differentiable forms for training (torch.autograd over the same kernels):
+    dit_attention_b200.autograd.dit_attention, dit_cross_attention
 """
 from __future__ import annotations
 
