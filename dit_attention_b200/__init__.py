@@ -14,7 +14,7 @@ Entry points (same names as the C ABI):
     regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
     regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream=None)
     regen_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Sq, Skv, D, scale, stream,
-                   workspace, workspace_bytes, accumulate_dq)
+                   workspace, workspace_bytes, accumulate)   # REGEN_ACCUM_DQ | REGEN_ACCUM_DKDV
     regen_attn_bwd_workspace_bytes(B, H, Sq, D)
     regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream=None)
     regen_rope3d_shard(q, k, T, Hh, Ww, theta, B, H, D, n0, S_local, inverse=0, stream=None)
@@ -63,6 +63,10 @@ _lib = None
 STATUS = {0: "REGEN_OK", -1: "REGEN_ERR_INVALID_ARG", -2: "REGEN_ERR_UNSUPPORTED",
           -3: "REGEN_ERR_MISALIGNED", -4: "REGEN_ERR_CUDA", -5: "REGEN_ERR_TIMEOUT"}
 
+
+# regen_attn_bwd's accumulate bits (include/regen_attn.h)
+REGEN_ACCUM_DQ = 1
+REGEN_ACCUM_DKDV = 2
 
 class RegenError(RuntimeError):
     def __init__(self, status: int, what: str):
@@ -211,10 +215,10 @@ def regen_lse_merge(o_a, lse_a, o_b, lse_b, out, lse_out, rows, D, stream=None) 
 
 
 def regen_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Sq, Skv, D, scale, stream, workspace,
-                   workspace_bytes, accumulate_dq=0) -> None:
+                   workspace_bytes, accumulate=0) -> None:
     _check(load().regen_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                                  _ptr(dv), B, H, Sq, Skv, D, float(scale), _stream(stream), _ptr(workspace),
-                                 int(workspace_bytes), int(accumulate_dq)), "regen_attn_bwd")
+                                 int(workspace_bytes), int(accumulate)), "regen_attn_bwd")
 
 
 def regen_attn_bwd_workspace_bytes(B, H, Sq, D) -> int:
@@ -360,11 +364,12 @@ def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None, stream=None):
 
 
 def attn_bwd(q, k, v, out, lse, dout, scale=None, dq=None, dk=None, dv=None, accumulate_dq=False,
-             workspace=None, stream=None):
+             workspace=None, stream=None, accumulate_dkdv=False):
     """Gradients of attn_fwd -> (dq, dk, dv), bf16 like the inputs.
 
     out and lse are the forward's (or, for one key block of a merged
-    attention, the merged ones). accumulate_dq adds into the given dq."""
+    attention, the merged ones). accumulate_dq adds into the given dq,
+    accumulate_dkdv into the given dk and dv."""
     import torch
     B, H, Sq, D = _bhsd(q, "q")
     Skv = _bhsd(k, "k")[2]
@@ -372,6 +377,8 @@ def attn_bwd(q, k, v, out, lse, dout, scale=None, dq=None, dk=None, dv=None, acc
         scale = 1.0 / math.sqrt(D)
     if accumulate_dq and dq is None:
         raise ValueError("accumulate_dq needs the dq to add into")
+    if accumulate_dkdv and (dk is None or dv is None):
+        raise ValueError("accumulate_dkdv needs the dk and dv to add into")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -379,7 +386,8 @@ def attn_bwd(q, k, v, out, lse, dout, scale=None, dq=None, dk=None, dv=None, acc
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     regen_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Sq, Skv, D, scale, stream, workspace,
-                   workspace.numel() * workspace.element_size(), 1 if accumulate_dq else 0)
+                   workspace.numel() * workspace.element_size(),
+                   (REGEN_ACCUM_DQ if accumulate_dq else 0) | (REGEN_ACCUM_DKDV if accumulate_dkdv else 0))
     return dq, dk, dv
 
 

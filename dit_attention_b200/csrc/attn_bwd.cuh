@@ -154,13 +154,16 @@ __device__ __forceinline__ void probs_pair(uint32_t &s0, uint32_t &s1, uint64_t 
 //   dV += P^T(i) dO(i) | S^T(i+1) | dK += dS^T(i) Q(i) | dP^T(i+1)
 // so the exponentials of tile i+1 overlap dK(i) and dP^T(i+1), and dS of
 // tile i overlaps dV(i) and S^T(i+1).
-template <int HD>
+// ACCUM: dK and dV are added to the bf16 values already in dk_old / dv_old
+// (the output buffers themselves: each CTA reads its own key rows before its
+// store), for gradients accumulated over several query blocks.
+template <int HD, bool ACCUM>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                          const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                          const float *__restrict__ ws, int Sq, int Skv, float scale, float scale_log2,
-                         uint64_t wait_limit_ns)
+                         uint64_t wait_limit_ns, const uint16_t *dk_old, const uint16_t *dv_old)
 {
     using C = BwdCfg<HD>;
     constexpr int NS = C::A_NS;
@@ -430,15 +433,35 @@ __global__ void __launch_bounds__(384, 1)
                 tmem_ld_32x32b_x32(tacc + c * 32, o);
                 tmem_ld_wait();
                 reg_fence(o);
+                float add[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) add[x] = 0.f;
+                if constexpr (ACCUM) {
+                    if (key0 + krow < Skv) {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(
+                            (w ? dk_old : dv_old) + (static_cast<int64_t>(bh) * Skv + key0 + krow) * HD + c * 32);
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const uint4 u = src[g];
+                            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                add[g * 8 + 2 * e] = __uint_as_float(uw[e] << 16);
+                                add[g * 8 + 2 * e + 1] = __uint_as_float(uw[e] & 0xFFFF0000u);
+                            }
+                        }
+                    }
+                }
+                auto val = [&](int x) { return fmaf(__uint_as_float(o[x]), mul, add[x]); };
                 const int half = c >> 1;
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     const int chunk = (c & 1) * 4 + g;
                     uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(o[g * 8 + 0]) * mul, __uint_as_float(o[g * 8 + 1]) * mul);
-                    v.y = pack_bf16x2(__uint_as_float(o[g * 8 + 2]) * mul, __uint_as_float(o[g * 8 + 3]) * mul);
-                    v.z = pack_bf16x2(__uint_as_float(o[g * 8 + 4]) * mul, __uint_as_float(o[g * 8 + 5]) * mul);
-                    v.w = pack_bf16x2(__uint_as_float(o[g * 8 + 6]) * mul, __uint_as_float(o[g * 8 + 7]) * mul);
+                    v.x = pack_bf16x2(val(g * 8 + 0), val(g * 8 + 1));
+                    v.y = pack_bf16x2(val(g * 8 + 2), val(g * 8 + 3));
+                    v.z = pack_bf16x2(val(g * 8 + 4), val(g * 8 + 5));
+                    v.w = pack_bf16x2(val(g * 8 + 6), val(g * 8 + 7));
                     *reinterpret_cast<uint4 *>(stage + half * C::HALF_BYTES + krow * 128 + ((chunk ^ (krow & 7)) << 4)) = v;
                 }
             }

@@ -229,7 +229,8 @@ int grid_for(int64_t work, int threads)
 template <int HD>
 int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, const regen_bf16 *out,
                const float *lse, const regen_bf16 *dout, regen_bf16 *dq, regen_bf16 *dk, regen_bf16 *dv,
-               int64_t BH, int Sq, int Skv, float scale, float *ws, bool accumulate, cudaStream_t stream)
+               int64_t BH, int Sq, int Skv, float scale, float *ws, bool acc_dq, bool acc_dkdv,
+               cudaStream_t stream)
 {
     using C = regen::BwdCfg<HD>;
     static std::once_flag once;
@@ -244,7 +245,9 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
             return fa.numRegs < C::MIN_LAUNCH_REGS ? static_cast<int>(REGEN_ERR_UNSUPPORTED)
                                                    : static_cast<int>(REGEN_OK);
         };
-        int st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dkdv_kernel<HD>), C::A_SMEM_BYTES);
+        int st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dkdv_kernel<HD, false>), C::A_SMEM_BYTES);
+        if (st == REGEN_OK)
+            st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dkdv_kernel<HD, true>), C::A_SMEM_BYTES);
         if (st == REGEN_OK)
             st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, false>), C::B_SMEM_BYTES);
         if (st == REGEN_OK)
@@ -267,10 +270,16 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
     if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
     const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     const uint64_t limit = g_wait_limit_ns.load();
-    regen::attn_bwd_dkdv_kernel<HD><<<static_cast<unsigned>(BH * nkv), C::THREADS, C::A_SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, tdk, tdv, ws, Sq, Skv, scale, scale_log2, limit);
+    const uint16_t *dk_old = reinterpret_cast<const uint16_t *>(dk);
+    const uint16_t *dv_old = reinterpret_cast<const uint16_t *>(dv);
+    if (acc_dkdv)
+        regen::attn_bwd_dkdv_kernel<HD, true><<<static_cast<unsigned>(BH * nkv), C::THREADS, C::A_SMEM_BYTES, stream>>>(
+            tq, tk, tv, tdo, tdk, tdv, ws, Sq, Skv, scale, scale_log2, limit, dk_old, dv_old);
+    else
+        regen::attn_bwd_dkdv_kernel<HD, false><<<static_cast<unsigned>(BH * nkv), C::THREADS, C::A_SMEM_BYTES, stream>>>(
+            tq, tk, tv, tdo, tdk, tdv, ws, Sq, Skv, scale, scale_log2, limit, dk_old, dv_old);
     if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
-    if (accumulate)
+    if (acc_dq)
         regen::attn_bwd_dq_kernel<HD, true><<<static_cast<unsigned>(BH * nq), C::THREADS, C::B_SMEM_BYTES, stream>>>(
             tq, tk, tv, tdo, tdq, dq, ws, Sq, Skv, scale, scale_log2, limit);
     else
@@ -515,21 +524,23 @@ REGEN_API int64_t regen_attn_bwd_workspace_bytes(int B, int H, int Sq, int D)
 REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
                              const regen_bf16 *out, const float *lse, const regen_bf16 *dout, regen_bf16 *dq,
                              regen_bf16 *dk, regen_bf16 *dv, int B, int H, int Sq, int Skv, int D, float scale,
-                             regen_stream_t stream, void *workspace, int64_t workspace_bytes, int accumulate_dq)
+                             regen_stream_t stream, void *workspace, int64_t workspace_bytes, int accumulate)
 {
     if (B < 0 || H < 0 || Sq < 0 || Skv < 0 || D < 0 || workspace_bytes < 0) return REGEN_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return REGEN_ERR_INVALID_ARG;
-    if (accumulate_dq != 0 && accumulate_dq != 1) return REGEN_ERR_INVALID_ARG;
+    if (accumulate < 0 || accumulate > (REGEN_ACCUM_DQ | REGEN_ACCUM_DKDV)) return REGEN_ERR_INVALID_ARG;
+    const bool acc_dq = (accumulate & REGEN_ACCUM_DQ) != 0, acc_dkdv = (accumulate & REGEN_ACCUM_DKDV) != 0;
     if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
     const int64_t BH = static_cast<int64_t>(B) * H;
     if (BH == 0 || (Sq == 0 && Skv == 0)) return REGEN_OK;
     if (BH > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
     const int64_t qbytes = BH * Sq * D * 2, kvbytes = BH * Skv * D * 2, lbytes = BH * Sq * 4;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (Sq == 0) {  // no query: dk = dv = 0
+    if (Sq == 0) {  // no query: dk = dv = 0 (unchanged when accumulating)
         if (!dk || !dv) return REGEN_ERR_INVALID_ARG;
         if (!aligned16(dk) || !aligned16(dv)) return REGEN_ERR_MISALIGNED;
         if (overlaps(dk, kvbytes, dv, kvbytes)) return REGEN_ERR_INVALID_ARG;
+        if (acc_dkdv) return REGEN_OK;
         for (regen_bf16 *z : {dk, dv}) {
             regen::attn_empty_kernel<<<grid_for(kvbytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(z),
                                                                                  kvbytes / 16, nullptr, 0);
@@ -540,7 +551,7 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
     if (Skv == 0) {  // no key: dq = 0 (unchanged when accumulating)
         if (!dq) return REGEN_ERR_INVALID_ARG;
         if (!aligned16(dq)) return REGEN_ERR_MISALIGNED;
-        if (accumulate_dq) return REGEN_OK;
+        if (acc_dq) return REGEN_OK;
         regen::attn_empty_kernel<<<grid_for(qbytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(dq),
                                                                             qbytes / 16, nullptr, 0);
         return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
@@ -563,8 +574,8 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
     }
     float *ws = static_cast<float *>(workspace);
     if (D == 128)
-        return launch_bwd<128>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, accumulate_dq != 0, st);
-    return launch_bwd<64>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, accumulate_dq != 0, st);
+        return launch_bwd<128>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, acc_dq, acc_dkdv, st);
+    return launch_bwd<64>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, acc_dq, acc_dkdv, st);
 }
 
 REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a, const regen_bf16 *o_b,

@@ -206,16 +206,21 @@ REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a,
  * Key blocks: when the keys were split into blocks whose partial results were
  * combined by regen_lse_merge, passing the MERGED out and lse with one
  * block's k, v gives that block's exact dk, dv and its share of dq; call once
- * per block with accumulate_dq = 1 after the first to sum the dq shares.
+ * per block with REGEN_ACCUM_DQ after the first to sum the dq shares.
+ * Query blocks (Ring attention's backward, where a key shard meets every
+ * rank's queries): REGEN_ACCUM_DKDV sums the dk, dv shares in the same way.
  *
  *   q, out, dout, dq  [B, H, Sq, D] bf16;  k, v, dk, dv  [B, H, Skv, D] bf16
  *   lse       [B, H, Sq] fp32 (the forward's, natural log)
  *   D         64 or 128 (else REGEN_ERR_UNSUPPORTED); scale finite
  *   workspace device scratch of at least regen_attn_bwd_workspace_bytes(B, H, Sq, D)
  *             bytes, 256-byte aligned, owned by the caller; overwritten.
- *   accumulate_dq  0: dq = result;  1: dq = bf16(dq + result) (dq read first)
+ *   accumulate  a bit set, each bit one output: 0 writes every result;
+ *             REGEN_ACCUM_DQ (1): dq = bf16(dq + result) (dq read first);
+ *             REGEN_ACCUM_DKDV (2): dk, dv = bf16(dk + result), bf16(dv + result);
+ *             any other value: REGEN_ERR_INVALID_ARG.
  * dq, dk, dv must not overlap each other, an input or the workspace.
- * Sq == 0: dk = dv = 0. Skv == 0: dq = 0 (unchanged when accumulating).
+ * Sq == 0: dk = dv = 0; Skv == 0: dq = 0 (each unchanged when it accumulates).
  * B or H == 0: REGEN_OK, nothing done.
  */
 REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
@@ -223,7 +228,8 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
                              regen_bf16 *dq, regen_bf16 *dk, regen_bf16 *dv,
                              int B, int H, int Sq, int Skv, int D, float scale,
                              regen_stream_t stream, void *workspace, int64_t workspace_bytes,
-                             int accumulate_dq);
+                             int accumulate);
+enum { REGEN_ACCUM_DQ = 1, REGEN_ACCUM_DKDV = 2 };
 
 /* Bytes of workspace regen_attn_bwd needs (B*H*ceil(Sq/128)*1024), or a
  * negative status for invalid sizes. */

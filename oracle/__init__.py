@@ -91,6 +91,12 @@ def _load():
             lib.oracle_attention_bwd_bf16.argtypes = [_u16p, _u16p, _u16p, _u16p, _i64, _i64, _i64, _i64,
                                                       ctypes.c_double, _dp, _dp, _dp]
             lib.oracle_attention_bwd_bf16.restype = ctypes.c_int
+            lib.oracle_attention_bwd_block_f64.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64,
+                                                           ctypes.c_double, _dp, _dp, _dp]
+            lib.oracle_attention_bwd_block_f64.restype = None
+            lib.oracle_attention_bwd_block_bf16.argtypes = [_u16p, _u16p, _u16p, _u16p, _dp, _u16p, _i64, _i64,
+                                                            _i64, _i64, ctypes.c_double, _dp, _dp, _dp]
+            lib.oracle_attention_bwd_block_bf16.restype = None
             lib.oracle_attention_bwd_rows_bf16.argtypes = [_u16p, _u16p, _u16p, _u16p, _i64, _i64, _i64, _i64,
                                                            ctypes.c_double, _i64p, _i64, _i64p, _i64, _dp, _dp,
                                                            _dp]
@@ -229,6 +235,38 @@ def attention_bwd(q, k, v, dout, scale: float):
         raise TypeError("inputs must all be uint16 (bf16 bits) or all float64")
     if rc != 0:
         raise MemoryError("oracle could not allocate its per-head P and dS")
+    return dq, dk, dv
+
+
+def attention_bwd_block(q, k, v, out, lse, dout, scale: float):
+    """The gradients contributed by one block of keys, given the whole
+    attention's out and lse: (dq share, dk, dv) in fp64.
+
+    q, out, dout [..., Sq, D]; k, v [..., Skv, D] -- all uint16 (bf16 bits) or
+    all float64; lse [..., Sq] (float64)."""
+    lib = _load()
+    q, k, v, out, dout = (np.ascontiguousarray(a) for a in (q, k, v, out, dout))
+    lse = np.ascontiguousarray(lse, dtype=np.float64)
+    Sq, D = q.shape[-2], q.shape[-1]
+    Skv = k.shape[-2]
+    lead = q.shape[:-2]
+    if (k.shape[:-2] != lead or v.shape != k.shape or out.shape != q.shape or dout.shape != q.shape
+            or k.shape[-1] != D or lse.shape != q.shape[:-1]):
+        raise ValueError("q, k, v, out, lse, dout shapes do not agree")
+    BH = int(np.prod(lead)) if lead else 1
+    dq = np.empty(q.shape, dtype=np.float64)
+    dk = np.empty(k.shape, dtype=np.float64)
+    dv = np.empty(k.shape, dtype=np.float64)
+    kinds = {a.dtype for a in (q, k, v, out, dout)}
+    if kinds == {np.dtype(np.uint16)}:
+        lib.oracle_attention_bwd_block_bf16(*(_ptr(a, _u16p) for a in (q, k, v, out)), _ptr(lse, _dp),
+                                            _ptr(dout, _u16p), BH, Sq, Skv, D, float(scale),
+                                            _ptr(dq, _dp), _ptr(dk, _dp), _ptr(dv, _dp))
+    elif kinds == {np.dtype(np.float64)}:
+        lib.oracle_attention_bwd_block_f64(*(_ptr(a, _dp) for a in (q, k, v, out, lse, dout)), BH, Sq, Skv, D,
+                                           float(scale), _ptr(dq, _dp), _ptr(dk, _dp), _ptr(dv, _dp))
+    else:
+        raise TypeError("q, k, v, out, dout must all be uint16 (bf16 bits) or all float64")
     return dq, dk, dv
 
 

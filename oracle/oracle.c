@@ -17,6 +17,10 @@
  *                          with the natural-log LSE of the scaled logits.
  *   oracle_attention_bwd_f64  the gradients dQ, dK, dV of that attention for an
  *                          upstream dO (chain rule through the softmax).
+ *   oracle_attention_bwd_block_f64  the same chain rule for one block of the
+ *                          keys, with the whole attention's out and LSE given
+ *                          (the step Ring attention's backward repeats per
+ *                          key shard).
  *   oracle_lse_merge_f64   the two-block combination of (O, LSE) that Ring
  *                          attention applies between KV blocks.
  *   oracle_rope3d_f64      3D rotary position embedding of the Wan2.1 DiT
@@ -278,6 +282,73 @@ int oracle_attention_bwd_bf16(const uint16_t *q, const uint16_t *k, const uint16
 {
     src_t sq = {q, 1}, sk = {k, 1}, sv = {v, 1}, sd = {dout, 1};
     return attention_bwd(sq, sk, sv, sd, BH, Sq, Skv, D, scale, dq, dk, dv);
+}
+
+/*
+ * The gradients contributed by one block of keys when the softmax runs over
+ * more keys than the block holds, and its statistics are given: out_i and
+ * lse_i of the whole attention (as Ring attention's backward receives them,
+ * the merged result of every key block). By the chain rule of the full
+ * attention, restricted to the block's keys j:
+ *   P_ij   = exp(scale <q_i, k_j> - lse_i)      (the block's slice of the softmax)
+ *   dP_ij  = <dO_i, v_j>
+ *   delta_i = <dO_i, out_i>                      (= sum over ALL keys of P dP)
+ *   dS_ij  = P_ij (dP_ij - delta_i)
+ *   dq_i  += scale sum_j dS_ij k_j               (this block's share of dq)
+ *   dk_j   = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dO_i   (complete)
+ * Inputs per head [Sq][D] / [Skv][D], lse [Sq]; outputs dq [Sq][D] (the
+ * share), dk, dv [Skv][D].
+ */
+static void attention_bwd_block_head(src_t q, int64_t qo, src_t k, src_t v, int64_t ko, src_t out, src_t dout,
+                                     const double *lse, int64_t Sq, int64_t Skv, int64_t D, double scale,
+                                     double *dq, double *dk, double *dv)
+{
+    for (int64_t x = 0; x < Sq * D; ++x) dq[x] = 0.0;
+    for (int64_t x = 0; x < Skv * D; ++x) { dk[x] = 0.0; dv[x] = 0.0; }
+    for (int64_t i = 0; i < Sq; ++i) {
+        double delta = 0.0;
+        for (int64_t d = 0; d < D; ++d) delta += at(dout, qo + i * D + d) * at(out, qo + i * D + d);
+        for (int64_t j = 0; j < Skv; ++j) {
+            double s = 0.0, dp = 0.0;
+            for (int64_t d = 0; d < D; ++d) {
+                s += at(q, qo + i * D + d) * at(k, ko + j * D + d);
+                dp += at(dout, qo + i * D + d) * at(v, ko + j * D + d);
+            }
+            const double p = exp(scale * s - lse[i]);
+            const double ds = p * (dp - delta);
+            for (int64_t d = 0; d < D; ++d) {
+                dq[i * D + d] += scale * ds * at(k, ko + j * D + d);
+                dk[j * D + d] += scale * ds * at(q, qo + i * D + d);
+                dv[j * D + d] += p * at(dout, qo + i * D + d);
+            }
+        }
+    }
+}
+
+static void attention_bwd_block(src_t q, src_t k, src_t v, src_t out, src_t dout, const double *lse, int64_t BH,
+                                int64_t Sq, int64_t Skv, int64_t D, double scale, double *dq, double *dk,
+                                double *dv)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < BH; ++bh)
+        attention_bwd_block_head(q, bh * Sq * D, k, v, bh * Skv * D, out, dout, lse + bh * Sq, Sq, Skv, D, scale,
+                                 dq + bh * Sq * D, dk + bh * Skv * D, dv + bh * Skv * D);
+}
+
+void oracle_attention_bwd_block_f64(const double *q, const double *k, const double *v, const double *out,
+                                    const double *lse, const double *dout, int64_t BH, int64_t Sq, int64_t Skv,
+                                    int64_t D, double scale, double *dq, double *dk, double *dv)
+{
+    src_t sq = {q, 0}, sk = {k, 0}, sv = {v, 0}, so = {out, 0}, sd = {dout, 0};
+    attention_bwd_block(sq, sk, sv, so, sd, lse, BH, Sq, Skv, D, scale, dq, dk, dv);
+}
+
+void oracle_attention_bwd_block_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *out,
+                                     const double *lse, const uint16_t *dout, int64_t BH, int64_t Sq, int64_t Skv,
+                                     int64_t D, double scale, double *dq, double *dk, double *dv)
+{
+    src_t sq = {q, 1}, sk = {k, 1}, sv = {v, 1}, so = {out, 1}, sd = {dout, 1};
+    attention_bwd_block(sq, sk, sv, so, sd, lse, BH, Sq, Skv, D, scale, dq, dk, dv);
 }
 
 /*

@@ -36,6 +36,8 @@ MUTANTS = {
                            "dS[i * Skv + j] = P[i * Skv + j] * dS[i * Skv + j];"),
     "bwd: dK without scale": ("dk[j * D + d] += scale * dS[i * Skv + j] * at(q, qo + i * D + d);",
                               "dk[j * D + d] += dS[i * Skv + j] * at(q, qo + i * D + d);"),
+    "block bwd: lse not subtracted": ("const double p = exp(scale * s - lse[i]);", "const double p = exp(scale * s);"),
+    "block bwd: delta dropped": ("const double ds = p * (dp - delta);", "const double ds = p * dp;"),
     "bwd: dV uses dS": ("dv[j * D + d] += P[i * Skv + j] * at(dout, doo + i * D + d);",
                         "dv[j * D + d] += dS[i * Skv + j] * at(dout, doo + i * D + d);"),
     "rope bwd: forward rotation used": ("row[base[a] + 2 * j + 1] = c * x1 - s * x0;",

@@ -421,6 +421,40 @@ def test_attention_bwd_rows_equals_full():
     np.testing.assert_allclose(sv, dv[:, :, kr], rtol=1e-12, atol=1e-14)
 
 
+
+def test_attention_bwd_block_with_all_keys_is_the_full_gradient():
+    # one block holding every key, with the attention's own out and lse, is the
+    # full chain rule -- computed independently (softmax and delta recomputed
+    # from q, k, v) by attention_bwd
+    rng = np.random.default_rng(11)
+    q, k, v, g = (rng.normal(size=s) for s in ((2, 2, 29, 16), (2, 2, 41, 16), (2, 2, 41, 16), (2, 2, 29, 16)))
+    out, lse = oracle.attention(q, k, v, 0.37)
+    for a, b in zip(oracle.attention_bwd(q, k, v, g, 0.37), oracle.attention_bwd_block(q, k, v, out, lse, g, 0.37)):
+        np.testing.assert_allclose(b, a, rtol=1e-11, atol=1e-13)
+    # the bf16 entry widens exactly: same numbers on bf16-representable inputs
+    qb, kb, vb, gb, ob = (oracle.f64_to_bf16(x) for x in (q, k, v, g, out))
+    wide = [oracle.bf16_to_f64(x) for x in (qb, kb, vb, ob)]
+    ref = oracle.attention_bwd_block(*wide, lse, oracle.bf16_to_f64(gb), 0.37)
+    for a, b in zip(ref, oracle.attention_bwd_block(qb, kb, vb, ob, lse, gb, 0.37)):
+        np.testing.assert_array_equal(b, a)
+
+
+def test_attention_bwd_block_shares_add_up_over_key_blocks():
+    # keys in three blocks: each block's dk, dv are the full gradient's rows,
+    # and the three dq shares sum to the full dq
+    rng = np.random.default_rng(12)
+    q, g = rng.normal(size=(1, 3, 23, 8)), rng.normal(size=(1, 3, 23, 8))
+    k, v = rng.normal(size=(1, 3, 50, 8)) * 1.5, rng.normal(size=(1, 3, 50, 8))
+    out, lse = oracle.attention(q, k, v, 0.5)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, g, 0.5)
+    share = np.zeros_like(dq)
+    for a, b in ((0, 7), (7, 31), (31, 50)):
+        sq, sk, sv = oracle.attention_bwd_block(q, k[:, :, a:b], v[:, :, a:b], out, lse, g, 0.5)
+        share += sq
+        np.testing.assert_allclose(sk, dk[:, :, a:b], rtol=1e-11, atol=1e-13)
+        np.testing.assert_allclose(sv, dv[:, :, a:b], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(share, dq, rtol=1e-11, atol=1e-13)
+
 # ------------------------------------------------------------- FP8 e4m3 ---
 
 def test_e4m3_decode_table():
