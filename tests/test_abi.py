@@ -133,7 +133,7 @@ _BWD = dict(q=FAKE, k=FAKE + 10 * MB, v=FAKE + 20 * MB, out=FAKE + 30 * MB, lse=
 
 
 @pytest.mark.parametrize("args,status", [
-    (dict(D=96), -2), (dict(B=-1), -1), (dict(Skv=-1), -1), (dict(scale=float("nan")), -1), (dict(acc=2), -1),
+    (dict(D=96), -2), (dict(B=-1), -1), (dict(Skv=-1), -1), (dict(scale=float("nan")), -1), (dict(acc=4), -1), (dict(acc=-1), -1),
     (dict(wsb=-1), -1), (dict(wsb=2047), -1), (dict(ws=None), -1), (dict(lse=None), -1), (dict(dout=None), -1),
     (dict(dk=None), -1), (dict(ws=FAKE + 90 * MB + 16), -3), (dict(dq=FAKE + 60 * MB + 2), -3),
     (dict(dq=FAKE + 4096), -1),            # dq overlaps q
@@ -143,6 +143,7 @@ _BWD = dict(q=FAKE, k=FAKE + 10 * MB, v=FAKE + 20 * MB, out=FAKE + 30 * MB, lse=
     (dict(B=0), 0), (dict(H=0, q=None), 0), (dict(Sq=0, Skv=0), 0),
     (dict(Sq=0, dk=None), -1), (dict(Skv=0, dq=FAKE + 60 * MB + 8), -3),
     (dict(Skv=0, acc=1, dq=FAKE + 60 * MB), 0),   # accumulating nothing: dq unchanged, no launch
+    (dict(Sq=0, acc=2), 0),                       # accumulating nothing: dk, dv unchanged, no launch
 ])
 def test_attn_bwd_validation(lib, args, status):
     a = dict(_BWD)
