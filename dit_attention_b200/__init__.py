@@ -24,6 +24,7 @@ Entry points (same names as the C ABI):
                    workspace, workspace_bytes);  regen_qkv_proj_workspace_bytes(T, Hh, Ww, D)
     regen_out_proj(o, w, bias, y, B, S, H, D, N, stream=None)
     regen_last_device_error() -> (status, site)
+    regen_last_cuda_error() -> (code, name)   (behind this thread's last REGEN_ERR_CUDA)
     regen_set_wait_limit_ns(ns)
 Convenience wrappers that allocate outputs with torch:
     attn_fwd(q, k, v, scale=None) -> (out, lse)
@@ -47,7 +48,7 @@ import threading
 
 __all__ = [
     "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
-    "regen_status_str", "regen_last_device_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
+    "regen_status_str", "regen_last_device_error", "regen_last_cuda_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
     "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes", "regen_attn_fwd_rope3d_noalloc",
     "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd", "regen_rope3d_shard", "regen_quant_e4m3",
     "regen_attn_fwd_fp8", "quant_e4m3", "attn_fwd_fp8", "regen_qkv_proj", "regen_qkv_proj_workspace_bytes",
@@ -69,9 +70,11 @@ REGEN_ACCUM_DQ = 1
 REGEN_ACCUM_DKDV = 2
 
 class RegenError(RuntimeError):
-    def __init__(self, status: int, what: str):
+    def __init__(self, status: int, what: str, cuda_error=None):
         self.status = status
-        super().__init__(f"{what}: {STATUS.get(status, status)} ({_status_text(status)})")
+        self.cuda_error = cuda_error    # (code, name) behind a REGEN_ERR_CUDA, when known
+        detail = f"; CUDA {cuda_error[1]} ({cuda_error[0]})" if cuda_error else ""
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({_status_text(status)}){detail}")
 
 
 def library_path() -> str:
@@ -131,6 +134,8 @@ def load():
         L.regen_selftest_exp2.restype = i32
         L.regen_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp, vp]
         L.regen_selftest_bounded_wait.restype = i32
+        L.regen_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
+        L.regen_last_cuda_error.restype = i32
         L.regen_version.argtypes = []
         L.regen_version.restype = i32
         _lib = L
@@ -164,7 +169,8 @@ def _stream(stream):
 
 def _check(rc: int, what: str) -> None:
     if rc != 0:
-        raise RegenError(rc, what)
+        cuda = regen_last_cuda_error() if rc == -4 else None   # REGEN_ERR_CUDA
+        raise RegenError(rc, what, cuda)
 
 
 # ------------------------------------------------------------- C names ---
@@ -287,6 +293,14 @@ def regen_last_device_error():
     site = ctypes.c_uint32(0)
     rc = load().regen_last_device_error(ctypes.byref(site))
     return rc, site.value
+
+
+def regen_last_cuda_error():
+    """(code, name) of the CUDA result behind this thread's last REGEN_ERR_CUDA
+    (0, "none" when there is none); reading clears it."""
+    name = ctypes.c_char_p()
+    code = load().regen_last_cuda_error(ctypes.byref(name))
+    return code, (name.value or b"").decode()
 
 
 def regen_set_wait_limit_ns(ns: int) -> None:

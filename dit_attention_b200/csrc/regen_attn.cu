@@ -29,6 +29,28 @@ namespace {
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 
+// The CUDA result behind this thread's last REGEN_ERR_CUDA: a cudaError_t, or a
+// driver CUresult + kDriverErrorBase (descriptor encoding); 0 when none.
+constexpr int kDriverErrorBase = 100000;
+thread_local int g_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return REGEN_OK;
+    g_last_cuda_error = static_cast<int>(e);
+    return REGEN_ERR_CUDA;
+}
+
+// Status of the launches issued so far on this thread (and clears the runtime's record).
+int launched() { return cuda_status(cudaGetLastError()); }
+
+bool encoded(CUresult r)
+{
+    if (r == CUDA_SUCCESS) return true;
+    g_last_cuda_error = kDriverErrorBase + static_cast<int>(r);
+    return false;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool overlaps(const void *a, int64_t abytes, const void *b, int64_t bbytes)
@@ -53,6 +75,33 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
+// Make the GPU that holds the device pointer `p` this host thread's current
+// device, with its primary context current (cudaSetDevice does both). The
+// caller's framework usually has done so already; a thread on which no CUDA
+// call has run yet (an autograd worker, a user's own thread) has no current
+// context: the TMA descriptor encoding fails there, and a launch would go to
+// the runtime's default device whatever device the data lives on. The device
+// comes from the pointer (cuPointerGetAttribute needs no context), so no other
+// GPU is touched.
+int bind_device(const void *p)
+{
+    using PFN = CUresult (*)(void *, CUpointer_attribute, CUdeviceptr);
+    static PFN get_attr = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuPointerGetAttribute", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_attr = reinterpret_cast<PFN>(f);
+    });
+    if (!get_attr) return cuda_status(cudaErrorNotSupported);
+    int ordinal = -1;
+    if (!encoded(get_attr(&ordinal, CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL, reinterpret_cast<CUdeviceptr>(p))))
+        return REGEN_ERR_CUDA;
+    return cuda_status(cudaSetDevice(ordinal));
+}
+
 // [BH, S, D] bf16 viewed as a 3D tensor (D innermost), boxes of 64 x 128 x 1
 // with the 128-byte swizzle; out-of-range rows read as zero.
 bool make_bhsd_map(CUtensorMap *map, const void *base, int64_t BH, int64_t S, int64_t D)
@@ -67,7 +116,7 @@ bool make_bhsd_map(CUtensorMap *map, const void *base, int64_t BH, int64_t S, in
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return encoded(r);
 }
 
 // [BH, S, 128] E4M3 codes as a 3D tensor (128 codes innermost), boxes of
@@ -83,7 +132,7 @@ bool make_u8_map(CUtensorMap *map, const void *base, int64_t BH, int64_t S)
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return encoded(r);
 }
 
 // bf16 [d2][d1][d0] (d0 innermost) as a 3D tensor with boxes of box0 x box1 x 1
@@ -100,7 +149,7 @@ bool make_bf16_map3(CUtensorMap *map, const void *base, int64_t d0, int64_t d1, 
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return encoded(r);
 }
 
 int num_sms()
@@ -147,7 +196,7 @@ int launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const regen::ProjS
     const uint64_t limit = g_wait_limit_ns.load();
     if (cudaLaunchKernelEx(&cfg, regen::proj_gemm_kernel<MODE>, ta, tb, shape, ep, limit) != cudaSuccess)
         return REGEN_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
 }
 
 template <bool NEG>
@@ -177,7 +226,7 @@ int launch_attn_fp8(const uint8_t *q8, const float *qs, const uint8_t *k8, const
     const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     regen::attn_fwd_fp8_kernel<NEG><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
         tq, tk, tv, to, qs, ks, vs, lse, Sq, Skv, scale_log2, g_wait_limit_ns.load());
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
 }
 
 template <int HD, bool NEG, bool ROPE_Q = false>
@@ -209,7 +258,7 @@ int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, r
     const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     regen::attn_fwd_kernel<HD, NEG, ROPE_Q><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
         tq, tk, tv, to, lse, Sq, Skv, scale_log2, g_wait_limit_ns.load(), rope_tab, geom);
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
 }
 
 // Gradient launches: prep (delta, lse2) -> dK/dV -> dQ, all on `stream`.
@@ -267,7 +316,7 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
     const int64_t prep_work = BH * nq * 128 * (HD / 8);
     regen::attn_bwd_prep_kernel<<<grid_for(prep_work, 256), 256, 0, stream>>>(
         reinterpret_cast<const uint4 *>(out), reinterpret_cast<const uint4 *>(dout), lse, ws, BH, Sq, HD, nq);
-    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     const uint64_t limit = g_wait_limit_ns.load();
     const uint16_t *dk_old = reinterpret_cast<const uint16_t *>(dk);
@@ -278,14 +327,14 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
     else
         regen::attn_bwd_dkdv_kernel<HD, false><<<static_cast<unsigned>(BH * nkv), C::THREADS, C::A_SMEM_BYTES, stream>>>(
             tq, tk, tv, tdo, tdk, tdv, ws, Sq, Skv, scale, scale_log2, limit, dk_old, dv_old);
-    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     if (acc_dq)
         regen::attn_bwd_dq_kernel<HD, true><<<static_cast<unsigned>(BH * nq), C::THREADS, C::B_SMEM_BYTES, stream>>>(
             tq, tk, tv, tdo, tdq, dq, ws, Sq, Skv, scale, scale_log2, limit);
     else
         regen::attn_bwd_dq_kernel<HD, false><<<static_cast<unsigned>(BH * nq), C::THREADS, C::B_SMEM_BYTES, stream>>>(
             tq, tk, tv, tdo, tdq, dq, ws, Sq, Skv, scale, scale_log2, limit);
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
 }
 
 int64_t bwd_workspace_bytes(int64_t BH, int64_t Sq) { return BH * ((Sq + 127) / 128) * 1024; }
@@ -309,11 +358,11 @@ int attn_rope3d_with_scratch(const regen_bf16 *q, const regen_bf16 *k, const reg
     double *tab = reinterpret_cast<double *>(scratch);
     regen_bf16 *k_rot = reinterpret_cast<regen_bf16 *>(scratch + rope_table_bytes(geom));
     regen::rope_table_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
-    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     const int64_t chunks = BH * S * (D / 8);
     regen::rope_apply_kernel<<<grid_for(chunks, 256), 256, 0, st>>>(
         reinterpret_cast<const uint4 *>(k), reinterpret_cast<uint4 *>(k_rot), BH, S, D, geom, tab);
-    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     const bool neg = scale < 0.0f;
     if (D == 128)
         return neg ? launch_attn<128, true, true>(q, k_rot, v, out, lse, BH, S, S, scale, st, tab, geom)
@@ -372,9 +421,10 @@ int rope3d_common(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float the
     const int threads = 128;
     const int64_t blocks = (work + threads - 1) / threads;
     if (blocks > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (const int rc = bind_device(q ? q : k); rc != REGEN_OK) return rc;
     regen::rope3d_kernel<<<static_cast<unsigned>(blocks), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         q, k, BH, static_cast<int>(S), Hh, Ww, D, static_cast<double>(theta), inverse, S_local >= 0 ? n0 : 0);
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
 }
 
 
@@ -401,12 +451,13 @@ REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const reg
         overlaps(lse, lbytes, k, kvbytes) || overlaps(lse, lbytes, v, kvbytes) ||
         overlaps(lse, lbytes, out, qbytes))
         return REGEN_ERR_INVALID_ARG;
+    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (Skv == 0) {
         const int64_t n16 = qbytes / 16;
         regen::attn_empty_kernel<<<grid_for(n16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(out), n16,
                                                                       lse, BH * Sq);
-        return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+        return launched();
     }
     const bool neg = scale < 0.0f;
     if (D == 128)
@@ -456,6 +507,7 @@ REGEN_API int regen_attn_fwd_rope3d(const regen_bf16 *q, const regen_bf16 *k, co
     if (overlaps(lse, lbytes, out, tbytes) || overlaps(workspace, need, out, tbytes) ||
         overlaps(workspace, need, lse, lbytes))
         return REGEN_ERR_INVALID_ARG;
+    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
     return attn_rope3d_with_scratch(q, k, v, out, lse, BH, static_cast<int>(S), D, scale, theta, geom,
                                     static_cast<uint8_t *>(workspace), reinterpret_cast<cudaStream_t>(stream));
 }
@@ -486,6 +538,7 @@ REGEN_API int regen_attn_fwd_rope3d_noalloc(const regen_bf16 *q, const regen_bf1
     for (const void *in : ins)
         if (overlaps(out, tbytes, in, tbytes) || overlaps(lse, lbytes, in, tbytes)) return REGEN_ERR_INVALID_ARG;
     if (overlaps(lse, lbytes, out, tbytes)) return REGEN_ERR_INVALID_ARG;
+    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
     uint8_t *scratch = noalloc_scratch_on_current_device();
     if (!scratch) return REGEN_ERR_CUDA;
     // Every scratch byte this call reads is written earlier in the same call
@@ -541,10 +594,11 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
         if (!aligned16(dk) || !aligned16(dv)) return REGEN_ERR_MISALIGNED;
         if (overlaps(dk, kvbytes, dv, kvbytes)) return REGEN_ERR_INVALID_ARG;
         if (acc_dkdv) return REGEN_OK;
+        if (const int rc = bind_device(dk); rc != REGEN_OK) return rc;
         for (regen_bf16 *z : {dk, dv}) {
             regen::attn_empty_kernel<<<grid_for(kvbytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(z),
                                                                                  kvbytes / 16, nullptr, 0);
-            if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+            if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
         }
         return REGEN_OK;
     }
@@ -552,9 +606,10 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
         if (!dq) return REGEN_ERR_INVALID_ARG;
         if (!aligned16(dq)) return REGEN_ERR_MISALIGNED;
         if (acc_dq) return REGEN_OK;
+        if (const int rc = bind_device(dq); rc != REGEN_OK) return rc;
         regen::attn_empty_kernel<<<grid_for(qbytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(dq),
                                                                             qbytes / 16, nullptr, 0);
-        return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+        return launched();
     }
     if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace) return REGEN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
@@ -573,6 +628,7 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
             if (overlaps(outs[a].p, outs[a].n, outs[b].p, outs[b].n)) return REGEN_ERR_INVALID_ARG;
     }
     float *ws = static_cast<float *>(workspace);
+    if (const int rc = bind_device(dq); rc != REGEN_OK) return rc;
     if (D == 128)
         return launch_bwd<128>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, acc_dq, acc_dkdv, st);
     return launch_bwd<64>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, acc_dq, acc_dkdv, st);
@@ -600,10 +656,11 @@ REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a, const r
     if ((overlaps(out, obytes, o_a, obytes) && out != o_a) || (overlaps(out, obytes, o_b, obytes) && out != o_b))
         return REGEN_ERR_INVALID_ARG;
     const int64_t work = rows * (D / 8);
+    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
     regen::lse_merge_kernel<<<grid_for(work, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const uint4 *>(o_a), lse_a, reinterpret_cast<const uint4 *>(o_b), lse_b,
         reinterpret_cast<uint4 *>(out), lse_out, rows, D);
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
 }
 
 REGEN_API int regen_quant_e4m3(const regen_bf16 *x, uint8_t *codes, float *scales, int B, int H, int S, int D,
@@ -621,6 +678,7 @@ REGEN_API int regen_quant_e4m3(const regen_bf16 *x, uint8_t *codes, float *scale
     if (overlaps(codes, cbytes, x, xbytes) || overlaps(scales, sbytes, x, xbytes) ||
         overlaps(scales, sbytes, codes, cbytes))
         return REGEN_ERR_INVALID_ARG;
+    if (const int rc = bind_device(codes); rc != REGEN_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const unsigned grid = static_cast<unsigned>(BH * nb);
     if (D == 128)
@@ -631,7 +689,7 @@ REGEN_API int regen_quant_e4m3(const regen_bf16 *x, uint8_t *codes, float *scale
         regen::quant_e4m3_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(x),
                                                            reinterpret_cast<uint2 *>(codes), scales, S,
                                                            static_cast<int>(nb));
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
 }
 
 REGEN_API int regen_attn_fwd_fp8(const uint8_t *q8, const float *q_scale, const uint8_t *k8, const float *k_scale,
@@ -657,11 +715,12 @@ REGEN_API int regen_attn_fwd_fp8(const uint8_t *q8, const float *q_scale, const 
     for (const Span &in : ins)
         if (overlaps(out, obytes, in.p, in.n) || overlaps(lse, lbytes, in.p, in.n)) return REGEN_ERR_INVALID_ARG;
     if (overlaps(lse, lbytes, out, obytes)) return REGEN_ERR_INVALID_ARG;
+    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (Skv == 0) {
         regen::attn_empty_kernel<<<grid_for(obytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(out),
                                                                             obytes / 16, lse, BH * Sq);
-        return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+        return launched();
     }
     return scale < 0.0f ? launch_attn_fp8<true>(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, BH, Sq, Skv, scale, st)
                         : launch_attn_fp8<false>(q8, q_scale, k8, k_scale, v8, v_scale, out, lse, BH, Sq, Skv, scale, st);
@@ -706,10 +765,11 @@ REGEN_API int regen_qkv_proj(const regen_bf16 *x, const regen_bf16 *w, const flo
     }
     for (int a = 0; a < 5; ++a)
         if (overlaps(workspace, tab_bytes, ins[a].p, ins[a].n)) return REGEN_ERR_INVALID_ARG;
+    if (const int rc = bind_device(q); rc != REGEN_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float2 *tab = static_cast<float2 *>(workspace);
     regen::rope_table_f32_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
-    if (cudaGetLastError() != cudaSuccess) return REGEN_ERR_CUDA;
+    if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     CUtensorMap ta, tb;
     if (!make_bf16_map3(&ta, x, C, S, B, 64, 128) || !make_bf16_map3(&tb, w, C, N, 1, 64, 128)) return REGEN_ERR_CUDA;
     regen::ProjShape shape{B, S, C, static_cast<int>(N), H, B * ((S + 255) / 256), static_cast<int>((N + 255) / 256)};
@@ -733,6 +793,7 @@ REGEN_API int regen_out_proj(const regen_bf16 *o, const regen_bf16 *w, const flo
                   ybytes = static_cast<int64_t>(B) * S * N * 2;
     if (overlaps(y, ybytes, o, obytes) || overlaps(y, ybytes, w, wbytes) || overlaps(y, ybytes, bias, N * 4LL))
         return REGEN_ERR_INVALID_ARG;
+    if (const int rc = bind_device(y); rc != REGEN_OK) return rc;
     CUtensorMap ta, tb;
     if (!make_bhsd_map(&ta, o, static_cast<int64_t>(B) * H, S, 128) || !make_bf16_map3(&tb, w, K, N, 1, 64, 128))
         return REGEN_ERR_CUDA;
@@ -747,17 +808,35 @@ REGEN_API int regen_selftest_exp2(const float *x, float *y, int64_t n, regen_str
     if (n == 0) return REGEN_OK;
     if (!x || !y) return REGEN_ERR_INVALID_ARG;
     const int64_t npairs = n / 2;
+    if (const int rc = bind_device(y); rc != REGEN_OK) return rc;
     regen::exp2_poly_selftest_kernel<<<grid_for(npairs, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         x, y, npairs);
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
 }
 
 REGEN_API int regen_selftest_bounded_wait(uint64_t limit_ns, int *done, regen_stream_t stream)
 {
     if (!done) return REGEN_ERR_INVALID_ARG;
     if (limit_ns == 0 || limit_ns > 5000000000ull) return REGEN_ERR_INVALID_ARG;
+    if (const int rc = bind_device(done); rc != REGEN_OK) return rc;
     regen::bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, done);
-    return cudaGetLastError() == cudaSuccess ? REGEN_OK : REGEN_ERR_CUDA;
+    return launched();
+}
+
+REGEN_API int regen_last_cuda_error(const char **name)
+{
+    const int e = g_last_cuda_error;
+    g_last_cuda_error = 0;
+    if (name) {
+        if (e == 0) {
+            *name = "none";
+        } else if (e >= kDriverErrorBase) {
+            *name = "tensor-map encoding failed (CUresult = code - 100000)";
+        } else {
+            *name = cudaGetErrorName(static_cast<cudaError_t>(e));
+        }
+    }
+    return e;
 }
 
 REGEN_API const char *regen_status_str(int status)

@@ -39,6 +39,12 @@ def _kernel_merge(o_a, lse_a, o_b, lse_b):
     return lse_merge(o_a, lse_a, o_b, lse_b)
 
 
+def _kernel_bwd(q, k, v, out, lse, dout, scale, dq, dk, dv, acc_dq, acc_dkdv):
+    from . import attn_bwd
+    return attn_bwd(q, k, v, out, lse, dout, scale, dq=dq, dk=dk, dv=dv, accumulate_dq=acc_dq,
+                    accumulate_dkdv=acc_dkdv)
+
+
 def shard_range(S: int, index: int, count: int):
     """Token range [start, stop) of shard `index` of `count` equal shards of S tokens."""
     if S % count:
@@ -78,6 +84,53 @@ def ring_attention(q, k, v, group=None, scale=None, attn=None, merge=None):
         if step < R - 1:
             cur_k, cur_v = nk, nv
     return out, lse
+
+
+def ring_attention_bwd(q, k, v, out, lse, dout, group=None, scale=None, bwd=None):
+    """Gradients (dq, dk, dv) of ring_attention for this rank's q, k, v shards.
+
+    out, lse: this rank's ring_attention result (the attention over every
+    rank's keys); dout: its upstream gradient. Step s: the key shard of rank
+    (r - s) mod R visits together with the dk, dv that the ranks before have
+    accumulated for it; this rank adds its queries' contribution (the gradient
+    kernel with the merged out and lse, accumulating into the visiting dk, dv)
+    and its own dq gathers that shard's share. The key shards travel on while
+    the step is computed; the accumulators follow once it is done, and a last
+    hop returns each shard's dk, dv to its owner.
+
+    bwd(q, k, v, out, lse, dout, scale, dq, dk, dv, acc_dq, acc_dkdv) -> (dq, dk, dv)
+    computes (or accumulates, when acc_*) one step; by default the library's
+    regen_attn_bwd."""
+    bwd = bwd or _kernel_bwd
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    nxt = dist.get_global_rank(group, (r + 1) % R) if group is not None else (r + 1) % R
+    prv = dist.get_global_rank(group, (r - 1) % R) if group is not None else (r - 1) % R
+    q, out, dout = q.contiguous(), out.contiguous(), dout.contiguous()
+    cur_k, cur_v = k.contiguous(), v.contiguous()
+    dq, cur_dk, cur_dv = torch.empty_like(q), torch.empty_like(cur_k), torch.empty_like(cur_v)
+    for step in range(R):
+        reqs = []
+        if step < R - 1:
+            nk, nv = torch.empty_like(cur_k), torch.empty_like(cur_v)
+            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur_k, nxt, group),
+                                           dist.P2POp(dist.irecv, nk, prv, group),
+                                           dist.P2POp(dist.isend, cur_v, nxt, group),
+                                           dist.P2POp(dist.irecv, nv, prv, group)])
+        dq, cur_dk, cur_dv = bwd(q, cur_k, cur_v, out, lse, dout, scale, dq, cur_dk, cur_dv, step > 0, step > 0)
+        ndk, ndv = torch.empty_like(cur_dk), torch.empty_like(cur_dv)
+        reqs += dist.batch_isend_irecv([dist.P2POp(dist.isend, cur_dk.contiguous(), nxt, group),
+                                        dist.P2POp(dist.irecv, ndk, prv, group),
+                                        dist.P2POp(dist.isend, cur_dv.contiguous(), nxt, group),
+                                        dist.P2POp(dist.irecv, ndv, prv, group)])
+        for req in reqs:
+            req.wait()
+        cur_dk, cur_dv = ndk, ndv
+        if step < R - 1:
+            cur_k, cur_v = nk, nv
+    return dq, cur_dk, cur_dv
 
 
 def seq_to_heads(x, group=None):
@@ -135,3 +188,33 @@ def usp_attention(q, k, v, ulysses_group, ring_group, scale=None, attn=None, mer
     qh, kh, vh = (seq_to_heads(t, ulysses_group) for t in (q, k, v))       # [B, H/U, S/R, D]
     out, lse = ring_attention(qh, kh, vh, ring_group, scale, attn, merge)
     return heads_to_seq(out, ulysses_group), heads_to_seq(lse, ulysses_group)
+
+
+class _USPAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, ulysses_group, ring_group, scale, attn, merge, bwd):
+        qh, kh, vh = (seq_to_heads(t.contiguous(), ulysses_group) for t in (q, k, v))
+        oh, lh = ring_attention(qh, kh, vh, ring_group, scale, attn, merge)
+        ctx.save_for_backward(qh, kh, vh, oh, lh)
+        ctx.groups, ctx.scale, ctx.bwd = (ulysses_group, ring_group), scale, bwd
+        return heads_to_seq(oh, ulysses_group)
+
+    @staticmethod
+    def backward(ctx, dout):
+        qh, kh, vh, oh, lh = ctx.saved_tensors
+        ug, rg_ = ctx.groups
+        # the all-to-all is a permutation of the data over the ranks: its
+        # adjoint is the inverse all-to-all
+        doh = seq_to_heads(dout.contiguous(), ug)
+        dqh, dkh, dvh = ring_attention_bwd(qh, kh, vh, oh, lh, doh, rg_, ctx.scale, ctx.bwd)
+        return (heads_to_seq(dqh, ug), heads_to_seq(dkh, ug), heads_to_seq(dvh, ug),
+                None, None, None, None, None, None)
+
+
+def usp_attention_autograd(q, k, v, ulysses_group, ring_group, scale=None, attn=None, merge=None, bwd=None):
+    """usp_attention as a differentiable function of this rank's q, k, v
+    shards (RoPE already applied): the backward runs the Ulysses all-to-alls
+    in reverse around ring_attention_bwd. Returns this rank's out shard."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    return _USPAttention.apply(q, k, v, ulysses_group, ring_group, float(scale), attn, merge, bwd)

@@ -342,6 +342,15 @@ REGEN_API int regen_selftest_bounded_wait(uint64_t limit_ns, int *done, regen_st
 REGEN_API const char *regen_status_str(int status);
 
 /*
+ * regen_last_cuda_error -- the CUDA result behind the last REGEN_ERR_CUDA that
+ * a call on THIS host thread returned: a cudaError_t (its name in *name when
+ * name is not NULL), or 100000 + a driver CUresult when a TMA descriptor could
+ * not be encoded; 0 (name "none") when there is none. Reading clears it.
+ * The string is static; the caller does not free it.
+ */
+REGEN_API int regen_last_cuda_error(const char **name);
+
+/*
  * regen_last_device_error -- REGEN_OK, or REGEN_ERR_TIMEOUT when a kernel of
  * this library gave up on a bounded wait since the previous call; clears the
  * record. It synchronises the device first (cudaDeviceSynchronize) and

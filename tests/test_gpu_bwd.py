@@ -126,6 +126,28 @@ def test_attn_bwd_key_blocks_with_merged_stats():
     check_grad(np.concatenate([to_bits(dva), to_bits(dvb)], axis=2), rv, "merged dv")
 
 
+def test_attn_bwd_query_blocks_accumulate_dkdv():
+    # queries in two blocks (as Ring attention's backward meets a key shard once
+    # per rank): the second call adds its dk, dv into the first's, and the sums
+    # equal the gradient over all queries; dq rows are independent per block
+    B, H, Skv, D = 1, 2, 300, 128
+    s1, s2 = 197, 230
+    q, g = rand_bf16((B, H, s1 + s2, D)), rand_bf16((B, H, s1 + s2, D))
+    k, v = rand_bf16((B, H, Skv, D)), rand_bf16((B, H, Skv, D))
+    scale = 1 / np.sqrt(D)
+    tq, tk, tv, tg = to_dev(q), to_dev(k), to_dev(v), to_dev(g)
+    out, lse = rg.attn_fwd(tq, tk, tv, scale)
+    c = lambda t, a, b: t[:, :, a:b].contiguous()  # noqa: E731
+    dq1, dk, dv = rg.attn_bwd(c(tq, 0, s1), tk, tv, c(out, 0, s1), c(lse, 0, s1), c(tg, 0, s1), scale)
+    dq2, _, _ = rg.attn_bwd(c(tq, s1, s1 + s2), tk, tv, c(out, s1, s1 + s2), c(lse, s1, s1 + s2),
+                            c(tg, s1, s1 + s2), scale, dk=dk, dv=dv, accumulate_dkdv=True)
+    torch.cuda.synchronize()
+    rq, rk, rv = oracle.attention_bwd(q, k, v, g, scale)
+    check_grad(np.concatenate([to_bits(dq1), to_bits(dq2)], axis=2), rq, "query-block dq")
+    check_grad(to_bits(dk), rk, "dk accumulated over two query blocks")
+    check_grad(to_bits(dv), rv, "dv accumulated over two query blocks")
+
+
 def test_attn_bwd_empty_sides():
     t = lambda *s: torch.full(s, 3.0, dtype=torch.bfloat16, device="cuda")  # noqa: E731
     q, out, g = t(1, 2, 0, 128), t(1, 2, 0, 128), t(1, 2, 0, 128)
@@ -144,6 +166,12 @@ def test_attn_bwd_empty_sides():
     rg.attn_bwd(q, k, v, out, lse, g, 0.1, dq=dq, accumulate_dq=True)
     torch.cuda.synchronize()
     assert float(dq.min()) == 3.0 and float(dq.max()) == 3.0                 # accumulating nothing
+    q, out, g = t(1, 2, 0, 128), t(1, 2, 0, 128), t(1, 2, 0, 128)
+    k, v = t(1, 2, 50, 128), t(1, 2, 50, 128)
+    dk, dv = t(1, 2, 50, 128), t(1, 2, 50, 128)
+    rg.attn_bwd(q, k, v, out, torch.zeros((1, 2, 0), device="cuda"), g, 0.1, dk=dk, dv=dv, accumulate_dkdv=True)
+    torch.cuda.synchronize()
+    assert float(torch.stack([dk, dv]).min()) == 3.0 and float(torch.stack([dk, dv]).max()) == 3.0
 
 
 def test_attn_bwd_workspace_errors():

@@ -351,3 +351,34 @@ def test_attention_ragged_multi_tile(B, H, Sq, Skv):
     ref, rl = oracle.attention(q, k, v, 1 / math.sqrt(128))
     check_attention(to_bits(out).reshape(-1, 128), lse.cpu().numpy().reshape(-1), ref.reshape(-1, 128),
                     rl.reshape(-1), f"{B}x{H}x{Sq}x{Skv}")
+
+
+def test_calls_from_a_fresh_host_thread():
+    # A thread on which no CUDA call has run has no current context (a torch
+    # autograd worker, a user's own thread). Every entry point binds the device
+    # that holds its data first: the same calls there give the same bits, after
+    # the main thread has already used the library.
+    import threading
+    B, H, S, D = 1, 2, 300, 128
+    q, k, v, g = (synth.f64_to_bf16_bits(RNG.normal(size=(B, H, S, D))) for _ in range(4))
+    tq, tk, tv, tg = to_dev(q), to_dev(k), to_dev(v), to_dev(g)
+    out, lse = rg.attn_fwd(tq, tk, tv)
+    grads = rg.attn_bwd(tq, tk, tv, out, lse, tg)
+    torch.cuda.synchronize()
+    res = {}
+
+    def worker():
+        try:
+            o2, l2 = rg.attn_fwd(tq, tk, tv)
+            g2 = rg.attn_bwd(tq, tk, tv, o2, l2, tg)
+            torch.cuda.synchronize()
+            res["ok"] = (o2, l2) + tuple(g2)
+        except Exception as e:  # reported below, on the main thread
+            res["err"] = repr(e)
+
+    t = threading.Thread(target=worker)
+    t.start()
+    t.join()
+    assert "err" not in res, res.get("err")
+    for a, b in zip((out, lse) + tuple(grads), res["ok"]):
+        assert torch.equal(a, b)

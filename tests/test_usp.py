@@ -117,6 +117,65 @@ def test_unified_sequence_parallel_ulysses2_ring2():
         assert eo < 1e-12 and el < 1e-12, (r, eo, el)
 
 
+def _oracle_bwd(q, k, v, out, lse, dout, scale, dq, dk, dv, acc_dq, acc_dkdv):
+    sq, sk, sv = (torch.from_numpy(x) for x in oracle.attention_bwd_block(
+        q.numpy(), k.numpy(), v.numpy(), out.numpy(), lse.numpy(), dout.numpy(), scale))
+    return (dq + sq if acc_dq else sq), (dk + sk if acc_dkdv else sk), (dv + sv if acc_dkdv else sv)
+
+
+def _dout(B=1, H=4, S=96, D=16, seed=6):
+    return np.random.default_rng(seed).normal(size=(B, H, S, D))
+
+
+def _rel(a, b):
+    return float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-300))
+
+
+def _ring_bwd_case(rank, world, S):
+    q, k, v = _window(S=S)
+    g = _dout(S=S)
+    scale = 0.25
+    a, b = usp.shard_range(S, rank, world)
+    sl = lambda x: torch.from_numpy(x[:, :, a:b].copy())  # noqa: E731
+    o, l = usp.ring_attention(sl(q), sl(k), sl(v), None, scale, _oracle_attn, _oracle_merge)
+    dq, dk, dv = usp.ring_attention_bwd(sl(q), sl(k), sl(v), o, l, sl(g), None, scale, _oracle_bwd)
+    rq, rk, rv = oracle.attention_bwd(q, k, v, g, scale)
+    return (_rel(dq.numpy(), rq[:, :, a:b]), _rel(dk.numpy(), rk[:, :, a:b]), _rel(dv.numpy(), rv[:, :, a:b]))
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ring_attention_backward_is_exact(world):
+    # every rank's dq, dk, dv of its own shards equal the oracle's gradient of
+    # the whole window: the key shards and their accumulators went all the way round
+    res = _run(world, _ring_bwd_case, 96)
+    assert sorted(res) == list(range(world))
+    for r, errs in res.items():
+        assert max(errs) < 1e-10, (r, errs)
+
+
+def _usp_autograd_case(rank, world, U, R):
+    ug, rg_ = usp.usp_groups(U, R)
+    q, k, v = _window(H=4, S=96)
+    g = _dout(H=4, S=96)
+    scale = 0.25
+    a, b = usp.shard_range(96, rank, world)
+    leaf = lambda x: torch.from_numpy(x[:, :, a:b].copy()).requires_grad_(True)  # noqa: E731
+    tq, tk, tv = leaf(q), leaf(k), leaf(v)
+    out = usp.usp_attention_autograd(tq, tk, tv, ug, rg_, scale, _oracle_attn, _oracle_merge, _oracle_bwd)
+    out.backward(torch.from_numpy(g[:, :, a:b].copy()))
+    ref, _ = oracle.attention(q, k, v, scale)
+    rq, rk, rv = oracle.attention_bwd(q, k, v, g, scale)
+    return (_rel(out.detach().numpy(), ref[:, :, a:b]), _rel(tq.grad.numpy(), rq[:, :, a:b]),
+            _rel(tk.grad.numpy(), rk[:, :, a:b]), _rel(tv.grad.numpy(), rv[:, :, a:b]))
+
+
+def test_unified_sequence_parallel_autograd_ulysses2_ring2():
+    # forward and backward through the all-to-alls and the ring on 2 x 2 ranks
+    res = _run(4, _usp_autograd_case, 2, 2)
+    for r, errs in res.items():
+        assert max(errs) < 1e-10, (r, errs)
+
+
 def test_shard_range():
     assert usp.shard_range(31200, 3, 8) == (11700, 15600)
     with pytest.raises(ValueError):
@@ -167,3 +226,54 @@ def test_ring_attention_with_kernels_two_ranks_one_gpu():
         np.testing.assert_array_equal(gk, kr[:, :, a:b])
         check_attention(o.reshape(-1, 128), l.reshape(-1), ref[:, :, a:b].reshape(-1, 128), rl[:, :, a:b].reshape(-1),
                         f"ring rank {r}")
+
+
+def _gpu_ring_bwd_case(rank, world):
+    import dit_attention_b200 as rg
+    torch.cuda.set_device(0)
+    w = synth.Workload("usp", B=1, H=4, D=128, Sq=1040, Skv=1040, seed=9, grid=(2, 20, 26), rope=True, rmsnorm=True)
+    q, k, v = synth.make_inputs(w)
+    g = synth.make_dout(w)
+    a, b = usp.shard_range(w.Sq, rank, world)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
+    tq, tk, tv, tg = dev(q[:, :, a:b]), dev(k[:, :, a:b]), dev(v[:, :, a:b]), dev(g[:, :, a:b])
+    T, Hh, Ww = w.grid
+    rg.regen_rope3d_shard(tq, tk, T, Hh, Ww, w.theta, w.B, w.H, w.D, a, b - a, 0)
+
+    # per-rank compute in the library's kernels; the shards travel as host tensors
+    def attn(qh, kh, vh, scale):
+        o, l = rg.attn_fwd(qh.cuda(), kh.cuda(), vh.cuda(), scale)
+        return o.cpu(), l.cpu()
+
+    def merge(oa, la, ob, lb):
+        o, l = rg.lse_merge(oa.cuda(), la.cuda(), ob.cuda(), lb.cuda())
+        return o.cpu(), l.cpu()
+
+    def bwd(q_, k_, v_, out, lse, dout, scale, dq, dk, dv, acc_dq, acc_dkdv):
+        c = lambda t: t.cuda()  # noqa: E731
+        r = rg.attn_bwd(c(q_), c(k_), c(v_), c(out), c(lse), c(dout), scale, dq=c(dq), dk=c(dk), dv=c(dv),
+                        accumulate_dq=acc_dq, accumulate_dkdv=acc_dkdv)
+        return tuple(t.cpu() for t in r)
+
+    o, l = usp.ring_attention(tq.cpu(), tk.cpu(), tv.cpu(), None, w.scale, attn, merge)
+    dq, dk, dv = usp.ring_attention_bwd(tq.cpu(), tk.cpu(), tv.cpu(), o, l, tg.cpu(), None, w.scale, bwd)
+    torch.cuda.synchronize()
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    return bits(dq), bits(dk), bits(dv), a, b
+
+
+@pytest.mark.gpu
+def test_ring_attention_backward_with_kernels_two_ranks_one_gpu():
+    from util import check_grad
+    assert torch.cuda.is_available()
+    res = _run(2, _gpu_ring_bwd_case)
+    w = synth.Workload("usp", B=1, H=4, D=128, Sq=1040, Skv=1040, seed=9, grid=(2, 20, 26), rope=True, rmsnorm=True)
+    q, k, v = synth.make_inputs(w)
+    g = synth.make_dout(w)
+    qr, kr = oracle.rope3d(q, w.grid, w.theta), oracle.rope3d(k, w.grid, w.theta)
+    rq, rk, rv = oracle.attention_bwd(qr, kr, v, g, w.scale)
+    for r, (dq, dk, dv, a, b) in res.items():
+        # gradients with respect to the rotated shards (RoPE's own gradient is pinned elsewhere)
+        check_grad(dq, rq[:, :, a:b], f"ring dq rank {r}")
+        check_grad(dk, rk[:, :, a:b], f"ring dk rank {r}")
+        check_grad(dv, rv[:, :, a:b], f"ring dv rank {r}")
