@@ -75,32 +75,85 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// Make the GPU that holds the device pointer `p` this host thread's current
-// device, with its primary context current (cudaSetDevice does both). The
-// caller's framework usually has done so already; a thread on which no CUDA
-// call has run yet (an autograd worker, a user's own thread) has no current
-// context: the TMA descriptor encoding fails there, and a launch would go to
-// the runtime's default device whatever device the data lives on. The device
-// comes from the pointer (cuPointerGetAttribute needs no context), so no other
-// GPU is touched.
-int bind_device(const void *p)
+// Driver entry points, through the runtime (no libcuda link).
+struct DriverCalls {
+    CUresult (*pointer_attr)(void *, CUpointer_attribute, CUdeviceptr) = nullptr;
+    CUresult (*ctx_get_current)(CUcontext *) = nullptr;
+    CUresult (*ctx_get_device)(CUdevice *) = nullptr;
+    CUresult (*ctx_set_current)(CUcontext) = nullptr;
+    bool ok() const { return pointer_attr && ctx_get_current && ctx_get_device && ctx_set_current; }
+};
+
+const DriverCalls &driver()
 {
-    using PFN = CUresult (*)(void *, CUpointer_attribute, CUdeviceptr);
-    static PFN get_attr = nullptr;
+    static DriverCalls d;
     static std::once_flag once;
     std::call_once(once, [] {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuPointerGetAttribute", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_attr = reinterpret_cast<PFN>(f);
+        auto get = [](const char *name) -> void * {
+            void *f = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            return cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) == cudaSuccess &&
+                           q == cudaDriverEntryPointSuccess ? f : nullptr;
+        };
+        d.pointer_attr = reinterpret_cast<decltype(d.pointer_attr)>(get("cuPointerGetAttribute"));
+        d.ctx_get_current = reinterpret_cast<decltype(d.ctx_get_current)>(get("cuCtxGetCurrent"));
+        d.ctx_get_device = reinterpret_cast<decltype(d.ctx_get_device)>(get("cuCtxGetDevice"));
+        d.ctx_set_current = reinterpret_cast<decltype(d.ctx_set_current)>(get("cuCtxSetCurrent"));
     });
-    if (!get_attr) return cuda_status(cudaErrorNotSupported);
-    int ordinal = -1;
-    if (!encoded(get_attr(&ordinal, CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL, reinterpret_cast<CUdeviceptr>(p))))
-        return REGEN_ERR_CUDA;
-    return cuda_status(cudaSetDevice(ordinal));
+    return d;
 }
+
+// For the duration of one call: the GPU that holds the device pointer `p` is
+// current on this host thread, with a context. The caller's framework has
+// usually made it current already, and then nothing changes. A thread on
+// which no CUDA call has run (an autograd worker, a user's own thread) has no
+// current context: the TMA descriptor encoding fails there and a launch would
+// go to the runtime's default device, so the data's device is made current
+// (cudaSetDevice, which binds its primary context) and left so, as the
+// framework itself would. When another device's context is current, it is
+// switched for the call and restored afterwards. The device comes from the
+// pointer, so no other GPU's context is created.
+class DeviceScope {
+public:
+    explicit DeviceScope(const void *p)
+    {
+        const DriverCalls &d = driver();
+        if (!d.ok()) {
+            status = cuda_status(cudaErrorNotSupported);
+            return;
+        }
+        int ordinal = -1;
+        if (!encoded(d.pointer_attr(&ordinal, CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL, reinterpret_cast<CUdeviceptr>(p)))) {
+            status = REGEN_ERR_CUDA;
+            return;
+        }
+        CUcontext cur = nullptr;
+        if (!encoded(d.ctx_get_current(&cur))) {
+            status = REGEN_ERR_CUDA;
+            return;
+        }
+        if (cur != nullptr) {
+            CUdevice dev = -1;
+            if (!encoded(d.ctx_get_device(&dev))) {
+                status = REGEN_ERR_CUDA;
+                return;
+            }
+            if (static_cast<int>(dev) == ordinal) return;   // already the data's device
+            prev_ = cur;
+        }
+        status = cuda_status(cudaSetDevice(ordinal));
+    }
+    ~DeviceScope()
+    {
+        if (prev_ != nullptr) driver().ctx_set_current(prev_);
+    }
+    DeviceScope(const DeviceScope &) = delete;
+    DeviceScope &operator=(const DeviceScope &) = delete;
+    int status = REGEN_OK;
+
+private:
+    CUcontext prev_ = nullptr;
+};
 
 // [BH, S, D] bf16 viewed as a 3D tensor (D innermost), boxes of 64 x 128 x 1
 // with the 128-byte swizzle; out-of-range rows read as zero.
@@ -421,7 +474,8 @@ int rope3d_common(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float the
     const int threads = 128;
     const int64_t blocks = (work + threads - 1) / threads;
     if (blocks > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
-    if (const int rc = bind_device(q ? q : k); rc != REGEN_OK) return rc;
+    const DeviceScope device(q ? q : k);
+    if (device.status != REGEN_OK) return device.status;
     regen::rope3d_kernel<<<static_cast<unsigned>(blocks), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         q, k, BH, static_cast<int>(S), Hh, Ww, D, static_cast<double>(theta), inverse, S_local >= 0 ? n0 : 0);
     return launched();
@@ -451,7 +505,8 @@ REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const reg
         overlaps(lse, lbytes, k, kvbytes) || overlaps(lse, lbytes, v, kvbytes) ||
         overlaps(lse, lbytes, out, qbytes))
         return REGEN_ERR_INVALID_ARG;
-    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
+    const DeviceScope device(out);
+    if (device.status != REGEN_OK) return device.status;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (Skv == 0) {
         const int64_t n16 = qbytes / 16;
@@ -507,7 +562,8 @@ REGEN_API int regen_attn_fwd_rope3d(const regen_bf16 *q, const regen_bf16 *k, co
     if (overlaps(lse, lbytes, out, tbytes) || overlaps(workspace, need, out, tbytes) ||
         overlaps(workspace, need, lse, lbytes))
         return REGEN_ERR_INVALID_ARG;
-    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
+    const DeviceScope device(out);
+    if (device.status != REGEN_OK) return device.status;
     return attn_rope3d_with_scratch(q, k, v, out, lse, BH, static_cast<int>(S), D, scale, theta, geom,
                                     static_cast<uint8_t *>(workspace), reinterpret_cast<cudaStream_t>(stream));
 }
@@ -538,7 +594,8 @@ REGEN_API int regen_attn_fwd_rope3d_noalloc(const regen_bf16 *q, const regen_bf1
     for (const void *in : ins)
         if (overlaps(out, tbytes, in, tbytes) || overlaps(lse, lbytes, in, tbytes)) return REGEN_ERR_INVALID_ARG;
     if (overlaps(lse, lbytes, out, tbytes)) return REGEN_ERR_INVALID_ARG;
-    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
+    const DeviceScope device(out);
+    if (device.status != REGEN_OK) return device.status;
     uint8_t *scratch = noalloc_scratch_on_current_device();
     if (!scratch) return REGEN_ERR_CUDA;
     // Every scratch byte this call reads is written earlier in the same call
@@ -594,7 +651,8 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
         if (!aligned16(dk) || !aligned16(dv)) return REGEN_ERR_MISALIGNED;
         if (overlaps(dk, kvbytes, dv, kvbytes)) return REGEN_ERR_INVALID_ARG;
         if (acc_dkdv) return REGEN_OK;
-        if (const int rc = bind_device(dk); rc != REGEN_OK) return rc;
+        const DeviceScope device(dk);
+        if (device.status != REGEN_OK) return device.status;
         for (regen_bf16 *z : {dk, dv}) {
             regen::attn_empty_kernel<<<grid_for(kvbytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(z),
                                                                                  kvbytes / 16, nullptr, 0);
@@ -606,7 +664,8 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
         if (!dq) return REGEN_ERR_INVALID_ARG;
         if (!aligned16(dq)) return REGEN_ERR_MISALIGNED;
         if (acc_dq) return REGEN_OK;
-        if (const int rc = bind_device(dq); rc != REGEN_OK) return rc;
+        const DeviceScope device(dq);
+        if (device.status != REGEN_OK) return device.status;
         regen::attn_empty_kernel<<<grid_for(qbytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(dq),
                                                                             qbytes / 16, nullptr, 0);
         return launched();
@@ -628,7 +687,8 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
             if (overlaps(outs[a].p, outs[a].n, outs[b].p, outs[b].n)) return REGEN_ERR_INVALID_ARG;
     }
     float *ws = static_cast<float *>(workspace);
-    if (const int rc = bind_device(dq); rc != REGEN_OK) return rc;
+    const DeviceScope device(dq);
+    if (device.status != REGEN_OK) return device.status;
     if (D == 128)
         return launch_bwd<128>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, acc_dq, acc_dkdv, st);
     return launch_bwd<64>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, acc_dq, acc_dkdv, st);
@@ -656,7 +716,8 @@ REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a, const r
     if ((overlaps(out, obytes, o_a, obytes) && out != o_a) || (overlaps(out, obytes, o_b, obytes) && out != o_b))
         return REGEN_ERR_INVALID_ARG;
     const int64_t work = rows * (D / 8);
-    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
+    const DeviceScope device(out);
+    if (device.status != REGEN_OK) return device.status;
     regen::lse_merge_kernel<<<grid_for(work, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const uint4 *>(o_a), lse_a, reinterpret_cast<const uint4 *>(o_b), lse_b,
         reinterpret_cast<uint4 *>(out), lse_out, rows, D);
@@ -678,7 +739,8 @@ REGEN_API int regen_quant_e4m3(const regen_bf16 *x, uint8_t *codes, float *scale
     if (overlaps(codes, cbytes, x, xbytes) || overlaps(scales, sbytes, x, xbytes) ||
         overlaps(scales, sbytes, codes, cbytes))
         return REGEN_ERR_INVALID_ARG;
-    if (const int rc = bind_device(codes); rc != REGEN_OK) return rc;
+    const DeviceScope device(codes);
+    if (device.status != REGEN_OK) return device.status;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const unsigned grid = static_cast<unsigned>(BH * nb);
     if (D == 128)
@@ -715,7 +777,8 @@ REGEN_API int regen_attn_fwd_fp8(const uint8_t *q8, const float *q_scale, const 
     for (const Span &in : ins)
         if (overlaps(out, obytes, in.p, in.n) || overlaps(lse, lbytes, in.p, in.n)) return REGEN_ERR_INVALID_ARG;
     if (overlaps(lse, lbytes, out, obytes)) return REGEN_ERR_INVALID_ARG;
-    if (const int rc = bind_device(out); rc != REGEN_OK) return rc;
+    const DeviceScope device(out);
+    if (device.status != REGEN_OK) return device.status;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (Skv == 0) {
         regen::attn_empty_kernel<<<grid_for(obytes / 16, 256), 256, 0, st>>>(reinterpret_cast<uint4 *>(out),
@@ -765,7 +828,8 @@ REGEN_API int regen_qkv_proj(const regen_bf16 *x, const regen_bf16 *w, const flo
     }
     for (int a = 0; a < 5; ++a)
         if (overlaps(workspace, tab_bytes, ins[a].p, ins[a].n)) return REGEN_ERR_INVALID_ARG;
-    if (const int rc = bind_device(q); rc != REGEN_OK) return rc;
+    const DeviceScope device(q);
+    if (device.status != REGEN_OK) return device.status;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float2 *tab = static_cast<float2 *>(workspace);
     regen::rope_table_f32_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
@@ -793,7 +857,8 @@ REGEN_API int regen_out_proj(const regen_bf16 *o, const regen_bf16 *w, const flo
                   ybytes = static_cast<int64_t>(B) * S * N * 2;
     if (overlaps(y, ybytes, o, obytes) || overlaps(y, ybytes, w, wbytes) || overlaps(y, ybytes, bias, N * 4LL))
         return REGEN_ERR_INVALID_ARG;
-    if (const int rc = bind_device(y); rc != REGEN_OK) return rc;
+    const DeviceScope device(y);
+    if (device.status != REGEN_OK) return device.status;
     CUtensorMap ta, tb;
     if (!make_bhsd_map(&ta, o, static_cast<int64_t>(B) * H, S, 128) || !make_bf16_map3(&tb, w, K, N, 1, 64, 128))
         return REGEN_ERR_CUDA;
@@ -808,7 +873,8 @@ REGEN_API int regen_selftest_exp2(const float *x, float *y, int64_t n, regen_str
     if (n == 0) return REGEN_OK;
     if (!x || !y) return REGEN_ERR_INVALID_ARG;
     const int64_t npairs = n / 2;
-    if (const int rc = bind_device(y); rc != REGEN_OK) return rc;
+    const DeviceScope device(y);
+    if (device.status != REGEN_OK) return device.status;
     regen::exp2_poly_selftest_kernel<<<grid_for(npairs, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         x, y, npairs);
     return launched();
@@ -818,7 +884,8 @@ REGEN_API int regen_selftest_bounded_wait(uint64_t limit_ns, int *done, regen_st
 {
     if (!done) return REGEN_ERR_INVALID_ARG;
     if (limit_ns == 0 || limit_ns > 5000000000ull) return REGEN_ERR_INVALID_ARG;
-    if (const int rc = bind_device(done); rc != REGEN_OK) return rc;
+    const DeviceScope device(done);
+    if (device.status != REGEN_OK) return device.status;
     regen::bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, done);
     return launched();
 }
