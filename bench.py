@@ -324,6 +324,15 @@ def run_native(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     value = aggregate_tflops(flops_step, world, ms_step)
 
+    # The last timed step's self-attention, exactly: its bf16 inputs (q and k
+    # as that step's RoPE left them) and its output, for the CPU leg's
+    # accuracy check (rank 0 only, and only when that leg runs).
+    snap = None
+    if rank == 0 and not args.no_cpu_baseline:
+        bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
+        snap = dict(q=bits(d["q"]), k=bits(d["k"]), v=bits(d["v"]), out=bits(out), lse=lse.cpu().numpy(),
+                    scale=scale)
+
     # ---- backward: the gradient step of the same window (the decoder is trained by
     # distillation). dO synthetic; the forward's out/lse of the last timed step
     # (taken before anything else overwrites them).
@@ -458,7 +467,7 @@ def run_native(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.barrier()
     if rank != 0:
-        return None
+        return None, None
 
     pk, pk_src = peaks()
     t_self = per_kernel["attn_self"]
@@ -525,7 +534,7 @@ def run_native(args, rank, world, local_rank):
         "lse_merge_gbs": round((3 * B * H * S * D * 2 + 3 * B * H * S * 4) / (s_merge * 1e-3) / 1e9, 1),
         "peak_gbs": float(pk["hbm_gbs"]),
     }
-    return line
+    return line, snap
 
 
 def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, barrier, to_dev):
@@ -740,15 +749,19 @@ def run_fp8(args, rg, d, ws, dev, stream, world, barrier):
 
 # ------------------------------------------------------ CPU (oracle) ---
 
-def cpu_sample_rate(target_s: float, seed_rows: int = 0):
+def cpu_sample_rate(target_s: float, seed_rows: int = 0, snap=None):
     """Time the fp64 oracle on a bounded sample of query rows of the 77-frame
-    self-attention. RoPE is not applied to the sample's inputs: the values do
-    not change the oracle's cost, and the oracle's RoPE adds no FLOPs counted here."""
+    self-attention. With `snap` (the last timed GPU step's bf16 inputs and
+    output) the oracle runs on exactly those inputs, so that its rows also
+    check the GPU's; without it (the reference arm) on the workload's
+    generated inputs, whose values do not change the oracle's cost."""
     import oracle
     from dit_attention_b200 import synth
     w = synth.WORKLOADS[SELF]
-    q, k, v = synth.make_inputs(w)
-    qr, kr = q, k
+    if snap is not None:
+        qr, kr, v = snap["q"], snap["k"], snap["v"]
+    else:
+        qr, kr, v = synth.make_inputs(w)
     rng = np.random.default_rng(seed_rows)
     BH = w.B * w.H
     # calibrate t(rows) = a + b*rows on two sizes, then size the sample to about target_s
@@ -765,15 +778,43 @@ def cpu_sample_rate(target_s: float, seed_rows: int = 0):
     return dict(q=qr, k=kr, v=v, w=w, rng=rng, rows=n_full, threads=oracle.num_threads())
 
 
-def time_cpu(sample, rows):
+def time_cpu(sample, rows, keep=None):
+    """TFLOP/s and seconds of the oracle on `rows` random query rows; with a
+    dict `keep`, also stores the row indices and the oracle's out and lse rows."""
     import oracle
     w = sample["w"]
     r = sample["rng"].choice(w.B * w.H * w.Sq, size=rows, replace=False)
     t = time.perf_counter()
-    oracle.attention(sample["q"], sample["k"], sample["v"], w.scale, rows=r)
+    ref, ref_lse = oracle.attention(sample["q"], sample["k"], sample["v"], w.scale, rows=r)
     dt = time.perf_counter() - t
+    if keep is not None:
+        keep.update(rows=r, out=ref, lse=ref_lse)
     flops = 4.0 * rows * w.Skv * w.D
     return flops / dt / 1e12, dt
+
+
+def accuracy(snap, kept):
+    """The GPU's rows against the oracle's on the same bf16 inputs: the
+    attention contract |out - ref| <= 1e-2 + 1e-2|ref|, |lse - ref| <= 1e-3, and
+    the error normalised by RMS(ref). The diagnostic flag is on the MEAN error
+    over RMS(ref), above 5e-3: the roundings of P and of the output keep it
+    near u/4 (u = 2^-8), while a real defect (a wrong scale, a dropped block)
+    moves every element. The maximum is reported beside it: over a million
+    elements the rounding of P alone reaches ~2 % of RMS on a few of them."""
+    import oracle
+    D = snap["out"].shape[-1]
+    got = oracle.bf16_to_f64(snap["out"].reshape(-1, D)[kept["rows"]])
+    ref = kept["out"].reshape(got.shape)
+    err = np.abs(got - ref)
+    rms = float(np.sqrt(np.mean(ref ** 2))) or 1.0
+    lse_err = np.abs(snap["lse"].reshape(-1)[kept["rows"]].astype(np.float64) - kept["lse"].reshape(-1))
+    within = bool(np.all(err <= 1e-2 + 1e-2 * np.abs(ref)) and np.all(lse_err <= 1e-3))
+    return {"rows": int(len(kept["rows"])), "inputs": "the last timed step's bf16 q, k (after its RoPE), v",
+            "max_abs_err": float(err.max()), "max_err_over_rms": float(err.max() / rms),
+            "mean_rel_err": float(np.mean(err) / (np.mean(np.abs(ref)) or 1.0)),
+            "max_lse_err": float(lse_err.max()), "contract": "|out-ref| <= 1e-2 + 1e-2|ref|, |lse-ref| <= 1e-3",
+            "mean_err_over_rms": float(np.mean(err) / rms), "within_contract": within,
+            "flag_mean_err_over_rms_5e-3": bool(np.mean(err) / rms > 5e-3)}
 
 
 def run_configs(args):
@@ -903,11 +944,13 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    line = run_native(args, rank, world, local_rank)
+    line, snap = run_native(args, rank, world, local_rank)
     if line is not None and not args.no_cpu_baseline:
         import oracle
-        sample = cpu_sample_rate(args.cpu_seconds)
-        v, dt = time_cpu(sample, sample["rows"])
+        sample = cpu_sample_rate(args.cpu_seconds, snap=snap)
+        kept = {}
+        v, dt = time_cpu(sample, sample["rows"], keep=kept)
+        line["accuracy"] = accuracy(snap, kept)
         # the same oracle once more on one thread, on a smaller sample (~1/3 of the time above)
         threads = sample["threads"]
         rows1 = max(16, sample["rows"] // max(1, 3 * threads))

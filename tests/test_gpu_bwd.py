@@ -244,12 +244,12 @@ def _workload_bwd(name, heads, nq_rows=24, nk_rows=24, delta_term=False):
     gv = to_bits(dv).reshape(BH, w.Skv, w.D)
     # identities of every head: sum_j dv_j = sum_i dO_i (rows of P sum to 1),
     # sum_j dk_j = 0 (shifting every key leaves the softmax unchanged)
-    # (bounds: a few bf16 roundings, u = 2^-9, of every summand)
+    # (bounds: 4u of every summand, u = 2^-8 the bf16 unit roundoff: a few roundings)
     fv = bits_to_f64(gv)
     sg = bits_to_f64(g.reshape(BH, w.Sq, w.D)).sum(axis=1)
-    assert np.all(np.abs(fv.sum(axis=1) - sg) <= 8 * 2.0 ** -9 * np.abs(fv).sum(axis=1) + 1e-3)
+    assert np.all(np.abs(fv.sum(axis=1) - sg) <= 4 * 2.0 ** -8 * np.abs(fv).sum(axis=1) + 1e-3)
     fk = bits_to_f64(gk)
-    assert np.all(np.abs(fk.sum(axis=1)) <= 8 * 2.0 ** -9 * np.abs(fk).sum(axis=1) + 1e-6)
+    assert np.all(np.abs(fk.sum(axis=1)) <= 4 * 2.0 ** -8 * np.abs(fk).sum(axis=1) + 1e-6)
     qrows, krows = _sample(w.Sq, nq_rows, 1), _sample(w.Skv, nk_rows, 2)
     qh = q.reshape(BH, w.Sq, w.D)[heads]
     kh = k.reshape(BH, w.Skv, w.D)[heads]
