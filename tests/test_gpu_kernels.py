@@ -382,3 +382,51 @@ def test_calls_from_a_fresh_host_thread():
     assert "err" not in res, res.get("err")
     for a, b in zip((out, lse) + tuple(grads), res["ok"]):
         assert torch.equal(a, b)
+
+
+def test_forward_step_under_cuda_graph_capture():
+    # The step's five launches (RoPE, self-attention, two cross-attention
+    # calls, merge) captured once into a CUDA graph and replayed on new inputs
+    # copied into the captured buffers: the same bits as eager calls. (Capture
+    # runs each entry point's host work once: argument checks, device binding,
+    # descriptor encoding; the descriptors travel in the kernel parameters.)
+    B, H, D, grid = 1, 2, 128, (2, 6, 11)
+    S = grid[0] * grid[1] * grid[2]
+    n_ref, n_ctx = 150, 70
+
+    def inputs():
+        q, k, v = (synth.f64_to_bf16_bits(RNG.normal(size=(B, H, S, D))) for _ in range(3))
+        kc, vc = (synth.f64_to_bf16_bits(RNG.normal(size=(B, H, n_ref + n_ctx, D))) for _ in range(2))
+        return [to_dev(x) for x in (q, k, v, kc[:, :, :n_ref], vc[:, :, :n_ref], kc[:, :, n_ref:], vc[:, :, n_ref:])]
+
+    def step(q, k, v, kr, vr, kx, vx, o):
+        rg.rope3d_(q, k, grid)
+        rg.attn_fwd(q, k, v, out=o["out"], lse=o["lse"])
+        rg.attn_fwd(q, kr, vr, out=o["oa"], lse=o["la"])
+        rg.attn_fwd(q, kx, vx, out=o["ob"], lse=o["lb"])
+        rg.lse_merge(o["oa"], o["la"], o["ob"], o["lb"], out=o["oc"], lse_out=o["lc"])
+
+    def outs():
+        o = {n: torch.empty((B, H, S, D), dtype=torch.bfloat16, device="cuda") for n in ("out", "oa", "ob", "oc")}
+        o.update({n: torch.empty((B, H, S), dtype=torch.float32, device="cuda") for n in ("lse", "la", "lb", "lc")})
+        return o
+
+    static_in, static_out = inputs(), outs()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):                 # warm up off the capture (one-time setup)
+        step(*[t.clone() for t in static_in], outs())
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(*static_in, static_out)
+    for _ in range(2):
+        fresh = inputs()
+        for dst, src in zip(static_in, fresh):
+            dst.copy_(src)
+        graph.replay()
+        eager = outs()
+        step(*fresh, eager)
+        torch.cuda.synchronize()
+        for n in static_out:
+            assert torch.equal(static_out[n], eager[n]), n
