@@ -11,17 +11,23 @@
 // Work unit = one CTA = one (batch*head, 256 query rows) = two 128-row Q tiles;
 // grid = B*H*ceil(Sq/256) CTAs.
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles once, then K/V tiles through NS-stage rings
-//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma and commit
-//   warps 2-3   idle
+//   warp 0      TMA producer: Q tiles once, then K tiles through an NS-stage ring
+//   warp 3      TMA producer: V tiles through an NS-stage ring
+//   warp 1      TMEM allocator; lane 0 issues the S = QK^T MMAs and their commits
+//   warp 2      lane 0 issues the O += PV MMAs and their commits
 //   warps 4-7   softmax + correction + epilogue for Q tile 0 (one thread per row)
 //   warps 8-11  the same for Q tile 1
-// Tensor memory (512 columns, fp32): S0 [0,128), S1 [128,256), O0 and O1 after
-// them (HD columns each). P (bf16) is written over the first 64 columns of
-// its S and fed to the PV MMA straight from TMEM.
-// MMA order, ping-ponging the two tiles so that one tile's softmax overlaps
-// the other tile's MMAs:
-//   S0(0) S1(0) | PV0(0) S0(1) | PV1(0) S1(1) | PV0(1) S0(2) | ...
+// Tensor memory (512 columns, fp32): one S buffer [0,128) shared by the two
+// tiles, P0 [128,192) and P1 [192,256) (bf16, two per column), then O0 and O1
+// (HD columns each). P feeds the PV MMA straight from TMEM. Because P has
+// columns of its own, the next S of a tile need not wait for that tile's PV:
+// S is free as soon as the softmax warps have copied it into registers.
+// The S MMAs (S0(0) S1(0) S0(1) S1(1) ..., the S buffer alternating between
+// the tiles) and the PV MMAs (PV0(0) PV1(0) PV0(1) ...) come from two issuing
+// threads: the tensor core queues only a few MMAs, so one thread that stops to
+// wait on a barrier between groups lets it run dry, while two keep it fed.
+// Each tile's softmax of block j+1 runs while its PV of block j does; it
+// waits for that PV only before it stores P (and rescales O, when it must).
 // Softmax keeps a per-row running max m (log2 units, scale folded in) and
 // sum l in fp32; O is rescaled only when the max grows by more than 8
 // (log2), which stays exact because P = 2^(s - m) is then at most 2^8 and
@@ -58,6 +64,8 @@ enum WaitSite : uint32_t {
     SITE_DRAIN = 9,
     SITE_SM_Q = 11,
     SITE_SELFTEST = 10,
+    SITE_MMA_S_FREE = 12,
+    SITE_SM_PV_DONE = 13,
 };
 
 __device__ __forceinline__ void record_timeout(uint32_t site)
@@ -107,9 +115,9 @@ struct AttnCfg {
     static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
     static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
     static constexpr int BAR_OFF = V_OFF + NS * TILE_BYTES;
-    // barriers: q, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2],
-    // o_full[2], drain, q_rotated
-    static constexpr int NBARS = 1 + 4 * NS + 6 + 1 + 1;
+    // barriers: q, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], s_free,
+    // p_full[2], pv_done[2], drain, q_rotated
+    static constexpr int NBARS = 1 + 4 * NS + 7 + 1 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;  // abort flag, TMEM base
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -151,10 +159,11 @@ __global__ void __launch_bounds__(384, 1)
     auto bar_v_full = [&](int s) { return bar0 + 8u * (1 + 2 * C::NS + s); };
     auto bar_v_empty = [&](int s) { return bar0 + 8u * (1 + 3 * C::NS + s); };
     auto bar_s_full = [&](int t) { return bar0 + 8u * (1 + 4 * C::NS + t); };
-    auto bar_p_full = [&](int t) { return bar0 + 8u * (3 + 4 * C::NS + t); };
-    auto bar_o_full = [&](int t) { return bar0 + 8u * (5 + 4 * C::NS + t); };
-    const uint32_t bar_drain = bar0 + 8u * (7 + 4 * C::NS);
-    const uint32_t bar_qrot = bar0 + 8u * (8 + 4 * C::NS);  // Q tiles rotated (ROPE_Q)
+    const uint32_t bar_s_free = bar0 + 8u * (3 + 4 * C::NS);  // S copied out by a softmax warpgroup
+    auto bar_p_full = [&](int t) { return bar0 + 8u * (4 + 4 * C::NS + t); };
+    auto bar_pv_done = [&](int t) { return bar0 + 8u * (6 + 4 * C::NS + t); };
+    const uint32_t bar_drain = bar0 + 8u * (8 + 4 * C::NS);
+    const uint32_t bar_qrot = bar0 + 8u * (9 + 4 * C::NS);  // Q tiles rotated (ROPE_Q)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 8);
 
@@ -169,9 +178,10 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar_s_full(t), 1);
             mbar_init(bar_p_full(t), 128);
-            mbar_init(bar_o_full(t), 1);
+            mbar_init(bar_pv_done(t), 1);
         }
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_s_free, 128);
+        mbar_init(bar_drain, 2);
         mbar_init(bar_qrot, 256);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -199,32 +209,73 @@ __global__ void __launch_bounds__(384, 1)
     // Each register region runs to its own final barrier (no shared tail).
     if (warp < 4) {
     setmaxnreg_dec<C::REGS_LOW>();
+    // Aborting: wait (bounded) for the copies a producer may still have in
+    // flight -- at most the last NS of its ring (and the Q tiles) -- so that
+    // none lands in shared memory after the CTA has exited. (copies complete
+    // in microseconds; the drain never uses less than kDrainFloorNs even when
+    // the caller's wait limit is tiny)
+    const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
+    auto drain_copies = [&](uint32_t bar, uint32_t parity) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
+        }
+    };
+    // Before TMEM is freed nothing may still run on the tensor core: each MMA
+    // issuer commits to bar_drain (count 2) and waits for both commits.
+    auto drain_mmas = [&]() {
+        tc_commit(bar_drain);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar_drain, 0)) {
+            if (global_timer_ns() - t0 > drain_ns) {
+                record_timeout(SITE_DRAIN);
+                break;
+            }
+        }
+    };
+    // Tensor-memory columns: S at 0 (the two tiles in turn), P_t at 128 + t*64,
+    // O_t at 256 + t*HD (computed, not indexed, so nothing lands in local memory)
+    auto tm_p = [&](int t) { return tmem + 128u + static_cast<uint32_t>(t) * 64u; };
+    auto tm_o = [&](int t) { return tmem + 256u + static_cast<uint32_t>(t) * HD; };
     if (warp == 0) {
-        // ------------------------------------------------------ producer ---
+        // ------------------------------------------- producer: Q, then K ---
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            const uint64_t keep = l2_policy_evict_last();   // K/V: re-read by every Q tile of the head
+            const uint64_t keep = l2_policy_evict_last();   // K: re-read by every Q tile of the head
             const uint64_t once = l2_policy_evict_first();  // Q: read once
             mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
             for (int t = 0; t < 2; ++t)
                 for (int h = 0; h < C::HALVES; ++h)
                     tma_load_3d(sbase + C::Q_OFF + t * C::TILE_BYTES + h * C::HALF_BYTES, &tm_q, bar_q,
                                 h * 64, q0 + t * C::BM, bh, once);
-            int nk = 0, nv = 0;  // K and V block loads issued so far
+            int nk = 0;  // K block loads issued so far
             bool ok = true;
             for (int j = 0; j < nkv; ++j) {
                 const int s = j % C::NS;
-                const uint32_t ph = (j / C::NS) & 1;
-                ok = wait_phase(bar_k_empty(s), ph ^ 1, SITE_PROD_K_EMPTY, wc);
+                ok = wait_phase(bar_k_empty(s), ((j / C::NS) & 1) ^ 1, SITE_PROD_K_EMPTY, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_k_full(s), C::TILE_BYTES);
                 for (int h = 0; h < C::HALVES; ++h)
                     tma_load_3d(sbase + C::K_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_k,
                                 bar_k_full(s), h * 64, j * C::BN, bh, keep);
                 ++nk;
-                ok = wait_phase(bar_v_empty(s), ph ^ 1, SITE_PROD_V_EMPTY, wc);
+            }
+            if (!ok) {
+                for (int j = (nk > C::NS ? nk - C::NS : 0); j < nk; ++j)
+                    drain_copies(bar_k_full(j % C::NS), (j / C::NS) & 1);
+                drain_copies(bar_q, 0);
+            }
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------- producer: V ---
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_v);
+            const uint64_t keep = l2_policy_evict_last();   // V: re-read by every Q tile of the head
+            int nv = 0;
+            bool ok = true;
+            for (int j = 0; j < nkv; ++j) {
+                const int s = j % C::NS;
+                ok = wait_phase(bar_v_empty(s), ((j / C::NS) & 1) ^ 1, SITE_PROD_V_EMPTY, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_v_full(s), C::TILE_BYTES);
                 for (int h = 0; h < C::HALVES; ++h)
@@ -232,111 +283,89 @@ __global__ void __launch_bounds__(384, 1)
                                 bar_v_full(s), h * 64, j * C::BN, bh, keep);
                 ++nv;
             }
-            if (!ok) {
-                // Aborting: wait (bounded) for the copies this warp may still have
-                // in flight -- at most the last NS of each ring and the Q tiles --
-                // so that none lands in shared memory after the CTA has exited.
-                // (copies complete in microseconds; the drain never uses less than
-                // kDrainFloorNs even when the caller's wait limit is tiny)
-                const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
-                auto drain = [&](uint32_t bar, uint32_t parity) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
-                    }
-                };
-                for (int j = (nk > C::NS ? nk - C::NS : 0); j < nk; ++j)
-                    drain(bar_k_full(j % C::NS), (j / C::NS) & 1);
+            if (!ok)
                 for (int j = (nv > C::NS ? nv - C::NS : 0); j < nv; ++j)
-                    drain(bar_v_full(j % C::NS), (j / C::NS) & 1);
-                drain(bar_q, 0);
-            }
+                    drain_copies(bar_v_full(j % C::NS), (j / C::NS) & 1);
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------- MMA issuer ---
+        // -------------------------------------------- MMA issuer: S = QK^T ---
+        // S = Q_t K_j^T : M=128, N=128, K=HD in steps of 16 (32 bytes) inside
+        // each 128-byte swizzle row; the second 64-column half starts HALF_BYTES on.
+        // The S buffer's copy-outs complete bar_s_free's phases in a fixed
+        // order: S0(0), S1(0), S0(1), S1(1), ... So S1(j) waits for the phase
+        // of S0(j) (even, parity 0) and S0(j+1) for that of S1(j) (odd,
+        // parity 1); this thread is the only waiter and waits for every
+        // phase in turn, so no wait can be two phases behind.
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false);  // Q.K^T, both K-major
-            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, true);    // P.V, V is MN-major
-            // TMEM columns: S_t at t*128, O_t at 256 + t*HD (computed, not indexed,
-            // so nothing lands in local memory)
-            auto tm_s = [&](int t) { return tmem + static_cast<uint32_t>(t) * 128u; };
-            auto tm_o = [&](int t) { return tmem + 256u + static_cast<uint32_t>(t) * HD; };
-            // S_t = Q_t K_j^T : M=128, N=128, K=HD in steps of 16 (32 bytes) inside
-            // each 128-byte swizzle row; the second 64-column half starts HALF_BYTES on.
             auto issue_s = [&](int t, int s) {
                 const uint32_t qa = sbase + C::Q_OFF + t * C::TILE_BYTES;
                 const uint32_t kb = sbase + C::K_OFF + s * C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t off = (kk / 4) * C::HALF_BYTES + (kk % 4) * 32;
-                    mma_ss(tm_s(t), smem_desc_sw128(qa + off, 16, 1024),
+                    mma_ss(tmem, smem_desc_sw128(qa + off, 16, 1024),
                            smem_desc_sw128(kb + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_t += P_t V_j : M=128, N=HD, K=128 keys in steps of 16. P comes from
-            // TMEM (16 keys = 8 columns); V rows are 128-byte swizzled, 16 keys =
-            // 2048 bytes, the two 64-wide D halves are HALF_BYTES apart (LBO).
+            bool ok = wait_phase(ROPE_Q ? bar_qrot : bar_q, 0, SITE_MMA_Q, wc);
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int s = j % C::NS;
+                ok = wait_phase(bar_k_full(s), (j / C::NS) & 1, SITE_MMA_K_FULL, wc);
+                if (!ok) break;
+                if (j > 0) {
+                    ok = wait_phase(bar_s_free, 1, SITE_MMA_S_FREE, wc);  // S1(j-1) copied out
+                    if (!ok) break;
+                }
+                tc_fence_after_sync();
+                issue_s(0, s);
+                tc_commit(bar_s_full(0));
+                ok = wait_phase(bar_s_free, 0, SITE_MMA_S_FREE, wc);      // S0(j) copied out
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_s(1, s);
+                tc_commit(bar_s_full(1));
+                tc_commit(bar_k_empty(s));
+            }
+            drain_mmas();
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------ MMA issuer: O += P V ---
+        // O_t += P_t V_j : M=128, N=HD, K=128 keys in steps of 16. P comes from
+        // TMEM (16 keys = 8 columns); V rows are 128-byte swizzled, 16 keys =
+        // 2048 bytes, the two 64-wide D halves are HALF_BYTES apart (LBO).
+        // Its MMAs touch none of the S issuer's columns (P_t and O_t only), so
+        // the two streams need no order between them beyond the softmax's
+        // barriers; each issuer's commits track its own MMAs.
+        if (lane == 0) {
+            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HD, true);  // P.V, V is MN-major
             auto issue_pv = [&](int t, int s, bool acc) {
                 const uint32_t vb = sbase + C::V_OFF + s * C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    mma_ts(tm_o(t), tm_s(t) + kk * 8, smem_desc_sw128(vb + kk * 2048, C::HALF_BYTES, 1024),
+                    mma_ts(tm_o(t), tm_p(t) + kk * 8, smem_desc_sw128(vb + kk * 2048, C::HALF_BYTES, 1024),
                            IDESC_O, (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            bool ok = wait_phase(ROPE_Q ? bar_qrot : bar_q, 0, SITE_MMA_Q, wc);
-            if (ok) ok = wait_phase(bar_k_full(0), 0, SITE_MMA_K_FULL, wc);
-            if (ok) {
-                tc_fence_after_sync();
-                issue_s(0, 0);
-                tc_commit(bar_s_full(0));
-                issue_s(1, 0);
-                tc_commit(bar_s_full(1));
-                tc_commit(bar_k_empty(0));
-            }
+            bool ok = true;
             for (int j = 0; j < nkv && ok; ++j) {
                 const int s = j % C::NS;
-                const uint32_t ph = (j / C::NS) & 1;
-                const int s1 = (j + 1) % C::NS;
-                const uint32_t ph1 = ((j + 1) / C::NS) & 1;
-                const bool more = j + 1 < nkv;
-                ok = wait_phase(bar_v_full(s), ph, SITE_MMA_V_FULL, wc);
+                ok = wait_phase(bar_v_full(s), (j / C::NS) & 1, SITE_MMA_V_FULL, wc);
                 if (!ok) break;
                 ok = wait_phase(bar_p_full(0), j & 1, SITE_MMA_P_FULL, wc);
                 if (!ok) break;
                 tc_fence_after_sync();
                 issue_pv(0, s, j > 0);
-                if (more) {
-                    ok = wait_phase(bar_k_full(s1), ph1, SITE_MMA_K_FULL, wc);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                    issue_s(0, s1);
-                    tc_commit(bar_s_full(0));
-                } else {
-                    tc_commit(bar_o_full(0));
-                }
+                tc_commit(bar_pv_done(0));
                 ok = wait_phase(bar_p_full(1), j & 1, SITE_MMA_P_FULL, wc);
                 if (!ok) break;
                 tc_fence_after_sync();
                 issue_pv(1, s, j > 0);
+                tc_commit(bar_pv_done(1));
                 tc_commit(bar_v_empty(s));
-                if (more) {
-                    issue_s(1, s1);
-                    tc_commit(bar_s_full(1));
-                    tc_commit(bar_k_empty(s1));
-                } else {
-                    tc_commit(bar_o_full(1));
-                }
             }
-            // Drain: nothing may still be running on the tensor core when TMEM is freed.
-            tc_commit(bar_drain);
-            const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(bar_drain, 0)) {
-                if (global_timer_ns() - t0 > drain_ns) {
-                    record_timeout(SITE_DRAIN);
-                    break;
-                }
-            }
+            drain_mmas();
         }
         __syncwarp();
     }
@@ -353,7 +382,8 @@ __global__ void __launch_bounds__(384, 1)
         const int quad = warp & 3;         // TMEM lane quadrant this warp may access
         const int row = quad * 32 + lane;  // row inside the tile
         const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t ts = tmem + lane_bits + t * 128u;
+        const uint32_t ts = tmem + lane_bits;                 // the shared S buffer
+        const uint32_t tp = tmem + lane_bits + 128u + t * 64u;  // this tile's P
         const uint32_t to = tmem + lane_bits + 256u + t * HD;
         const int kv_tail = Skv - (nkv - 1) * C::BN;  // valid keys in the last block (1..128)
         float m = 0.f;   // running max of scaled logits (log2 units); set by block 0
@@ -388,6 +418,9 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+            // S is in registers: the buffer may take the other tile's next S.
+            tc_fence_before_sync();
+            mbar_arrive(bar_s_free);
             // One block of the online softmax. MASKED: the last block, whose
             // columns >= kv_tail lie past Skv (their logits are zero-filled
             // loads) and get probability 0.
@@ -429,12 +462,14 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 // P = 2^(s*scale_log2 - m): packed FMA for the affine step, MUFU
                 // ex2, fp32 row sum (4 packed accumulators) before rounding to bf16.
+                // All 64 packed columns are formed in registers first: only
+                // their stores need PV_t(j-1) to have finished reading P_t.
                 const uint64_t c2 = f2_pack(scale_log2, scale_log2);
                 const uint64_t nm2 = f2_pack(-m, -m);
                 uint64_t rs2[4] = {0, 0, 0, 0};
+                uint32_t pk[2][32];
 #pragma unroll
                 for (int hv = 0; hv < 2; ++hv) {   // 64 keys -> 32 packed columns per half
-                    uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 64; i += 2) {
                         const int x = hv * 64 + i;
@@ -452,10 +487,17 @@ __global__ void __launch_bounds__(384, 1)
                             if (x + 1 >= kv_tail) p1 = 0.f;
                         }
                         rs2[(i >> 1) & 3] = f2_add(rs2[(i >> 1) & 3], f2_pack(p0, p1));
-                        pk[i >> 1] = pack_bf16x2(p0, p1);
+                        pk[hv][i >> 1] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st_32x32b_x32(ts + hv * 32, pk);
                 }
+                // P_t and O_t are free once PV_t(j-1) has completed.
+                if (j > 0) {
+                    ok = __all_sync(0xffffffffu, wait_phase(bar_pv_done(t), (j - 1) & 1, SITE_SM_PV_DONE, wc));
+                    if (!ok) return;
+                    tc_fence_after_sync();
+                }
+                tmem_st_32x32b_x32(tp, pk[0]);
+                tmem_st_32x32b_x32(tp + 32, pk[1]);
                 float r0, r1, r2, r3;
                 f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), r0, r1);
                 (void)r2;
@@ -466,8 +508,9 @@ __global__ void __launch_bounds__(384, 1)
                 block(std::true_type{});
             else
                 block(std::false_type{});
-            // O_t holds exactly PV_t(0..j-1) here: the commit that signalled S_t(j)
-            // follows PV_t(j-1), and PV_t(j) waits for this warpgroup's arrive.
+            if (!ok) break;
+            // O_t holds exactly PV_t(0..j-1) here: block() waited for PV_t(j-1)
+            // before writing P, and PV_t(j) waits for this warpgroup's arrive.
             if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
                 for (int c = 0; c < HD / 32; ++c) {
@@ -484,7 +527,7 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_before_sync();
             mbar_arrive(bar_p_full(t));
         }
-        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_o_full(t), 0, SITE_SM_O_FULL, wc));
+        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_pv_done(t), (nkv - 1) & 1, SITE_SM_O_FULL, wc));
         if (ok) {
             tc_fence_after_sync();
             // Epilogue: O / l -> bf16 into this tile's Q buffer (free now: every
