@@ -40,11 +40,16 @@
 #include "rope3d.cuh"
 
 // Pairs of every 8 probabilities whose 2^x runs on the FMA pipe (exp2_poly_pair)
-// instead of MUFU, in the forward and the gradient kernels. On the 77-frame
-// window 1 measured equal to 2 for the forward and ~2 % faster for the
-// gradient; 3 is slower for both.
+// instead of MUFU. Gradient kernels: on the 77-frame window 1 measured ~2 %
+// faster than 2, and 3 slower. Forward: with its two MMA issuers the kernel
+// runs at the 1 kW power cap, where the polynomial's FMA-pipe work costs more
+// than the MUFU time it frees: 0 measured 15.2-15.3 ms, 1 16.1-16.2 ms and 2
+// 17.4-17.6 ms on the 77-frame window, so the forward uses MUFU alone.
 #ifndef REGEN_EXP2_EMU_PER8
 #define REGEN_EXP2_EMU_PER8 1
+#endif
+#ifndef REGEN_FWD_EXP2_EMU_PER8
+#define REGEN_FWD_EXP2_EMU_PER8 0
 #endif
 
 namespace regen {
@@ -127,9 +132,9 @@ struct AttnCfg {
     // need (REGS_HIGH - R) * 256 <= (R - REGS_LOW) * 128, i.e. R >= 160
     static constexpr int MIN_LAUNCH_REGS = 160;
     // Of every 8 pairs of probabilities, this many are evaluated on the FMA
-    // pipe (exp2_poly_pair) instead of MUFU: ex2 throughput (16/clk/SM) alone
-    // equals the tensor time of a key block, so part of it moves to the FMAs.
-    static constexpr int EMU_PER8 = REGEN_EXP2_EMU_PER8;
+    // pipe (exp2_poly_pair) instead of MUFU (ex2 throughput, 16/clk/SM, alone
+    // equals the tensor time of a key block; the power cap decides the split).
+    static constexpr int EMU_PER8 = REGEN_FWD_EXP2_EMU_PER8;
 };
 
 // ROPE_Q: the Q tiles are rotated by the 3D RoPE in shared memory right after
