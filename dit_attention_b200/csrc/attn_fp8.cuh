@@ -15,6 +15,9 @@
 // down to ~2^-10 of the row max in E4M3's normal range (3 significant bits)
 // instead of its subnormals. D = 128 only: a row of codes is exactly one
 // 128-byte swizzle row.
+// Structure as in the bf16 kernel (attn_fwd.cuh): two 128-row Q tiles per CTA
+// sharing one S buffer in tensor memory, each with its own P8 and O; K and V
+// from two producer warps; S and PV MMAs from two issuing threads.
 #pragma once
 
 #include "attn_fwd.cuh"
@@ -135,8 +138,9 @@ struct Fp8Cfg {
     static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
     static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
     static constexpr int BAR_OFF = V_OFF + NS * TILE_BYTES;
-    // q, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2], o_full[2], drain
-    static constexpr int NBARS = 1 + 4 * NS + 6 + 1;
+    // q, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], s_free, p_full[2],
+    // pv_done[2], drain
+    static constexpr int NBARS = 1 + 4 * NS + 7 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;  // abort flag, TMEM base, 8 warp maxima
     static constexpr int SMEM_BYTES = MISC_OFF + 48 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -172,9 +176,10 @@ __global__ void __launch_bounds__(384, 1)
     auto bar_v_full = [&](int s) { return bar0 + 8u * (1 + 2 * C::NS + s); };
     auto bar_v_empty = [&](int s) { return bar0 + 8u * (1 + 3 * C::NS + s); };
     auto bar_s_full = [&](int t) { return bar0 + 8u * (1 + 4 * C::NS + t); };
-    auto bar_p_full = [&](int t) { return bar0 + 8u * (3 + 4 * C::NS + t); };
-    auto bar_o_full = [&](int t) { return bar0 + 8u * (5 + 4 * C::NS + t); };
-    const uint32_t bar_drain = bar0 + 8u * (7 + 4 * C::NS);
+    const uint32_t bar_s_free = bar0 + 8u * (3 + 4 * C::NS);  // S copied out by a softmax warpgroup
+    auto bar_p_full = [&](int t) { return bar0 + 8u * (4 + 4 * C::NS + t); };
+    auto bar_pv_done = [&](int t) { return bar0 + 8u * (6 + 4 * C::NS + t); };
+    const uint32_t bar_drain = bar0 + 8u * (8 + 4 * C::NS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 8);
     float *warp_max = reinterpret_cast<float *>(smem + C::MISC_OFF + 16);
@@ -190,9 +195,10 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar_s_full(t), 1);
             mbar_init(bar_p_full(t), 128);
-            mbar_init(bar_o_full(t), 1);
+            mbar_init(bar_pv_done(t), 1);
         }
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_s_free, 128);
+        mbar_init(bar_drain, 2);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -214,125 +220,142 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp < 4) {
     setmaxnreg_dec<C::REGS_LOW>();
+    // Aborting producers wait (bounded) for their copies still in flight; the
+    // two MMA issuers each commit to bar_drain (count 2) and wait for both
+    // before TMEM is freed (same protocol as the bf16 kernel).
+    const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
+    auto drain_copies = [&](uint32_t bar, uint32_t parity) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
+        }
+    };
+    auto drain_mmas = [&]() {
+        tc_commit(bar_drain);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar_drain, 0)) {
+            if (global_timer_ns() - t0 > drain_ns) {
+                record_timeout(SITE_DRAIN);
+                break;
+            }
+        }
+    };
+    // Tensor-memory columns: S at 0 (the two tiles in turn), P8_t at 128 + t*32
+    // (128 codes per row, 4 per column), O_t at 256 + t*128.
+    auto tm_p = [&](int t) { return tmem + 128u + static_cast<uint32_t>(t) * 32u; };
+    auto tm_o = [&](int t) { return tmem + 256u + static_cast<uint32_t>(t) * 128u; };
     if (warp == 0) {
-        // ------------------------------------------------------ producer ---
+        // ------------------------------------------- producer: Q, then K ---
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
             const uint64_t keep = l2_policy_evict_last();
             const uint64_t once = l2_policy_evict_first();
             mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
             for (int t = 0; t < 2; ++t)
                 tma_load_3d(sbase + C::Q_OFF + t * C::TILE_BYTES, &tm_q, bar_q, 0, q0 + t * C::BM, bh, once);
-            int nk = 0, nv = 0;
+            int nk = 0;
             bool ok = true;
             for (int j = 0; j < nkv; ++j) {
                 const int s = j % C::NS;
-                const uint32_t ph = (j / C::NS) & 1;
-                ok = wait_phase(bar_k_empty(s), ph ^ 1, SITE_PROD_K_EMPTY, wc);
+                ok = wait_phase(bar_k_empty(s), ((j / C::NS) & 1) ^ 1, SITE_PROD_K_EMPTY, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_k_full(s), C::TILE_BYTES);
                 tma_load_3d(sbase + C::K_OFF + s * C::TILE_BYTES, &tm_k, bar_k_full(s), 0, j * C::BN, bh, keep);
                 ++nk;
-                ok = wait_phase(bar_v_empty(s), ph ^ 1, SITE_PROD_V_EMPTY, wc);
+            }
+            if (!ok) {
+                for (int j = (nk > C::NS ? nk - C::NS : 0); j < nk; ++j)
+                    drain_copies(bar_k_full(j % C::NS), (j / C::NS) & 1);
+                drain_copies(bar_q, 0);
+            }
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------- producer: V ---
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_v);
+            const uint64_t keep = l2_policy_evict_last();
+            int nv = 0;
+            bool ok = true;
+            for (int j = 0; j < nkv; ++j) {
+                const int s = j % C::NS;
+                ok = wait_phase(bar_v_empty(s), ((j / C::NS) & 1) ^ 1, SITE_PROD_V_EMPTY, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_v_full(s), C::TILE_BYTES);
                 tma_load_3d(sbase + C::V_OFF + s * C::TILE_BYTES, &tm_v, bar_v_full(s), 0, j * C::BN, bh, keep);
                 ++nv;
             }
-            if (!ok) {
-                const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
-                auto drain = [&](uint32_t bar, uint32_t parity) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
-                    }
-                };
-                for (int j = (nk > C::NS ? nk - C::NS : 0); j < nk; ++j)
-                    drain(bar_k_full(j % C::NS), (j / C::NS) & 1);
+            if (!ok)
                 for (int j = (nv > C::NS ? nv - C::NS : 0); j < nv; ++j)
-                    drain(bar_v_full(j % C::NS), (j / C::NS) & 1);
-                drain(bar_q, 0);
-            }
+                    drain_copies(bar_v_full(j % C::NS), (j / C::NS) & 1);
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------- MMA issuer ---
+        // ----------------------------------------- MMA issuer: S = Q8 K8^T ---
+        // S_t = Q_t K_j^T: K = 128 codes = one 128-byte swizzle row, 32 codes
+        // (32 bytes) per MMA. bar_s_free's phases complete in the order S0(0),
+        // S1(0), S0(1), ...: S1(j) waits for parity 0, S0(j+1) for parity 1.
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_e4m3_f32(128, 128, false);  // Q8 K8^T, both K-major
-            constexpr uint32_t IDESC_O = idesc_e4m3_f32(128, 128, true);   // P8 V8, V MN-major
-            auto tm_s = [&](int t) { return tmem + static_cast<uint32_t>(t) * 128u; };
-            auto tm_o = [&](int t) { return tmem + 256u + static_cast<uint32_t>(t) * 128u; };
-            // S_t = Q_t K_j^T: K = 128 codes = one 128-byte swizzle row, 32 codes (32 bytes) per MMA.
             auto issue_s = [&](int t, int s) {
                 const uint32_t qa = sbase + C::Q_OFF + t * C::TILE_BYTES;
                 const uint32_t kb = sbase + C::K_OFF + s * C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ss_f8(tm_s(t), smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024),
+                    mma_ss_f8(tmem, smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024),
                               IDESC_S, kk > 0 ? 1u : 0u);
             };
-            // O_t += P8_t V8_j: 32 keys per MMA = 8 TMEM columns of P8 and 32 rows
-            // (4096 bytes) of V, whose 128 codes per row are the N extent.
+            bool ok = wait_phase(bar_q, 0, SITE_MMA_Q, wc);
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int s = j % C::NS;
+                ok = wait_phase(bar_k_full(s), (j / C::NS) & 1, SITE_MMA_K_FULL, wc);
+                if (!ok) break;
+                if (j > 0) {
+                    ok = wait_phase(bar_s_free, 1, SITE_MMA_S_FREE, wc);  // S1(j-1) copied out
+                    if (!ok) break;
+                }
+                tc_fence_after_sync();
+                issue_s(0, s);
+                tc_commit(bar_s_full(0));
+                ok = wait_phase(bar_s_free, 0, SITE_MMA_S_FREE, wc);      // S0(j) copied out
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_s(1, s);
+                tc_commit(bar_s_full(1));
+                tc_commit(bar_k_empty(s));
+            }
+            drain_mmas();
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------- MMA issuer: O += P8 V8 ---
+        // O_t += P8_t V8_j: 32 keys per MMA = 8 TMEM columns of P8 and 32 rows
+        // (4096 bytes) of V, whose 128 codes per row are the N extent.
+        if (lane == 0) {
+            constexpr uint32_t IDESC_O = idesc_e4m3_f32(128, 128, true);   // P8 V8, V MN-major
             auto issue_pv = [&](int t, int s, bool acc) {
                 const uint32_t vb = sbase + C::V_OFF + s * C::TILE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts_f8(tm_o(t), tm_s(t) + kk * 8, smem_desc_sw128(vb + kk * 4096, C::TILE_BYTES, 1024), IDESC_O,
+                    mma_ts_f8(tm_o(t), tm_p(t) + kk * 8, smem_desc_sw128(vb + kk * 4096, C::TILE_BYTES, 1024), IDESC_O,
                               (acc || kk > 0) ? 1u : 0u);
             };
-            bool ok = wait_phase(bar_q, 0, SITE_MMA_Q, wc);
-            if (ok) ok = wait_phase(bar_k_full(0), 0, SITE_MMA_K_FULL, wc);
-            if (ok) {
-                tc_fence_after_sync();
-                issue_s(0, 0);
-                tc_commit(bar_s_full(0));
-                issue_s(1, 0);
-                tc_commit(bar_s_full(1));
-                tc_commit(bar_k_empty(0));
-            }
+            bool ok = true;
             for (int j = 0; j < nkv && ok; ++j) {
                 const int s = j % C::NS;
-                const uint32_t ph = (j / C::NS) & 1;
-                const int s1 = (j + 1) % C::NS;
-                const uint32_t ph1 = ((j + 1) / C::NS) & 1;
-                const bool more = j + 1 < nkv;
-                ok = wait_phase(bar_v_full(s), ph, SITE_MMA_V_FULL, wc);
+                ok = wait_phase(bar_v_full(s), (j / C::NS) & 1, SITE_MMA_V_FULL, wc);
                 if (!ok) break;
                 ok = wait_phase(bar_p_full(0), j & 1, SITE_MMA_P_FULL, wc);
                 if (!ok) break;
                 tc_fence_after_sync();
                 issue_pv(0, s, j > 0);
-                if (more) {
-                    ok = wait_phase(bar_k_full(s1), ph1, SITE_MMA_K_FULL, wc);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                    issue_s(0, s1);
-                    tc_commit(bar_s_full(0));
-                } else {
-                    tc_commit(bar_o_full(0));
-                }
+                tc_commit(bar_pv_done(0));
                 ok = wait_phase(bar_p_full(1), j & 1, SITE_MMA_P_FULL, wc);
                 if (!ok) break;
                 tc_fence_after_sync();
                 issue_pv(1, s, j > 0);
+                tc_commit(bar_pv_done(1));
                 tc_commit(bar_v_empty(s));
-                if (more) {
-                    issue_s(1, s1);
-                    tc_commit(bar_s_full(1));
-                    tc_commit(bar_k_empty(s1));
-                } else {
-                    tc_commit(bar_o_full(1));
-                }
             }
-            tc_commit(bar_drain);
-            const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(bar_drain, 0)) {
-                if (global_timer_ns() - t0 > drain_ns) {
-                    record_timeout(SITE_DRAIN);
-                    break;
-                }
-            }
+            drain_mmas();
         }
         __syncwarp();
     }
@@ -349,7 +372,8 @@ __global__ void __launch_bounds__(384, 1)
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t ts = tmem + lane_bits + t * 128u;
+        const uint32_t ts = tmem + lane_bits;                 // the shared S buffer
+        const uint32_t tp = tmem + lane_bits + 128u + t * 32u;  // this tile's P8
         const uint32_t to = tmem + lane_bits + 256u + t * 128u;
         const int kv_tail = Skv - (nkv - 1) * C::BN;
         const float *ksc = k_scale + static_cast<int64_t>(bh) * nkv;
@@ -389,6 +413,9 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) reg_fence(sr[cc]);
+            // S is in registers: the buffer may take the other tile's next S.
+            tc_fence_before_sync();
+            mbar_arrive(bar_s_free);
             bool grow = false;
             float alpha = 1.0f;
             auto block = [&](auto masked_tag) {
@@ -449,7 +476,13 @@ __global__ void __launch_bounds__(384, 1)
                     }
                     pk[i >> 2] = pack_e4m3x4(p[0], p[1], p[2], p[3]);
                 }
-                tmem_st_32x32b_x32(ts, pk);
+                // P8_t and O_t are free once PV_t(j-1) has completed.
+                if (j > 0) {
+                    ok = __all_sync(0xffffffffu, wait_phase(bar_pv_done(t), (j - 1) & 1, SITE_SM_PV_DONE, wc));
+                    if (!ok) return;
+                    tc_fence_after_sync();
+                }
+                tmem_st_32x32b_x32(tp, pk);
                 float r0, r1;
                 f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), r0, r1);
                 l += (r0 + r1) * ex2_approx(-bj - C::BIAS);
@@ -458,6 +491,7 @@ __global__ void __launch_bounds__(384, 1)
                 block(std::true_type{});
             else
                 block(std::false_type{});
+            if (!ok) break;
             if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
@@ -474,7 +508,11 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_before_sync();
             mbar_arrive(bar_p_full(t));
         }
-        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_o_full(t), 0, SITE_SM_O_FULL, wc));
+        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_pv_done(t), (nkv - 1) & 1, SITE_SM_O_FULL, wc));
+        // The output is staged in the K ring, tile t in stages 2t and 2t+1. The S
+        // MMAs come from the other issuing thread: tile 1 saw every one of them
+        // complete (its last S is the last one issued), tile 0 waits for that too.
+        if (ok && t == 0) ok = __all_sync(0xffffffffu, wait_phase(bar_s_full(1), (nkv - 1) & 1, SITE_SM_O_FULL, wc));
         if (ok) {
             tc_fence_after_sync();
             // Epilogue: O * sv_max / (2^BIAS l) -> bf16 (P' carried the factor
