@@ -40,6 +40,7 @@ enum BwdWaitSite : uint32_t {
     SITE_BWD_MMA = 13,    // the MMA issuer waiting for operands, P or dS
     SITE_BWD_SM = 14,     // the elementwise warps waiting for S or dP
     SITE_BWD_ACC = 15,    // the epilogue waiting for the accumulators
+    SITE_BWD_SMEM = 16,   // the dynamic shared memory did not start 1024-byte aligned
 };
 
 template <int HD>
@@ -57,18 +58,25 @@ struct BwdCfg {
     static constexpr int MIN_LAUNCH_REGS = 160;
     static constexpr int EMU_PER8 = REGEN_EXP2_EMU_PER8;
 
-    // dK/dV kernel: K and V tiles resident, Q / dO / stats through an NS-stage ring.
-    static constexpr int A_NS = (HD == 128) ? 2 : 4;
+    // dK/dV kernel: K and V tiles resident; Q through an NQ-stage ring and dO with
+    // the per-row stats through an ND-stage ring, both released after dK.
+    // barriers: kv, q_full[NQ], q_empty[NQ], do_full[ND], do_empty[ND], x_full, x_free,
+    // p_full, ds_full, dv_done, dk_done, drain
+    // At D = 128, 3 + 2 stages need 231.6 KB: that fits only without slack for
+    // aligning the base, so the kernel checks that the dynamic shared memory
+    // starts on a 1024-byte boundary (it does when, as here, no static shared
+    // memory precedes it) and refuses to run otherwise.
+    static constexpr int A_NQ = (HD == 128) ? 3 : 4;
+    static constexpr int A_ND = (HD == 128) ? 2 : 4;
     static constexpr int A_K_OFF = 0;
     static constexpr int A_V_OFF = TILE_BYTES;
     static constexpr int A_Q_OFF = 2 * TILE_BYTES;
-    static constexpr int A_DO_OFF = A_Q_OFF + A_NS * TILE_BYTES;
-    static constexpr int A_ST_OFF = A_DO_OFF + A_NS * TILE_BYTES;
-    static constexpr int A_BAR_OFF = A_ST_OFF + A_NS * STAT_BYTES;
-    // kv, full[NS], empty[NS], s_full, dp_full, p_full, ds_full, acc_full, drain
-    static constexpr int A_NBARS = 1 + 2 * A_NS + 6;
+    static constexpr int A_DO_OFF = A_Q_OFF + A_NQ * TILE_BYTES;
+    static constexpr int A_ST_OFF = A_DO_OFF + A_ND * TILE_BYTES;
+    static constexpr int A_BAR_OFF = A_ST_OFF + A_ND * STAT_BYTES;
+    static constexpr int A_NBARS = 1 + 2 * A_NQ + 2 * A_ND + 7;
     static constexpr int A_MISC_OFF = A_BAR_OFF + A_NBARS * 8;
-    static constexpr int A_SMEM_BYTES = A_MISC_OFF + 16 + 1024;
+    static constexpr int A_SMEM_BYTES = A_MISC_OFF + 16;
 
     // dQ kernel: Q and dO resident, K and V through rings of NK and NV stages.
     static constexpr int B_NK = (HD == 128) ? 3 : 4;
@@ -148,12 +156,18 @@ __device__ __forceinline__ void probs_pair(uint32_t &s0, uint32_t &s1, uint64_t 
 // warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-7 and 8-11
 // the elementwise warpgroups; warpgroup w owns query columns [64w, 64w + 64)
 // of the transposed tiles, thread = key row (TMEM lane).
-// TMEM columns: S^T [0,128) (P^T as bf16 over [64w, 64w+32) for each w),
-// dP^T [128,256) (dS^T likewise), dV [256, 256+HD), dK [256+HD, 256+2HD).
-// MMA order per query tile i (one issuing thread, so they run in this order):
-//   dV += P^T(i) dO(i) | S^T(i+1) | dK += dS^T(i) Q(i) | dP^T(i+1)
-// so the exponentials of tile i+1 overlap dK(i) and dP^T(i+1), and dS of
-// tile i overlaps dV(i) and S^T(i+1).
+// TMEM columns: X [0,128) holds S^T(i), then dP^T(i) (fp32; warpgroup w reads
+// [64w, 64w+64)); P^T [128,192) and dS^T [192,256) as bf16 (warpgroup w at
+// +32w); dV [256, 256+HD), dK [256+HD, 256+2HD).
+// The elementwise warps keep P in registers from the moment they copy S^T out,
+// so S^T and dP^T never need tensor memory at the same time, and P^T, dS^T
+// have columns of their own. Two MMA issuers:
+//   warp 1:  S^T(i) = K Q(i)^T, then dP^T(i) = V dO(i)^T, each into X once the
+//            elementwise warps have copied the previous product out;
+//   warp 2:  dV += P^T(i) dO(i) once P^T(i) is stored, dK += dS^T(i) Q(i) once
+//            dS^T(i) is stored.
+// So S^T(i+1) need not wait for dV(i): the elementwise warps wait for dV(i-1)
+// (dK(i-1)) only before storing P^T(i) (dS^T(i)).
 // ACCUM: dK and dV are added to the bf16 values already in dk_old / dv_old
 // (the output buffers themselves: each CTA reads its own key rows before its
 // store), for gradients accumulated over several query blocks.
@@ -166,39 +180,56 @@ __global__ void __launch_bounds__(384, 1)
                          uint64_t wait_limit_ns, const uint16_t *dk_old, const uint16_t *dv_old)
 {
     using C = BwdCfg<HD>;
-    constexpr int NS = C::A_NS;
+    constexpr int NQ = C::A_NQ, ND = C::A_ND;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+    uint8_t *smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    if (sbase & 1023u) {  // uniform over the CTA: nothing has been initialised yet
+        if (threadIdx.x == 0 && atomicCAS(&g_regen_err, 0, -2 /* REGEN_ERR_UNSUPPORTED */) == 0)
+            g_regen_err_site = SITE_BWD_SMEM;
+        return;
+    }
 
     const uint32_t bar0 = sbase + C::A_BAR_OFF;
     const uint32_t bar_kv = bar0;
-    auto bar_full = [&](int s) { return bar0 + 8u * (1 + s); };
-    auto bar_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
-    const uint32_t bar_s_full = bar0 + 8u * (1 + 2 * NS);
-    const uint32_t bar_dp_full = bar0 + 8u * (2 + 2 * NS);
+    auto bar_q_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto bar_q_empty = [&](int s) { return bar0 + 8u * (1 + NQ + s); };
+    auto bar_do_full = [&](int s) { return bar0 + 8u * (1 + 2 * NQ + s); };
+    auto bar_do_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NQ + ND + s); };
+    constexpr int NS = NQ + ND;  // barrier slots taken by the two rings
+    // X's products complete bar_x_full in the order S^T(0), dP^T(0), S^T(1), ...
+    // (parity 0 for S^T, 1 for dP^T) and their copy-outs complete bar_x_free in
+    // the same order: no waiter can fall two phases behind, since the next
+    // product is issued only after the copy-out of the previous one.
+    const uint32_t bar_x_full = bar0 + 8u * (1 + 2 * NS);
+    const uint32_t bar_x_free = bar0 + 8u * (2 + 2 * NS);
     const uint32_t bar_p_full = bar0 + 8u * (3 + 2 * NS);
     const uint32_t bar_ds_full = bar0 + 8u * (4 + 2 * NS);
-    const uint32_t bar_acc_full = bar0 + 8u * (5 + 2 * NS);
-    const uint32_t bar_drain = bar0 + 8u * (6 + 2 * NS);
+    const uint32_t bar_dv_done = bar0 + 8u * (5 + 2 * NS);
+    const uint32_t bar_dk_done = bar0 + 8u * (6 + 2 * NS);
+    const uint32_t bar_drain = bar0 + 8u * (7 + 2 * NS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::A_MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::A_MISC_OFF + 8);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 1);
+        for (int s = 0; s < NQ; ++s) {
+            mbar_init(bar_q_full(s), 1);
+            mbar_init(bar_q_empty(s), 1);
         }
-        mbar_init(bar_s_full, 1);
-        mbar_init(bar_dp_full, 1);
+        for (int s = 0; s < ND; ++s) {
+            mbar_init(bar_do_full(s), 1);
+            mbar_init(bar_do_empty(s), 1);
+        }
+        mbar_init(bar_x_full, 1);
+        mbar_init(bar_x_free, 256);
         mbar_init(bar_p_full, 256);
         mbar_init(bar_ds_full, 256);
-        mbar_init(bar_acc_full, 1);
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_dv_done, 1);
+        mbar_init(bar_dk_done, 1);
+        mbar_init(bar_drain, 2);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -219,14 +250,21 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp < 4) {
     setmaxnreg_dec<C::REGS_LOW>();
+    const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
+    // Aborting: a producer waits (bounded) for its copies still in flight -- at
+    // most the last stages of its ring -- before the CTA exits.
+    auto drain_copies = [&](uint32_t bar, uint32_t parity) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
+        }
+    };
     if (warp == 0) {
-        // ------------------------------------------------------ producer ---
+        // -------------------------------------- producer: K, V, then Q ---
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            tma_prefetch_desc(&tm_do);
-            const uint64_t keep = l2_policy_evict_last();   // Q, dO: re-read by every key tile of the head
+            const uint64_t keep = l2_policy_evict_last();   // Q: re-read by every key tile of the head
             const uint64_t once = l2_policy_evict_first();  // K, V: read by this CTA only
             mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
             for (int h = 0; h < C::HALVES; ++h) {
@@ -236,102 +274,121 @@ __global__ void __launch_bounds__(384, 1)
             int n = 0;  // query tiles issued
             bool ok = true;
             for (int i = 0; i < nq; ++i) {
-                const int s = i % NS;
-                ok = wait_phase(bar_empty(s), ((i / NS) & 1) ^ 1, SITE_BWD_PROD, wc);
+                const int s = i % NQ;
+                ok = wait_phase(bar_q_empty(s), ((i / NQ) & 1) ^ 1, SITE_BWD_PROD, wc);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar_full(s), 2 * C::TILE_BYTES + C::STAT_BYTES);
-                for (int h = 0; h < C::HALVES; ++h) {
-                    tma_load_3d(sbase + C::A_Q_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_q, bar_full(s),
+                mbar_arrive_expect_tx(bar_q_full(s), C::TILE_BYTES);
+                for (int h = 0; h < C::HALVES; ++h)
+                    tma_load_3d(sbase + C::A_Q_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_q, bar_q_full(s),
                                 h * 64, i * C::BM, bh, keep);
-                    tma_load_3d(sbase + C::A_DO_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_do, bar_full(s),
-                                h * 64, i * C::BM, bh, keep);
-                }
-                bulk_load_1d(sbase + C::A_ST_OFF + s * C::STAT_BYTES,
-                             ws + (static_cast<int64_t>(bh) * nq + i) * 256, C::STAT_BYTES, bar_full(s));
                 ++n;
             }
             if (!ok) {
-                // Aborting: wait (bounded) for the copies still in flight -- at most
-                // the last NS stages and the K/V tiles -- before the CTA exits.
-                const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
-                auto drain = [&](uint32_t bar, uint32_t parity) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
-                    }
-                };
-                for (int i = (n > NS ? n - NS : 0); i < n; ++i) drain(bar_full(i % NS), (i / NS) & 1);
-                drain(bar_kv, 0);
+                for (int i = (n > NQ ? n - NQ : 0); i < n; ++i) drain_copies(bar_q_full(i % NQ), (i / NQ) & 1);
+                drain_copies(bar_kv, 0);
             }
         }
-    } else if (warp == 1) {
-        // ---------------------------------------------------- MMA issuer ---
+    } else if (warp == 3) {
+        // ------------------------------------- producer: dO and the stats ---
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_do);
+            const uint64_t keep = l2_policy_evict_last();   // dO: re-read by every key tile of the head
+            int n = 0;
+            bool ok = true;
+            for (int i = 0; i < nq; ++i) {
+                const int s = i % ND;
+                ok = wait_phase(bar_do_empty(s), ((i / ND) & 1) ^ 1, SITE_BWD_PROD, wc);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_do_full(s), C::TILE_BYTES + C::STAT_BYTES);
+                for (int h = 0; h < C::HALVES; ++h)
+                    tma_load_3d(sbase + C::A_DO_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_do, bar_do_full(s),
+                                h * 64, i * C::BM, bh, keep);
+                bulk_load_1d(sbase + C::A_ST_OFF + s * C::STAT_BYTES,
+                             ws + (static_cast<int64_t>(bh) * nq + i) * 256, C::STAT_BYTES, bar_do_full(s));
+                ++n;
+            }
+            if (!ok)
+                for (int i = (n > ND ? n - ND : 0); i < n; ++i) drain_copies(bar_do_full(i % ND), (i / ND) & 1);
+        }
+    } else {
+        // ------------------------------------------- MMA issuers (warps 1, 2) ---
         if (lane == 0) {
             constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 128, false);  // K Q^T, V dO^T: both K-major
             constexpr uint32_t IDESC_G = idesc_bf16_f32(128, HD, true);    // P^T dO, dS^T Q: B MN-major
-            const uint32_t tm_st = tmem, tm_dpt = tmem + 128u;
+            const uint32_t tm_x = tmem, tm_pt = tmem + 128u, tm_dst = tmem + 192u;
             const uint32_t tm_dv = tmem + 256u, tm_dk = tmem + 256u + HD;
-            // D[128 x 128] = A[128 x HD] B[128 x HD]^T, both operands row-major
-            // 128-byte-swizzled tiles: K steps of 16 (32 bytes) inside a swizzle row,
-            // the second 64-column half HALF_BYTES on.
-            auto issue_t = [&](uint32_t d, uint32_t a, uint32_t b) {
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * C::HALF_BYTES + (kk % 4) * 32;
-                    mma_ss(d, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), IDESC_T,
-                           kk > 0 ? 1u : 0u);
-                }
-            };
-            // D[128 x HD] += A[128 keys x 128 queries] (bf16 in TMEM) B[128 queries x HD]:
-            // query steps of 16 = 8 TMEM columns; warpgroup w's 64 queries sit at
-            // column 64w; B rows (queries) 128-byte swizzled, 16 rows = 2048 bytes.
-            auto issue_g = [&](uint32_t d, uint32_t a, uint32_t b, bool acc) {
-#pragma unroll
-                for (int kk = 0; kk < C::BM / 16; ++kk)
-                    mma_ts(d, a + 64u * (kk >> 2) + 8u * (kk & 3),
-                           smem_desc_sw128(b + kk * 2048, C::HALF_BYTES, 1024), IDESC_G,
-                           (acc || kk > 0) ? 1u : 0u);
-            };
             const uint32_t k_s = sbase + C::A_K_OFF, v_s = sbase + C::A_V_OFF;
-            auto q_s = [&](int s) { return sbase + C::A_Q_OFF + s * C::TILE_BYTES; };
-            auto do_s = [&](int s) { return sbase + C::A_DO_OFF + s * C::TILE_BYTES; };
-            bool ok = wait_phase(bar_kv, 0, SITE_BWD_MMA, wc);
-            if (ok) ok = wait_phase(bar_full(0), 0, SITE_BWD_MMA, wc);
-            if (ok) {
-                tc_fence_after_sync();
-                issue_t(tm_st, k_s, q_s(0));
-                tc_commit(bar_s_full);
-                issue_t(tm_dpt, v_s, do_s(0));
-                tc_commit(bar_dp_full);
-            }
-            for (int i = 0; i < nq && ok; ++i) {
-                const int s = i % NS;
-                const int s1 = (i + 1) % NS;
-                const bool more = i + 1 < nq;
-                ok = wait_phase(bar_p_full, i & 1, SITE_BWD_MMA, wc);
-                if (!ok) break;
-                tc_fence_after_sync();
-                issue_g(tm_dv, tm_st, do_s(s), i > 0);
-                if (more) {
-                    ok = wait_phase(bar_full(s1), ((i + 1) / NS) & 1, SITE_BWD_MMA, wc);
+            auto q_s = [&](int i) { return sbase + C::A_Q_OFF + (i % NQ) * C::TILE_BYTES; };
+            auto do_s = [&](int i) { return sbase + C::A_DO_OFF + (i % ND) * C::TILE_BYTES; };
+            bool ok = true;
+            if (warp == 1) {
+                // D[128 x 128] = A[128 x HD] B[128 x HD]^T, both operands row-major
+                // 128-byte-swizzled tiles: K steps of 16 (32 bytes) inside a swizzle row,
+                // the second 64-column half HALF_BYTES on.
+                auto issue_t = [&](uint32_t a, uint32_t b) {
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        const uint32_t off = (kk / 4) * C::HALF_BYTES + (kk % 4) * 32;
+                        mma_ss(tm_x, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024),
+                               IDESC_T, kk > 0 ? 1u : 0u);
+                    }
+                };
+                ok = wait_phase(bar_kv, 0, SITE_BWD_MMA, wc);
+                for (int i = 0; i < nq && ok; ++i) {
+                    ok = wait_phase(bar_q_full(i % NQ), (i / NQ) & 1, SITE_BWD_MMA, wc);
+                    if (!ok) break;
+                    if (i > 0) {
+                        ok = wait_phase(bar_x_free, 1, SITE_BWD_MMA, wc);  // dP^T(i-1) copied out
+                        if (!ok) break;
+                    }
+                    tc_fence_after_sync();
+                    issue_t(k_s, q_s(i));
+                    tc_commit(bar_x_full);
+                    ok = wait_phase(bar_x_free, 0, SITE_BWD_MMA, wc);      // S^T(i) copied out
+                    if (!ok) break;
+                    ok = wait_phase(bar_do_full(i % ND), (i / ND) & 1, SITE_BWD_MMA, wc);
                     if (!ok) break;
                     tc_fence_after_sync();
-                    issue_t(tm_st, k_s, q_s(s1));
-                    tc_commit(bar_s_full);
+                    issue_t(v_s, do_s(i));
+                    tc_commit(bar_x_full);
                 }
-                ok = wait_phase(bar_ds_full, i & 1, SITE_BWD_MMA, wc);
-                if (!ok) break;
-                tc_fence_after_sync();
-                issue_g(tm_dk, tm_dpt, q_s(s), i > 0);
-                tc_commit(bar_empty(s));
-                if (more) {
-                    issue_t(tm_dpt, v_s, do_s(s1));
-                    tc_commit(bar_dp_full);
-                } else {
-                    tc_commit(bar_acc_full);
+            } else {
+                // D[128 x HD] += A[128 keys x 128 queries] (bf16 in TMEM) B[128 queries x HD]:
+                // query steps of 16 = 8 TMEM columns; warpgroup w's 64 queries sit at
+                // column 32w of the operand; B rows (queries) 128-byte swizzled, 16 rows
+                // = 2048 bytes.
+                auto issue_g = [&](uint32_t d, uint32_t a, uint32_t b, bool acc) {
+#pragma unroll
+                    for (int kk = 0; kk < C::BM / 16; ++kk)
+                        mma_ts(d, a + 32u * (kk >> 2) + 8u * (kk & 3),
+                               smem_desc_sw128(b + kk * 2048, C::HALF_BYTES, 1024), IDESC_G,
+                               (acc || kk > 0) ? 1u : 0u);
+                };
+                for (int i = 0; i < nq && ok; ++i) {
+                    // both stages are complete by now (S^T(i) and dP^T(i) read them)
+                    ok = wait_phase(bar_do_full(i % ND), (i / ND) & 1, SITE_BWD_MMA, wc);
+                    if (ok) ok = wait_phase(bar_q_full(i % NQ), (i / NQ) & 1, SITE_BWD_MMA, wc);
+                    if (!ok) break;
+                    ok = wait_phase(bar_p_full, i & 1, SITE_BWD_MMA, wc);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    issue_g(tm_dv, tm_pt, do_s(i), i > 0);
+                    tc_commit(bar_dv_done);
+                    ok = wait_phase(bar_ds_full, i & 1, SITE_BWD_MMA, wc);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    issue_g(tm_dk, tm_dst, q_s(i), i > 0);
+                    tc_commit(bar_dk_done);
+                    // every product that read the two stages has completed: S^T(i)
+                    // and dP^T(i) before the elementwise warps could form dS^T(i),
+                    // which also finished reading the stats in the dO stage
+                    tc_commit(bar_q_empty(i % NQ));
+                    tc_commit(bar_do_empty(i % ND));
                 }
             }
+            // Each issuer commits to bar_drain (count 2) and waits for both, so
+            // that nothing runs on the tensor core when TMEM is freed.
             tc_commit(bar_drain);
-            const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(bar_drain, 0)) {
                 if (global_timer_ns() - t0 > drain_ns) {
@@ -355,69 +412,97 @@ __global__ void __launch_bounds__(384, 1)
         const int quad = warp & 3;
         const int krow = quad * 32 + lane;  // key row inside the tile
         const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t tst = tmem + lane_bits + 64u * w;
-        const uint32_t tdp = tmem + lane_bits + 128u + 64u * w;
+        const uint32_t tx = tmem + lane_bits + 64u * w;           // this warpgroup's columns of X
+        const uint32_t tpt = tmem + lane_bits + 128u + 32u * w;   // its P^T
+        const uint32_t tds = tmem + lane_bits + 192u + 32u * w;   // its dS^T
         const uint64_t c2 = f2_pack(scale_log2, scale_log2);
         bool ok = true;
         for (int i = 0; ok && i < nq; ++i) {
-            const float *st = reinterpret_cast<const float *>(smem + C::A_ST_OFF + (i % NS) * C::STAT_BYTES);
-            const float2 *lse2 = reinterpret_cast<const float2 *>(st + 64 * w);
-            const float2 *dlt = reinterpret_cast<const float2 *>(st + 128 + 64 * w);
-            ok = __all_sync(0xffffffffu, wait_phase(bar_s_full, i & 1, SITE_BWD_SM, wc));
+            const float *st = reinterpret_cast<const float *>(smem + C::A_ST_OFF + (i % ND) * C::STAT_BYTES);
+            const float4 *lse4 = reinterpret_cast<const float4 *>(st + 64 * w);         // two column pairs each
+            const float4 *dlt4 = reinterpret_cast<const float4 *>(st + 128 + 64 * w);
+            ok = __all_sync(0xffffffffu, wait_phase(bar_x_full, 0, SITE_BWD_SM, wc));   // S^T(i)
             // the stats were written by the bulk copy: observe its barrier too
-            // (complete by now; the stage is refilled only after ds_full below)
-            if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_full(i % NS), (i / NS) & 1, SITE_BWD_SM, wc));
+            // (complete by now; the stage is refilled only after dK(i))
+            if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_do_full(i % ND), (i / ND) & 1, SITE_BWD_SM, wc));
             if (!ok) break;
             tc_fence_after_sync();
             uint32_t pr[2][32];
-            tmem_ld_32x32b_x32(tst, pr[0]);
-            tmem_ld_32x32b_x32(tst + 32, pr[1]);
+            tmem_ld_32x32b_x32(tx, pr[0]);
+            tmem_ld_32x32b_x32(tx + 32, pr[1]);
             tmem_ld_wait();
             reg_fence(pr[0]);
             reg_fence(pr[1]);
+            tc_fence_before_sync();
+            mbar_arrive(bar_x_free);
             // P^T = 2^(S^T * scale*log2(e) - lse2[column]); rows past Sq have lse2 = +inf.
+            uint32_t pk[2][16];
+            auto probs_half = [&](int hv) {
 #pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const float2 l = lse2[hv * 16 + c];
+                for (int c = 0; c < 16; c += 2) {
+                    const float4 l = lse4[hv * 8 + c / 2];
                     probs_pair<C::EMU_PER8>(pr[hv][2 * c], pr[hv][2 * c + 1], c2, f2_pack(-l.x, -l.y), c);
-                    pk[c] = pack_bf16x2(__uint_as_float(pr[hv][2 * c]), __uint_as_float(pr[hv][2 * c + 1]));
+                    probs_pair<C::EMU_PER8>(pr[hv][2 * c + 2], pr[hv][2 * c + 3], c2, f2_pack(-l.z, -l.w), c + 1);
+                    pk[hv][c] = pack_bf16x2(__uint_as_float(pr[hv][2 * c]), __uint_as_float(pr[hv][2 * c + 1]));
+                    pk[hv][c + 1] = pack_bf16x2(__uint_as_float(pr[hv][2 * c + 2]), __uint_as_float(pr[hv][2 * c + 3]));
                 }
-                tmem_st_32x32b_x16(tst + 16u * hv, pk);
+            };
+            probs_half(0);
+            // dP^T(i) is ready about now: copying it out halfway through P frees X
+            // for S^T(i+1) one half-block earlier.
+            ok = __all_sync(0xffffffffu, wait_phase(bar_x_full, 1, SITE_BWD_SM, wc));   // dP^T(i)
+            if (!ok) break;
+            tc_fence_after_sync();
+            uint32_t dr[2][32];
+            tmem_ld_32x32b_x32(tx, dr[0]);
+            tmem_ld_32x32b_x32(tx + 32, dr[1]);
+            tmem_ld_wait();
+            reg_fence(dr[0]);
+            reg_fence(dr[1]);
+            tc_fence_before_sync();
+            mbar_arrive(bar_x_free);
+            probs_half(1);
+            if (i > 0) {  // P^T is free once dV(i-1) has read it
+                ok = __all_sync(0xffffffffu, wait_phase(bar_dv_done, (i - 1) & 1, SITE_BWD_SM, wc));
+                if (!ok) break;
+                tc_fence_after_sync();
             }
+            tmem_st_32x32b_x16(tpt, pk[0]);
+            tmem_st_32x32b_x16(tpt + 16u, pk[1]);
             tmem_st_wait();
             tc_fence_before_sync();
             mbar_arrive(bar_p_full);
-            ok = __all_sync(0xffffffffu, wait_phase(bar_dp_full, i & 1, SITE_BWD_SM, wc));
-            if (!ok) break;
-            tc_fence_after_sync();
-            // dS^T = P^T (dP^T - delta[column]), fp32, then bf16 over the dP^T columns.
+            // dS^T = P^T (dP^T - delta[column]), fp32, then bf16.
 #pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-                uint32_t dr[32];
-                tmem_ld_32x32b_x32(tdp + 32u * hv, dr);
-                tmem_ld_wait();
-                reg_fence(dr);
-                uint32_t pk[16];
+            for (int hv = 0; hv < 2; ++hv)
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const float2 d = dlt[hv * 16 + c];
-                    const uint64_t ds = f2_mul(f2_pack(__uint_as_float(pr[hv][2 * c]), __uint_as_float(pr[hv][2 * c + 1])),
-                                               f2_sub(f2_pack(__uint_as_float(dr[2 * c]), __uint_as_float(dr[2 * c + 1])),
-                                                      f2_pack(d.x, d.y)));
-                    float a, b;
-                    f2_unpack(ds, a, b);
-                    pk[c] = pack_bf16x2(a, b);
+                for (int c = 0; c < 16; c += 2) {
+                    const float4 d = dlt4[hv * 8 + c / 2];
+                    const uint64_t ds0 = f2_mul(f2_pack(__uint_as_float(pr[hv][2 * c]), __uint_as_float(pr[hv][2 * c + 1])),
+                                                f2_sub(f2_pack(__uint_as_float(dr[hv][2 * c]), __uint_as_float(dr[hv][2 * c + 1])),
+                                                       f2_pack(d.x, d.y)));
+                    const uint64_t ds1 = f2_mul(f2_pack(__uint_as_float(pr[hv][2 * c + 2]), __uint_as_float(pr[hv][2 * c + 3])),
+                                                f2_sub(f2_pack(__uint_as_float(dr[hv][2 * c + 2]), __uint_as_float(dr[hv][2 * c + 3])),
+                                                       f2_pack(d.z, d.w)));
+                    float a0, b0, a1, b1;
+                    f2_unpack(ds0, a0, b0);
+                    f2_unpack(ds1, a1, b1);
+                    pk[hv][c] = pack_bf16x2(a0, b0);
+                    pk[hv][c + 1] = pack_bf16x2(a1, b1);
                 }
-                tmem_st_32x32b_x16(tdp + 16u * hv, pk);
+            if (i > 0) {  // dS^T is free once dK(i-1) has read it
+                ok = __all_sync(0xffffffffu, wait_phase(bar_dk_done, (i - 1) & 1, SITE_BWD_SM, wc));
+                if (!ok) break;
+                tc_fence_after_sync();
             }
+            tmem_st_32x32b_x16(tds, pk[0]);
+            tmem_st_32x32b_x16(tds + 16u, pk[1]);
             tmem_st_wait();
             tc_fence_before_sync();
             mbar_arrive(bar_ds_full);
         }
-        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_acc_full, 0, SITE_BWD_ACC, wc));
+        // dK(nq-1) is the last product; the commit after it covers dV(nq-1) too
+        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar_dk_done, (nq - 1) & 1, SITE_BWD_ACC, wc));
         if (ok) {
             tc_fence_after_sync();
             // Epilogue: warpgroup 0 writes dV, warpgroup 1 writes scale * dK, each
