@@ -86,8 +86,9 @@ struct BwdCfg {
     static constexpr int B_K_OFF = 2 * TILE_BYTES;
     static constexpr int B_V_OFF = B_K_OFF + B_NK * TILE_BYTES;
     static constexpr int B_BAR_OFF = B_V_OFF + B_NV * TILE_BYTES;
-    // qdo, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], dp_full, ds_full, acc_full, drain
-    static constexpr int B_NBARS = 1 + 2 * B_NK + 2 * B_NV + 2 + 4;
+    // qdo, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], dp_full, ds_full, acc_full,
+    // drain, dp_free, s_free[2]
+    static constexpr int B_NBARS = 1 + 2 * B_NK + 2 * B_NV + 2 + 7;
     static constexpr int B_MISC_OFF = B_BAR_OFF + B_NBARS * 8;
     static constexpr int B_SMEM_BYTES = B_MISC_OFF + 16 + 1024;
 };
@@ -571,9 +572,14 @@ __global__ void __launch_bounds__(384, 1)
 // warpgroup w owns key columns [64w, 64w + 64) of each key tile.
 // TMEM columns: S in two buffers [0,128) and [128,256) (dS as bf16 over
 // [64w, 64w+32) of its buffer), dP [256,384), dQ [384, 384+HD).
-// MMA order per key tile j:  dQ += dS(j) K(j) | dP(j+1) | S(j+2)
-// with S(j+1) already issued, so the exponentials of tile j+1 overlap dQ(j)
-// and dP(j+1). ACCUM: dQ is added to the bf16 values already in dq.
+// Two MMA issuers. Warp 1 issues S(j) = Q K(j)^T into buffer j & 1 once dQ(j-2)
+// has released it, and dP(j) = dO V(j)^T once the elementwise warps have
+// copied dP(j-1) out; neither waits for dS, so both run about a tile ahead.
+// Warp 2 issues dQ += dS(j) K(j) as soon as dS(j) is stored. (With one issuing
+// thread, in the order dQ(j) | dP(j+1) | S(j+2), a clock64 trace showed that
+// thread busy for the whole tile and the elementwise warps idle ~45 % of it.)
+// K and V come from two producer warps (0 and 3).
+// ACCUM: dQ is added to the bf16 values already in dq.
 template <int HD, bool ACCUM>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -602,6 +608,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t bar_ds_full = bar0 + 8u * (4 + 2 * NK + 2 * NV);
     const uint32_t bar_acc_full = bar0 + 8u * (5 + 2 * NK + 2 * NV);
     const uint32_t bar_drain = bar0 + 8u * (6 + 2 * NK + 2 * NV);
+    const uint32_t bar_dp_free = bar0 + 8u * (7 + 2 * NK + 2 * NV);                   // dP copied out
+    auto bar_s_free = [&](int b) { return bar0 + 8u * (8 + 2 * NK + 2 * NV + b); };  // dQ read dS(b)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::B_MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::B_MISC_OFF + 8);
 
@@ -617,10 +625,13 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(bar_s_full(0), 1);
         mbar_init(bar_s_full(1), 1);
+        mbar_init(bar_s_free(0), 1);
+        mbar_init(bar_s_free(1), 1);
         mbar_init(bar_dp_full, 1);
+        mbar_init(bar_dp_free, 256);
         mbar_init(bar_ds_full, 256);
         mbar_init(bar_acc_full, 1);
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_drain, 2);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -642,24 +653,46 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp < 4) {
     setmaxnreg_dec<C::REGS_LOW>();
+    const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
+    auto drain_copies = [&](uint32_t bar, uint32_t parity) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
+        }
+    };
+    // Each MMA issuer commits to bar_drain (count 2) and waits for both before
+    // TMEM is freed.
+    auto drain_mmas = [&]() {
+        tc_commit(bar_drain);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar_drain, 0)) {
+            if (global_timer_ns() - t0 > drain_ns) {
+                record_timeout(SITE_DRAIN);
+                break;
+            }
+        }
+    };
+    auto tm_sb = [&](int b) { return tmem + 128u * static_cast<uint32_t>(b); };
+    const uint32_t tm_dp = tmem + 256u, tm_dq = tmem + 384u;
+    const uint32_t q_s = sbase + C::B_Q_OFF, do_s = sbase + C::B_DO_OFF;
+    auto k_s = [&](int s) { return sbase + C::B_K_OFF + s * C::TILE_BYTES; };
+    auto v_s = [&](int s) { return sbase + C::B_V_OFF + s * C::TILE_BYTES; };
     if (warp == 0) {
-        // ------------------------------------------------------ producer ---
+        // --------------------------------------- producer: Q, dO, then K ---
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            const uint64_t keep = l2_policy_evict_last();   // K, V: re-read by every query tile of the head
+            const uint64_t keep = l2_policy_evict_last();   // K: re-read by every query tile of the head
             const uint64_t once = l2_policy_evict_first();  // Q, dO: read by this CTA only
             mbar_arrive_expect_tx(bar_qdo, 2 * C::TILE_BYTES);
             for (int h = 0; h < C::HALVES; ++h) {
                 tma_load_3d(sbase + C::B_Q_OFF + h * C::HALF_BYTES, &tm_q, bar_qdo, h * 64, q0, bh, once);
                 tma_load_3d(sbase + C::B_DO_OFF + h * C::HALF_BYTES, &tm_do, bar_qdo, h * 64, q0, bh, once);
             }
-            int nk = 0, nv = 0;
+            int nk = 0;
             bool ok = true;
             for (int j = 0; j < nkv; ++j) {
-                const int sk = j % NK, sv = j % NV;
+                const int sk = j % NK;
                 ok = wait_phase(bar_k_empty(sk), ((j / NK) & 1) ^ 1, SITE_BWD_PROD, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_k_full(sk), C::TILE_BYTES);
@@ -667,6 +700,21 @@ __global__ void __launch_bounds__(384, 1)
                     tma_load_3d(sbase + C::B_K_OFF + sk * C::TILE_BYTES + h * C::HALF_BYTES, &tm_k, bar_k_full(sk),
                                 h * 64, j * C::BN, bh, keep);
                 ++nk;
+            }
+            if (!ok) {
+                for (int j = (nk > NK ? nk - NK : 0); j < nk; ++j) drain_copies(bar_k_full(j % NK), (j / NK) & 1);
+                drain_copies(bar_qdo, 0);
+            }
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------- producer: V ---
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_v);
+            const uint64_t keep = l2_policy_evict_last();   // V: re-read by every query tile of the head
+            int nv = 0;
+            bool ok = true;
+            for (int j = 0; j < nkv; ++j) {
+                const int sv = j % NV;
                 ok = wait_phase(bar_v_empty(sv), ((j / NV) & 1) ^ 1, SITE_BWD_PROD, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_v_full(sv), C::TILE_BYTES);
@@ -675,25 +723,18 @@ __global__ void __launch_bounds__(384, 1)
                                 h * 64, j * C::BN, bh, keep);
                 ++nv;
             }
-            if (!ok) {
-                const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
-                auto drain = [&](uint32_t bar, uint32_t parity) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < drain_ns) {
-                    }
-                };
-                for (int j = (nk > NK ? nk - NK : 0); j < nk; ++j) drain(bar_k_full(j % NK), (j / NK) & 1);
-                for (int j = (nv > NV ? nv - NV : 0); j < nv; ++j) drain(bar_v_full(j % NV), (j / NV) & 1);
-                drain(bar_qdo, 0);
-            }
+            if (!ok)
+                for (int j = (nv > NV ? nv - NV : 0); j < nv; ++j) drain_copies(bar_v_full(j % NV), (j / NV) & 1);
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------- MMA issuer ---
+        // ----------------------------- MMA issuer: S = Q K^T and dP = dO V^T ---
+        // S(j) goes into buffer j & 1 once dQ(j-2) has read the dS written over
+        // it; dP(j) into its buffer once the elementwise warps have copied dP(j-1)
+        // out. Neither waits for dS, so both run ahead of the elementwise work.
+        // This thread is the only waiter on bar_s_free(b) and bar_dp_free and
+        // waits for each of their completions in turn.
         if (lane == 0) {
             constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 128, false);  // Q K^T, dO V^T
-            constexpr uint32_t IDESC_G = idesc_bf16_f32(128, HD, true);    // dS K: K tile MN-major
-            auto tm_sb = [&](int b) { return tmem + 128u * static_cast<uint32_t>(b); };
-            const uint32_t tm_dp = tmem + 256u, tm_dq = tmem + 384u;
             auto issue_t = [&](uint32_t d, uint32_t a, uint32_t b) {
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
@@ -702,6 +743,36 @@ __global__ void __launch_bounds__(384, 1)
                            kk > 0 ? 1u : 0u);
                 }
             };
+            bool ok = wait_phase(bar_qdo, 0, SITE_BWD_MMA, wc);
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int b = j & 1;
+                if (j >= 2) {
+                    ok = wait_phase(bar_s_free(b), ((j - 2) >> 1) & 1, SITE_BWD_MMA, wc);
+                    if (!ok) break;
+                }
+                ok = wait_phase(bar_k_full(j % NK), (j / NK) & 1, SITE_BWD_MMA, wc);
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_t(tm_sb(b), q_s, k_s(j % NK));
+                tc_commit(bar_s_full(b));
+                if (j >= 1) {
+                    ok = wait_phase(bar_dp_free, (j - 1) & 1, SITE_BWD_MMA, wc);
+                    if (!ok) break;
+                }
+                ok = wait_phase(bar_v_full(j % NV), (j / NV) & 1, SITE_BWD_MMA, wc);
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_t(tm_dp, do_s, v_s(j % NV));
+                tc_commit(bar_dp_full);
+                tc_commit(bar_v_empty(j % NV));
+            }
+            drain_mmas();
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------- MMA issuer: dQ += dS K ---
+        if (lane == 0) {
+            constexpr uint32_t IDESC_G = idesc_bf16_f32(128, HD, true);    // dS K: K tile MN-major
             auto issue_dq = [&](uint32_t a, uint32_t kb, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)
@@ -709,67 +780,21 @@ __global__ void __launch_bounds__(384, 1)
                            smem_desc_sw128(kb + kk * 2048, C::HALF_BYTES, 1024), IDESC_G,
                            (acc || kk > 0) ? 1u : 0u);
             };
-            const uint32_t q_s = sbase + C::B_Q_OFF, do_s = sbase + C::B_DO_OFF;
-            auto k_s = [&](int s) { return sbase + C::B_K_OFF + s * C::TILE_BYTES; };
-            auto v_s = [&](int s) { return sbase + C::B_V_OFF + s * C::TILE_BYTES; };
-            bool ok = wait_phase(bar_qdo, 0, SITE_BWD_MMA, wc);
-            if (ok) ok = wait_phase(bar_k_full(0), 0, SITE_BWD_MMA, wc);
-            if (ok) {
-                tc_fence_after_sync();
-                issue_t(tm_sb(0), q_s, k_s(0));
-                tc_commit(bar_s_full(0));
-                ok = wait_phase(bar_v_full(0), 0, SITE_BWD_MMA, wc);
-            }
-            if (ok) {
-                tc_fence_after_sync();
-                issue_t(tm_dp, do_s, v_s(0));
-                tc_commit(bar_dp_full);
-                tc_commit(bar_v_empty(0));
-                if (nkv > 1) {
-                    ok = wait_phase(bar_k_full(1 % NK), (1 / NK) & 1, SITE_BWD_MMA, wc);
-                    if (ok) {
-                        tc_fence_after_sync();
-                        issue_t(tm_sb(1), q_s, k_s(1 % NK));
-                        tc_commit(bar_s_full(1));
-                    }
-                }
-            }
+            bool ok = true;
             for (int j = 0; j < nkv && ok; ++j) {
                 const int b = j & 1;
-                ok = wait_phase(bar_ds_full, j & 1, SITE_BWD_MMA, wc);
+                ok = wait_phase(bar_k_full(j % NK), (j / NK) & 1, SITE_BWD_MMA, wc);  // complete by now
+                if (ok) ok = wait_phase(bar_ds_full, j & 1, SITE_BWD_MMA, wc);
                 if (!ok) break;
                 tc_fence_after_sync();
                 issue_dq(tm_sb(b), k_s(j % NK), j > 0);
+                tc_commit(bar_s_free(b));
+                // K(j) was read by S(j) too; that MMA completed before the
+                // elementwise warps could form dS(j).
                 tc_commit(bar_k_empty(j % NK));
-                if (j + 1 < nkv) {
-                    const int sv = (j + 1) % NV;
-                    ok = wait_phase(bar_v_full(sv), ((j + 1) / NV) & 1, SITE_BWD_MMA, wc);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                    issue_t(tm_dp, do_s, v_s(sv));
-                    tc_commit(bar_dp_full);
-                    tc_commit(bar_v_empty(sv));
-                } else {
-                    tc_commit(bar_acc_full);
-                }
-                if (j + 2 < nkv) {
-                    const int sk = (j + 2) % NK;
-                    ok = wait_phase(bar_k_full(sk), ((j + 2) / NK) & 1, SITE_BWD_MMA, wc);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                    issue_t(tm_sb(b), q_s, k_s(sk));
-                    tc_commit(bar_s_full(b));
-                }
+                if (j + 1 == nkv) tc_commit(bar_acc_full);
             }
-            tc_commit(bar_drain);
-            const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(bar_drain, 0)) {
-                if (global_timer_ns() - t0 > drain_ns) {
-                    record_timeout(SITE_DRAIN);
-                    break;
-                }
-            }
+            drain_mmas();
         }
         __syncwarp();
     }
@@ -819,17 +844,22 @@ __global__ void __launch_bounds__(384, 1)
             ok = __all_sync(0xffffffffu, wait_phase(bar_dp_full, j & 1, SITE_BWD_SM, wc));
             if (!ok) break;
             tc_fence_after_sync();
+            uint32_t dr[2][32];
+            tmem_ld_32x32b_x32(tmem + lane_bits + 256u + 64u * w, dr[0]);
+            tmem_ld_32x32b_x32(tmem + lane_bits + 256u + 64u * w + 32u, dr[1]);
+            tmem_ld_wait();
+            reg_fence(dr[0]);
+            reg_fence(dr[1]);
+            // dP is in registers: the buffer may take dP(j+1).
+            tc_fence_before_sync();
+            mbar_arrive(bar_dp_free);
 #pragma unroll
             for (int hv = 0; hv < 2; ++hv) {
-                uint32_t dr[32];
-                tmem_ld_32x32b_x32(tmem + lane_bits + 256u + 64u * w + 32u * hv, dr);
-                tmem_ld_wait();
-                reg_fence(dr);
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
                     const uint64_t ds = f2_mul(f2_pack(__uint_as_float(pr[hv][2 * c]), __uint_as_float(pr[hv][2 * c + 1])),
-                                               f2_sub(f2_pack(__uint_as_float(dr[2 * c]), __uint_as_float(dr[2 * c + 1])), dl2));
+                                               f2_sub(f2_pack(__uint_as_float(dr[hv][2 * c]), __uint_as_float(dr[hv][2 * c + 1])), dl2));
                     float a, bb;
                     f2_unpack(ds, a, bb);
                     pk[c] = pack_bf16x2(a, bb);

@@ -115,14 +115,21 @@ struct AttnCfg {
     static constexpr int HALVES = HD / 64;                // 128-byte column groups per row
     static constexpr int TILE_BYTES = 128 * HD * 2;       // one 128-row bf16 tile
     static constexpr int HALF_BYTES = 128 * 128;          // 128 rows x 128 bytes
-    static constexpr int NS = (HD == 128) ? 2 : 4;        // K ring and V ring depth
+#ifndef REGEN_FWD_K_STAGES
+#define REGEN_FWD_K_STAGES 2
+#endif
+#ifndef REGEN_FWD_V_STAGES
+#define REGEN_FWD_V_STAGES 2
+#endif
+    static constexpr int NSK = (HD == 128) ? REGEN_FWD_K_STAGES : 4;  // K ring depth
+    static constexpr int NSV = (HD == 128) ? REGEN_FWD_V_STAGES : 4;  // V ring depth
     static constexpr int Q_OFF = 0;
     static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
-    static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
-    static constexpr int BAR_OFF = V_OFF + NS * TILE_BYTES;
-    // barriers: q, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], s_free,
+    static constexpr int V_OFF = K_OFF + NSK * TILE_BYTES;
+    static constexpr int BAR_OFF = V_OFF + NSV * TILE_BYTES;
+    // barriers: q, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[2], s_free,
     // p_full[2], pv_done[2], drain, q_rotated
-    static constexpr int NBARS = 1 + 4 * NS + 7 + 1 + 1;
+    static constexpr int NBARS = 1 + 2 * NSK + 2 * NSV + 7 + 1 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;  // abort flag, TMEM base
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -160,23 +167,26 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t bar0 = sbase + C::BAR_OFF;
     const uint32_t bar_q = bar0;
     auto bar_k_full = [&](int s) { return bar0 + 8u * (1 + s); };
-    auto bar_k_empty = [&](int s) { return bar0 + 8u * (1 + C::NS + s); };
-    auto bar_v_full = [&](int s) { return bar0 + 8u * (1 + 2 * C::NS + s); };
-    auto bar_v_empty = [&](int s) { return bar0 + 8u * (1 + 3 * C::NS + s); };
-    auto bar_s_full = [&](int t) { return bar0 + 8u * (1 + 4 * C::NS + t); };
-    const uint32_t bar_s_free = bar0 + 8u * (3 + 4 * C::NS);  // S copied out by a softmax warpgroup
-    auto bar_p_full = [&](int t) { return bar0 + 8u * (4 + 4 * C::NS + t); };
-    auto bar_pv_done = [&](int t) { return bar0 + 8u * (6 + 4 * C::NS + t); };
-    const uint32_t bar_drain = bar0 + 8u * (8 + 4 * C::NS);
-    const uint32_t bar_qrot = bar0 + 8u * (9 + 4 * C::NS);  // Q tiles rotated (ROPE_Q)
+    constexpr int NB = 2 * C::NSK + 2 * C::NSV;  // slots of the two rings' barriers
+    auto bar_k_empty = [&](int s) { return bar0 + 8u * (1 + C::NSK + s); };
+    auto bar_v_full = [&](int s) { return bar0 + 8u * (1 + 2 * C::NSK + s); };
+    auto bar_v_empty = [&](int s) { return bar0 + 8u * (1 + 2 * C::NSK + C::NSV + s); };
+    auto bar_s_full = [&](int t) { return bar0 + 8u * (1 + NB + t); };
+    const uint32_t bar_s_free = bar0 + 8u * (3 + NB);  // S copied out by a softmax warpgroup
+    auto bar_p_full = [&](int t) { return bar0 + 8u * (4 + NB + t); };
+    auto bar_pv_done = [&](int t) { return bar0 + 8u * (6 + NB + t); };
+    const uint32_t bar_drain = bar0 + 8u * (8 + NB);
+    const uint32_t bar_qrot = bar0 + 8u * (9 + NB);  // Q tiles rotated (ROPE_Q)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 8);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        for (int s = 0; s < C::NS; ++s) {
+        for (int s = 0; s < C::NSK; ++s) {
             mbar_init(bar_k_full(s), 1);
             mbar_init(bar_k_empty(s), 1);
+        }
+        for (int s = 0; s < C::NSV; ++s) {
             mbar_init(bar_v_full(s), 1);
             mbar_init(bar_v_empty(s), 1);
         }
@@ -256,8 +266,8 @@ __global__ void __launch_bounds__(384, 1)
             int nk = 0;  // K block loads issued so far
             bool ok = true;
             for (int j = 0; j < nkv; ++j) {
-                const int s = j % C::NS;
-                ok = wait_phase(bar_k_empty(s), ((j / C::NS) & 1) ^ 1, SITE_PROD_K_EMPTY, wc);
+                const int s = j % C::NSK;
+                ok = wait_phase(bar_k_empty(s), ((j / C::NSK) & 1) ^ 1, SITE_PROD_K_EMPTY, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_k_full(s), C::TILE_BYTES);
                 for (int h = 0; h < C::HALVES; ++h)
@@ -266,8 +276,8 @@ __global__ void __launch_bounds__(384, 1)
                 ++nk;
             }
             if (!ok) {
-                for (int j = (nk > C::NS ? nk - C::NS : 0); j < nk; ++j)
-                    drain_copies(bar_k_full(j % C::NS), (j / C::NS) & 1);
+                for (int j = (nk > C::NSK ? nk - C::NSK : 0); j < nk; ++j)
+                    drain_copies(bar_k_full(j % C::NSK), (j / C::NSK) & 1);
                 drain_copies(bar_q, 0);
             }
         }
@@ -279,8 +289,8 @@ __global__ void __launch_bounds__(384, 1)
             int nv = 0;
             bool ok = true;
             for (int j = 0; j < nkv; ++j) {
-                const int s = j % C::NS;
-                ok = wait_phase(bar_v_empty(s), ((j / C::NS) & 1) ^ 1, SITE_PROD_V_EMPTY, wc);
+                const int s = j % C::NSV;
+                ok = wait_phase(bar_v_empty(s), ((j / C::NSV) & 1) ^ 1, SITE_PROD_V_EMPTY, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_v_full(s), C::TILE_BYTES);
                 for (int h = 0; h < C::HALVES; ++h)
@@ -289,8 +299,8 @@ __global__ void __launch_bounds__(384, 1)
                 ++nv;
             }
             if (!ok)
-                for (int j = (nv > C::NS ? nv - C::NS : 0); j < nv; ++j)
-                    drain_copies(bar_v_full(j % C::NS), (j / C::NS) & 1);
+                for (int j = (nv > C::NSV ? nv - C::NSV : 0); j < nv; ++j)
+                    drain_copies(bar_v_full(j % C::NSV), (j / C::NSV) & 1);
         }
     } else if (warp == 1) {
         // -------------------------------------------- MMA issuer: S = QK^T ---
@@ -315,8 +325,8 @@ __global__ void __launch_bounds__(384, 1)
             };
             bool ok = wait_phase(ROPE_Q ? bar_qrot : bar_q, 0, SITE_MMA_Q, wc);
             for (int j = 0; j < nkv && ok; ++j) {
-                const int s = j % C::NS;
-                ok = wait_phase(bar_k_full(s), (j / C::NS) & 1, SITE_MMA_K_FULL, wc);
+                const int s = j % C::NSK;
+                ok = wait_phase(bar_k_full(s), (j / C::NSK) & 1, SITE_MMA_K_FULL, wc);
                 if (!ok) break;
                 if (j > 0) {
                     ok = wait_phase(bar_s_free, 1, SITE_MMA_S_FREE, wc);  // S1(j-1) copied out
@@ -355,8 +365,8 @@ __global__ void __launch_bounds__(384, 1)
             };
             bool ok = true;
             for (int j = 0; j < nkv && ok; ++j) {
-                const int s = j % C::NS;
-                ok = wait_phase(bar_v_full(s), (j / C::NS) & 1, SITE_MMA_V_FULL, wc);
+                const int s = j % C::NSV;
+                ok = wait_phase(bar_v_full(s), (j / C::NSV) & 1, SITE_MMA_V_FULL, wc);
                 if (!ok) break;
                 ok = wait_phase(bar_p_full(0), j & 1, SITE_MMA_P_FULL, wc);
                 if (!ok) break;
