@@ -351,11 +351,15 @@ REGEN_API const char *regen_status_str(int status);
 REGEN_API int regen_last_cuda_error(const char **name);
 
 /*
- * regen_last_device_error -- REGEN_OK, or REGEN_ERR_TIMEOUT when a kernel of
- * this library gave up on a bounded wait since the previous call; clears the
- * record. It synchronises the device first (cudaDeviceSynchronize) and
- * returns REGEN_ERR_CUDA if that fails. *detail (may be NULL) receives a code
- * naming the wait that expired (0 if none).
+ * regen_last_device_error -- REGEN_OK, or the first error a kernel of this
+ * library recorded since the previous call; clears the record:
+ *   REGEN_ERR_TIMEOUT      a kernel gave up on a bounded wait;
+ *   REGEN_ERR_UNSUPPORTED  the gradient's dK/dV kernel found its dynamic shared
+ *                          memory not 1024-byte aligned and did nothing (detail 16;
+ *                          it needs all 227 KB, with no room to realign).
+ * It synchronises the device first (cudaDeviceSynchronize) and returns
+ * REGEN_ERR_CUDA if that fails. *detail (may be NULL) receives a code naming
+ * the wait or check that failed (0 if none).
  */
 REGEN_API int regen_last_device_error(uint32_t *detail);
 
