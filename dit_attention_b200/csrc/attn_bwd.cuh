@@ -437,10 +437,16 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_before_sync();
             mbar_arrive(bar_x_free);
             // P^T = 2^(S^T * scale*log2(e) - lse2[column]); rows past Sq have lse2 = +inf.
+            // Computed in quarters of 8 column pairs. dP^T(i) is copied out of X as
+            // soon as a non-blocking test after a quarter finds it ready (a blocking
+            // wait only after the last), so that X takes S^T(i+1) as early as possible.
             uint32_t pk[2][16];
-            auto probs_half = [&](int hv) {
+            uint32_t dr[2][32];
+            bool have_dp = false;
+            auto probs_quarter = [&](int qtr) {
+                const int hv = qtr >> 1;
 #pragma unroll
-                for (int c = 0; c < 16; c += 2) {
+                for (int c = (qtr & 1) * 8; c < (qtr & 1) * 8 + 8; c += 2) {
                     const float4 l = lse4[hv * 8 + c / 2];
                     probs_pair<C::EMU_PER8>(pr[hv][2 * c], pr[hv][2 * c + 1], c2, f2_pack(-l.x, -l.y), c);
                     probs_pair<C::EMU_PER8>(pr[hv][2 * c + 2], pr[hv][2 * c + 3], c2, f2_pack(-l.z, -l.w), c + 1);
@@ -448,21 +454,28 @@ __global__ void __launch_bounds__(384, 1)
                     pk[hv][c + 1] = pack_bf16x2(__uint_as_float(pr[hv][2 * c + 2]), __uint_as_float(pr[hv][2 * c + 3]));
                 }
             };
-            probs_half(0);
-            // dP^T(i) is ready about now: copying it out halfway through P frees X
-            // for S^T(i+1) one half-block earlier.
-            ok = __all_sync(0xffffffffu, wait_phase(bar_x_full, 1, SITE_BWD_SM, wc));   // dP^T(i)
-            if (!ok) break;
-            tc_fence_after_sync();
-            uint32_t dr[2][32];
-            tmem_ld_32x32b_x32(tx, dr[0]);
-            tmem_ld_32x32b_x32(tx + 32, dr[1]);
-            tmem_ld_wait();
-            reg_fence(dr[0]);
-            reg_fence(dr[1]);
-            tc_fence_before_sync();
-            mbar_arrive(bar_x_free);
-            probs_half(1);
+            auto copy_dp = [&]() {
+                tc_fence_after_sync();
+                tmem_ld_32x32b_x32(tx, dr[0]);
+                tmem_ld_32x32b_x32(tx + 32, dr[1]);
+                tmem_ld_wait();
+                reg_fence(dr[0]);
+                reg_fence(dr[1]);
+                tc_fence_before_sync();
+                mbar_arrive(bar_x_free);
+                have_dp = true;
+            };
+#pragma unroll
+            for (int qtr = 0; qtr < 3; ++qtr) {
+                probs_quarter(qtr);
+                if (!have_dp && __all_sync(0xffffffffu, mbar_test_wait(bar_x_full, 1))) copy_dp();
+            }
+            probs_quarter(3);
+            if (!have_dp) {
+                ok = __all_sync(0xffffffffu, wait_phase(bar_x_full, 1, SITE_BWD_SM, wc));   // dP^T(i)
+                if (!ok) break;
+                copy_dp();
+            }
             if (i > 0) {  // P^T is free once dV(i-1) has read it
                 ok = __all_sync(0xffffffffu, wait_phase(bar_dv_done, (i - 1) & 1, SITE_BWD_SM, wc));
                 if (!ok) break;
