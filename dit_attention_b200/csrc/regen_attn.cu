@@ -412,8 +412,8 @@ int attn_rope3d_with_scratch(const regen_bf16 *q, const regen_bf16 *k, const reg
     regen_bf16 *k_rot = reinterpret_cast<regen_bf16 *>(scratch + rope_table_bytes(geom));
     regen::rope_table_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
     if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
-    const int64_t chunks = BH * S * (D / 8);
-    regen::rope_apply_kernel<<<grid_for(chunks, 256), 256, 0, st>>>(
+    const int64_t chunks = static_cast<int64_t>(S) * (D / 8);  // one thread per (token, chunk), all rows
+    regen::rope_apply_kernel<<<grid_for(chunks, 128), 128, 0, st>>>(
         reinterpret_cast<const uint4 *>(k), reinterpret_cast<uint4 *>(k_rot), BH, S, D, geom, tab);
     if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     const bool neg = scale < 0.0f;

@@ -128,22 +128,38 @@ __device__ __forceinline__ uint4 rotate_chunk(uint4 v, int c, int n, const RopeG
 __global__ void rope_apply_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int64_t rows, int S,
                                   int D, RopeGeom g, const double *__restrict__ tab)
 {
+    // One thread per (token, 16-byte chunk): the chunk's four (cos, sin) pairs
+    // are read from the table once and applied to that chunk of every row
+    // (consecutive threads, consecutive chunks of one row: coalesced).
     const int chunks = D >> 3;
     const int64_t per_row = static_cast<int64_t>(S) * chunks;
-    const int64_t total = rows * per_row;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total; i += stride) {
-        const int64_t in_row = i % per_row;
-        const int n = static_cast<int>(in_row / chunks);
-        const int c = static_cast<int>(in_row % chunks);
-        dst[i] = rotate_chunk(src[i], c, n, g, tab);
+    for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < per_row; t += stride) {
+        const int n = static_cast<int>(t / chunks);
+        const int c = static_cast<int>(t % chunks);
+        double cs[4], sn[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const int64_t e = g.entry(n, c * 8 + 2 * p);
+            cs[p] = __ldg(tab + 2 * e);
+            sn[p] = __ldg(tab + 2 * e + 1);
+        }
+        auto rot = [&](uint4 v) {
+            return make_uint4(rotate_pair(v.x, cs[0], sn[0]), rotate_pair(v.y, cs[1], sn[1]),
+                              rotate_pair(v.z, cs[2], sn[2]), rotate_pair(v.w, cs[3], sn[3]));
+        };
+        int64_t r = 0;
+        for (; r + 4 <= rows; r += 4) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = src[(r + u) * per_row + t];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) dst[(r + u) * per_row + t] = rot(v[u]);
+        }
+        for (; r < rows; ++r) dst[r * per_row + t] = rot(src[r * per_row + t]);
     }
 }
 
-// grid: ceil(S * D/8 / blockDim) blocks; x (q then k) has `rows` rows of S x D
-// holding the latent tokens n0 .. n0 + S - 1 (a sequence shard when n0 > 0).
-// inverse: turn every pair back by its angle (sine negated), the transposed
-// rotation that carries gradients through the RoPE.
 __global__ void rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k, int64_t rows,
                               int S, int Hh, int Ww, int D, double theta, bool inverse, int n0)
 {
