@@ -50,6 +50,7 @@ __all__ = [
     "RegenError", "library_path", "load", "regen_attn_fwd", "regen_rope3d", "regen_lse_merge",
     "regen_status_str", "regen_last_device_error", "regen_last_cuda_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
     "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes", "regen_attn_fwd_rope3d_noalloc",
+    "regen_noalloc_scratch_bytes",
     "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd", "regen_rope3d_shard", "regen_quant_e4m3",
     "regen_attn_fwd_fp8", "quant_e4m3", "attn_fwd_fp8", "regen_qkv_proj", "regen_qkv_proj_workspace_bytes",
     "regen_out_proj", "qkv_proj", "out_proj",
@@ -99,6 +100,8 @@ def load():
         L.regen_attn_fwd_rope3d_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp,
                                                     i32, i32, i32, f32]
         L.regen_attn_fwd_rope3d_noalloc.restype = i32
+        L.regen_noalloc_scratch_bytes.argtypes = []
+        L.regen_noalloc_scratch_bytes.restype = i64
         L.regen_attn_fwd_rope3d_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
         L.regen_attn_fwd_rope3d_workspace_bytes.restype = i64
         L.regen_rope3d.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, vp]
@@ -187,7 +190,9 @@ def regen_attn_fwd_rope3d(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream, T,
                                         int(workspace_bytes)), "regen_attn_fwd_rope3d")
 
 
-NOALLOC_SCRATCH_BYTES = 64 << 20   # REGEN_NOALLOC_SCRATCH_BYTES
+def regen_noalloc_scratch_bytes() -> int:
+    """Size of the fixed scratch array built into the library."""
+    return int(load().regen_noalloc_scratch_bytes())
 
 
 def regen_attn_fwd_rope3d_noalloc(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream, T, Hh, Ww, theta) -> None:
@@ -197,9 +202,10 @@ def regen_attn_fwd_rope3d_noalloc(q, k, v, out, lse, B, H, Sq, Skv, D, scale, st
                                               float(scale), _stream(stream), T, Hh, Ww, float(theta))
     if rc == -2 and D in (64, 128) and T > 0 and Hh > 0 and Ww > 0:
         need = load().regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
-        if need > NOALLOC_SCRATCH_BYTES:
+        have = regen_noalloc_scratch_bytes()
+        if need > have:
             raise RegenError(rc, f"regen_attn_fwd_rope3d_noalloc: needs {need} bytes of scratch, "
-                                 f"the fixed array holds {NOALLOC_SCRATCH_BYTES}")
+                                 f"the fixed array holds {have}")
     _check(rc, "regen_attn_fwd_rope3d_noalloc")
 
 

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libregen_attn.so")
 SOURCES = ["regen_attn.cu"]
-HEADERS = ["ptx.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "attn_fp8.cuh", "proj_gemm.cuh", "rope3d.cuh", "lse_merge.cuh"]
+HEADERS = ["ctx_cache.h", "ptx.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "attn_fp8.cuh", "proj_gemm.cuh", "rope3d.cuh", "lse_merge.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 

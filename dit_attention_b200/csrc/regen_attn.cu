@@ -14,8 +14,11 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "regen_attn.h"
+
+#include "ctx_cache.h"
 
 #include "attn_bwd.cuh"
 #include "attn_fp8.cuh"
@@ -81,7 +84,8 @@ struct DriverCalls {
     CUresult (*ctx_get_current)(CUcontext *) = nullptr;
     CUresult (*ctx_get_device)(CUdevice *) = nullptr;
     CUresult (*ctx_set_current)(CUcontext) = nullptr;
-    bool ok() const { return pointer_attr && ctx_get_current && ctx_get_device && ctx_set_current; }
+    CUresult (*ctx_get_id)(CUcontext, unsigned long long *) = nullptr;
+    bool ok() const { return pointer_attr && ctx_get_current && ctx_get_device && ctx_set_current && ctx_get_id; }
 };
 
 const DriverCalls &driver()
@@ -99,6 +103,7 @@ const DriverCalls &driver()
         d.ctx_get_current = reinterpret_cast<decltype(d.ctx_get_current)>(get("cuCtxGetCurrent"));
         d.ctx_get_device = reinterpret_cast<decltype(d.ctx_get_device)>(get("cuCtxGetDevice"));
         d.ctx_set_current = reinterpret_cast<decltype(d.ctx_set_current)>(get("cuCtxSetCurrent"));
+        d.ctx_get_id = reinterpret_cast<decltype(d.ctx_get_id)>(get("cuCtxGetId"));
     });
     return d;
 }
@@ -154,6 +159,54 @@ public:
 private:
     CUcontext prev_ = nullptr;
 };
+
+// The driver's unique ID of the context current on this thread (the one
+// DeviceScope bound); false when there is none or the driver cannot say.
+bool current_context_id(unsigned long long *id)
+{
+    const DriverCalls &d = driver();
+    CUcontext cur = nullptr;
+    if (!d.ok() || !encoded(d.ctx_get_current(&cur))) return false;
+    if (cur == nullptr) {
+        g_last_cuda_error = kDriverErrorBase + static_cast<int>(CUDA_ERROR_INVALID_CONTEXT);
+        return false;
+    }
+    return encoded(d.ctx_get_id(cur, id));
+}
+
+// One value per CUDA context, computed on the first call made in that context
+// (ctx_cache.h): a kernel's shared-memory limit and a __device__ symbol's
+// address belong to the module as loaded in one context, not to the process.
+template <typename T>
+class PerContext {
+public:
+    template <typename F>
+    int get(F &&setup, T *value)
+    {
+        unsigned long long id = 0;
+        if (!current_context_id(&id)) return REGEN_ERR_CUDA;
+        return cache_.get(id, std::forward<F>(setup), value);
+    }
+
+private:
+    regen::CtxCache<T, REGEN_ERR_CUDA> cache_;
+};
+
+// Raise a kernel's dynamic shared-memory limit in the current context and
+// check that its compiled register count leaves room for the in-kernel
+// register re-allocation (else REGEN_ERR_UNSUPPORTED: the split would wait
+// forever, so the kernel is never launched).
+int kernel_setup(const void *fn, int smem_bytes, int min_regs)
+{
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, fn);
+    if (e != cudaSuccess) {
+        cudaGetLastError();   // not sticky: clear the runtime's record
+        return cuda_status(e);
+    }
+    return fa.numRegs < min_regs ? static_cast<int>(REGEN_ERR_UNSUPPORTED) : static_cast<int>(REGEN_OK);
+}
 
 // [BH, S, D] bf16 viewed as a 3D tensor (D innermost), boxes of 64 x 128 x 1
 // with the 128-byte swizzle; out-of-range rows read as zero.
@@ -218,17 +271,11 @@ int launch_proj(const CUtensorMap &ta, const CUtensorMap &tb, const regen::ProjS
                 const regen::ProjEpi &ep, cudaStream_t stream)
 {
     using C = regen::ProjCfg;
-    static std::once_flag once;
-    static int attr_status = REGEN_OK;
-    std::call_once(once, [] {
-        cudaFuncAttributes fa;
-        if (cudaFuncSetAttribute(regen::proj_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncGetAttributes(&fa, regen::proj_gemm_kernel<MODE>) != cudaSuccess)
-            attr_status = REGEN_ERR_CUDA;
-        else if (fa.numRegs < C::MIN_LAUNCH_REGS)
-            attr_status = REGEN_ERR_UNSUPPORTED;
-    });
+    static PerContext<int> ready;
+    const int attr_status = ready.get([](int *) {
+        return kernel_setup(reinterpret_cast<const void *>(regen::proj_gemm_kernel<MODE>), C::SMEM_BYTES,
+                            C::MIN_LAUNCH_REGS);
+    }, nullptr);
     if (attr_status != REGEN_OK) return attr_status;
     const int64_t total = static_cast<int64_t>(shape.num_mt) * shape.num_nt;   // pair tiles
     const int sms = num_sms();
@@ -258,17 +305,11 @@ int launch_attn_fp8(const uint8_t *q8, const float *qs, const uint8_t *k8, const
                     cudaStream_t stream)
 {
     using C = regen::Fp8Cfg;
-    static std::once_flag once;
-    static int attr_status = REGEN_OK;
-    std::call_once(once, [] {
-        cudaFuncAttributes fa;
-        if (cudaFuncSetAttribute(regen::attn_fwd_fp8_kernel<NEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncGetAttributes(&fa, regen::attn_fwd_fp8_kernel<NEG>) != cudaSuccess)
-            attr_status = REGEN_ERR_CUDA;
-        else if (fa.numRegs < C::MIN_LAUNCH_REGS)
-            attr_status = REGEN_ERR_UNSUPPORTED;
-    });
+    static PerContext<int> ready;
+    const int attr_status = ready.get([](int *) {
+        return kernel_setup(reinterpret_cast<const void *>(regen::attn_fwd_fp8_kernel<NEG>), C::SMEM_BYTES,
+                            C::MIN_LAUNCH_REGS);
+    }, nullptr);
     if (attr_status != REGEN_OK) return attr_status;
     CUtensorMap tq, tk, tv, to;
     if (!make_u8_map(&tq, q8, BH, Sq) || !make_u8_map(&tk, k8, BH, Skv) || !make_u8_map(&tv, v8, BH, Skv) ||
@@ -288,18 +329,11 @@ int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, r
                 const double *rope_tab = nullptr, regen::RopeGeom geom = regen::RopeGeom{})
 {
     using C = regen::AttnCfg<HD>;
-    static std::once_flag once;
-    static int attr_status = REGEN_OK;
-    std::call_once(once, [] {
-        cudaFuncAttributes fa;
-        if (cudaFuncSetAttribute(regen::attn_fwd_kernel<HD, NEG, ROPE_Q>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncGetAttributes(&fa, regen::attn_fwd_kernel<HD, NEG, ROPE_Q>) != cudaSuccess)
-            attr_status = REGEN_ERR_CUDA;
-        else if (fa.numRegs < C::MIN_LAUNCH_REGS)
-            // the in-kernel register re-allocation would not fit: refuse to launch
-            attr_status = REGEN_ERR_UNSUPPORTED;
-    });
+    static PerContext<int> ready;
+    const int attr_status = ready.get([](int *) {
+        return kernel_setup(reinterpret_cast<const void *>(regen::attn_fwd_kernel<HD, NEG, ROPE_Q>), C::SMEM_BYTES,
+                            C::MIN_LAUNCH_REGS);
+    }, nullptr);
     if (attr_status != REGEN_OK) return attr_status;
     CUtensorMap tq, tk, tv, to;
     if (!make_bhsd_map(&tq, q, BH, Sq, HD) || !make_bhsd_map(&tk, k, BH, Skv, HD) ||
@@ -335,27 +369,21 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
                cudaStream_t stream)
 {
     using C = regen::BwdCfg<HD>;
-    static std::once_flag once;
-    static int attr_status = REGEN_OK;
-    std::call_once(once, [] {
-        auto setup = [](const void *fn, int smem) {
-            cudaFuncAttributes fa;
-            if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-                cudaFuncGetAttributes(&fa, fn) != cudaSuccess)
-                return static_cast<int>(REGEN_ERR_CUDA);
-            // the in-kernel register re-allocation would not fit: refuse to launch
-            return fa.numRegs < C::MIN_LAUNCH_REGS ? static_cast<int>(REGEN_ERR_UNSUPPORTED)
-                                                   : static_cast<int>(REGEN_OK);
-        };
-        int st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dkdv_kernel<HD, false>), C::A_SMEM_BYTES);
+    static PerContext<int> ready;
+    const int attr_status = ready.get([](int *) {
+        int st = kernel_setup(reinterpret_cast<const void *>(regen::attn_bwd_dkdv_kernel<HD, false>),
+                              C::A_SMEM_BYTES, C::MIN_LAUNCH_REGS);
         if (st == REGEN_OK)
-            st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dkdv_kernel<HD, true>), C::A_SMEM_BYTES);
+            st = kernel_setup(reinterpret_cast<const void *>(regen::attn_bwd_dkdv_kernel<HD, true>),
+                              C::A_SMEM_BYTES, C::MIN_LAUNCH_REGS);
         if (st == REGEN_OK)
-            st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, false>), C::B_SMEM_BYTES);
+            st = kernel_setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, false>),
+                              C::B_SMEM_BYTES, C::MIN_LAUNCH_REGS);
         if (st == REGEN_OK)
-            st = setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, true>), C::B_SMEM_BYTES);
-        attr_status = st;
-    });
+            st = kernel_setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, true>),
+                              C::B_SMEM_BYTES, C::MIN_LAUNCH_REGS);
+        return st;
+    }, nullptr);
     if (attr_status != REGEN_OK) return attr_status;
     CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
     if (!make_bhsd_map(&tq, q, BH, Sq, HD) || !make_bhsd_map(&tk, k, BH, Skv, HD) ||
@@ -429,27 +457,36 @@ int attn_rope3d_with_scratch(const regen_bf16 *q, const regen_bf16 *k, const reg
 // The array belongs to this library: every device that loads the library
 // holds it until the process exits. In host code `g_noalloc_scratch` names
 // only a host-side stand-in; the device address comes from
-// cudaGetSymbolAddress, resolved once per device (with that device current)
-// on the first call made on that device, and cached.
+// cudaGetSymbolAddress, looked up in the current context on the first call
+// made in that context (the array has one copy per context that loads the
+// module) and cached per context.
 constexpr int64_t kNoAllocScratchBytes = REGEN_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-uint8_t *g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the fixed scratch on the current device (nullptr on error).
-uint8_t *noalloc_scratch_on_current_device()
+// Device address of the fixed scratch in the current context. REGEN_ERR_INVALID_ARG
+// when the address is not known yet and `st` is capturing a graph: the lookup
+// may load the module, which a capture does not allow, so the first call in a
+// context must come before any capture.
+int noalloc_scratch_in_current_context(cudaStream_t st, uint8_t **scratch)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
-        g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
-    }
-    return g_noalloc_ptr[dev];
+    static PerContext<uint8_t *> addr;
+    return addr.get([st](uint8_t **p) {
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        const cudaError_t qe = cudaStreamIsCapturing(st, &cap);
+        if (qe != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_status(qe);
+        }
+        if (cap != cudaStreamCaptureStatusNone) return static_cast<int>(REGEN_ERR_INVALID_ARG);
+        void *a = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
+        if (e != cudaSuccess || a == nullptr) {
+            cudaGetLastError();
+            return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+        }
+        *p = static_cast<uint8_t *>(a);
+        return static_cast<int>(REGEN_OK);
+    }, scratch);
 }
 
 // S_local < 0: the whole grid (n0 = 0, S = T*Hh*Ww).
@@ -596,13 +633,16 @@ REGEN_API int regen_attn_fwd_rope3d_noalloc(const regen_bf16 *q, const regen_bf1
     if (overlaps(lse, lbytes, out, tbytes)) return REGEN_ERR_INVALID_ARG;
     const DeviceScope device(out);
     if (device.status != REGEN_OK) return device.status;
-    uint8_t *scratch = noalloc_scratch_on_current_device();
-    if (!scratch) return REGEN_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *scratch = nullptr;
+    const int found = noalloc_scratch_in_current_context(st, &scratch);
+    if (found != REGEN_OK) return found;
     // Every scratch byte this call reads is written earlier in the same call
     // (table, then rotated K), so nothing left by a previous call matters.
-    return attn_rope3d_with_scratch(q, k, v, out, lse, BH, static_cast<int>(S), D, scale, theta, geom, scratch,
-                                    reinterpret_cast<cudaStream_t>(stream));
+    return attn_rope3d_with_scratch(q, k, v, out, lse, BH, static_cast<int>(S), D, scale, theta, geom, scratch, st);
 }
+
+REGEN_API int64_t regen_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 
 REGEN_API int regen_rope3d(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float theta, int B,
@@ -898,7 +938,7 @@ REGEN_API int regen_last_cuda_error(const char **name)
         if (e == 0) {
             *name = "none";
         } else if (e >= kDriverErrorBase) {
-            *name = "tensor-map encoding failed (CUresult = code - 100000)";
+            *name = "a driver call failed: descriptor encoding or context query (CUresult = code - 100000)";
         } else {
             *name = cudaGetErrorName(static_cast<cudaError_t>(e));
         }

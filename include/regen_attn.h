@@ -125,15 +125,20 @@ REGEN_API int64_t regen_attn_fwd_rope3d_workspace_bytes(int B, int H, int T, int
  *    regen_attn_fwd_rope3d_workspace_bytes reports -- exceeds it is rejected
  *    with REGEN_ERR_UNSUPPORTED before anything is launched (that admits e.g.
  *    12 heads of 10920 tokens at D = 128, not 40 heads of 31200).
- *  - Set-up: the first call made on a device, with that device current, looks
- *    up the array's device address (cudaGetSymbolAddress) and caches it;
- *    make that first call before any stream capture on that device.
+ *  - Set-up: the first call made in a CUDA context (the one current when the
+ *    call binds the data's device: normally that device's primary context)
+ *    looks up the array's device address there (cudaGetSymbolAddress) and
+ *    caches it for that context. Make that first call before any stream
+ *    capture: a first call whose stream is capturing is refused with
+ *    REGEN_ERR_INVALID_ARG, since the lookup may load the module.
  *  - Sharing: all calls use the same array, which keeps whatever the last
  *    call left in it. Nothing there needs clearing, since each call writes
  *    every byte it later reads. Calls whose work overlaps on the GPU (for
  *    example on two unordered streams) race on the array: order them.
  */
 #define REGEN_NOALLOC_SCRATCH_BYTES (64LL << 20)
+/* Size in bytes of that fixed array, as built into this library. */
+REGEN_API int64_t regen_noalloc_scratch_bytes(void);
 REGEN_API int regen_attn_fwd_rope3d_noalloc(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v,
                                             regen_bf16 *out, float *lse,
                                             int B, int H, int Sq, int Skv, int D, float scale,
@@ -344,8 +349,9 @@ REGEN_API const char *regen_status_str(int status);
 /*
  * regen_last_cuda_error -- the CUDA result behind the last REGEN_ERR_CUDA that
  * a call on THIS host thread returned: a cudaError_t (its name in *name when
- * name is not NULL), or 100000 + a driver CUresult when a TMA descriptor could
- * not be encoded; 0 (name "none") when there is none. Reading clears it.
+ * name is not NULL), or 100000 + a driver CUresult when a driver call failed
+ * (a TMA descriptor could not be encoded, or the current context could not be
+ * queried); 0 (name "none") when there is none. Reading clears it.
  * The string is static; the caller does not free it.
  */
 REGEN_API int regen_last_cuda_error(const char **name);

@@ -234,3 +234,50 @@ def test_rope3d_shard_validation(lib, args, status):
     rc = lib.regen_rope3d_shard(a["q"], a["k"], a["T"], a["Hh"], a["Ww"], a["theta"], a["B"], a["H"], a["D"], a["n0"],
                                 a["S"], a["inv"], None)
     assert rc == status
+
+
+def test_noalloc_scratch_size_matches_header(lib):
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+REGEN_NOALLOC_SCRATCH_BYTES\s+\((\d+)LL\s*<<\s*(\d+)\)", text)
+    assert m, "REGEN_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert rg.regen_noalloc_scratch_bytes() == int(m.group(1)) << int(m.group(2))
+
+
+CTX_CACHE_TEST = r"""
+#include <cstdio>
+#include "ctx_cache.h"
+int main() {
+    regen::CtxCache<int, -4> cache;
+    int calls = 0, v = 0;
+    auto setup = [&](int value, int status) {
+        return [&calls, value, status](int *out) { ++calls; *out = value; return status; };
+    };
+    // context 7: set up once, then served from the cache
+    if (cache.get(7, setup(70, 0), &v) != 0 || v != 70 || calls != 1) return 1;
+    if (cache.get(7, setup(71, 0), &v) != 0 || v != 70 || calls != 1) return 2;
+    // a second context (another GPU, or a context the host created) gets its own set-up
+    if (cache.get(9, setup(90, 0), &v) != 0 || v != 90 || calls != 2) return 3;
+    if (cache.get(7, setup(72, 0), &v) != 0 || v != 70 || calls != 2) return 4;
+    // a failing CUDA call (-4) is not cached: the next call retries
+    if (cache.get(11, setup(0, -4), &v) != -4 || calls != 3) return 5;
+    if (cache.get(11, setup(110, 0), &v) != 0 || v != 110 || calls != 4) return 6;
+    // a refusal that a retry cannot change (-2) is cached like a success
+    if (cache.get(13, setup(0, -2), &v) != -2 || calls != 5) return 7;
+    if (cache.get(13, setup(130, 0), &v) != -2 || calls != 5) return 8;
+    std::puts("ok");
+    return 0;
+}
+"""
+
+
+def test_per_context_setup_cache(tmp_path):
+    """Kernel attributes and the fixed scratch's address are set up per CUDA
+    context: each context runs the set-up once, failures of the CUDA call
+    itself are retried, refusals are kept."""
+    src = tmp_path / "ctx_cache_test.cpp"
+    src.write_text(CTX_CACHE_TEST)
+    exe = tmp_path / "ctx_cache_test"
+    subprocess.run(["g++", "-std=c++17", "-O1", "-I", os.path.join(ROOT, "dit_attention_b200", "csrc"),
+                    str(src), "-o", str(exe), "-pthread"], check=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert res.returncode == 0 and res.stdout.strip() == "ok", (res.returncode, res.stdout)

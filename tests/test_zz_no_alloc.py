@@ -60,10 +60,32 @@ def test_no_alloc_matches_workspace_entry_on_two_calls_in_a_row():
     assert rg.regen_last_device_error() == (0, 0)
 
 
+def test_no_alloc_call_leaves_device_memory_unchanged():
+    # After a first call in this context (which may load the module and looks
+    # up the array's address), a call takes no device memory: the device's
+    # free bytes are the same before and after it.
+    w25 = synth.WORKLOADS["win25_s10920"]
+    q, k, v = synth.make_inputs(w25)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    out, lse = _no_alloc(dq, dk, dv, w25.grid, w25.theta)       # first call: set-up
+    out2 = torch.empty_like(out)
+    lse2 = torch.empty_like(lse)
+    B, H, S, D = dq.shape
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    rg.regen_attn_fwd_rope3d_noalloc(dq, dk, dv, out2, lse2, B, H, S, S, D, 1.0 / math.sqrt(D), None,
+                                     *w25.grid, w25.theta)
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before
+    np.testing.assert_array_equal(to_bits(out2), to_bits(out))
+    assert rg.regen_last_device_error() == (0, 0)
+
+
 def test_no_alloc_rejects_problems_larger_than_its_scratch():
     # 40 heads of 31200 tokens need ~320 MB of rotated K: more than the 64 MiB array
     need = rg.regen_attn_fwd_rope3d_workspace_bytes(1, 40, 20, 30, 52, 128)
-    assert need > rg.NOALLOC_SCRATCH_BYTES
+    assert need > rg.regen_noalloc_scratch_bytes()
     fake = 0x7F0000000000
     with pytest.raises(rg.RegenError) as e:
         rg.regen_attn_fwd_rope3d_noalloc(fake, fake + (1 << 30), fake + (2 << 30), fake + (3 << 30),
