@@ -54,7 +54,7 @@ __all__ = [
     "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd", "regen_rope3d_shard", "regen_quant_e4m3",
     "regen_attn_fwd_fp8", "quant_e4m3", "attn_fwd_fp8", "regen_qkv_proj", "regen_qkv_proj_workspace_bytes",
     "regen_out_proj", "qkv_proj", "out_proj",
-    "attn_fwd", "attn_fwd_rope3d", "rope3d_", "lse_merge", "attn_bwd", "rope3d_bwd_", "STATUS",
+    "attn_fwd", "attn_fwd_kv2", "regen_attn_fwd_kv2", "attn_fwd_rope3d", "rope3d_", "lse_merge", "attn_bwd", "rope3d_bwd_", "STATUS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -94,6 +94,8 @@ def load():
         vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
         L.regen_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp]
         L.regen_attn_fwd.restype = i32
+        L.regen_attn_fwd_kv2.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
+        L.regen_attn_fwd_kv2.restype = i32
         L.regen_attn_fwd_rope3d.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp,
                                             i32, i32, i32, f32, vp, i64]
         L.regen_attn_fwd_rope3d.restype = i32
@@ -181,6 +183,12 @@ def _check(rc: int, what: str) -> None:
 def regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream=None) -> None:
     _check(load().regen_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D,
                                  float(scale), _stream(stream)), "regen_attn_fwd")
+
+
+def regen_attn_fwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, B, H, Sq, Skv_a, Skv_b, D, scale, stream=None) -> None:
+    _check(load().regen_attn_fwd_kv2(_ptr(q), _ptr(k_a), _ptr(v_a), _ptr(k_b), _ptr(v_b), _ptr(out), _ptr(lse),
+                                     B, H, Sq, Skv_a, Skv_b, D, float(scale), _stream(stream)),
+           "regen_attn_fwd_kv2")
 
 
 def regen_attn_fwd_rope3d(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream, T, Hh, Ww, theta,
@@ -337,6 +345,22 @@ def attn_fwd(q, k, v, scale=None, out=None, lse=None, stream=None):
     if lse is None:
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
     regen_attn_fwd(q, k, v, out, lse, B, H, Sq, Skv, D, scale, stream)
+    return out, lse
+
+
+def attn_fwd_kv2(q, k_a, v_a, k_b, v_b, scale=None, out=None, lse=None, stream=None):
+    """Attention of q over two key/value sources as one softmax over their
+    concatenation [k_a; k_b] -> (out bf16, lse fp32)."""
+    import torch
+    B, H, Sq, D = _bhsd(q, "q")
+    Skv_a, Skv_b = _bhsd(k_a, "k_a")[2], _bhsd(k_b, "k_b")[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    regen_attn_fwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, B, H, Sq, Skv_a, Skv_b, D, scale, stream)
     return out, lse
 
 

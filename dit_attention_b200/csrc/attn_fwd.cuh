@@ -128,8 +128,8 @@ struct AttnCfg {
     static constexpr int V_OFF = K_OFF + NSK * TILE_BYTES;
     static constexpr int BAR_OFF = V_OFF + NSV * TILE_BYTES;
     // barriers: q, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[2], s_free,
-    // p_full[2], pv_done[2], drain, q_rotated
-    static constexpr int NBARS = 1 + 2 * NSK + 2 * NSV + 7 + 1 + 1;
+    // p_full[2], pv_done[2], drain, q_rotated[2]
+    static constexpr int NBARS = 1 + 2 * NSK + 2 * NSV + 7 + 1 + 2;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;  // abort flag, TMEM base
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -144,18 +144,28 @@ struct AttnCfg {
     static constexpr int EMU_PER8 = REGEN_FWD_EXP2_EMU_PER8;
 };
 
-// ROPE_Q: the Q tiles are rotated by the 3D RoPE in shared memory right after
+// RoPE (rope_tab.t32 not null, single key source): the Q tiles are rotated by
+// the 3D RoPE in shared memory right after
 // their TMA load (each softmax thread rotates its own row, from the (cos, sin)
-// table `rope_tab`), before the first S MMA reads them; the rotation is the
-// same fp64 arithmetic and rounding as rope3d_kernel, so the result equals
-// rotating Q in HBM first.
-template <int HD, bool NEG_SCALE, bool ROPE_Q>
+// table `rope_tab`), before the first S MMA of that tile reads them; the
+// rotation gives the same bits as rope_stream_kernel (fp32 with a per-pair
+// certificate, else fp64), so the result equals rotating Q in HBM first.
+// KV2: the keys come from two sources, tm_k/tm_v (the first Skv1 keys) and
+// tm_k2/tm_v2 (the other Skv - Skv1), under one online softmax: the result is
+// the attention over the two sources concatenated. The blocks of source 1 come
+// first, then those of source 2; each source's last block is masked past its
+// own end. (Other instantiations ignore tm_k2, tm_v2 and Skv1.)
+// The RoPE choice is a run-time flag, not a template parameter, so that the
+// plain and the RoPE-fused attention run the same compiled main loop.
+template <int HD, bool NEG_SCALE, bool KV2 = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                    float *__restrict__ lse, int Sq, int Skv, float scale_log2,
-                    uint64_t wait_limit_ns, const double *__restrict__ rope_tab, RopeGeom rope_geom)
+                    const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_v2,
+                    float *__restrict__ lse, int Sq, int Skv, int Skv1, float scale_log2,
+                    uint64_t wait_limit_ns, RopeTabs rope_tab, RopeGeom rope_geom)
 {
+    const bool rope_q = !KV2 && rope_tab.t32 != nullptr;
     using C = AttnCfg<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -176,7 +186,7 @@ __global__ void __launch_bounds__(384, 1)
     auto bar_p_full = [&](int t) { return bar0 + 8u * (4 + NB + t); };
     auto bar_pv_done = [&](int t) { return bar0 + 8u * (6 + NB + t); };
     const uint32_t bar_drain = bar0 + 8u * (8 + NB);
-    const uint32_t bar_qrot = bar0 + 8u * (9 + NB);  // Q tiles rotated (ROPE_Q)
+    auto bar_qrot = [&](int t) { return bar0 + 8u * (9 + NB + t); };  // Q tile t rotated (rope_q)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 8);
 
@@ -197,7 +207,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(bar_s_free, 128);
         mbar_init(bar_drain, 2);
-        mbar_init(bar_qrot, 256);
+        mbar_init(bar_qrot(0), 128);
+        mbar_init(bar_qrot(1), 128);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -211,7 +222,19 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tmem = *tmem_slot;
 
     const WaitCtl wc{abort_flag, wait_limit_ns};
-    const int nkv = (Skv + C::BN - 1) / C::BN;
+    // key blocks: source 1's, then (KV2) source 2's
+    const int nkv1 = KV2 ? (Skv1 + C::BN - 1) / C::BN : 0;
+    const int nkv = KV2 ? nkv1 + (Skv - Skv1 + C::BN - 1) / C::BN : (Skv + C::BN - 1) / C::BN;
+    // the map and first key row of key block j
+    auto kv_src = [&](int j, const CUtensorMap *m1, const CUtensorMap *m2, const CUtensorMap *&m, int &row) {
+        if (KV2 && j >= nkv1) {
+            m = m2;
+            row = (j - nkv1) * C::BN;
+        } else {
+            m = m1;
+            row = j * C::BN;
+        }
+    };
     // 1-D grid, query-tile pairs of one head adjacent so that the CTAs resident
     // at any time share the K/V of one or two heads in L2.
     const int npairs = (Sq + 2 * C::BM - 1) / (2 * C::BM);
@@ -256,6 +279,7 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
+            if (KV2) tma_prefetch_desc(&tm_k2);
             const uint64_t keep = l2_policy_evict_last();   // K: re-read by every Q tile of the head
             const uint64_t once = l2_policy_evict_first();  // Q: read once
             mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
@@ -269,10 +293,13 @@ __global__ void __launch_bounds__(384, 1)
                 const int s = j % C::NSK;
                 ok = wait_phase(bar_k_empty(s), ((j / C::NSK) & 1) ^ 1, SITE_PROD_K_EMPTY, wc);
                 if (!ok) break;
+                const CUtensorMap *mk;
+                int krow;
+                kv_src(j, &tm_k, &tm_k2, mk, krow);
                 mbar_arrive_expect_tx(bar_k_full(s), C::TILE_BYTES);
                 for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_3d(sbase + C::K_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_k,
-                                bar_k_full(s), h * 64, j * C::BN, bh, keep);
+                    tma_load_3d(sbase + C::K_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, mk,
+                                bar_k_full(s), h * 64, krow, bh, keep);
                 ++nk;
             }
             if (!ok) {
@@ -285,6 +312,7 @@ __global__ void __launch_bounds__(384, 1)
         // ------------------------------------------------- producer: V ---
         if (lane == 0) {
             tma_prefetch_desc(&tm_v);
+            if (KV2) tma_prefetch_desc(&tm_v2);
             const uint64_t keep = l2_policy_evict_last();   // V: re-read by every Q tile of the head
             int nv = 0;
             bool ok = true;
@@ -292,10 +320,13 @@ __global__ void __launch_bounds__(384, 1)
                 const int s = j % C::NSV;
                 ok = wait_phase(bar_v_empty(s), ((j / C::NSV) & 1) ^ 1, SITE_PROD_V_EMPTY, wc);
                 if (!ok) break;
+                const CUtensorMap *mv;
+                int vrow;
+                kv_src(j, &tm_v, &tm_v2, mv, vrow);
                 mbar_arrive_expect_tx(bar_v_full(s), C::TILE_BYTES);
                 for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_3d(sbase + C::V_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, &tm_v,
-                                bar_v_full(s), h * 64, j * C::BN, bh, keep);
+                    tma_load_3d(sbase + C::V_OFF + s * C::TILE_BYTES + h * C::HALF_BYTES, mv,
+                                bar_v_full(s), h * 64, vrow, bh, keep);
                 ++nv;
             }
             if (!ok)
@@ -323,7 +354,9 @@ __global__ void __launch_bounds__(384, 1)
                            smem_desc_sw128(kb + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
                 }
             };
-            bool ok = wait_phase(ROPE_Q ? bar_qrot : bar_q, 0, SITE_MMA_Q, wc);
+            // Q tile t is ready when its TMA load landed (rope_q: when its rows
+            // have been rotated); S_t(0) waits for that tile alone.
+            bool ok = rope_q ? true : wait_phase(bar_q, 0, SITE_MMA_Q, wc);
             for (int j = 0; j < nkv && ok; ++j) {
                 const int s = j % C::NSK;
                 ok = wait_phase(bar_k_full(s), (j / C::NSK) & 1, SITE_MMA_K_FULL, wc);
@@ -332,11 +365,19 @@ __global__ void __launch_bounds__(384, 1)
                     ok = wait_phase(bar_s_free, 1, SITE_MMA_S_FREE, wc);  // S1(j-1) copied out
                     if (!ok) break;
                 }
+                if (rope_q && j == 0) {
+                    ok = wait_phase(bar_qrot(0), 0, SITE_MMA_Q, wc);
+                    if (!ok) break;
+                }
                 tc_fence_after_sync();
                 issue_s(0, s);
                 tc_commit(bar_s_full(0));
                 ok = wait_phase(bar_s_free, 0, SITE_MMA_S_FREE, wc);      // S0(j) copied out
                 if (!ok) break;
+                if (rope_q && j == 0) {
+                    ok = wait_phase(bar_qrot(1), 0, SITE_MMA_Q, wc);
+                    if (!ok) break;
+                }
                 tc_fence_after_sync();
                 issue_s(1, s);
                 tc_commit(bar_s_full(1));
@@ -400,26 +441,49 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t ts = tmem + lane_bits;                 // the shared S buffer
         const uint32_t tp = tmem + lane_bits + 128u + t * 64u;  // this tile's P
         const uint32_t to = tmem + lane_bits + 256u + t * HD;
-        const int kv_tail = Skv - (nkv - 1) * C::BN;  // valid keys in the last block (1..128)
+        // valid keys of block j (1..128): fewer only in the last block of a source
+        auto valid_keys = [&](int j) -> int {
+            if constexpr (KV2) {
+                if (j == nkv1 - 1) return Skv1 - (nkv1 - 1) * C::BN;
+                if (j == nkv - 1) return Skv - Skv1 - (nkv - 1 - nkv1) * C::BN;
+                return C::BN;
+            } else {
+                return j == nkv - 1 ? Skv - (nkv - 1) * C::BN : C::BN;
+            }
+        };
         float m = 0.f;   // running max of scaled logits (log2 units); set by block 0
         float l = 0.f;   // running sum of 2^(s - m)
         bool ok = true;
-        if constexpr (ROPE_Q) {
+        if (rope_q) {
             // Rotate this thread's row of its Q tile in place in shared memory
             // (128-byte swizzled rows: 16-byte chunk cw of row r sits at chunk
-            // cw ^ (r & 7)), then hand the tile to the MMA issuer.
-            ok = __all_sync(0xffffffffu, wait_phase(bar_q, 0, SITE_SM_Q, wc));
+            // cw ^ (r & 7)), then hand the tile to the S issuer. The row's 64
+            // fp32 (cos, sin) pairs depend only on its token, so they are
+            // loaded while the Q tile is still on its way from HBM.
+            constexpr int DH = 2 * (HD / 6), DT = HD - 2 * DH;   // axis widths t, h, w = DT, DH, DH
+            constexpr int NP = HD / 2;                           // pairs per row
             const int n = q0 + t * C::BM + row;
-            if (ok && n < Sq) {
+            const bool live = n < Sq;
+            const RopeRowEntries re = RopeRowEntries::of(rope_geom, live ? n : 0);
+            float2 cs[NP];
+#pragma unroll
+            for (int p = 0; p < NP; ++p) cs[p] = __ldg(rope_tab.t32 + re.entry(2 * p, DT, DH));
+            ok = __all_sync(0xffffffffu, wait_phase(bar_q, 0, SITE_SM_Q, wc));
+            if (ok && live) {
                 uint8_t *rowp = smem + C::Q_OFF + t * C::TILE_BYTES + row * 128;
-#pragma unroll 4
+#pragma unroll
                 for (int c = 0; c < HD / 8; ++c) {
-                    uint4 *p = reinterpret_cast<uint4 *>(rowp + (c >> 3) * C::HALF_BYTES + (((c & 7) ^ (row & 7)) << 4));
-                    *p = rotate_chunk(*p, c, n, rope_geom, rope_tab);
+                    uint4 *ptr = reinterpret_cast<uint4 *>(rowp + (c >> 3) * C::HALF_BYTES + (((c & 7) ^ (row & 7)) << 4));
+                    const uint4 v = *ptr;
+                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p)
+                        w[p] = rotate_pair_tab(w[p], cs[4 * c + p], rope_tab.t64, re.entry(8 * c + 2 * p, DT, DH));
+                    *ptr = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(bar_qrot);
+            mbar_arrive(bar_qrot(t));
         }
         for (int j = 0; ok && j < nkv; ++j) {
             // every lane waits; the outcome is made warp-uniform so that the
@@ -436,9 +500,10 @@ __global__ void __launch_bounds__(384, 1)
             // S is in registers: the buffer may take the other tile's next S.
             tc_fence_before_sync();
             mbar_arrive(bar_s_free);
-            // One block of the online softmax. MASKED: the last block, whose
-            // columns >= kv_tail lie past Skv (their logits are zero-filled
-            // loads) and get probability 0.
+            // One block of the online softmax. MASKED: the last block of a key
+            // source, whose columns >= kv_tail lie past that source's end (their
+            // logits are zero-filled loads) and get probability 0.
+            const int kv_tail = valid_keys(j);
             bool grow = false;
             float alpha = 1.0f;
             auto block = [&](auto masked_tag) {
@@ -519,7 +584,7 @@ __global__ void __launch_bounds__(384, 1)
                 (void)r3;
                 l += r0 + r1;
             };
-            if (j == nkv - 1 && kv_tail < C::BN)
+            if (kv_tail < C::BN)
                 block(std::true_type{});
             else
                 block(std::false_type{});

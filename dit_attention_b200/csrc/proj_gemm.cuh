@@ -80,25 +80,25 @@ __device__ __forceinline__ void proj_tile(int t, const ProjShape &p, int &mt, in
 }
 
 // (cos, sin) in fp32 of every RoPE table entry (RopeGeom layout), from fp64.
-__global__ void rope_table_f32_kernel(float2 *__restrict__ tab, RopeGeom g, double theta)
+__global__ void rope_table_f32_kernel(float2 *__restrict__ tab, RopeGeom g, const __grid_constant__ RopeFreqs fr)
 {
     const int64_t n = g.entries();
     const int64_t base_h = static_cast<int64_t>(g.T) * (g.dt / 2);
     const int64_t base_w = base_h + static_cast<int64_t>(g.Hh) * (g.dh / 2);
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n; e += stride) {
-        int pos, j, width;
+        int pos, pair;   // pair: index of the pair within the head dimension
         if (e < base_h) {
-            pos = static_cast<int>(e / (g.dt / 2)); j = static_cast<int>(e % (g.dt / 2)); width = g.dt;
+            pos = static_cast<int>(e / (g.dt / 2)); pair = static_cast<int>(e % (g.dt / 2));
         } else if (e < base_w) {
-            pos = static_cast<int>((e - base_h) / (g.dh / 2)); j = static_cast<int>((e - base_h) % (g.dh / 2));
-            width = g.dh;
+            pos = static_cast<int>((e - base_h) / (g.dh / 2));
+            pair = g.dt / 2 + static_cast<int>((e - base_h) % (g.dh / 2));
         } else {
-            pos = static_cast<int>((e - base_w) / (g.dh / 2)); j = static_cast<int>((e - base_w) % (g.dh / 2));
-            width = g.dh;
+            pos = static_cast<int>((e - base_w) / (g.dh / 2));
+            pair = (g.dt + g.dh) / 2 + static_cast<int>((e - base_w) % (g.dh / 2));
         }
         double c, s;
-        rope_angle(pos, 2 * j, width, theta, c, s);
+        rope_angle(pos, fr.f[pair], c, s);
         tab[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
     }
 }

@@ -323,28 +323,41 @@ int launch_attn_fp8(const uint8_t *q8, const float *qs, const uint8_t *k8, const
     return launched();
 }
 
-template <int HD, bool NEG, bool ROPE_Q = false>
+// Skv keys in k, v; with KV2 the first Skv1 of them in k, v and the other
+// Skv - Skv1 in k2, v2 (one softmax over both).
+template <int HD, bool NEG, bool ROPE_Q = false, bool KV2 = false>
 int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, regen_bf16 *out,
                 float *lse, int64_t BH, int Sq, int Skv, float scale, cudaStream_t stream,
-                const double *rope_tab = nullptr, regen::RopeGeom geom = regen::RopeGeom{})
+                regen::RopeTabs rope_tab = regen::RopeTabs{}, regen::RopeGeom geom = regen::RopeGeom{},
+                const regen_bf16 *k2 = nullptr, const regen_bf16 *v2 = nullptr, int Skv1 = 0)
 {
     using C = regen::AttnCfg<HD>;
     static PerContext<int> ready;
     const int attr_status = ready.get([](int *) {
-        return kernel_setup(reinterpret_cast<const void *>(regen::attn_fwd_kernel<HD, NEG, ROPE_Q>), C::SMEM_BYTES,
-                            C::MIN_LAUNCH_REGS);
+        return kernel_setup(reinterpret_cast<const void *>(regen::attn_fwd_kernel<HD, NEG, KV2>),
+                            C::SMEM_BYTES, C::MIN_LAUNCH_REGS);
     }, nullptr);
     if (attr_status != REGEN_OK) return attr_status;
-    CUtensorMap tq, tk, tv, to;
-    if (!make_bhsd_map(&tq, q, BH, Sq, HD) || !make_bhsd_map(&tk, k, BH, Skv, HD) ||
-        !make_bhsd_map(&tv, v, BH, Skv, HD) || !make_bhsd_map(&to, out, BH, Sq, HD))
+    CUtensorMap tq, tk, tv, to, tk2, tv2;
+    const int skv_a = KV2 ? Skv1 : Skv;
+    if (!make_bhsd_map(&tq, q, BH, Sq, HD) || !make_bhsd_map(&tk, k, BH, skv_a, HD) ||
+        !make_bhsd_map(&tv, v, BH, skv_a, HD) || !make_bhsd_map(&to, out, BH, Sq, HD))
         return REGEN_ERR_CUDA;
+    if (KV2) {
+        if (!make_bhsd_map(&tk2, k2, BH, Skv - Skv1, HD) || !make_bhsd_map(&tv2, v2, BH, Skv - Skv1, HD))
+            return REGEN_ERR_CUDA;
+    } else {
+        tk2 = tk;   // unused by this instantiation
+        tv2 = tv;
+    }
     const int64_t npairs = (Sq + 2 * C::BM - 1) / (2 * C::BM);
     const int64_t grid = npairs * BH;
     if (grid > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
     const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    regen::attn_fwd_kernel<HD, NEG, ROPE_Q><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, to, lse, Sq, Skv, scale_log2, g_wait_limit_ns.load(), rope_tab, geom);
+    static_assert(!(ROPE_Q && KV2), "the RoPE-fused attention has one key source");
+    if (ROPE_Q != (rope_tab.t32 != nullptr)) return REGEN_ERR_INVALID_ARG;   // the kernel keys on the table
+    regen::attn_fwd_kernel<HD, NEG, KV2><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, to, tk2, tv2, lse, Sq, Skv, Skv1, scale_log2, g_wait_limit_ns.load(), rope_tab, geom);
     return launched();
 }
 
@@ -420,13 +433,55 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
 
 int64_t bwd_workspace_bytes(int64_t BH, int64_t Sq) { return BH * ((Sq + 127) / 128) * 1024; }
 
-// Scratch of the RoPE-fused attention: the fp64 (cos, sin) table, then the
-// rotated K ([B*H, S, D] bf16), each starting on a 256-byte boundary.
-int64_t rope_table_bytes(const regen::RopeGeom &g) { return (g.entries() * 16 + 255) / 256 * 256; }
+// Scratch of the RoPE-fused attention: the fp64 (cos, sin) table, its fp32
+// copy, then the rotated K ([B*H, S, D] bf16), each starting on a 256-byte boundary.
+int64_t rope_tab64_bytes(const regen::RopeGeom &g) { return (g.entries() * 16 + 255) / 256 * 256; }
+int64_t rope_table_bytes(const regen::RopeGeom &g)
+{
+    return rope_tab64_bytes(g) + (g.entries() * 8 + 255) / 256 * 256;
+}
 
 int64_t rope_workspace_bytes(int64_t BH, int64_t S, const regen::RopeGeom &g, int D)
 {
     return rope_table_bytes(g) + BH * S * D * 2;
+}
+
+// theta^(-local/width) for every pair of head dimension D (<= 512), in the
+// RoPE's axis blocks t, h, w of widths D - 4*floor(D/6), 2*floor(D/6), 2*floor(D/6).
+regen::RopeFreqs make_rope_freqs(int D, float theta)
+{
+    regen::RopeFreqs fr{};
+    const int dh = 2 * (D / 6), dt = D - 2 * dh;
+    for (int d = 0; d + 1 < D && d / 2 < 256; d += 2) {
+        int local, width;
+        if (d < dt) {
+            local = d; width = dt;
+        } else if (d < dt + dh) {
+            local = d - dt; width = dh;
+        } else {
+            local = d - dt - dh; width = dh;
+        }
+        fr.f[d / 2] = std::pow(static_cast<double>(theta), -static_cast<double>(local) / static_cast<double>(width));
+    }
+    return fr;
+}
+
+// Rows per thread of a RoPE kernel whose grid has `blocks_x` blocks per row
+// group: the fewest groups (each thread's angles serve the most rows) that
+// still give about one wave of 128-thread blocks on a 148-SM part, and at
+// least 4 rows per group (one load batch). Returns the rows per group;
+// *groups receives the number of groups.
+int rope_rows_per_group(int64_t blocks_x, int64_t rows, int64_t *groups)
+{
+    const int64_t target = 148LL * 8;
+    int64_t g = (target + blocks_x - 1) / blocks_x;
+    const int64_t gmax = (rows + 3) / 4;
+    if (g > gmax) g = gmax;
+    if (g > 32767) g = 32767;
+    if (g < 1) g = 1;
+    const int64_t per = (rows + g - 1) / g;
+    *groups = (rows + per - 1) / per;
+    return static_cast<int>(per);
 }
 
 // Table -> rotated K -> attention with Q rotated in shared memory; every
@@ -436,13 +491,19 @@ int attn_rope3d_with_scratch(const regen_bf16 *q, const regen_bf16 *k, const reg
                              float *lse, int64_t BH, int S, int D, float scale, float theta,
                              const regen::RopeGeom &geom, uint8_t *scratch, cudaStream_t st)
 {
-    double *tab = reinterpret_cast<double *>(scratch);
+    double *tab64 = reinterpret_cast<double *>(scratch);
+    float2 *tab32 = reinterpret_cast<float2 *>(scratch + rope_tab64_bytes(geom));
+    const regen::RopeTabs tab{tab64, tab32};
     regen_bf16 *k_rot = reinterpret_cast<regen_bf16 *>(scratch + rope_table_bytes(geom));
-    regen::rope_table_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
+    regen::rope_table_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab64, tab32, geom,
+                                                                           make_rope_freqs(D, theta));
     if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
-    const int64_t chunks = static_cast<int64_t>(S) * (D / 8);  // one thread per (token, chunk), all rows
-    regen::rope_apply_kernel<<<grid_for(chunks, 128), 128, 0, st>>>(
-        reinterpret_cast<const uint4 *>(k), reinterpret_cast<uint4 *>(k_rot), BH, S, D, geom, tab);
+    const int64_t chunks = static_cast<int64_t>(S) * (D / 8);  // one thread per (token, chunk) and row group
+    const int64_t bx = (chunks + 127) / 128;
+    int64_t groups = 1;
+    const int per = rope_rows_per_group(bx, BH, &groups);
+    regen::rope_apply_kernel<<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(groups)), 128, 0, st>>>(
+        k, k_rot, BH, S, D, geom, tab, per);
     if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     const bool neg = scale < 0.0f;
     if (D == 128)
@@ -511,10 +572,14 @@ int rope3d_common(regen_bf16 *q, regen_bf16 *k, int T, int Hh, int Ww, float the
     const int threads = 128;
     const int64_t blocks = (work + threads - 1) / threads;
     if (blocks > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    int64_t groups = 1;   // row groups per tensor (q, then k: blockIdx.y)
+    const int per = rope_rows_per_group((q && k) ? 2 * blocks : blocks, BH, &groups);
     const DeviceScope device(q ? q : k);
     if (device.status != REGEN_OK) return device.status;
-    regen::rope3d_kernel<<<static_cast<unsigned>(blocks), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        q, k, BH, static_cast<int>(S), Hh, Ww, D, static_cast<double>(theta), inverse, S_local >= 0 ? n0 : 0);
+    const dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(2 * groups));
+    regen::rope3d_kernel<<<grid, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<uint16_t *>(q), reinterpret_cast<uint16_t *>(k), BH, static_cast<int>(S), Hh, Ww, D,
+        make_rope_freqs(D, theta), inverse, S_local >= 0 ? n0 : 0, per, static_cast<int>(groups));
     return launched();
 }
 
@@ -557,6 +622,49 @@ REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const reg
                    : launch_attn<128, false>(q, k, v, out, lse, BH, Sq, Skv, scale, st);
     return neg ? launch_attn<64, true>(q, k, v, out, lse, BH, Sq, Skv, scale, st)
                : launch_attn<64, false>(q, k, v, out, lse, BH, Sq, Skv, scale, st);
+}
+
+REGEN_API int regen_attn_fwd_kv2(const regen_bf16 *q, const regen_bf16 *k_a, const regen_bf16 *v_a,
+                                 const regen_bf16 *k_b, const regen_bf16 *v_b, regen_bf16 *out, float *lse, int B,
+                                 int H, int Sq, int Skv_a, int Skv_b, int D, float scale, regen_stream_t stream)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Skv_a < 0 || Skv_b < 0 || D < 0) return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(Skv_a) + Skv_b > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    // one source empty: the plain attention over the other
+    if (Skv_b == 0) return regen_attn_fwd(q, k_a, v_a, out, lse, B, H, Sq, Skv_a, D, scale, stream);
+    if (Skv_a == 0) return regen_attn_fwd(q, k_b, v_b, out, lse, B, H, Sq, Skv_b, D, scale, stream);
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0 || Sq == 0) return REGEN_OK;
+    if (BH > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (!q || !out || !k_a || !v_a || !k_b || !v_b) return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || !aligned16(k_a) || !aligned16(v_a) ||
+        !aligned16(k_b) || !aligned16(v_b))
+        return REGEN_ERR_MISALIGNED;
+    const int64_t qbytes = BH * Sq * D * 2, abytes = BH * Skv_a * D * 2, bbytes = BH * Skv_b * D * 2,
+                  lbytes = BH * Sq * 4;
+    struct Span { const void *p; int64_t n; };
+    const Span ins[5] = {{q, qbytes}, {k_a, abytes}, {v_a, abytes}, {k_b, bbytes}, {v_b, bbytes}};
+    for (const Span &in : ins)
+        if (overlaps(out, qbytes, in.p, in.n) || overlaps(lse, lbytes, in.p, in.n)) return REGEN_ERR_INVALID_ARG;
+    if (overlaps(lse, lbytes, out, qbytes)) return REGEN_ERR_INVALID_ARG;
+    const DeviceScope device(out);
+    if (device.status != REGEN_OK) return device.status;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int Skv = Skv_a + Skv_b;
+    const bool neg = scale < 0.0f;
+    const regen::RopeTabs nt{};
+    const regen::RopeGeom ng{};
+    if (D == 128)
+        return neg ? launch_attn<128, true, false, true>(q, k_a, v_a, out, lse, BH, Sq, Skv, scale, st, nt, ng, k_b,
+                                                         v_b, Skv_a)
+                   : launch_attn<128, false, false, true>(q, k_a, v_a, out, lse, BH, Sq, Skv, scale, st, nt, ng,
+                                                          k_b, v_b, Skv_a);
+    return neg ? launch_attn<64, true, false, true>(q, k_a, v_a, out, lse, BH, Sq, Skv, scale, st, nt, ng, k_b, v_b,
+                                                    Skv_a)
+               : launch_attn<64, false, false, true>(q, k_a, v_a, out, lse, BH, Sq, Skv, scale, st, nt, ng, k_b, v_b,
+                                                     Skv_a);
 }
 
 REGEN_API int64_t regen_attn_fwd_rope3d_workspace_bytes(int B, int H, int T, int Hh, int Ww, int D)
@@ -872,7 +980,7 @@ REGEN_API int regen_qkv_proj(const regen_bf16 *x, const regen_bf16 *w, const flo
     if (device.status != REGEN_OK) return device.status;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float2 *tab = static_cast<float2 *>(workspace);
-    regen::rope_table_f32_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, static_cast<double>(theta));
+    regen::rope_table_f32_kernel<<<grid_for(geom.entries(), 128), 128, 0, st>>>(tab, geom, make_rope_freqs(D, theta));
     if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     CUtensorMap ta, tb;
     if (!make_bf16_map3(&ta, x, C, S, B, 64, 128) || !make_bf16_map3(&tb, w, C, N, 1, 64, 128)) return REGEN_ERR_CUDA;

@@ -1,4 +1,4 @@
-// rope3d.cuh -- 3D rotary position embedding of Q and K, in place (sm_100a).
+// rope3d.cuh -- 3D rotary position embedding of Q and K (sm_100a).
 //
 // The ReGenVC decoder's DiT matches the Wan2.1-Fun-Control architecture (blog
 // page, "Methodology -- deep read"), whose attention rotates Q and K by a 3D
@@ -7,16 +7,25 @@
 // D - 4*floor(D/6), 2*floor(D/6), 2*floor(D/6); pair (2j, 2j+1) of a block of
 // width d turns by pos * theta^(-2j/d).
 //
+// Result contract: the angle's cosine and sine in fp64, the rotation in fp64,
+// one rounding to bf16 (nearest even). The kernels reach that result with
+// fp32 arithmetic on the fp32 roundings of the fp64 cosine and sine, and prove
+// per element that the fp32 value rounds to the same bf16 as the fp64 one
+// (rotate_pair_f32); the few pairs it cannot prove (about one in a thousand,
+// near a bf16 rounding boundary) are redone in fp64 (rotate_pair).
+//
 // HBM-bound: every element is read and written once. One thread owns one
-// 16-byte chunk (4 pairs) of one token's row; it evaluates its 4 angles once
-// (fp64 sincos) and then walks the same chunk through every (batch, head) row
-// of Q and then of K, so the trigonometry is amortised over 2*B*H rows.
-// Adjacent threads own adjacent chunks of a row: each warp access is two
-// contiguous 256-byte rows. The rotation is done in fp64 and rounded once to
-// bf16 (one direct fp64 -> bf16 conversion, nearest-even).
+// 16-byte chunk (4 pairs) of one token's row and walks that chunk through
+// every row of Q (or of K): its 4 angles are evaluated once and stay in
+// registers in fp64 (for the rare fp64 redo) and fp32 (for the rotation), and
+// the next four rows' loads are in flight while it rotates and stores the
+// current four. Adjacent threads own adjacent chunks of a row: each warp
+// access is two contiguous 256-byte rows.
 #pragma once
 
 #include <stdint.h>
+
+#include "ptx.cuh"
 
 namespace regen {
 
@@ -49,11 +58,43 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t packed, double c, doubl
     return double_to_bf16_bits(y0) | (double_to_bf16_bits(y1) << 16);
 }
 
-// cos and sin of pos * theta^(-local/width) for the pair starting at
-// dimension `local` of an axis block of `width` dimensions (fp64).
-__device__ __forceinline__ void rope_angle(int pos, int local, int width, double theta, double &c, double &s)
+// The same pair rotated in fp32 from c32 = fp32(c) and s32 = fp32(s), with a
+// proof that it rounds like rotate_pair: returns true when both packed results
+// in `out` equal rotate_pair(packed, c, s), false when it cannot tell.
+// Bound: with X = |x0| + |x1|, the fp32 value differs from the fp64 one by at
+// most 3.0001 * 2^-24 * X + 2^-148 (the fp32 roundings of c and s, of the
+// product, of the fused result, and the fp64 path's own 2^-52 X; the last
+// term covers results among the fp32 subnormals). If no bf16 rounding
+// boundary -- the midpoint between two neighbouring bf16 values -- lies
+// within that distance of the fp32 value, both round to the same bf16. The
+// test uses 2^-21 X + 2^-146 (twice the bound, which also absorbs the
+// rounding of X itself), and the midpoint of the bf16 cell that holds y,
+// whose distance to y is exact in fp32 (same sign and binade). A NaN or
+// infinite value fails the test and goes to fp64.
+__device__ __forceinline__ bool rotate_pair_f32(uint32_t packed, float c32, float s32, uint32_t &out)
 {
-    const double freq = pow(theta, -static_cast<double>(local) / static_cast<double>(width));
+    const float x0 = __uint_as_float(packed << 16);
+    const float x1 = __uint_as_float(packed & 0xFFFF0000u);
+    const float y0 = __fmaf_rn(x0, c32, -__fmul_rn(x1, s32));
+    const float y1 = __fmaf_rn(x0, s32, __fmul_rn(x1, c32));
+    const float bound = __fmaf_rn(__fadd_rn(fabsf(x0), fabsf(x1)), 0x1p-21f, 0x1p-146f);
+    const float g0 = fabsf(__fsub_rn(y0, __uint_as_float((__float_as_uint(y0) & 0xFFFF0000u) | 0x8000u)));
+    const float g1 = fabsf(__fsub_rn(y1, __uint_as_float((__float_as_uint(y1) & 0xFFFF0000u) | 0x8000u)));
+    out = pack_bf16x2(y0, y1);
+    return g0 > bound && g1 > bound;
+}
+
+// Frequencies theta^(-local/width) of the pairs of a head dimension D <= 512,
+// indexed by pair (d/2 for the pair starting at dimension d): they depend on
+// D and theta only, so the host evaluates them once per call (fp64 pow) and
+// passes them by value.
+struct RopeFreqs {
+    double f[256];
+};
+
+// cos and sin of pos * freq (fp64).
+__device__ __forceinline__ void rope_angle(int pos, double freq, double &c, double &s)
+{
     sincos(static_cast<double>(pos) * freq, &s, &c);
 }
 
@@ -86,135 +127,183 @@ struct RopeGeom {
     }
 };
 
-// tab[2e], tab[2e+1] = cos, sin of every table entry e (grid-stride).
-__global__ void rope_table_kernel(double *__restrict__ tab, RopeGeom g, double theta)
+// Table entries of a token's three axis blocks: the pair starting at head
+// dimension d < dt has entry t0 + d/2, then h0 + (d - dt)/2, then w0 + (d - dt - dh)/2.
+struct RopeRowEntries {
+    int64_t t0, h0, w0;
+    __device__ __forceinline__ static RopeRowEntries of(const RopeGeom &g, int n)
+    {
+        RopeRowEntries r;
+        const int t = n / (g.Hh * g.Ww), y = (n / g.Ww) % g.Hh, x = n % g.Ww;
+        const int64_t base_h = static_cast<int64_t>(g.T) * (g.dt / 2);
+        const int64_t base_w = base_h + static_cast<int64_t>(g.Hh) * (g.dh / 2);
+        r.t0 = static_cast<int64_t>(t) * (g.dt / 2);
+        r.h0 = base_h + static_cast<int64_t>(y) * (g.dh / 2);
+        r.w0 = base_w + static_cast<int64_t>(x) * (g.dh / 2);
+        return r;
+    }
+    __device__ __forceinline__ int64_t entry(int d, int dt, int dh) const
+    {
+        return d < dt ? t0 + d / 2 : (d < dt + dh ? h0 + (d - dt) / 2 : w0 + (d - dt - dh) / 2);
+    }
+};
+
+// The 3D RoPE table: (cos, sin) per (axis, position, pair) in fp64 (tab64,
+// two doubles per entry) and their fp32 roundings (tab32, one float2 per
+// entry), laid out as RopeGeom describes.
+struct RopeTabs {
+    const double *t64;
+    const float2 *t32;
+};
+
+// The fp64 rotation from fp64 table entry e (out of line: one copy of the
+// cold path keeps unrolled callers small for the instruction cache).
+__device__ __noinline__ uint32_t rotate_pair_tab64(uint32_t packed, const double *__restrict__ t64, int64_t e)
+{
+    return rotate_pair(packed, __ldg(t64 + 2 * e), __ldg(t64 + 2 * e + 1));
+}
+
+// Rotate one packed pair from table entry e: fp32 when the certificate
+// holds, else fp64 from the fp64 entry (rare, so the branch seldom diverges).
+__device__ __forceinline__ uint32_t rotate_pair_tab(uint32_t packed, float2 cs32, const double *__restrict__ t64,
+                                                    int64_t e)
+{
+    uint32_t r;
+    if (__builtin_expect(rotate_pair_f32(packed, cs32.x, cs32.y, r), 1)) return r;
+    return rotate_pair_tab64(packed, t64, e);
+}
+
+// tab64[2e], tab64[2e+1] = cos, sin of every table entry e, and tab32[e]
+// their fp32 roundings (grid-stride).
+__global__ void rope_table_kernel(double *__restrict__ tab64, float2 *__restrict__ tab32, RopeGeom g,
+                                  const __grid_constant__ RopeFreqs fr)
 {
     const int64_t n = g.entries();
     const int64_t base_h = static_cast<int64_t>(g.T) * (g.dt / 2);
     const int64_t base_w = base_h + static_cast<int64_t>(g.Hh) * (g.dh / 2);
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n; e += stride) {
-        int pos, j, width;
+        int pos, pair;   // pair: index of the pair within the head dimension
         if (e < base_h) {
-            pos = static_cast<int>(e / (g.dt / 2)); j = static_cast<int>(e % (g.dt / 2)); width = g.dt;
+            pos = static_cast<int>(e / (g.dt / 2)); pair = static_cast<int>(e % (g.dt / 2));
         } else if (e < base_w) {
-            pos = static_cast<int>((e - base_h) / (g.dh / 2)); j = static_cast<int>((e - base_h) % (g.dh / 2));
-            width = g.dh;
+            pos = static_cast<int>((e - base_h) / (g.dh / 2));
+            pair = g.dt / 2 + static_cast<int>((e - base_h) % (g.dh / 2));
         } else {
-            pos = static_cast<int>((e - base_w) / (g.dh / 2)); j = static_cast<int>((e - base_w) % (g.dh / 2));
-            width = g.dh;
+            pos = static_cast<int>((e - base_w) / (g.dh / 2));
+            pair = (g.dt + g.dh) / 2 + static_cast<int>((e - base_w) % (g.dh / 2));
         }
         double c, s;
-        rope_angle(pos, 2 * j, width, theta, c, s);
-        tab[2 * e] = c;
-        tab[2 * e + 1] = s;
+        rope_angle(pos, fr.f[pair], c, s);
+        tab64[2 * e] = c;
+        tab64[2 * e + 1] = s;
+        tab32[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
     }
 }
 
-// Rotate the 16-byte chunk holding dimensions [8c, 8c + 8) of token n's row.
-__device__ __forceinline__ uint4 rotate_chunk(uint4 v, int c, int n, const RopeGeom &g,
-                                              const double *__restrict__ tab)
+// Walk rows [r0, r1) of one 16-byte chunk (element offset `off` in a row of
+// `row_stride` elements): dst row r = rot(src row r), four rows at a time
+// with the next four rows' loads issued before the current four are stored.
+template <typename Rot>
+__device__ __forceinline__ void rope_walk_rows(const uint16_t *src, uint16_t *dst, int64_t r0, int64_t r1,
+                                               int64_t row_stride, int64_t off, Rot rot)
 {
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    auto ld = [&](int64_t r) { return *reinterpret_cast<const uint4 *>(src + r * row_stride + off); };
+    uint4 cur[4];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const int64_t e = g.entry(n, c * 8 + 2 * p);
-        w[p] = rotate_pair(w[p], __ldg(tab + 2 * e), __ldg(tab + 2 * e + 1));
+    for (int u = 0; u < 4; ++u)
+        if (r0 + u < r1) cur[u] = ld(r0 + u);
+    for (int64_t r = r0; r < r1; r += 4) {
+        uint4 nxt[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (r + 4 + u < r1) nxt[u] = ld(r + 4 + u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (r + u < r1) *reinterpret_cast<uint4 *>(dst + (r + u) * row_stride + off) = rot(cur[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
     }
-    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // dst = RoPE(src) for `rows` rows of S x D (out of place), from the table.
-__global__ void rope_apply_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int64_t rows, int S,
-                                  int D, RopeGeom g, const double *__restrict__ tab)
+// Thread = (token, 16-byte chunk) x one group of `rows_per_group` rows
+// (blockIdx.y): the chunk's four table entries are read once per group.
+__global__ void __launch_bounds__(128, 6) rope_apply_kernel(const uint16_t *__restrict__ src,
+                                                            uint16_t *__restrict__ dst, int64_t rows, int S, int D,
+                                                            RopeGeom g, RopeTabs tab, int rows_per_group)
 {
-    // One thread per (token, 16-byte chunk): the chunk's four (cos, sin) pairs
-    // are read from the table once and applied to that chunk of every row
-    // (consecutive threads, consecutive chunks of one row: coalesced).
     const int chunks = D >> 3;
     const int64_t per_row = static_cast<int64_t>(S) * chunks;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < per_row; t += stride) {
-        const int n = static_cast<int>(t / chunks);
-        const int c = static_cast<int>(t % chunks);
-        double cs[4], sn[4];
+    const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+    if (t >= per_row) return;
+    const int n = static_cast<int>(t / chunks);
+    const int c = static_cast<int>(t % chunks);
+    const RopeRowEntries re = RopeRowEntries::of(g, n);
+    int64_t e[4];
+    float2 cs[4];
+    double c64[4], s64[4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const int64_t e = g.entry(n, c * 8 + 2 * p);
-            cs[p] = __ldg(tab + 2 * e);
-            sn[p] = __ldg(tab + 2 * e + 1);
-        }
-        auto rot = [&](uint4 v) {
-            return make_uint4(rotate_pair(v.x, cs[0], sn[0]), rotate_pair(v.y, cs[1], sn[1]),
-                              rotate_pair(v.z, cs[2], sn[2]), rotate_pair(v.w, cs[3], sn[3]));
-        };
-        int64_t r = 0;
-        for (; r + 4 <= rows; r += 4) {
-            uint4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = src[(r + u) * per_row + t];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) dst[(r + u) * per_row + t] = rot(v[u]);
-        }
-        for (; r < rows; ++r) dst[r * per_row + t] = rot(src[r * per_row + t]);
+    for (int p = 0; p < 4; ++p) {
+        e[p] = re.entry(c * 8 + 2 * p, g.dt, g.dh);
+        cs[p] = __ldg(tab.t32 + e[p]);
+        c64[p] = __ldg(tab.t64 + 2 * e[p]);
+        s64[p] = __ldg(tab.t64 + 2 * e[p] + 1);
     }
+    auto rot1 = [&](uint32_t w, int p) {
+        uint32_t r;
+        if (__builtin_expect(rotate_pair_f32(w, cs[p].x, cs[p].y, r), 1)) return r;
+        return rotate_pair(w, c64[p], s64[p]);
+    };
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_group;
+    const int64_t r1 = r0 + rows_per_group < rows ? r0 + rows_per_group : rows;
+    rope_walk_rows(src, dst, r0, r1, static_cast<int64_t>(S) * D, t * 8, [&](uint4 v) {
+        return make_uint4(rot1(v.x, 0), rot1(v.y, 1), rot1(v.z, 2), rot1(v.w, 3));
+    });
 }
 
-__global__ void rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k, int64_t rows,
-                              int S, int Hh, int Ww, int D, double theta, bool inverse, int n0)
+// In place on q and k: thread = (token, 16-byte chunk) x one group of rows
+// (blockIdx.y in [0, 2*groups): groups of q's rows, then of k's). The four
+// angles come from fp64 sincos once per thread. inverse: the transposed
+// rotation (sine negated), the RoPE's gradient. n0: position of token 0 of
+// this sequence shard on the latent grid.
+__global__ void __launch_bounds__(128, 8) rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k,
+                                                        int64_t rows, int S, int Hh, int Ww, int D,
+                                                        const __grid_constant__ RopeFreqs fr, bool inverse, int n0,
+                                                        int rows_per_group, int groups)
 {
     const int chunks = D >> 3;
     const int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
     if (gid >= static_cast<int64_t>(S) * chunks) return;
+    const int which = static_cast<int>(blockIdx.y) / groups;   // 0: q, 1: k
+    uint16_t *x = which == 0 ? q : k;
+    if (x == nullptr) return;
     const int n = static_cast<int>(gid / chunks);
     const int c = static_cast<int>(gid % chunks);
     const int tok = n0 + n;   // position on the latent grid
-    const int pos[3] = {tok / (Hh * Ww), (tok / Ww) % Hh, tok % Ww};
+    const int pt = tok / (Hh * Ww), ph = (tok / Ww) % Hh, pw = tok % Ww;
     const int dh = 2 * (D / 6);
     const int dt = D - 2 * dh;
     double cs[4], sn[4];
+    float cs32[4], sn32[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const int d = c * 8 + 2 * p;
-        int axis, local, width;
-        if (d < dt) {
-            axis = 0; local = d; width = dt;
-        } else if (d < dt + dh) {
-            axis = 1; local = d - dt; width = dh;
-        } else {
-            axis = 2; local = d - dt - dh; width = dh;
-        }
-        rope_angle(pos[axis], local, width, theta, cs[p], sn[p]);
+        rope_angle(d < dt ? pt : (d < dt + dh ? ph : pw), fr.f[d / 2], cs[p], sn[p]);
         if (inverse) sn[p] = -sn[p];
+        cs32[p] = static_cast<float>(cs[p]);
+        sn32[p] = static_cast<float>(sn[p]);
     }
-    const int64_t row_stride = static_cast<int64_t>(S) * D;
-    const int64_t off = static_cast<int64_t>(n) * D + c * 8;
-    for (int which = 0; which < 2; ++which) {
-        uint16_t *x = which == 0 ? q : k;
-        if (x == nullptr) continue;
-        int64_t r = 0;
-        for (; r + 4 <= rows; r += 4) {
-            uint4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint4 *>(x + (r + u) * row_stride + off);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                v[u].x = rotate_pair(v[u].x, cs[0], sn[0]);
-                v[u].y = rotate_pair(v[u].y, cs[1], sn[1]);
-                v[u].z = rotate_pair(v[u].z, cs[2], sn[2]);
-                v[u].w = rotate_pair(v[u].w, cs[3], sn[3]);
-                *reinterpret_cast<uint4 *>(x + (r + u) * row_stride + off) = v[u];
-            }
-        }
-        for (; r < rows; ++r) {
-            uint4 v = *reinterpret_cast<const uint4 *>(x + r * row_stride + off);
-            v.x = rotate_pair(v.x, cs[0], sn[0]);
-            v.y = rotate_pair(v.y, cs[1], sn[1]);
-            v.z = rotate_pair(v.z, cs[2], sn[2]);
-            v.w = rotate_pair(v.w, cs[3], sn[3]);
-            *reinterpret_cast<uint4 *>(x + r * row_stride + off) = v;
-        }
-    }
+    auto rot1 = [&](uint32_t w, int p) {
+        uint32_t r;
+        if (__builtin_expect(rotate_pair_f32(w, cs32[p], sn32[p], r), 1)) return r;
+        return rotate_pair(w, cs[p], sn[p]);
+    };
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y % groups) * rows_per_group;
+    const int64_t r1 = r0 + rows_per_group < rows ? r0 + rows_per_group : rows;
+    rope_walk_rows(x, x, r0, r1, static_cast<int64_t>(S) * D, static_cast<int64_t>(n) * D + c * 8, [&](uint4 v) {
+        return make_uint4(rot1(v.x, 0), rot1(v.y, 1), rot1(v.z, 2), rot1(v.w, 3));
+    });
 }
 
 }  // namespace regen

@@ -75,6 +75,31 @@ REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const reg
                              regen_stream_t stream);
 
 /*
+ * regen_attn_fwd_kv2 -- regen_attn_fwd over keys held in two separate
+ * buffers: the cross-attention of the video tokens to the reference-frame
+ * latent tokens and to the conditioning tokens (mlsanity.com abstract; blog
+ * page, "Methodology -- deep read"), as one softmax over the two key sets
+ * concatenated, [k_a ; k_b] with their values [v_a ; v_b]:
+ *     out_i = sum_j softmax(s)_j v_j,  lse_i = ln sum_j exp(s_j),  j over Skv_a + Skv_b keys
+ * In one launch: the kernel takes key blocks from source a, then from source
+ * b, and masks each source's last block past that source's end, so nothing is
+ * copied and no partial results are merged. Same arithmetic and rounding as
+ * regen_attn_fwd on the concatenated keys (bit for bit when Skv_a is a
+ * multiple of 128).
+ *
+ *   q    [B, H, Sq, D] bf16;  k_a, v_a [B, H, Skv_a, D];  k_b, v_b [B, H, Skv_b, D] bf16
+ *   out  [B, H, Sq, D] bf16;  lse [B, H, Sq] fp32 or NULL
+ *   D, scale and edge cases as regen_attn_fwd; Skv_a + Skv_b < 2^31. One
+ *   source empty: the same as regen_attn_fwd over the other (its pointers
+ *   may then be NULL). out and lse must not overlap any input.
+ */
+REGEN_API int regen_attn_fwd_kv2(const regen_bf16 *q, const regen_bf16 *k_a, const regen_bf16 *v_a,
+                                 const regen_bf16 *k_b, const regen_bf16 *v_b,
+                                 regen_bf16 *out, float *lse,
+                                 int B, int H, int Sq, int Skv_a, int Skv_b, int D, float scale,
+                                 regen_stream_t stream);
+
+/*
  * regen_attn_fwd_rope3d -- self-attention with the 3D RoPE applied on the
  * way in: the same result, bit for bit, as regen_rope3d(q, k, ...) followed
  * by regen_attn_fwd(...), but q and k are left unmodified.
@@ -84,7 +109,7 @@ REGEN_API int regen_attn_fwd(const regen_bf16 *q, const regen_bf16 *k, const reg
  *    every key tile, so rotating K per load would repeat the work for each of
  *    the ceil(S/256) query-tile pairs.
  *  - The (cos, sin) of every (axis, position, pair) are computed once, in fp64,
- *    into a small table at the start of the workspace.
+ *    into a small table at the start of the workspace, with its fp32 copy.
  *
  *   q, k, v, out, lse, B, H, D, scale, stream: as regen_attn_fwd
  *   Sq == Skv == T*Hh*Ww (else REGEN_ERR_INVALID_ARG); T, Hh, Ww, theta: as regen_rope3d
@@ -103,9 +128,10 @@ REGEN_API int regen_attn_fwd_rope3d(const regen_bf16 *q, const regen_bf16 *k, co
                                     void *workspace, int64_t workspace_bytes);
 
 /*
- * Bytes of workspace regen_attn_fwd_rope3d needs: a 256-byte-rounded table of
- * 16 * (T*(D - 4*floor(D/6))/2 + (Hh + Ww)*floor(D/6)) bytes plus B*H*S*D*2
- * bytes of rotated K. Negative (a regen_status) for invalid sizes.
+ * Bytes of workspace regen_attn_fwd_rope3d needs: with E = T*(D - 4*floor(D/6))/2
+ * + (Hh + Ww)*floor(D/6) table entries, 16*E bytes of fp64 table and 8*E bytes
+ * of fp32 table (each rounded up to a multiple of 256) plus B*H*S*D*2 bytes of
+ * rotated K. Negative (a regen_status) for invalid sizes.
  */
 REGEN_API int64_t regen_attn_fwd_rope3d_workspace_bytes(int B, int H, int T, int Hh, int Ww, int D);
 
@@ -153,8 +179,10 @@ REGEN_API int regen_attn_fwd_rope3d_noalloc(const regen_bf16 *q, const regen_bf1
  * D - 4*floor(D/6), 2*floor(D/6), 2*floor(D/6) (44/42/42 at D = 128); in a
  * block of width d_a the pair (2j, 2j+1) turns by pos_a * theta^(-2j/d_a):
  *     x'_{2j} = x_{2j} cos - x_{2j+1} sin,   x'_{2j+1} = x_{2j} sin + x_{2j+1} cos
- * Angles and the rotation are evaluated in fp64 and the result is rounded
- * once to bf16 (nearest even).
+ * The result is that of fp64 angles and an fp64 rotation rounded once to
+ * bf16 (nearest even). The kernel computes it in fp32 and proves, pair by
+ * pair, that the fp32 value rounds to the same bf16; the pairs it cannot
+ * prove (near a bf16 rounding boundary) are redone in fp64.
  *
  *   q, k   [B, H, S, D] bf16, rotated in place; either may be NULL (skipped),
  *          not both. q and k must not overlap.

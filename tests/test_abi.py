@@ -93,9 +93,11 @@ def test_python_binding_raises(lib):
 
 
 def test_rope3d_fused_workspace_bytes(lib):
-    # table: 16 * (T*dt/2 + (Hh + Ww)*dh/2), rounded up to 256; plus B*H*S*D*2 of rotated K
+    # E = T*dt/2 + (Hh + Ww)*dh/2 table entries: 16 E bytes (fp64) and 8 E bytes (fp32),
+    # each rounded up to 256; plus B*H*S*D*2 of rotated K
     T, Hh, Ww, D = 20, 30, 52, 128
-    table = (16 * (T * 22 + (Hh + Ww) * 21) + 255) // 256 * 256
+    E = T * 22 + (Hh + Ww) * 21
+    table = (16 * E + 255) // 256 * 256 + (8 * E + 255) // 256 * 256
     assert rg.regen_attn_fwd_rope3d_workspace_bytes(1, 40, T, Hh, Ww, D) == table + 40 * T * Hh * Ww * D * 2
     assert lib.regen_attn_fwd_rope3d_workspace_bytes(1, 1, 0, 1, 1, 128) == -1
     assert lib.regen_attn_fwd_rope3d_workspace_bytes(1, 1, 1, 1, 1, 96) == -2
@@ -281,3 +283,18 @@ def test_per_context_setup_cache(tmp_path):
                     str(src), "-o", str(exe), "-pthread"], check=True)
     res = subprocess.run([str(exe)], capture_output=True, text=True)
     assert res.returncode == 0 and res.stdout.strip() == "ok", (res.returncode, res.stdout)
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=96), -2), (dict(B=-1), -1), (dict(Skv_a=-1), -1), (dict(Skv_b=-2), -1), (dict(scale=float("nan")), -1),
+    (dict(k_b=None), -1), (dict(v_a=None), -1), (dict(k_a=FAKE + 10 * MB + 8), -3), (dict(lse=FAKE + 60 * MB + 4), -3),
+    (dict(out=FAKE + 20 * MB), -1), (dict(lse=FAKE + 40 * MB), -1), (dict(Skv_a=2**30, Skv_b=2**30), -2),
+    (dict(B=0), 0), (dict(Sq=0), 0),
+])
+def test_attn_fwd_kv2_validation(lib, args, status):
+    a = dict(q=FAKE, k_a=FAKE + 10 * MB, v_a=FAKE + 20 * MB, k_b=FAKE + 30 * MB, v_b=FAKE + 40 * MB,
+             out=FAKE + 50 * MB, lse=FAKE + 60 * MB, B=1, H=2, Sq=100, Skv_a=60, Skv_b=40, D=128, scale=0.125)
+    a.update(args)
+    rc = lib.regen_attn_fwd_kv2(a["q"], a["k_a"], a["v_a"], a["k_b"], a["v_b"], a["out"], a["lse"], a["B"], a["H"],
+                                a["Sq"], a["Skv_a"], a["Skv_b"], a["D"], a["scale"], None)
+    assert rc == status

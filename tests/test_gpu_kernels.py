@@ -74,6 +74,39 @@ def test_rope3d_full_77_frame_window_sampled_heads():
         np.testing.assert_array_equal(gk[0, h], oracle.rope3d(k[0, h], w.grid, w.theta))
 
 
+def _all_finite_bf16_patterns(n_rows, D, seed):
+    """Every finite bf16 bit pattern (zeros, subnormals, up to +-max) once,
+    shuffled, then filled up with random ones: [n_rows, D]."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]                   # drop inf and NaN
+    rng = np.random.default_rng(seed)
+    need = n_rows * D
+    assert need >= bits.size
+    fill = rng.choice(bits, size=need - bits.size)
+    return rng.permutation(np.concatenate([bits, fill])).reshape(n_rows, D)
+
+
+def test_rope3d_every_finite_bf16_pattern_bit_exact():
+    # The rotation runs in fp32 and proves per pair that it rounds like fp64,
+    # else redoes the pair in fp64: across every finite bf16 magnitude
+    # (subnormals, values whose products overflow fp32, exact zeros) the bits
+    # must equal the oracle's fp64 rotation, forward and inverse.
+    grid, D, H = (3, 5, 7), 128, 6          # 105 tokens x 128 x 6 heads = 80640 values
+    S = grid[0] * grid[1] * grid[2]
+    q = _all_finite_bf16_patterns(H * S, D, 1).reshape(1, H, S, D)
+    k = _all_finite_bf16_patterns(H * S, D, 2).reshape(1, H, S, D)
+    for theta in (10000.0, 3.0):
+        dq, dk = to_dev(q), to_dev(k)
+        rg.rope3d_(dq, dk, grid, theta)
+        torch.cuda.synchronize()
+        gq, gk = to_bits(dq), to_bits(dk)
+        np.testing.assert_array_equal(gq, oracle.rope3d(q, grid, theta))
+        np.testing.assert_array_equal(gk, oracle.rope3d(k, grid, theta))
+        rg.rope3d_bwd_(dq, None, grid, theta)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(to_bits(dq), oracle.rope3d_bwd(gq, grid, theta))
+
+
 # ------------------------------------------------------------- LSE merge ---
 
 @pytest.mark.parametrize("rows,D", [(1, 128), (2, 128), (777, 128), (4096, 64), (33, 8)])
