@@ -1,14 +1,16 @@
 """Benchmark of the DiT attention hot path (one line of JSON on rank 0).
 
-One step = one pass of the whole hot path for one denoising step of the
-77-frame window (B=1, H=40, D=128, latent grid 20 x 30 x 52 -> S = 31200):
-  1. rope3d on Q and K (in place)                       regen_rope3d
-  2. self-attention, 31200 x 31200                      regen_attn_fwd
-  3. cross-attention of the 31200 video tokens to the 1560 reference-frame
-     tokens and, separately, to the 512 conditioning tokens   regen_attn_fwd x2
-  4. the two cross-attention partials merged by LSE     regen_lse_merge
-(3+4 equal one softmax over the 2072 concatenated keys.) Each step rotates
-the Q/K left by the previous step again: the same work on the same shapes.
+One step = one pass of the hot path for one denoising step of the 77-frame
+window (B=1, H=40, D=128, latent grid 20 x 30 x 52 -> S = 31200):
+  1. self-attention, 31200 x 31200, with the 3D RoPE fused into the Q load
+     (K rotated once into workspace)                    regen_attn_fwd_rope3d
+  2. cross-attention of the 31200 video tokens to the 1560 reference-frame
+     and 512 conditioning tokens, one softmax over both key buffers in one
+     launch                                             regen_attn_fwd_kv2
+Beside it, timed in alternating rounds on the same box: the step with the
+RoPE as a pre-pass (regen_rope3d + regen_attn_fwd); and the cross-attention
+paths on the step's shapes, including the Ring form (one call per key block
+merged by regen_lse_merge) and one call over concatenated keys.
 
 value = attention FLOPs of the step (4*B*H*Sq*Skv*D, self + cross) / device
 time of the step, summed over ranks (weak scaling: every rank runs its own
@@ -215,8 +217,9 @@ def step_config(world):
     ws, wc = synth.WORKLOADS[SELF], synth.WORKLOADS[CROSS]
     T, Hh, Ww = ws.grid
     return {
-        "workload": "win77_s31200 self-attention + RoPE, cross-attention to 1560 reference + 512 "
-                    "conditioning tokens merged by LSE (one denoising step of the 77-frame window)",
+        "workload": "win77_s31200 self-attention with the 3D RoPE fused into the Q load, cross-attention to "
+                    "1560 reference + 512 conditioning tokens under one softmax (one denoising step of the "
+                    "77-frame window)",
         "B": ws.B, "H": ws.H, "S": ws.Sq, "D": ws.D, "Skv_cross": [N_REF, wc.Skv - N_REF],
         "latent_grid": [T, Hh, Ww], "scale": 1.0 / math.sqrt(ws.D),
         "l2": "inputs larger than L2 (320 MB per tensor vs 126 MB); no flush",
@@ -247,6 +250,57 @@ def traffic_from_profile():
         return None
 
 
+def tensor_roofline(kernel, flops, ms, region_ms, clk, pk, pk_src, peak_mult=1.0, peak_note="bf16"):
+    """Roofline of a tensor-core kernel: achieved = algorithmic FLOPs per launch
+    / its event-timed duration, against the measured burst peak when the timed
+    region is short (under 3 s: the part runs at its boost clock before the
+    power cap settles) or the sustained one otherwise; also the fractions of
+    both peaks, of the sustained peak scaled to this run's SM clock, and the
+    cycles per launch at the run's median SM clock (comparable across boxes)."""
+    burst = float(pk["bf16_tflops"]) * peak_mult
+    sust = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]) * peak_mult
+    achieved = flops / (ms * 1e-3) / 1e12
+    short = region_ms < 3000.0
+    peak = burst if short else sust
+    d = {"bound": "tensor", "kernel": kernel, "achieved": round(achieved, 2), "peak": round(peak, 1),
+         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+         "peak_source": (f"{pk_src} {'bf16_tflops (burst)' if short else 'bf16_tflops_sustained'}"
+                         f"{'' if peak_mult == 1.0 else ' x %g (%s)' % (peak_mult, peak_note)}: the timed region "
+                         f"lasts {region_ms / 1000:.2f} s"),
+         "frac_of_burst_peak": round(achieved / burst, 4), "frac_of_sustained_peak": round(achieved / sust, 4),
+         "frac_of_nominal": round(achieved / (2250.0 * peak_mult), 4),
+         "algorithmic_flops_per_launch": flops, "ms_per_launch": round(ms, 4)}
+    mhz = clk.get("sm_mhz") if clk else None
+    if mhz:
+        d["sm_mhz_median"] = mhz
+        d["cycles_per_launch"] = int(round(ms * 1e-3 * mhz * 1e6))
+        sust_mhz = (pk.get("clocks_under_load") or {}).get("sm_mhz_median")
+        if sust_mhz:
+            d["frac_of_sustained_peak_at_this_clock"] = round(achieved / (sust * mhz / float(sust_mhz)), 4)
+    return d
+
+
+def timed_region(fn, n, stream, world, dev, barrier, with_clocks=True):
+    """n calls of fn between two events on `stream` (barrier + synchronize on
+    both sides), max over ranks; returns (ms per call, clocks dict, region ms)."""
+    import torch
+    clocks = ClockSampler(dev) if with_clocks else None
+    barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else {}
+    barrier()
+    total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return total / n, clk, total
+
+
 def run_native(args, rank, world, local_rank):
     import torch
     import dit_attention_b200 as rg
@@ -270,19 +324,26 @@ def run_native(args, rank, world, local_rank):
     }
     d = {name: to_dev(a) for name, a in host.items()}
     B, H, S, D = ws.B, ws.H, ws.Sq, ws.D
+    n_ctx = wc.Skv - N_REF
     out = torch.empty_like(d["q"])
     lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
-    oa, ob, oc = (torch.empty_like(d["qc"]) for _ in range(3))
-    la, lb, lc = (torch.empty((B, H, S), dtype=torch.float32, device=dev) for _ in range(3))
+    oc = torch.empty_like(d["qc"])
+    lc = torch.empty((B, H, S), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     scale = 1.0 / math.sqrt(D)
     T, Hh, Ww = ws.grid
+    rope_ws_bytes = rg.regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
+    rope_ws = torch.empty(rope_ws_bytes, dtype=torch.uint8, device=dev)
 
-    names = ["rope3d", "attn_self", "attn_cross_ref", "attn_cross_ctx", "lse_merge"]
-    LAUNCHES_PER_STEP = len(names)
-
-    outs0 = dict(out=out, lse=lse, oa=oa, la=la, ob=ob, lb=lb, oc=oc, lc=lc)
+    # One step: the self-attention with the 3D RoPE fused into its Q load (the
+    # table, the K pass and the attention: 3 launches; q and k are not
+    # modified, so every step starts from the same inputs) and the
+    # cross-attention to the reference-frame and conditioning keys in one
+    # launch over the two key buffers.
+    names = ["attn_self_rope_fused", "attn_cross_kv2"]
+    LAUNCHES_PER_STEP = 4
+    outs0 = dict(out=out, lse=lse, oc=oc, lc=lc)
 
     def step(ev=None, inp=None, o=None):
         inp = d if inp is None else inp
@@ -292,16 +353,12 @@ def run_native(args, rank, world, local_rank):
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        rg.regen_rope3d(inp["q"], inp["k"], T, Hh, Ww, ws.theta, B, H, D, sh)
+        rg.regen_attn_fwd_rope3d(inp["q"], inp["k"], inp["v"], o["out"], o["lse"], B, H, S, S, D, scale, sh,
+                                 T, Hh, Ww, ws.theta, rope_ws, rope_ws_bytes)
         mark(1)
-        rg.regen_attn_fwd(inp["q"], inp["k"], inp["v"], o["out"], o["lse"], B, H, S, S, D, scale, sh)
+        rg.regen_attn_fwd_kv2(inp["qc"], inp["kr"], inp["vr"], inp["kx"], inp["vx"], o["oc"], o["lc"], B, H, S,
+                              N_REF, n_ctx, D, scale, sh)
         mark(2)
-        rg.regen_attn_fwd(inp["qc"], inp["kr"], inp["vr"], o["oa"], o["la"], B, H, S, N_REF, D, scale, sh)
-        mark(3)
-        rg.regen_attn_fwd(inp["qc"], inp["kx"], inp["vx"], o["ob"], o["lb"], B, H, S, wc.Skv - N_REF, D, scale, sh)
-        mark(4)
-        rg.regen_lse_merge(o["oa"], o["la"], o["ob"], o["lb"], o["oc"], o["lc"], B * H * S, D, sh)
-        mark(5)
 
     def barrier():
         if world > 1:
@@ -312,8 +369,8 @@ def run_native(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
 
-    # ---- device-resident timing: K steps between two events, per-kernel events inside
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    # ---- device-resident timing: K steps between two events, per-call events inside
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clocks = ClockSampler(dev)
     barrier()
     torch.cuda.synchronize()
@@ -339,60 +396,98 @@ def run_native(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     value = aggregate_tflops(flops_step, world, ms_step)
 
-    # The last timed step's self-attention, exactly: its bf16 inputs (q and k
-    # as that step's RoPE left them) and its output, for the CPU leg's
-    # accuracy check (rank 0 only, and only when that leg runs).
+    # The last timed step's self-attention inputs (unrotated q, k as given to
+    # the fused call) and its output, for the CPU leg's accuracy check (rank 0
+    # only, and only when that leg runs); the oracle rotates q and k itself.
     snap = None
     if rank == 0 and not args.no_cpu_baseline:
         bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
         snap = dict(q=bits(d["q"]), k=bits(d["k"]), v=bits(d["v"]), out=bits(out), lse=lse.cpu().numpy(),
-                    scale=scale)
+                    scale=scale, grid=ws.grid, theta=ws.theta)
+
+    # ---- the same step with the RoPE as a pre-pass (regen_rope3d on copies of q, k,
+    # then the plain attention), timed in rounds alternating with the fused step,
+    # on the same box and clocks. Each pre-pass step rotates its copies again: the
+    # same work on the same shapes.
+    qp, kp = d["q"].clone(), d["k"].clone()
+    pre_names = ["rope3d", "attn_self", "attn_cross_kv2"]
+
+    def step_prepass(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        rg.regen_rope3d(qp, kp, T, Hh, Ww, ws.theta, B, H, D, sh)
+        mark(1)
+        rg.regen_attn_fwd(qp, kp, d["v"], out, lse, B, H, S, S, D, scale, sh)
+        mark(2)
+        rg.regen_attn_fwd_kv2(d["qc"], d["kr"], d["vr"], d["kx"], d["vx"], oc, lc, B, H, S, N_REF, n_ctx, D, scale,
+                              sh)
+        mark(3)
+
+    n_alt = max(3, min(args.steps, 10))
+    for _ in range(args.warmup):
+        step_prepass()
+    fused_ms, pre_ms, pre_k = [], [], {n: [] for n in pre_names}
+    for rnd in range(3):
+        for which in ((0, 1) if rnd % 2 == 0 else (1, 0)):
+            if which == 0:
+                ms, _, _ = timed_region(step, n_alt, stream, world, dev, barrier, with_clocks=False)
+                fused_ms.append(ms)
+            else:
+                pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_alt)]
+                ms, _, _ = timed_region(lambda it=iter(pev): step_prepass(next(it)), n_alt, stream, world, dev,
+                                        barrier, with_clocks=False)
+                pre_ms.append(ms)
+                for j, n in enumerate(pre_names):
+                    pre_k[n].append(sum(e[j].elapsed_time(e[j + 1]) for e in pev) / n_alt)
+    del qp, kp
+
+    # ---- cross-attention paths on the step's shapes: the one-launch two-source
+    # call (the step's), the two key blocks as separate calls merged by
+    # regen_lse_merge (the Ring form of the same result), and one call over the
+    # keys concatenated in one buffer.
+    oa, ob = torch.empty_like(oc), torch.empty_like(oc)
+    la, lb = torch.empty_like(lc), torch.empty_like(lc)
+    kcat = torch.cat([d["kr"], d["kx"]], dim=2).contiguous()
+    vcat = torch.cat([d["vr"], d["vx"]], dim=2).contiguous()
+    cross_fns = {
+        "kv2": lambda: rg.regen_attn_fwd_kv2(d["qc"], d["kr"], d["vr"], d["kx"], d["vx"], oc, lc, B, H, S, N_REF,
+                                             n_ctx, D, scale, sh),
+        "ref_block": lambda: rg.regen_attn_fwd(d["qc"], d["kr"], d["vr"], oa, la, B, H, S, N_REF, D, scale, sh),
+        "ctx_block": lambda: rg.regen_attn_fwd(d["qc"], d["kx"], d["vx"], ob, lb, B, H, S, n_ctx, D, scale, sh),
+        "lse_merge": lambda: rg.regen_lse_merge(oa, la, ob, lb, oc, lc, B * H * S, D, sh),
+        "concat_one_call": lambda: rg.regen_attn_fwd(d["qc"], kcat, vcat, oc, lc, B, H, S, wc.Skv, D, scale, sh),
+    }
+    cross_ms = {}
+    for n, fn in cross_fns.items():
+        for _ in range(args.warmup):
+            fn()
+        cross_ms[n] = timed_region(fn, max(5, min(args.steps, 20)), stream, world, dev, barrier,
+                                   with_clocks=False)[0]
+    del oa, ob, la, lb, kcat, vcat
 
     # ---- backward: the gradient step of the same window (the decoder is trained by
     # distillation). dO synthetic; the forward's out/lse of the last timed step
     # (taken before anything else overwrites them).
     # Self: regen_attn_bwd then regen_rope3d_bwd on dq, dk (gradients w.r.t. the
-    # unrotated Q, K). Cross: one regen_attn_bwd per key block with the MERGED
-    # out/lse, the second accumulating dq. Each regen_attn_bwd is 3 launches
-    # (prep, dK/dV, dQ).
-    bwd = run_backward(args, rg, synth, d, outs0, ws, wc, rank, dev, stream, world, barrier, to_dev)
+    # unrotated Q, K); q, k enter it rotated (the pre-pass's output of the same
+    # inputs). Cross: one regen_attn_bwd per key block with the merged out/lse,
+    # the second accumulating dq. Each regen_attn_bwd is 3 launches.
+    step()            # the fused step's out/lse for these inputs
+    qrot, krot = d["q"].clone(), d["k"].clone()
+    rg.regen_rope3d(qrot, krot, T, Hh, Ww, ws.theta, B, H, D, sh)
+    dr = dict(d, q=qrot, k=krot)
+    bwd = run_backward(args, rg, synth, dr, outs0, ws, wc, rank, dev, stream, world, barrier, to_dev)
 
     # ---- the projections around the attention of a 14B-class DiT block on the same
     # window: fused QKV projection (+ RMSNorm + RoPE) and the output projection.
     proj = run_proj(args, rg, synth, ws, dev, stream, world, barrier, to_dev, rank)
 
-    # ---- the FP8 variant of the self-attention (after the same RoPE): blockwise
+    # ---- the FP8 variant of the self-attention (on the rotated q, k): blockwise
     # E4M3 quantisation of Q, K, V (3 launches) and the E4M3 attention.
-    fp8 = run_fp8(args, rg, d, ws, dev, stream, world, barrier)
-
-    # ---- the same step with the RoPE fused into the Q load (regen_attn_fwd_rope3d):
-    # Q rotated on its tiles in shared memory, K rotated once into the workspace;
-    # q and k are not modified, so every step starts from the unrotated inputs.
-    rope_ws_bytes = rg.regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
-    rope_ws = torch.empty(rope_ws_bytes, dtype=torch.uint8, device=dev)
-
-    def step_fused():
-        rg.regen_attn_fwd_rope3d(d["q"], d["k"], d["v"], out, lse, B, H, S, S, D, scale, sh, T, Hh, Ww,
-                                 ws.theta, rope_ws, rope_ws_bytes)
-        rg.regen_attn_fwd(d["qc"], d["kr"], d["vr"], oa, la, B, H, S, N_REF, D, scale, sh)
-        rg.regen_attn_fwd(d["qc"], d["kx"], d["vx"], ob, lb, B, H, S, wc.Skv - N_REF, D, scale, sh)
-        rg.regen_lse_merge(oa, la, ob, lb, oc, lc, B * H * S, D, sh)
-
-    n_alt = max(3, min(args.steps, 20))
-    for _ in range(args.warmup):
-        step_fused()
-    torch.cuda.synchronize()
-    barrier()
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(n_alt):
-        step_fused()
-    f1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms_fused = max_over_ranks(f0.elapsed_time(f1), world, dev) / n_alt
-    del rope_ws
+    fp8 = run_fp8(args, rg, dr, ws, dev, stream, world, barrier)
+    del qrot, krot, dr
 
     # ---- end to end: pinned host inputs -> device -> hot path -> outputs to pinned host
     pin = {n: torch.from_numpy(a.view(np.int16)).pin_memory() for n, a in host.items()}
@@ -418,17 +513,8 @@ def run_native(args, rank, world, local_rank):
 
     e2e_serial_step()
     torch.cuda.synchronize()
-    barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
     n_serial = max(2, min(args.e2e_steps, 5))
-    for _ in range(n_serial):
-        e2e_serial_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms_e2e_serial = max_over_ranks(e0.elapsed_time(e1), world, dev) / n_serial
+    ms_e2e_serial = timed_region(e2e_serial_step, n_serial, stream, world, dev, barrier, with_clocks=False)[0]
 
     # (b) pipelined: step i's host->device copies (stream h2d) and step i-1's
     # device->host read-back (stream d2h) overlap step i-1's / i's kernels
@@ -476,7 +562,7 @@ def run_native(args, rank, world, local_rank):
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
     e2e_value = aggregate_tflops(flops_step, world, ms_e2e)
-    del d_alt, outs_alt
+    del d_alt, outs_alt, rope_ws
 
     if world > 1:
         import torch.distributed as dist
@@ -485,9 +571,16 @@ def run_native(args, rank, world, local_rank):
         return None, None
 
     pk, pk_src = peaks()
-    t_self = per_kernel["attn_self"]
-    achieved = f_self / (t_self * 1e-3) / 1e12
-    peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
+    t_self = per_kernel["attn_self_rope_fused"]
+    roof = tensor_roofline("attn_fwd with the 3D RoPE fused into the Q load (31200 x 31200, H=40, D=128): the "
+                           "regen_attn_fwd_rope3d call, whose table and K-pass launches are included in its time",
+                           f_self, t_self, ms_total, clk, pk, pk_src)
+    roof["traffic"] = traffic_from_profile()
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    if "cycles_per_launch" in roof:
+        ctas = B * H * -(-S // 256)
+        roof["sm_cycles_per_key_block"] = round(roof["cycles_per_launch"] * n_sm / (ctas * -(-S // 128)), 1)
+    med = statistics.median
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -502,46 +595,54 @@ def run_native(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic (seeded splitmix64 normals; RMSNormed Q/K; no weights involved)",
         "config": step_config(world),
-        "roofline": {
-            "bound": "tensor",
-            "kernel": "attn_fwd (self-attention, 31200 x 31200, H=40, D=128)",
-            "achieved": round(achieved, 2),
-            "peak": peak,
-            "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4),
-            "peak_source": f"{pk_src} bf16_tflops_sustained (kernel timed inside a back-to-back loop)",
-            "frac_of_burst_peak": round(achieved / float(pk["bf16_tflops"]), 4),
-            "frac_of_nominal_2250": round(achieved / 2250.0, 4),
-            "traffic": traffic_from_profile(),
-            "algorithmic_flops_per_launch": f_self,
-        },
+        "roofline": roof,
         "kernels_ms": {n: round(t, 4) for n, t in per_kernel.items()},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(ms_e2e, 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-                "how": "pinned host inputs -> device -> the five launches -> outputs and LSEs to pinned host "
-                       "every step; copies on their own streams overlap the neighbouring steps' kernels "
-                       "(two device buffer sets); timed from the first copy to the last read-back",
+                "how": "pinned host inputs -> device -> the step's two C-ABI calls (four launches) -> outputs and "
+                       "LSEs to pinned host every step; copies on their own streams overlap the neighbouring "
+                       "steps' kernels (two device buffer sets); timed from the first copy to the last read-back",
                 "serial_ms_per_step": round(ms_e2e_serial, 3),
                 "serial_value": round(aggregate_tflops(flops_step, world, ms_e2e_serial), 2)},
         "clocks": clk,
     }
-    line["backward"] = bwd
-    line["fp8"] = fp8
-    line["projections"] = proj
-    line["rope_fused_step"] = {
-        "what": "the same step with regen_attn_fwd_rope3d (RoPE fused into the Q tile load, K rotated into "
-                "workspace) in place of regen_rope3d + regen_attn_fwd; 7 launches per step",
-        "steps": n_alt, "ms_per_step": round(ms_fused, 4),
-        "value": round(aggregate_tflops(flops_step, world, ms_fused), 2), "unit": "TFLOP/s",
+    line["rope_prepass_step"] = {
+        "what": "the same step with the RoPE as a pre-pass (regen_rope3d in place, then regen_attn_fwd) instead of "
+                "fused into the attention's Q load; 3 rounds of n steps alternating with the fused step",
+        "steps_per_round": n_alt,
+        "ms_per_step_rounds": [round(x, 4) for x in pre_ms],
+        "fused_ms_per_step_rounds": [round(x, 4) for x in fused_ms],
+        "ms_per_step": round(med(pre_ms), 4), "fused_ms_per_step": round(med(fused_ms), 4),
+        "fused_minus_prepass_ms": round(med(fused_ms) - med(pre_ms), 4),
+        "value": round(aggregate_tflops(flops_step, world, med(pre_ms)), 2), "unit": "TFLOP/s",
+        "kernels_ms": {n: round(med(x), 4) for n, x in pre_k.items()},
+        "attn_self_plain_tflops": round(f_self / (med(pre_k["attn_self"]) * 1e-3) / 1e12, 2),
     }
-    s_merge = per_kernel["lse_merge"]
-    s_rope = per_kernel["rope3d"]
+    f_ref = 4.0 * B * H * S * N_REF * D
+    line["cross_attention"] = {
+        "what": "cross-attention of the 31200 video tokens to 1560 reference-frame + 512 conditioning keys: the "
+                "step's one two-source launch, the Ring form (one call per key block merged by regen_lse_merge) "
+                "and one call over the keys concatenated in one buffer",
+        "ms": {n: round(x, 4) for n, x in cross_ms.items()},
+        "kv2_tflops": round(f_cross / (cross_ms["kv2"] * 1e-3) / 1e12, 2),
+        "two_calls_plus_merge_ms": round(cross_ms["ref_block"] + cross_ms["ctx_block"] + cross_ms["lse_merge"], 4),
+        "ref_block_tflops": round(f_ref / (cross_ms["ref_block"] * 1e-3) / 1e12, 2),
+        "ctx_block_tflops": round((f_cross - f_ref) / (cross_ms["ctx_block"] * 1e-3) / 1e12, 2),
+    }
+    s_merge = cross_ms["lse_merge"]
+    s_rope = med(pre_k["rope3d"])
     line["hbm"] = {
         "rope3d_gbs": round(4 * B * H * S * D * 2 / (s_rope * 1e-3) / 1e9, 1),
         "lse_merge_gbs": round((3 * B * H * S * D * 2 + 3 * B * H * S * 4) / (s_merge * 1e-3) / 1e9, 1),
         "peak_gbs": float(pk["hbm_gbs"]),
+        "rope3d_frac": round(4 * B * H * S * D * 2 / (s_rope * 1e-3) / 1e9 / float(pk["hbm_gbs"]), 4),
+        "lse_merge_frac": round((3 * B * H * S * D * 2 + 3 * B * H * S * 4) / (s_merge * 1e-3) / 1e9
+                                / float(pk["hbm_gbs"]), 4),
     }
+    line["backward"] = bwd
+    line["fp8"] = fp8
+    line["projections"] = proj
     return line, snap
 
 
@@ -585,19 +686,14 @@ def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, bar
     torch.cuda.synchronize()
     n = max(3, min(args.steps, 10))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n)]
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(n):
-        step(evs[i])
-    torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(evs[0][0].elapsed_time(evs[n - 1][4]), world, dev) / n
+    ms, clk, region = timed_region(lambda it=iter(evs): step(next(it)), n, stream, world, dev, barrier)
     per = {nm: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n)) / n for j, nm in enumerate(names)}
     f_self, f_cross = step_flops()
     flops = 2.5 * (f_self + f_cross)      # S, dP, dV, dK, dQ: five products of the forward's two sizes
     pk, pk_src = peaks()
-    peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
-    achieved = 2.5 * f_self / (per["attn_bwd_self"] * 1e-3) / 1e12
+    roof = tensor_roofline("regen_attn_bwd self-attention (prep + dK/dV + dQ launches)", 2.5 * f_self,
+                           per["attn_bwd_self"], region, clk, pk, pk_src)
+    roof["issued_tensor_flops_frac"] = round(roof["frac"] * 7 / 5, 4)
     del work
     return {
         "what": "gradient step of the same window: regen_attn_bwd (self) + regen_rope3d_bwd + regen_attn_bwd per "
@@ -608,11 +704,8 @@ def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, bar
                       "recompute QK^T and dO V^T once more (7 products in all, no atomics)",
         "kernels_ms": {nm: round(t, 4) for nm, t in per.items()},
         "launches_per_step": 3 + 1 + 3 + 3,
-        "roofline": {"bound": "tensor", "kernel": "regen_attn_bwd self-attention (prep + dK/dV + dQ launches)",
-                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4),
-                     "peak_source": f"{pk_src} bf16_tflops_sustained",
-                     "issued_tensor_flops_frac": round(achieved * 7 / 5 / peak, 4)},
+        "roofline": roof,
+        "clocks": clk,
     }
 
 
@@ -657,27 +750,19 @@ def run_proj(args, rg, synth, ws, dev, stream, world, barrier, to_dev, rank):
     def cublas_out():
         torch.matmul(om, wo.t(), out=reso)
 
-    def timed(fn, n):
+    def timed(fn, n, clocks=False):
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        return max_over_ranks(e0.elapsed_time(e1), world, dev) / n
+        return timed_region(fn, n, stream, world, dev, barrier, with_clocks=clocks)
 
     n = max(5, min(args.steps, 40))
-    t_qkv, t_out = timed(qkv, n), timed(outp, n)
-    t_cq, t_co = timed(cublas_qkv, n), timed(cublas_out, n)
+    t_qkv, clk_qkv, region_qkv = timed(qkv, n, clocks=True)
+    t_out = timed(outp, n)[0]
+    t_cq, t_co = timed(cublas_qkv, n)[0], timed(cublas_out, n)[0]
     f_qkv = 2.0 * B * S * C * 3 * H * D
     f_out = 2.0 * B * S * H * D * C
     pk, pk_src = peaks()
-    peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
     tf = lambda f, ms: f / (ms * 1e-3) / 1e12  # noqa: E731
     del work, x, w, wo, o, q, k, v, y, res, reso, om
     return {
@@ -690,9 +775,8 @@ def run_proj(args, rg, synth, ws, dev, stream, world, barrier, to_dev, rank):
                      "cublas_gemm_ms": round(t_cq, 4), "cublas_tflops": round(tf(f_qkv, t_cq), 2)},
         "out_proj": {"ms": round(t_out, 4), "tflops": round(tf(f_out, t_out), 2), "M": B * S, "N": C, "K": H * D,
                      "cublas_gemm_ms": round(t_co, 4), "cublas_tflops": round(tf(f_out, t_co), 2)},
-        "roofline": {"bound": "tensor", "kernel": "proj_gemm_kernel<QKV> (31200 x 15360 x 5120)",
-                     "achieved": round(tf(f_qkv, t_qkv), 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(tf(f_qkv, t_qkv) / peak, 4), "peak_source": f"{pk_src} bf16_tflops_sustained"},
+        "roofline": tensor_roofline("proj_gemm_kernel<QKV> (31200 x 15360 x 5120)", f_qkv, t_qkv, region_qkv, clk_qkv,
+                                    pk, pk_src),
         "launches_per_step": 3,
     }
 
@@ -726,19 +810,11 @@ def run_fp8(args, rg, d, ws, dev, stream, world, barrier):
     torch.cuda.synchronize()
     n = max(3, min(args.steps, 20))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(n):
-        step(evs[i])
-    torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(evs[0][0].elapsed_time(evs[n - 1][2]), world, dev) / n
+    ms, clk, region = timed_region(lambda it=iter(evs): step(next(it)), n, stream, world, dev, barrier)
     t_q = sum(e[0].elapsed_time(e[1]) for e in evs) / n
     t_a = sum(e[1].elapsed_time(e[2]) for e in evs) / n
     f_self = step_flops()[0]
     pk, pk_src = peaks()
-    peak8 = 2.0 * float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
-    achieved = f_self / (t_a * 1e-3) / 1e12
     qbytes = 3 * B * H * S * D * 3 + 3 * B * H * nb * 4    # read bf16, write codes, write scales
     return {
         "what": "FP8 (E4M3) variant of the 77-frame self-attention after its RoPE: blockwise quantisation of Q, K, V "
@@ -747,10 +823,9 @@ def run_fp8(args, rg, d, ws, dev, stream, world, barrier):
         "value": round(aggregate_tflops(f_self, world, ms), 2), "unit": "TFLOP/s",
         "kernels_ms": {"quant_e4m3_x3": round(t_q, 4), "attn_fwd_fp8": round(t_a, 4)},
         "quant_gbs": round(qbytes / (t_q * 1e-3) / 1e9, 1),
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_fp8 (31200 x 31200, H=40, D=128)",
-                     "achieved": round(achieved, 2), "peak": peak8, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak8, 4),
-                     "peak_source": f"{pk_src} bf16_tflops_sustained x 2 (dense E4M3 : BF16 nominal ratio)"},
+        "roofline": tensor_roofline("attn_fwd_fp8 (31200 x 31200, H=40, D=128)", f_self, t_a, region, clk, pk, pk_src,
+                                    peak_mult=2.0, peak_note="dense E4M3 : BF16 nominal ratio"),
+        "clocks": clk,
         "launches_per_step": 4,
     }
 
@@ -766,8 +841,10 @@ def cpu_sample_rate(target_s: float, seed_rows: int = 0, snap=None):
     import oracle
     from dit_attention_b200 import synth
     w = synth.WORKLOADS[SELF]
-    if snap is not None:
-        qr, kr, v = snap["q"], snap["k"], snap["v"]
+    if snap is not None:   # the step's unrotated inputs: the oracle applies the RoPE itself (not timed)
+        qr = oracle.rope3d(snap["q"], snap["grid"], snap["theta"])
+        kr = oracle.rope3d(snap["k"], snap["grid"], snap["theta"])
+        v = snap["v"]
     else:
         qr, kr, v = synth.make_inputs(w)
     rng = np.random.default_rng(seed_rows)
@@ -817,7 +894,8 @@ def accuracy(snap, kept):
     rms = float(np.sqrt(np.mean(ref ** 2))) or 1.0
     lse_err = np.abs(snap["lse"].reshape(-1)[kept["rows"]].astype(np.float64) - kept["lse"].reshape(-1))
     within = bool(np.all(err <= 1e-2 + 1e-2 * np.abs(ref)) and np.all(lse_err <= 1e-3))
-    return {"rows": int(len(kept["rows"])), "inputs": "the last timed step's bf16 q, k (after its RoPE), v",
+    return {"rows": int(len(kept["rows"])),
+            "inputs": "the last timed step's bf16 q, k, v; the oracle applies the 3D RoPE to q and k itself",
             "max_abs_err": float(err.max()), "max_err_over_rms": float(err.max() / rms),
             "mean_rel_err": float(np.mean(err) / (np.mean(np.abs(ref)) or 1.0)),
             "max_lse_err": float(lse_err.max()), "contract": "|out-ref| <= 1e-2 + 1e-2|ref|, |lse-ref| <= 1e-3",
