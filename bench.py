@@ -55,6 +55,13 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     p.add_argument("--configs", action="store_true",
                    help="instead of the step: CUDA-event medians of every workload's kernels (1 GPU)")
+    p.add_argument("--profile-case", choices=["attn", "fused", "kv2", "rope", "merge", "bwd", "fp8"], default=None,
+                   help="instead of the step: a short, bounded launch sequence of one kernel for ncu (no timing)")
+    p.add_argument("--heads", type=int, default=8, help="--profile-case: heads")
+    p.add_argument("--seq", type=int, default=31200, help="--profile-case: query tokens (31200, 10920 or 1024)")
+    p.add_argument("--kv", type=int, default=0, help="--profile-case: key count (default --seq; kv2: 1560 + rest)")
+    p.add_argument("--dim", type=int, default=128, help="--profile-case: head dimension")
+    p.add_argument("--iters", type=int, default=2, help="--profile-case: calls of the kernel")
     return p.parse_args()
 
 
@@ -985,6 +992,62 @@ def run_configs(args):
                     "between launches); TFLOP/s = 4 B H Sq Skv D / time", "configs": rows}
 
 
+PROFILE_GRIDS = {31200: (20, 30, 52), 10920: (7, 30, 52), 1024: (1, 32, 32)}
+
+
+def run_profile_case(args):
+    """One kernel of the hot path on a synthetic shape, --iters calls, for a
+    profiler (ncu): attn (self-attention over --seq keys, or --kv for
+    cross-attention), fused (the RoPE-fused self-attention: table, K pass and
+    attention launches), kv2 (two-source cross-attention: 1560 reference keys
+    plus the rest of --kv), rope (3D RoPE on the latent grid of --seq), merge
+    (two-block LSE merge), bwd (one forward, then gradient calls: prep, dK/dV
+    and dQ launches each) or fp8 (Q, K, V quantised once, then FP8 attention
+    calls). No timing is done here."""
+    import torch
+    import dit_attention_b200 as rg
+    from dit_attention_b200 import synth
+    skv = args.kv or args.seq
+    w = synth.Workload("profile", B=1, H=args.heads, D=args.dim, Sq=args.seq, Skv=skv, seed=7)
+    q, k, v = synth.make_inputs(w)
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+    dq, dk, dv = dev(q), dev(k), dev(v)
+    rg.load()
+    scale = 1.0 / math.sqrt(args.dim)
+    if args.kernel_case == "bwd":
+        out, lse = rg.attn_fwd(dq, dk, dv, scale)
+        g = dev(synth.make_dout(w))
+    if args.kernel_case == "fp8":
+        quant = [rg.quant_e4m3(x) for x in (dq, dk, dv)]
+    if args.kernel_case == "kv2":
+        n_ref = min(N_REF, skv - 1)
+        ka, va = dk[:, :, :n_ref].contiguous(), dv[:, :, :n_ref].contiguous()
+        kb, vb = dk[:, :, n_ref:].contiguous(), dv[:, :, n_ref:].contiguous()
+    for _ in range(args.iters):
+        if args.kernel_case == "fp8":
+            rg.attn_fwd_fp8(*quant[0], *quant[1], *quant[2], scale)
+        elif args.kernel_case == "attn":
+            rg.attn_fwd(dq, dk, dv, scale)
+        elif args.kernel_case == "fused":
+            rg.attn_fwd_rope3d(dq, dk, dv, PROFILE_GRIDS[args.seq], scale=scale)
+        elif args.kernel_case == "kv2":
+            rg.attn_fwd_kv2(dq, ka, va, kb, vb, scale)
+        elif args.kernel_case == "bwd":
+            rg.attn_bwd(dq, dk, dv, out, lse, g, scale)
+        elif args.kernel_case == "rope":
+            rg.rope3d_(dq, dk, PROFILE_GRIDS[args.seq])
+        else:
+            lse = torch.zeros((1, args.heads, args.seq), dtype=torch.float32, device="cuda")
+            rg.lse_merge(dq, lse, dk[:, :, :args.seq], lse)
+    torch.cuda.synchronize()
+    rc, site = rg.regen_last_device_error()
+    if rc != 0:
+        raise SystemExit(f"device error {rc} at wait site {site}")
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -1022,6 +1085,11 @@ def main():
     if args.configs:
         if rank == 0:
             print(json.dumps(run_configs(args)), flush=True)
+        return
+    if args.profile_case:
+        args.kernel_case = args.profile_case
+        if rank == 0:
+            run_profile_case(args)
         return
     if world > 1:
         import datetime

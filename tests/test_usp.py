@@ -277,3 +277,81 @@ def test_ring_attention_backward_with_kernels_two_ranks_one_gpu():
         check_grad(dq, rq[:, :, a:b], f"ring dq rank {r}")
         check_grad(dk, rk[:, :, a:b], f"ring dk rank {r}")
         check_grad(dv, rv[:, :, a:b], f"ring dv rank {r}")
+
+
+def _gpu_usp_case(rank, world, U, R):
+    # Unified sequence parallelism as the pages lay it out, scaled down to
+    # Ulysses 2 x Ring 2 ranks on one GPU: the RoPE of each rank's token shard
+    # at its global positions, the Ulysses all-to-alls, the ring with its LSE
+    # merges, and the backward through all of them, with the library's kernels
+    # as every rank's compute (regen_rope3d_shard, regen_attn_fwd,
+    # regen_lse_merge, regen_attn_bwd, and the RoPE's gradient); the shards and
+    # partial results travel as host tensors over gloo.
+    import dit_attention_b200 as rg
+    torch.cuda.set_device(0)
+    ug, rg_ = usp.usp_groups(U, R)
+    w = synth.Workload("usp", B=1, H=4, D=128, Sq=1040, Skv=1040, seed=9, grid=(2, 20, 26), rope=True, rmsnorm=True)
+    q, k, v = synth.make_inputs(w)
+    g = synth.make_dout(w)
+    a, b = usp.shard_range(w.Sq, rank, world)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
+    tq, tk = dev(q[:, :, a:b]), dev(k[:, :, a:b])
+    T, Hh, Ww = w.grid
+    rg.regen_rope3d_shard(tq, tk, T, Hh, Ww, w.theta, w.B, w.H, w.D, a, b - a, 0)   # RoPE at global positions
+
+    def attn(qh, kh, vh, scale):
+        o, l = rg.attn_fwd(qh.detach().cuda().contiguous(), kh.detach().cuda().contiguous(),
+                           vh.detach().cuda().contiguous(), scale)
+        return o.cpu(), l.cpu()
+
+    def merge(oa, la, ob, lb):
+        o, l = rg.lse_merge(oa.cuda(), la.cuda(), ob.cuda(), lb.cuda())
+        return o.cpu(), l.cpu()
+
+    def bwd(q_, k_, v_, out, lse, dout, scale, dq, dk, dv, acc_dq, acc_dkdv):
+        c = lambda t: t.detach().cuda().contiguous()  # noqa: E731
+        r = rg.attn_bwd(c(q_), c(k_), c(v_), c(out), c(lse), c(dout), scale, dq=c(dq), dk=c(dk), dv=c(dv),
+                        accumulate_dq=acc_dq, accumulate_dkdv=acc_dkdv)
+        return tuple(t.cpu() for t in r)
+
+    leaf = lambda t: t.cpu().requires_grad_(True)  # noqa: E731
+    lq, lk = leaf(tq), leaf(tk)
+    lv = torch.from_numpy(np.ascontiguousarray(v[:, :, a:b]).view(np.int16)).view(torch.bfloat16).requires_grad_(True)
+    out = usp.usp_attention_autograd(lq, lk, lv, ug, rg_, w.scale, attn, merge, bwd)
+    gout = torch.from_numpy(np.ascontiguousarray(g[:, :, a:b]).view(np.int16)).view(torch.bfloat16)
+    out.backward(gout)
+    # the RoPE's gradient of this rank's shard, at its global positions
+    gq, gk = lq.grad.cuda().contiguous(), lk.grad.cuda().contiguous()
+    rg.regen_rope3d_shard(gq, gk, T, Hh, Ww, w.theta, w.B, w.H, w.D, a, b - a, 1)
+    torch.cuda.synchronize()
+    bits = lambda t: t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    return (bits(out), bits(lq.grad), bits(lk.grad), bits(lv.grad), bits(gq), bits(gk), bits(tq), bits(tk), a, b)
+
+
+@pytest.mark.gpu
+def test_usp_ulysses2_ring2_forward_and_backward_with_kernels_four_ranks_one_gpu():
+    from util import check_attention, check_grad
+    assert torch.cuda.is_available()
+    res = _run(4, _gpu_usp_case, 2, 2)
+    assert sorted(res) == [0, 1, 2, 3]
+    w = synth.Workload("usp", B=1, H=4, D=128, Sq=1040, Skv=1040, seed=9, grid=(2, 20, 26), rope=True, rmsnorm=True)
+    q, k, v = synth.make_inputs(w)
+    g = synth.make_dout(w)
+    qr, kr = oracle.rope3d(q, w.grid, w.theta), oracle.rope3d(k, w.grid, w.theta)
+    ref, rl = oracle.attention(qr, kr, v, w.scale)
+    rq, rk, rv = oracle.attention_bwd(qr, kr, v, g, w.scale)
+    for r, (o, dq, dk, dv, gq, gk, tq, tk, a, b) in res.items():
+        np.testing.assert_array_equal(tq, qr[:, :, a:b])            # sharded RoPE == whole-grid RoPE
+        np.testing.assert_array_equal(tk, kr[:, :, a:b])
+        check_attention(o.reshape(-1, 128), None, ref[:, :, a:b].reshape(-1, 128), rl[:, :, a:b].reshape(-1),
+                        f"usp out rank {r}")
+        # gradients with respect to the rotated shards, against the oracle's chain rule over the whole window
+        check_grad(dq, rq[:, :, a:b], f"usp dq rank {r}")
+        check_grad(dk, rk[:, :, a:b], f"usp dk rank {r}")
+        check_grad(dv, rv[:, :, a:b], f"usp dv rank {r}")
+        # the RoPE's gradient of the shard at its global positions, bit for bit
+        full_q = np.zeros_like(q)
+        full_k = np.zeros_like(k)
+        full_q[:, :, a:b], full_k[:, :, a:b] = dq, dk
+        np.testing.assert_array_equal(gq, oracle.rope3d_bwd(full_q, w.grid, w.theta)[:, :, a:b], f"rank {r}")
+        np.testing.assert_array_equal(gk, oracle.rope3d_bwd(full_k, w.grid, w.theta)[:, :, a:b], f"rank {r}")
