@@ -144,8 +144,59 @@ struct AttnCfg {
     static constexpr int EMU_PER8 = REGEN_FWD_EXP2_EMU_PER8;
 };
 
-// RoPE (rope_tab.t32 not null, single key source): the Q tiles are rotated by
-// the 3D RoPE in shared memory right after
+// The RoPE of one row of a Q tile in shared memory (128-byte swizzled rows:
+// 16-byte chunk cw of row r sits at chunk cw ^ (r & 7)), for token n (rows
+// past Sq are left alone). The row's 64 fp32 (cos, sin) pairs depend only on
+// its token, so they are loaded before the wait for the tile's TMA load. Two
+// passes: every pair in fp32, stored where its certificate holds (the others
+// keep their input and a bit in `redo`); then the few uncertified pairs in
+// fp64 from the fp64 table. The fp32 pass has no branch, and the fp64 one
+// runs only as often as the warp's most unlucky lane needs it.
+// Returns the wait's outcome, made warp-uniform.
+template <int HD>
+__device__ __forceinline__ bool rope_q_tile_row(uint8_t *tile, int row, int n, int Sq, uint32_t bar_q, WaitCtl wc,
+                                                RopeTabs rope_tab, RopeGeom rope_geom)
+{
+    constexpr int DH = 2 * (HD / 6), DT = HD - 2 * DH;   // axis widths t, h, w = DT, DH, DH
+    constexpr int NP = HD / 2;                           // pairs per row
+    constexpr int HALF_BYTES = 128 * 128;
+    const bool live = n < Sq;
+    const RopeRowEntries re = RopeRowEntries::of(rope_geom, live ? n : 0);
+    float2 cs[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) cs[p] = __ldg(rope_tab.t32 + re.entry(2 * p, DT, DH));
+    const bool ok = __all_sync(0xffffffffu, wait_phase(bar_q, 0, SITE_SM_Q, wc));
+    if (ok && live) {
+        uint8_t *rowp = tile + row * 128;
+        auto chunk = [&](int c) {
+            return reinterpret_cast<uint4 *>(rowp + (c >> 3) * HALF_BYTES + (((c & 7) ^ (row & 7)) << 4));
+        };
+        uint64_t redo = 0;   // bit p: pair p was not certified
+#pragma unroll
+        for (int c = 0; c < HD / 8; ++c) {
+            const uint4 v = *chunk(c);
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                uint32_t r;
+                const bool certified = rotate_pair_f32(w[p], cs[4 * c + p].x, cs[4 * c + p].y, r);
+                redo |= static_cast<uint64_t>(!certified) << (4 * c + p);
+                w[p] = certified ? r : w[p];
+            }
+            *chunk(c) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        while (redo) {
+            const int p = __ffsll(static_cast<long long>(redo)) - 1;
+            redo &= redo - 1;
+            uint32_t *pair = reinterpret_cast<uint32_t *>(chunk(p >> 2)) + (p & 3);
+            const int64_t e = re.entry(2 * p, DT, DH);
+            *pair = rotate_pair(*pair, __ldg(rope_tab.t64 + 2 * e), __ldg(rope_tab.t64 + 2 * e + 1));
+        }
+    }
+    return ok;
+}
+
+// ROPE_Q: the Q tiles are rotated by the 3D RoPE in shared memory right after
 // their TMA load (each softmax thread rotates its own row, from the (cos, sin)
 // table `rope_tab`), before the first S MMA of that tile reads them; the
 // rotation gives the same bits as rope_stream_kernel (fp32 with a per-pair
@@ -155,9 +206,9 @@ struct AttnCfg {
 // the attention over the two sources concatenated. The blocks of source 1 come
 // first, then those of source 2; each source's last block is masked past its
 // own end. (Other instantiations ignore tm_k2, tm_v2 and Skv1.)
-// The RoPE choice is a run-time flag, not a template parameter, so that the
-// plain and the RoPE-fused attention run the same compiled main loop.
-template <int HD, bool NEG_SCALE, bool KV2 = false>
+// The plain instantiation holds no RoPE code at all (a run-time flag, or the
+// prologue in one instantiation, measurably changed the main loop's code).
+template <int HD, bool NEG_SCALE, bool ROPE_Q, bool KV2 = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -165,7 +216,8 @@ __global__ void __launch_bounds__(384, 1)
                     float *__restrict__ lse, int Sq, int Skv, int Skv1, float scale_log2,
                     uint64_t wait_limit_ns, RopeTabs rope_tab, RopeGeom rope_geom)
 {
-    const bool rope_q = !KV2 && rope_tab.t32 != nullptr;
+    static_assert(!(ROPE_Q && KV2), "the RoPE-fused attention has one key source");
+    constexpr bool rope_q = ROPE_Q;
     using C = AttnCfg<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -454,34 +506,9 @@ __global__ void __launch_bounds__(384, 1)
         float m = 0.f;   // running max of scaled logits (log2 units); set by block 0
         float l = 0.f;   // running sum of 2^(s - m)
         bool ok = true;
-        if (rope_q) {
-            // Rotate this thread's row of its Q tile in place in shared memory
-            // (128-byte swizzled rows: 16-byte chunk cw of row r sits at chunk
-            // cw ^ (r & 7)), then hand the tile to the S issuer. The row's 64
-            // fp32 (cos, sin) pairs depend only on its token, so they are
-            // loaded while the Q tile is still on its way from HBM.
-            constexpr int DH = 2 * (HD / 6), DT = HD - 2 * DH;   // axis widths t, h, w = DT, DH, DH
-            constexpr int NP = HD / 2;                           // pairs per row
-            const int n = q0 + t * C::BM + row;
-            const bool live = n < Sq;
-            const RopeRowEntries re = RopeRowEntries::of(rope_geom, live ? n : 0);
-            float2 cs[NP];
-#pragma unroll
-            for (int p = 0; p < NP; ++p) cs[p] = __ldg(rope_tab.t32 + re.entry(2 * p, DT, DH));
-            ok = __all_sync(0xffffffffu, wait_phase(bar_q, 0, SITE_SM_Q, wc));
-            if (ok && live) {
-                uint8_t *rowp = smem + C::Q_OFF + t * C::TILE_BYTES + row * 128;
-#pragma unroll
-                for (int c = 0; c < HD / 8; ++c) {
-                    uint4 *ptr = reinterpret_cast<uint4 *>(rowp + (c >> 3) * C::HALF_BYTES + (((c & 7) ^ (row & 7)) << 4));
-                    const uint4 v = *ptr;
-                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int p = 0; p < 4; ++p)
-                        w[p] = rotate_pair_tab(w[p], cs[4 * c + p], rope_tab.t64, re.entry(8 * c + 2 * p, DT, DH));
-                    *ptr = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
+        if constexpr (rope_q) {
+            ok = rope_q_tile_row<HD>(smem + C::Q_OFF + t * C::TILE_BYTES, row, q0 + t * C::BM + row, Sq, bar_q, wc,
+                                     rope_tab, rope_geom);
             fence_proxy_async_smem();
             mbar_arrive(bar_qrot(t));
         }

@@ -334,7 +334,7 @@ int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, r
     using C = regen::AttnCfg<HD>;
     static PerContext<int> ready;
     const int attr_status = ready.get([](int *) {
-        return kernel_setup(reinterpret_cast<const void *>(regen::attn_fwd_kernel<HD, NEG, KV2>),
+        return kernel_setup(reinterpret_cast<const void *>(regen::attn_fwd_kernel<HD, NEG, ROPE_Q, KV2>),
                             C::SMEM_BYTES, C::MIN_LAUNCH_REGS);
     }, nullptr);
     if (attr_status != REGEN_OK) return attr_status;
@@ -355,8 +355,7 @@ int launch_attn(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, r
     if (grid > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
     const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     static_assert(!(ROPE_Q && KV2), "the RoPE-fused attention has one key source");
-    if (ROPE_Q != (rope_tab.t32 != nullptr)) return REGEN_ERR_INVALID_ARG;   // the kernel keys on the table
-    regen::attn_fwd_kernel<HD, NEG, KV2><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
+    regen::attn_fwd_kernel<HD, NEG, ROPE_Q, KV2><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(
         tq, tk, tv, to, tk2, tv2, lse, Sq, Skv, Skv1, scale_log2, g_wait_limit_ns.load(), rope_tab, geom);
     return launched();
 }

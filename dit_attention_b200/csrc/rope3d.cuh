@@ -99,8 +99,10 @@ __device__ __forceinline__ void rope_angle(int pos, double freq, double &c, doub
 }
 
 // Geometry of the 3D RoPE for a latent grid and head dim: axis blocks t, h, w
-// of widths dt, dh, dh; table of (cos, sin) per (axis, position, pair) laid
-// out as [T][dt/2] then [Hh][dh/2] then [Ww][dh/2] entries of two doubles.
+// of widths dt, dh, dh, and T*dt/2 + (Hh + Ww)*dh/2 (cos, sin) table entries.
+// entry(n, d) indexes the position-major layout [T][dt/2], [Hh][dh/2],
+// [Ww][dh/2] of the projection epilogue's table; the fused attention's table
+// is pair-major (RopeRowEntries).
 struct RopeGeom {
     int T, Hh, Ww, dt, dh;
     __host__ __device__ static RopeGeom make(int T, int Hh, int Ww, int D)
@@ -127,24 +129,34 @@ struct RopeGeom {
     }
 };
 
-// Table entries of a token's three axis blocks: the pair starting at head
-// dimension d < dt has entry t0 + d/2, then h0 + (d - dt)/2, then w0 + (d - dt - dh)/2.
+// The RoPE table of the fused attention, pair-major within each axis block:
+// entries [dt/2][T], then [dh/2][Hh], then [dh/2][Ww] (pair j of position p of
+// the t axis is entry j*T + p, and so on). Consecutive tokens differ mostly in
+// their w position, so a warp's 32 rows read 32 consecutive entries of one
+// pair (and broadcast entries for t and h): coalesced loads. t0, h0, w0: the
+// token's entries of pair 0 in each block; a pair j further is j*T, j*Hh, j*Ww on.
 struct RopeRowEntries {
     int64_t t0, h0, w0;
+    int T, Hh, Ww;
     __device__ __forceinline__ static RopeRowEntries of(const RopeGeom &g, int n)
     {
         RopeRowEntries r;
         const int t = n / (g.Hh * g.Ww), y = (n / g.Ww) % g.Hh, x = n % g.Ww;
         const int64_t base_h = static_cast<int64_t>(g.T) * (g.dt / 2);
         const int64_t base_w = base_h + static_cast<int64_t>(g.Hh) * (g.dh / 2);
-        r.t0 = static_cast<int64_t>(t) * (g.dt / 2);
-        r.h0 = base_h + static_cast<int64_t>(y) * (g.dh / 2);
-        r.w0 = base_w + static_cast<int64_t>(x) * (g.dh / 2);
+        r.t0 = t;
+        r.h0 = base_h + y;
+        r.w0 = base_w + x;
+        r.T = g.T;
+        r.Hh = g.Hh;
+        r.Ww = g.Ww;
         return r;
     }
     __device__ __forceinline__ int64_t entry(int d, int dt, int dh) const
     {
-        return d < dt ? t0 + d / 2 : (d < dt + dh ? h0 + (d - dt) / 2 : w0 + (d - dt - dh) / 2);
+        return d < dt ? t0 + static_cast<int64_t>(d / 2) * T
+                      : (d < dt + dh ? h0 + static_cast<int64_t>((d - dt) / 2) * Hh
+                                     : w0 + static_cast<int64_t>((d - dt - dh) / 2) * Ww);
     }
 };
 
@@ -156,25 +168,8 @@ struct RopeTabs {
     const float2 *t32;
 };
 
-// The fp64 rotation from fp64 table entry e (out of line: one copy of the
-// cold path keeps unrolled callers small for the instruction cache).
-__device__ __noinline__ uint32_t rotate_pair_tab64(uint32_t packed, const double *__restrict__ t64, int64_t e)
-{
-    return rotate_pair(packed, __ldg(t64 + 2 * e), __ldg(t64 + 2 * e + 1));
-}
-
-// Rotate one packed pair from table entry e: fp32 when the certificate
-// holds, else fp64 from the fp64 entry (rare, so the branch seldom diverges).
-__device__ __forceinline__ uint32_t rotate_pair_tab(uint32_t packed, float2 cs32, const double *__restrict__ t64,
-                                                    int64_t e)
-{
-    uint32_t r;
-    if (__builtin_expect(rotate_pair_f32(packed, cs32.x, cs32.y, r), 1)) return r;
-    return rotate_pair_tab64(packed, t64, e);
-}
-
 // tab64[2e], tab64[2e+1] = cos, sin of every table entry e, and tab32[e]
-// their fp32 roundings (grid-stride).
+// their fp32 roundings (grid-stride; layout of RopeRowEntries).
 __global__ void rope_table_kernel(double *__restrict__ tab64, float2 *__restrict__ tab32, RopeGeom g,
                                   const __grid_constant__ RopeFreqs fr)
 {
@@ -185,13 +180,13 @@ __global__ void rope_table_kernel(double *__restrict__ tab64, float2 *__restrict
     for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n; e += stride) {
         int pos, pair;   // pair: index of the pair within the head dimension
         if (e < base_h) {
-            pos = static_cast<int>(e / (g.dt / 2)); pair = static_cast<int>(e % (g.dt / 2));
+            pos = static_cast<int>(e % g.T); pair = static_cast<int>(e / g.T);
         } else if (e < base_w) {
-            pos = static_cast<int>((e - base_h) / (g.dh / 2));
-            pair = g.dt / 2 + static_cast<int>((e - base_h) % (g.dh / 2));
+            pos = static_cast<int>((e - base_h) % g.Hh);
+            pair = g.dt / 2 + static_cast<int>((e - base_h) / g.Hh);
         } else {
-            pos = static_cast<int>((e - base_w) / (g.dh / 2));
-            pair = (g.dt + g.dh) / 2 + static_cast<int>((e - base_w) % (g.dh / 2));
+            pos = static_cast<int>((e - base_w) % g.Ww);
+            pair = (g.dt + g.dh) / 2 + static_cast<int>((e - base_w) / g.Ww);
         }
         double c, s;
         rope_angle(pos, fr.f[pair], c, s);
