@@ -2,15 +2,17 @@
 
 One step = one pass of the hot path for one denoising step of the 77-frame
 window (B=1, H=40, D=128, latent grid 20 x 30 x 52 -> S = 31200):
-  1. self-attention, 31200 x 31200, with the 3D RoPE fused into the Q load
-     (K rotated once into workspace)                    regen_attn_fwd_rope3d
-  2. cross-attention of the 31200 video tokens to the 1560 reference-frame
+  1. 3D RoPE of Q and K, in place                       regen_rope3d
+  2. self-attention, 31200 x 31200                      regen_attn_fwd
+  3. cross-attention of the 31200 video tokens to the 1560 reference-frame
      and 512 conditioning tokens, one softmax over both key buffers in one
      launch                                             regen_attn_fwd_kv2
-Beside it, timed in alternating rounds on the same box: the step with the
-RoPE as a pre-pass (regen_rope3d + regen_attn_fwd); and the cross-attention
-paths on the step's shapes, including the Ring form (one call per key block
-merged by regen_lse_merge) and one call over concatenated keys.
+Each step rotates the Q/K left by the previous step again: the same work on
+the same shapes. Beside it, timed in rounds alternating with it on the same
+box: the step with the RoPE fused into the attention's Q load
+(regen_attn_fwd_rope3d); and the cross-attention paths on the step's shapes,
+including the Ring form (one call per key block merged by regen_lse_merge)
+and one call over the concatenated keys.
 
 value = attention FLOPs of the step (4*B*H*Sq*Skv*D, self + cross) / device
 time of the step, summed over ranks (weak scaling: every rank runs its own
@@ -224,9 +226,8 @@ def step_config(world):
     ws, wc = synth.WORKLOADS[SELF], synth.WORKLOADS[CROSS]
     T, Hh, Ww = ws.grid
     return {
-        "workload": "win77_s31200 self-attention with the 3D RoPE fused into the Q load, cross-attention to "
-                    "1560 reference + 512 conditioning tokens under one softmax (one denoising step of the "
-                    "77-frame window)",
+        "workload": "win77_s31200 3D RoPE + self-attention, cross-attention to 1560 reference + 512 "
+                    "conditioning tokens under one softmax (one denoising step of the 77-frame window)",
         "B": ws.B, "H": ws.H, "S": ws.Sq, "D": ws.D, "Skv_cross": [N_REF, wc.Skv - N_REF],
         "latent_grid": [T, Hh, Ww], "scale": 1.0 / math.sqrt(ws.D),
         "l2": "inputs larger than L2 (320 MB per tensor vs 126 MB); no flush",
@@ -343,14 +344,14 @@ def run_native(args, rank, world, local_rank):
     rope_ws_bytes = rg.regen_attn_fwd_rope3d_workspace_bytes(B, H, T, Hh, Ww, D)
     rope_ws = torch.empty(rope_ws_bytes, dtype=torch.uint8, device=dev)
 
-    # One step: the self-attention with the 3D RoPE fused into its Q load (the
-    # table, the K pass and the attention: 3 launches; q and k are not
-    # modified, so every step starts from the same inputs) and the
+    # One step: the 3D RoPE of Q and K in place, the self-attention, and the
     # cross-attention to the reference-frame and conditioning keys in one
-    # launch over the two key buffers.
-    names = ["attn_self_rope_fused", "attn_cross_kv2"]
-    LAUNCHES_PER_STEP = 4
+    # launch over the two key buffers. In the timed loop each step rotates the
+    # Q and K the previous step left: the same work on the same shapes.
+    names = ["rope3d", "attn_self", "attn_cross_kv2"]
+    LAUNCHES_PER_STEP = 3
     outs0 = dict(out=out, lse=lse, oc=oc, lc=lc)
+    q_raw, k_raw = d["q"].clone(), d["k"].clone()   # the unrotated inputs, for the fused step and the snapshot
 
     def step(ev=None, inp=None, o=None):
         inp = d if inp is None else inp
@@ -360,12 +361,13 @@ def run_native(args, rank, world, local_rank):
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        rg.regen_attn_fwd_rope3d(inp["q"], inp["k"], inp["v"], o["out"], o["lse"], B, H, S, S, D, scale, sh,
-                                 T, Hh, Ww, ws.theta, rope_ws, rope_ws_bytes)
+        rg.regen_rope3d(inp["q"], inp["k"], T, Hh, Ww, ws.theta, B, H, D, sh)
         mark(1)
+        rg.regen_attn_fwd(inp["q"], inp["k"], inp["v"], o["out"], o["lse"], B, H, S, S, D, scale, sh)
+        mark(2)
         rg.regen_attn_fwd_kv2(inp["qc"], inp["kr"], inp["vr"], inp["kx"], inp["vx"], o["oc"], o["lc"], B, H, S,
                               N_REF, n_ctx, D, scale, sh)
-        mark(2)
+        mark(3)
 
     def barrier():
         if world > 1:
@@ -377,7 +379,7 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     # ---- device-resident timing: K steps between two events, per-call events inside
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     clocks = ClockSampler(dev)
     barrier()
     torch.cuda.synchronize()
@@ -403,52 +405,53 @@ def run_native(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     value = aggregate_tflops(flops_step, world, ms_step)
 
-    # The last timed step's self-attention inputs (unrotated q, k as given to
-    # the fused call) and its output, for the CPU leg's accuracy check (rank 0
-    # only, and only when that leg runs); the oracle rotates q and k itself.
-    snap = None
-    if rank == 0 and not args.no_cpu_baseline:
-        bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
-        snap = dict(q=bits(d["q"]), k=bits(d["k"]), v=bits(d["v"]), out=bits(out), lse=lse.cpu().numpy(),
-                    scale=scale, grid=ws.grid, theta=ws.theta)
+    # ---- the same step with the RoPE fused into the attention's Q load
+    # (regen_attn_fwd_rope3d: the table, the K pass into workspace, the attention
+    # with Q rotated in shared memory; q and k untouched), timed in rounds
+    # alternating with the pre-pass step above, on the same box and clocks.
+    fused_names = ["attn_self_rope_fused", "attn_cross_kv2"]
 
-    # ---- the same step with the RoPE as a pre-pass (regen_rope3d on copies of q, k,
-    # then the plain attention), timed in rounds alternating with the fused step,
-    # on the same box and clocks. Each pre-pass step rotates its copies again: the
-    # same work on the same shapes.
-    qp, kp = d["q"].clone(), d["k"].clone()
-    pre_names = ["rope3d", "attn_self", "attn_cross_kv2"]
-
-    def step_prepass(ev=None):
+    def step_fused(ev=None):
         def mark(i):
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        rg.regen_rope3d(qp, kp, T, Hh, Ww, ws.theta, B, H, D, sh)
+        rg.regen_attn_fwd_rope3d(q_raw, k_raw, d["v"], out, lse, B, H, S, S, D, scale, sh, T, Hh, Ww, ws.theta,
+                                 rope_ws, rope_ws_bytes)
         mark(1)
-        rg.regen_attn_fwd(qp, kp, d["v"], out, lse, B, H, S, S, D, scale, sh)
-        mark(2)
         rg.regen_attn_fwd_kv2(d["qc"], d["kr"], d["vr"], d["kx"], d["vx"], oc, lc, B, H, S, N_REF, n_ctx, D, scale,
                               sh)
-        mark(3)
+        mark(2)
 
     n_alt = max(3, min(args.steps, 10))
     for _ in range(args.warmup):
-        step_prepass()
-    fused_ms, pre_ms, pre_k = [], [], {n: [] for n in pre_names}
+        step_fused()
+    fused_ms, pre_ms, fused_k = [], [], {n: [] for n in fused_names}
     for rnd in range(3):
         for which in ((0, 1) if rnd % 2 == 0 else (1, 0)):
             if which == 0:
                 ms, _, _ = timed_region(step, n_alt, stream, world, dev, barrier, with_clocks=False)
-                fused_ms.append(ms)
-            else:
-                pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_alt)]
-                ms, _, _ = timed_region(lambda it=iter(pev): step_prepass(next(it)), n_alt, stream, world, dev,
-                                        barrier, with_clocks=False)
                 pre_ms.append(ms)
-                for j, n in enumerate(pre_names):
-                    pre_k[n].append(sum(e[j].elapsed_time(e[j + 1]) for e in pev) / n_alt)
-    del qp, kp
+            else:
+                fev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_alt)]
+                ms, _, _ = timed_region(lambda it=iter(fev): step_fused(next(it)), n_alt, stream, world, dev,
+                                        barrier, with_clocks=False)
+                fused_ms.append(ms)
+                for j, n in enumerate(fused_names):
+                    fused_k[n].append(sum(e[j].elapsed_time(e[j + 1]) for e in fev) / n_alt)
+
+    # One more step on the unrotated inputs: its out/lse serve the CPU leg's
+    # accuracy check (rank 0 only, when that leg runs; the oracle gets the
+    # host's unrotated q, k and applies the RoPE itself) and the backward below.
+    d["q"].copy_(q_raw)
+    d["k"].copy_(k_raw)
+    step()
+    torch.cuda.synchronize()
+    snap = None
+    if rank == 0 and not args.no_cpu_baseline:
+        snap = dict(q=host["q"], k=host["k"], v=host["v"],
+                    out=out.contiguous().view(torch.int16).cpu().numpy().view(np.uint16), lse=lse.cpu().numpy(),
+                    scale=scale, grid=ws.grid, theta=ws.theta)
 
     # ---- cross-attention paths on the step's shapes: the one-launch two-source
     # call (the step's), the two key blocks as separate calls merged by
@@ -475,17 +478,13 @@ def run_native(args, rank, world, local_rank):
     del oa, ob, la, lb, kcat, vcat
 
     # ---- backward: the gradient step of the same window (the decoder is trained by
-    # distillation). dO synthetic; the forward's out/lse of the last timed step
-    # (taken before anything else overwrites them).
+    # distillation). dO synthetic; the forward's out/lse of the snapshot step
+    # (its q, k rotated once: the inputs the gradient kernels take).
     # Self: regen_attn_bwd then regen_rope3d_bwd on dq, dk (gradients w.r.t. the
-    # unrotated Q, K); q, k enter it rotated (the pre-pass's output of the same
-    # inputs). Cross: one regen_attn_bwd per key block with the merged out/lse,
-    # the second accumulating dq. Each regen_attn_bwd is 3 launches.
-    step()            # the fused step's out/lse for these inputs
-    qrot, krot = d["q"].clone(), d["k"].clone()
-    rg.regen_rope3d(qrot, krot, T, Hh, Ww, ws.theta, B, H, D, sh)
-    dr = dict(d, q=qrot, k=krot)
-    bwd = run_backward(args, rg, synth, dr, outs0, ws, wc, rank, dev, stream, world, barrier, to_dev)
+    # unrotated Q, K). Cross: one regen_attn_bwd per key block with the merged
+    # out/lse, the second accumulating dq. Each regen_attn_bwd is 3 launches.
+    step_fused()          # cross out/lse again (the cross paths above overwrote them); same self out/lse
+    bwd = run_backward(args, rg, synth, d, outs0, ws, wc, rank, dev, stream, world, barrier, to_dev)
 
     # ---- the projections around the attention of a 14B-class DiT block on the same
     # window: fused QKV projection (+ RMSNorm + RoPE) and the output projection.
@@ -493,8 +492,7 @@ def run_native(args, rank, world, local_rank):
 
     # ---- the FP8 variant of the self-attention (on the rotated q, k): blockwise
     # E4M3 quantisation of Q, K, V (3 launches) and the E4M3 attention.
-    fp8 = run_fp8(args, rg, dr, ws, dev, stream, world, barrier)
-    del qrot, krot, dr
+    fp8 = run_fp8(args, rg, d, ws, dev, stream, world, barrier)
 
     # ---- end to end: pinned host inputs -> device -> hot path -> outputs to pinned host
     pin = {n: torch.from_numpy(a.view(np.int16)).pin_memory() for n, a in host.items()}
@@ -569,7 +567,7 @@ def run_native(args, rank, world, local_rank):
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
     e2e_value = aggregate_tflops(flops_step, world, ms_e2e)
-    del d_alt, outs_alt, rope_ws
+    del d_alt, outs_alt, rope_ws, q_raw, k_raw
 
     if world > 1:
         import torch.distributed as dist
@@ -578,10 +576,9 @@ def run_native(args, rank, world, local_rank):
         return None, None
 
     pk, pk_src = peaks()
-    t_self = per_kernel["attn_self_rope_fused"]
-    roof = tensor_roofline("attn_fwd with the 3D RoPE fused into the Q load (31200 x 31200, H=40, D=128): the "
-                           "regen_attn_fwd_rope3d call, whose table and K-pass launches are included in its time",
-                           f_self, t_self, ms_total, clk, pk, pk_src)
+    t_self = per_kernel["attn_self"]
+    roof = tensor_roofline("attn_fwd self-attention (31200 x 31200, H=40, D=128)", f_self, t_self, ms_total, clk,
+                           pk, pk_src)
     roof["traffic"] = traffic_from_profile()
     n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
     if "cycles_per_launch" in roof:
@@ -607,24 +604,25 @@ def run_native(args, rank, world, local_rank):
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(ms_e2e, 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-                "how": "pinned host inputs -> device -> the step's two C-ABI calls (four launches) -> outputs and "
+                "how": "pinned host inputs -> device -> the step's three C-ABI calls (three launches) -> outputs and "
                        "LSEs to pinned host every step; copies on their own streams overlap the neighbouring "
                        "steps' kernels (two device buffer sets); timed from the first copy to the last read-back",
                 "serial_ms_per_step": round(ms_e2e_serial, 3),
                 "serial_value": round(aggregate_tflops(flops_step, world, ms_e2e_serial), 2)},
         "clocks": clk,
     }
-    line["rope_prepass_step"] = {
-        "what": "the same step with the RoPE as a pre-pass (regen_rope3d in place, then regen_attn_fwd) instead of "
-                "fused into the attention's Q load; 3 rounds of n steps alternating with the fused step",
+    line["rope_fused_step"] = {
+        "what": "the same step with the RoPE fused into the attention's Q load (regen_attn_fwd_rope3d: table, K "
+                "rotated into workspace, Q rotated on its tiles in shared memory) instead of the pre-pass; 3 rounds "
+                "of n steps alternating with the pre-pass step",
         "steps_per_round": n_alt,
-        "ms_per_step_rounds": [round(x, 4) for x in pre_ms],
-        "fused_ms_per_step_rounds": [round(x, 4) for x in fused_ms],
-        "ms_per_step": round(med(pre_ms), 4), "fused_ms_per_step": round(med(fused_ms), 4),
+        "ms_per_step_rounds": [round(x, 4) for x in fused_ms],
+        "prepass_ms_per_step_rounds": [round(x, 4) for x in pre_ms],
+        "ms_per_step": round(med(fused_ms), 4), "prepass_ms_per_step": round(med(pre_ms), 4),
         "fused_minus_prepass_ms": round(med(fused_ms) - med(pre_ms), 4),
-        "value": round(aggregate_tflops(flops_step, world, med(pre_ms)), 2), "unit": "TFLOP/s",
-        "kernels_ms": {n: round(med(x), 4) for n, x in pre_k.items()},
-        "attn_self_plain_tflops": round(f_self / (med(pre_k["attn_self"]) * 1e-3) / 1e12, 2),
+        "value": round(aggregate_tflops(flops_step, world, med(fused_ms)), 2), "unit": "TFLOP/s",
+        "kernels_ms": {n: round(med(x), 4) for n, x in fused_k.items()},
+        "launches_per_step": 4,
     }
     f_ref = 4.0 * B * H * S * N_REF * D
     line["cross_attention"] = {
@@ -638,7 +636,7 @@ def run_native(args, rank, world, local_rank):
         "ctx_block_tflops": round((f_cross - f_ref) / (cross_ms["ctx_block"] * 1e-3) / 1e12, 2),
     }
     s_merge = cross_ms["lse_merge"]
-    s_rope = med(pre_k["rope3d"])
+    s_rope = per_kernel["rope3d"]
     line["hbm"] = {
         "rope3d_gbs": round(4 * B * H * S * D * 2 / (s_rope * 1e-3) / 1e9, 1),
         "lse_merge_gbs": round((3 * B * H * S * D * 2 + 3 * B * H * S * 4) / (s_merge * 1e-3) / 1e9, 1),
@@ -902,7 +900,8 @@ def accuracy(snap, kept):
     lse_err = np.abs(snap["lse"].reshape(-1)[kept["rows"]].astype(np.float64) - kept["lse"].reshape(-1))
     within = bool(np.all(err <= 1e-2 + 1e-2 * np.abs(ref)) and np.all(lse_err <= 1e-3))
     return {"rows": int(len(kept["rows"])),
-            "inputs": "the last timed step's bf16 q, k, v; the oracle applies the 3D RoPE to q and k itself",
+            "inputs": "one more step after the timed ones, on the unrotated bf16 q, k, v; the oracle applies the "
+                      "3D RoPE to q and k itself",
             "max_abs_err": float(err.max()), "max_err_over_rms": float(err.max() / rms),
             "mean_rel_err": float(np.mean(err) / (np.mean(np.abs(ref)) or 1.0)),
             "max_lse_err": float(lse_err.max()), "contract": "|out-ref| <= 1e-2 + 1e-2|ref|, |lse-ref| <= 1e-3",
