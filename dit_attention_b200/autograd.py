@@ -1,7 +1,7 @@
 """torch.autograd glue over the library's forward and gradient kernels.
 
 Argument marshalling only: the forward runs regen_rope3d, regen_attn_fwd and
-regen_lse_merge, the backward runs regen_attn_bwd and regen_rope3d_bwd; no
+regen_attn_fwd_kv2, the backward runs regen_attn_bwd and regen_rope3d_bwd; no
 arithmetic happens here. Tensors are bf16 [B, H, S, D] on the GPU.
 
     dit_attention(q, k, v, grid=None, theta=10000.0, scale=None) -> out
@@ -12,10 +12,10 @@ arithmetic happens here. Tensors are bf16 [B, H, S, D] on the GPU.
     dit_cross_attention(q, (k_a, v_a), (k_b, v_b), scale=None) -> out
         one softmax over the keys of two separately held sources (the DiT's
         reference-frame latents and conditioning tokens, ReGenVC blog page,
-        "Methodology -- deep read"), computed per source and merged by the
-        log-sum-exp. Its gradient runs per source with the MERGED output and
-        LSE, so that each source's P is its slice of the joint softmax, and
-        the two dq shares add up.
+        "Methodology -- deep read"), in one launch over both (regen_attn_fwd_kv2).
+        Its gradient runs per source with the joint output and LSE, so that
+        each source's P is its slice of the joint softmax, and the two dq
+        shares add up.
 """
 from __future__ import annotations
 
@@ -23,7 +23,7 @@ import math
 
 import torch
 
-from . import attn_bwd, attn_fwd, lse_merge, rope3d_, rope3d_bwd_
+from . import attn_bwd, attn_fwd, attn_fwd_kv2, rope3d_, rope3d_bwd_
 
 
 def _scale(scale, q):
@@ -55,9 +55,7 @@ class _TwoSourceAttention(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k_a, v_a, k_b, v_b, scale):
         q, k_a, v_a, k_b, v_b = (t.contiguous() for t in (q, k_a, v_a, k_b, v_b))
-        o_a, l_a = attn_fwd(q, k_a, v_a, scale)
-        o_b, l_b = attn_fwd(q, k_b, v_b, scale)
-        out, lse = lse_merge(o_a, l_a, o_b, l_b)
+        out, lse = attn_fwd_kv2(q, k_a, v_a, k_b, v_b, scale)
         ctx.save_for_backward(q, k_a, v_a, k_b, v_b, out, lse)
         ctx.scale = scale
         return out
