@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t src = sbase + (w ? C::A_DO_OFF : C::A_Q_OFF);
             for (int h = 0; h < C::HALVES; ++h) tma_store_3d(map, src + h * C::HALF_BYTES, h * 64, key0, bh);
             tma_store_commit();
-            tma_store_wait_all();
+            tma_store_wait_read_all();   // only the shared-memory reads must finish before the CTA exits
         }
         tc_fence_before_sync();
         __syncthreads();
@@ -938,7 +938,7 @@ __global__ void __launch_bounds__(384, 1)
             for (int h = 0; h < C::HALVES; ++h)
                 tma_store_3d(&tm_dq, sbase + C::B_Q_OFF + h * C::HALF_BYTES, h * 64, q0, bh);
             tma_store_commit();
-            tma_store_wait_all();
+            tma_store_wait_read_all();   // only the shared-memory reads must finish before the CTA exits
         }
         tc_fence_before_sync();
         __syncthreads();

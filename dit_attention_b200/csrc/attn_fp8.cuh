@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(384, 1)
                 tma_store_3d(&tm_o, sbase + C::K_OFF + t * 2 * C::OUT_HALF + h * C::OUT_HALF, h * 64,
                              q0 + t * C::BM, bh);
             tma_store_commit();
-            tma_store_wait_all();
+            tma_store_wait_read_all();   // only the shared-memory reads must finish before the CTA exits
         }
         tc_fence_before_sync();
         __syncthreads();

@@ -242,6 +242,11 @@ __global__ void __launch_bounds__(384, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF + 8);
 
+    // 1-D grid, query-tile pairs of one head adjacent so that the CTAs resident
+    // at any time share the K/V of one or two heads in L2.
+    const int npairs = (Sq + 2 * C::BM - 1) / (2 * C::BM);
+    const int bh = static_cast<int>(blockIdx.x / npairs);
+    const int q0 = static_cast<int>(blockIdx.x % npairs) * (2 * C::BM);
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
         for (int s = 0; s < C::NSK; ++s) {
@@ -263,6 +268,14 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(bar_qrot(1), 128);
         *abort_flag = 0;
         fence_mbarrier_init();
+        // The Q tiles' loads (this thread is also the Q/K producer) leave now,
+        // ahead of the TMEM allocation and the block-wide barrier.
+        tma_prefetch_desc(&tm_q);
+        mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+        for (int t = 0; t < 2; ++t)
+            for (int h = 0; h < C::HALVES; ++h)
+                tma_load_3d(sbase + C::Q_OFF + t * C::TILE_BYTES + h * C::HALF_BYTES, &tm_q, bar_q, h * 64,
+                            q0 + t * C::BM, bh, l2_policy_evict_first());
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -287,11 +300,6 @@ __global__ void __launch_bounds__(384, 1)
             row = j * C::BN;
         }
     };
-    // 1-D grid, query-tile pairs of one head adjacent so that the CTAs resident
-    // at any time share the K/V of one or two heads in L2.
-    const int npairs = (Sq + 2 * C::BM - 1) / (2 * C::BM);
-    const int bh = static_cast<int>(blockIdx.x / npairs);
-    const int q0 = static_cast<int>(blockIdx.x % npairs) * (2 * C::BM);
 
     // Registers: the producer/MMA warpgroup gives (R - REGS_LOW) per thread back,
     // the two softmax warpgroups take (REGS_HIGH - R) each; the host launches
@@ -329,17 +337,10 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 0) {
         // ------------------------------------------- producer: Q, then K ---
         if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             if (KV2) tma_prefetch_desc(&tm_k2);
             const uint64_t keep = l2_policy_evict_last();   // K: re-read by every Q tile of the head
-            const uint64_t once = l2_policy_evict_first();  // Q: read once
-            mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
-            for (int t = 0; t < 2; ++t)
-                for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_3d(sbase + C::Q_OFF + t * C::TILE_BYTES + h * C::HALF_BYTES, &tm_q, bar_q,
-                                h * 64, q0 + t * C::BM, bh, once);
-            int nk = 0;  // K block loads issued so far
+            int nk = 0;   // (the Q tiles' loads were issued at set-up, evict-first: read once)  // K block loads issued so far
             bool ok = true;
             for (int j = 0; j < nkv; ++j) {
                 const int s = j % C::NSK;
@@ -674,7 +675,7 @@ __global__ void __launch_bounds__(384, 1)
                 tma_store_3d(&tm_o, sbase + C::Q_OFF + t * C::TILE_BYTES + h * C::HALF_BYTES, h * 64,
                              q0 + t * C::BM, bh);
             tma_store_commit();
-            tma_store_wait_all();
+            tma_store_wait_read_all();   // only the shared-memory reads must finish before the CTA exits
         }
         tc_fence_before_sync();
         __syncthreads();
