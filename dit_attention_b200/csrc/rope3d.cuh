@@ -196,6 +196,23 @@ __global__ void rope_table_kernel(double *__restrict__ tab64, float2 *__restrict
     }
 }
 
+// The four pairs of a 16-byte chunk: fp32 with one certificate for the whole
+// chunk; if any pair is not certified (about one chunk in 80), the chunk is
+// redone in fp64 from the fp64 cosines and sines.
+__device__ __forceinline__ uint4 rotate_chunk_f32(uint4 v, const float2 (&cs)[4], const double (&c64)[4],
+                                                  const double (&s64)[4])
+{
+    uint4 r;
+    bool ok = rotate_pair_f32(v.x, cs[0].x, cs[0].y, r.x);
+    ok &= rotate_pair_f32(v.y, cs[1].x, cs[1].y, r.y);
+    ok &= rotate_pair_f32(v.z, cs[2].x, cs[2].y, r.z);
+    ok &= rotate_pair_f32(v.w, cs[3].x, cs[3].y, r.w);
+    if (__builtin_expect(!ok, 0))
+        r = make_uint4(rotate_pair(v.x, c64[0], s64[0]), rotate_pair(v.y, c64[1], s64[1]),
+                       rotate_pair(v.z, c64[2], s64[2]), rotate_pair(v.w, c64[3], s64[3]));
+    return r;
+}
+
 // Walk rows [r0, r1) of one 16-byte chunk (element offset `off` in a row of
 // `row_stride` elements): dst row r = rot(src row r), four rows at a time
 // with the next four rows' loads issued before the current four are stored.
@@ -245,15 +262,10 @@ __global__ void __launch_bounds__(128, 6) rope_apply_kernel(const uint16_t *__re
         c64[p] = __ldg(tab.t64 + 2 * e[p]);
         s64[p] = __ldg(tab.t64 + 2 * e[p] + 1);
     }
-    auto rot1 = [&](uint32_t w, int p) {
-        uint32_t r;
-        if (__builtin_expect(rotate_pair_f32(w, cs[p].x, cs[p].y, r), 1)) return r;
-        return rotate_pair(w, c64[p], s64[p]);
-    };
     const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_group;
     const int64_t r1 = r0 + rows_per_group < rows ? r0 + rows_per_group : rows;
     rope_walk_rows(src, dst, r0, r1, static_cast<int64_t>(S) * D, t * 8, [&](uint4 v) {
-        return make_uint4(rot1(v.x, 0), rot1(v.y, 1), rot1(v.z, 2), rot1(v.w, 3));
+        return rotate_chunk_f32(v, cs, c64, s64);
     });
 }
 
@@ -262,7 +274,7 @@ __global__ void __launch_bounds__(128, 6) rope_apply_kernel(const uint16_t *__re
 // angles come from fp64 sincos once per thread. inverse: the transposed
 // rotation (sine negated), the RoPE's gradient. n0: position of token 0 of
 // this sequence shard on the latent grid.
-__global__ void __launch_bounds__(128, 8) rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k,
+__global__ void __launch_bounds__(128, 7) rope3d_kernel(uint16_t *__restrict__ q, uint16_t *__restrict__ k,
                                                         int64_t rows, int S, int Hh, int Ww, int D,
                                                         const __grid_constant__ RopeFreqs fr, bool inverse, int n0,
                                                         int rows_per_group, int groups)
@@ -280,24 +292,18 @@ __global__ void __launch_bounds__(128, 8) rope3d_kernel(uint16_t *__restrict__ q
     const int dh = 2 * (D / 6);
     const int dt = D - 2 * dh;
     double cs[4], sn[4];
-    float cs32[4], sn32[4];
+    float2 cs2[4];   // their fp32 roundings
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const int d = c * 8 + 2 * p;
         rope_angle(d < dt ? pt : (d < dt + dh ? ph : pw), fr.f[d / 2], cs[p], sn[p]);
         if (inverse) sn[p] = -sn[p];
-        cs32[p] = static_cast<float>(cs[p]);
-        sn32[p] = static_cast<float>(sn[p]);
+        cs2[p] = make_float2(static_cast<float>(cs[p]), static_cast<float>(sn[p]));
     }
-    auto rot1 = [&](uint32_t w, int p) {
-        uint32_t r;
-        if (__builtin_expect(rotate_pair_f32(w, cs32[p], sn32[p], r), 1)) return r;
-        return rotate_pair(w, cs[p], sn[p]);
-    };
     const int64_t r0 = static_cast<int64_t>(blockIdx.y % groups) * rows_per_group;
     const int64_t r1 = r0 + rows_per_group < rows ? r0 + rows_per_group : rows;
     rope_walk_rows(x, x, r0, r1, static_cast<int64_t>(S) * D, static_cast<int64_t>(n) * D + c * 8, [&](uint4 v) {
-        return make_uint4(rot1(v.x, 0), rot1(v.y, 1), rot1(v.z, 2), rot1(v.w, 3));
+        return rotate_chunk_f32(v, cs2, cs, sn);
     });
 }
 
