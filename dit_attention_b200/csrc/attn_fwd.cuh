@@ -519,12 +519,12 @@ __global__ void __launch_bounds__(384, 1)
             ok = __all_sync(0xffffffffu, wait_phase(bar_s_full(t), j & 1, SITE_SM_S_FULL, wc));
             if (!ok) break;
             tc_fence_after_sync();
-            uint32_t sr[4][32];
+            uint32_t sr[2][64];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(ts + c * 32, sr[c]);
+            for (int c = 0; c < 2; ++c) tmem_ld_32x32b_x64(ts + c * 64, sr[c]);
             tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+            for (int c = 0; c < 2; ++c) reg_fence(sr[c]);
             // S is in registers: the buffer may take the other tile's next S.
             tc_fence_before_sync();
             mbar_arrive(bar_s_free);
@@ -536,11 +536,11 @@ __global__ void __launch_bounds__(384, 1)
             float alpha = 1.0f;
             auto block = [&](auto masked_tag) {
                 constexpr bool MASKED = decltype(masked_tag)::value;
-                auto S = [&](int x) { return __uint_as_float(sr[x >> 5][x & 31]); };
+                auto S = [&](int x) { return __uint_as_float(sr[x >> 6][x & 63]); };
                 if constexpr (MASKED) {
 #pragma unroll
                     for (int x = 0; x < 128; ++x)
-                        if (x >= kv_tail) sr[x >> 5][x & 31] = __float_as_uint(NEG_SCALE ? INFINITY : -INFINITY);
+                        if (x >= kv_tail) sr[x >> 6][x & 63] = __float_as_uint(NEG_SCALE ? INFINITY : -INFINITY);
                 }
                 // Row extreme of the raw logits: 8 independent 3-input chains.
                 float acc[8];
@@ -575,7 +575,7 @@ __global__ void __launch_bounds__(384, 1)
                 const uint64_t c2 = f2_pack(scale_log2, scale_log2);
                 const uint64_t nm2 = f2_pack(-m, -m);
                 uint64_t rs2[4] = {0, 0, 0, 0};
-                uint32_t pk[2][32];
+                uint32_t pk[64];
 #pragma unroll
                 for (int hv = 0; hv < 2; ++hv) {   // 64 keys -> 32 packed columns per half
 #pragma unroll
@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(384, 1)
                             if (x + 1 >= kv_tail) p1 = 0.f;
                         }
                         rs2[(i >> 1) & 3] = f2_add(rs2[(i >> 1) & 3], f2_pack(p0, p1));
-                        pk[hv][i >> 1] = pack_bf16x2(p0, p1);
+                        pk[hv * 32 + (i >> 1)] = pack_bf16x2(p0, p1);
                     }
                 }
                 // P_t and O_t are free once PV_t(j-1) has completed.
@@ -604,8 +604,7 @@ __global__ void __launch_bounds__(384, 1)
                     if (!ok) return;
                     tc_fence_after_sync();
                 }
-                tmem_st_32x32b_x32(tp, pk[0]);
-                tmem_st_32x32b_x32(tp + 32, pk[1]);
+                tmem_st_32x32b_x64(tp, pk);
                 float r0, r1, r2, r3;
                 f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), r0, r1);
                 (void)r2;
