@@ -667,7 +667,17 @@ def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, bar
     dkx, dvx = torch.empty_like(d["kx"]), torch.empty_like(d["vx"])
     wsb = rg.regen_attn_bwd_workspace_bytes(B, H, S, D)
     work = torch.empty(wsb, dtype=torch.uint8, device=dev)
-    names = ["attn_bwd_self", "rope3d_bwd", "attn_bwd_cross_ref", "attn_bwd_cross_ctx"]
+    names = ["attn_bwd_self", "rope3d_bwd", "attn_bwd_cross_kv2"]
+
+    def cross_kv2():
+        rg.regen_attn_bwd_kv2(d["qc"], d["kr"], d["vr"], d["kx"], d["vx"], outs["oc"], outs["lc"], g_cross, dqc,
+                              dkr, dvr, dkx, dvx, B, H, S, n_ref, n_ctx, D, scale, sh, work, wsb, 0)
+
+    def cross_per_source():
+        rg.regen_attn_bwd(d["qc"], d["kr"], d["vr"], outs["oc"], outs["lc"], g_cross, dqc, dkr, dvr, B, H, S,
+                          n_ref, D, scale, sh, work, wsb, 0)
+        rg.regen_attn_bwd(d["qc"], d["kx"], d["vx"], outs["oc"], outs["lc"], g_cross, dqc, dkx, dvx, B, H, S,
+                          n_ctx, D, scale, sh, work, wsb, 1)
 
     def step(ev=None):
         def mark(i):
@@ -679,20 +689,29 @@ def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, bar
         mark(1)
         rg.regen_rope3d_bwd(dq, dk, T, Hh, Ww, ws.theta, B, H, D, sh)
         mark(2)
-        rg.regen_attn_bwd(d["qc"], d["kr"], d["vr"], outs["oc"], outs["lc"], g_cross, dqc, dkr, dvr, B, H, S,
-                          n_ref, D, scale, sh, work, wsb, 0)
+        cross_kv2()
         mark(3)
-        rg.regen_attn_bwd(d["qc"], d["kx"], d["vx"], outs["oc"], outs["lc"], g_cross, dqc, dkx, dvx, B, H, S,
-                          n_ctx, D, scale, sh, work, wsb, 1)
-        mark(4)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     n = max(3, min(args.steps, 10))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
     ms, clk, region = timed_region(lambda it=iter(evs): step(next(it)), n, stream, world, dev, barrier)
     per = {nm: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n)) / n for j, nm in enumerate(names)}
+    # the cross-attention gradient in one two-source call against one call per
+    # key source (the second accumulating dq): alternating rounds, outside the step
+    cmp = {"kv2": [], "per_source": []}
+    for rnd in range(4):
+        order = (("kv2", cross_kv2), ("per_source", cross_per_source))
+        for nm, fn in (order if rnd % 2 == 0 else order[::-1]):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(3):
+                fn()
+            e1.record(stream)
+            e1.synchronize()
+            cmp[nm].append(e0.elapsed_time(e1) / 3)
     f_self, f_cross = step_flops()
     flops = 2.5 * (f_self + f_cross)      # S, dP, dV, dK, dQ: five products of the forward's two sizes
     pk, pk_src = peaks()
@@ -701,14 +720,17 @@ def run_backward(args, rg, synth, d, outs, ws, wc, rank, dev, stream, world, bar
     roof["issued_tensor_flops_frac"] = round(roof["frac"] * 7 / 5, 4)
     del work
     return {
-        "what": "gradient step of the same window: regen_attn_bwd (self) + regen_rope3d_bwd + regen_attn_bwd per "
-                "cross-attention key block with the merged out/LSE (dq of the second accumulated); synthetic dO",
+        "what": "gradient step of the same window: regen_attn_bwd (self) + regen_rope3d_bwd + regen_attn_bwd_kv2 "
+                "(the cross-attention's two key sources with the joint out/LSE, one dQ pass over both); synthetic dO",
         "steps": n, "ms_per_step": round(ms, 4),
         "value": round(aggregate_tflops(flops, world, ms), 2), "unit": "TFLOP/s",
         "flops_note": "algorithmic: 2.5x the forward's (QK^T, dO V^T, P^T dO, dS^T Q, dS K); the kernels also "
                       "recompute QK^T and dO V^T once more (7 products in all, no atomics)",
         "kernels_ms": {nm: round(t, 4) for nm, t in per.items()},
-        "launches_per_step": 3 + 1 + 3 + 3,
+        "launches_per_step": 3 + 1 + 3,
+        "cross_attention_ms": {"kv2": round(min(cmp["kv2"]), 4), "per_source_calls": round(min(cmp["per_source"]), 4),
+                               "what": "best of 4 alternating rounds of 3 calls: regen_attn_bwd_kv2 against one "
+                                       "regen_attn_bwd per key source (6 launches, dq accumulated)"},
         "roofline": roof,
         "clocks": clk,
     }

@@ -16,6 +16,8 @@ Entry points (same names as the C ABI):
     regen_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Sq, Skv, D, scale, stream,
                    workspace, workspace_bytes, accumulate)   # REGEN_ACCUM_DQ | REGEN_ACCUM_DKDV
     regen_attn_bwd_workspace_bytes(B, H, Sq, D)
+    regen_attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout, dq, dk_a, dv_a, dk_b, dv_b, B, H, Sq,
+                       Skv_a, Skv_b, D, scale, stream, workspace, workspace_bytes, accumulate)
     regen_rope3d_bwd(dq, dk, T, Hh, Ww, theta, B, H, D, stream=None)
     regen_rope3d_shard(q, k, T, Hh, Ww, theta, B, H, D, n0, S_local, inverse=0, stream=None)
     regen_quant_e4m3(x, codes, scales, B, H, S, D, stream=None)
@@ -32,6 +34,7 @@ Convenience wrappers that allocate outputs with torch:
     rope3d_(q, k, grid, theta=10000.0)
     lse_merge(o_a, lse_a, o_b, lse_b) -> (out, lse)
     attn_bwd(q, k, v, out, lse, dout, scale=None) -> (dq, dk, dv)
+    attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout, scale=None) -> (dq, dk_a, dv_a, dk_b, dv_b)
     rope3d_bwd_(dq, dk, grid, theta=10000.0)
     quant_e4m3(x) -> (codes, scales);  attn_fwd_fp8(q8, qs, k8, ks, v8, vs, scale=None) -> (out, lse)
     qkv_proj(x, w, heads, grid, bias=None, gamma_q=None, gamma_k=None) -> (q, k, v)
@@ -51,7 +54,7 @@ __all__ = [
     "regen_status_str", "regen_last_device_error", "regen_last_cuda_error", "regen_selftest_exp2", "regen_selftest_bounded_wait", "regen_set_wait_limit_ns", "regen_version",
     "regen_attn_fwd_rope3d", "regen_attn_fwd_rope3d_workspace_bytes", "regen_attn_fwd_rope3d_noalloc",
     "regen_noalloc_scratch_bytes",
-    "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_rope3d_bwd", "regen_rope3d_shard", "regen_quant_e4m3",
+    "regen_attn_bwd", "regen_attn_bwd_workspace_bytes", "regen_attn_bwd_kv2", "attn_bwd_kv2", "regen_rope3d_bwd", "regen_rope3d_shard", "regen_quant_e4m3",
     "regen_attn_fwd_fp8", "quant_e4m3", "attn_fwd_fp8", "regen_qkv_proj", "regen_qkv_proj_workspace_bytes",
     "regen_out_proj", "qkv_proj", "out_proj",
     "attn_fwd", "attn_fwd_kv2", "regen_attn_fwd_kv2", "attn_fwd_rope3d", "rope3d_", "lse_merge", "attn_bwd", "rope3d_bwd_", "STATUS",
@@ -115,6 +118,8 @@ def load():
         L.regen_attn_bwd.restype = i32
         L.regen_attn_bwd_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.regen_attn_bwd_workspace_bytes.restype = i64
+        L.regen_attn_bwd_kv2.argtypes = [vp] * 13 + [i32] * 6 + [f32, vp, vp, i64, i32]
+        L.regen_attn_bwd_kv2.restype = i32
         L.regen_rope3d_bwd.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, vp]
         L.regen_rope3d_bwd.restype = i32
         L.regen_rope3d_shard.argtypes = [vp, vp, i32, i32, i32, f32, i32, i32, i32, i32, i32, i32, vp]
@@ -239,6 +244,14 @@ def regen_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, Sq, Skv, D, scale,
     _check(load().regen_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                                  _ptr(dv), B, H, Sq, Skv, D, float(scale), _stream(stream), _ptr(workspace),
                                  int(workspace_bytes), int(accumulate)), "regen_attn_bwd")
+
+
+def regen_attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout, dq, dk_a, dv_a, dk_b, dv_b, B, H, Sq, Skv_a, Skv_b,
+                       D, scale, stream, workspace, workspace_bytes, accumulate=0) -> None:
+    _check(load().regen_attn_bwd_kv2(_ptr(q), _ptr(k_a), _ptr(v_a), _ptr(k_b), _ptr(v_b), _ptr(out), _ptr(lse),
+                                     _ptr(dout), _ptr(dq), _ptr(dk_a), _ptr(dv_a), _ptr(dk_b), _ptr(dv_b), B, H, Sq,
+                                     Skv_a, Skv_b, D, float(scale), _stream(stream), _ptr(workspace),
+                                     int(workspace_bytes), int(accumulate)), "regen_attn_bwd_kv2")
 
 
 def regen_attn_bwd_workspace_bytes(B, H, Sq, D) -> int:
@@ -433,6 +446,29 @@ def attn_bwd(q, k, v, out, lse, dout, scale=None, dq=None, dk=None, dv=None, acc
                    workspace.numel() * workspace.element_size(),
                    (REGEN_ACCUM_DQ if accumulate_dq else 0) | (REGEN_ACCUM_DKDV if accumulate_dkdv else 0))
     return dq, dk, dv
+
+
+def attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout, scale=None, dq=None, accumulate_dq=False, workspace=None,
+                 stream=None):
+    """Gradients of attn_fwd_kv2 -> (dq, dk_a, dv_a, dk_b, dv_b), bf16 like the
+    inputs; out and lse are the two-source forward's. accumulate_dq adds into
+    the given dq."""
+    import torch
+    B, H, Sq, D = _bhsd(q, "q")
+    Skv_a, Skv_b = _bhsd(k_a, "k_a")[2], _bhsd(k_b, "k_b")[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if accumulate_dq and dq is None:
+        raise ValueError("accumulate_dq needs the dq to add into")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk_a, dv_a, dk_b, dv_b = (torch.empty_like(t) for t in (k_a, v_a, k_b, v_b))
+    need = regen_attn_bwd_workspace_bytes(B, H, Sq, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    regen_attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout, dq, dk_a, dv_a, dk_b, dv_b, B, H, Sq, Skv_a, Skv_b, D,
+                       scale, stream, workspace, workspace.numel() * workspace.element_size(),
+                       REGEN_ACCUM_DQ if accumulate_dq else 0)
+    return dq, dk_a, dv_a, dk_b, dv_b
 
 
 def rope3d_bwd_(dq, dk, grid, theta=10000.0, stream=None):

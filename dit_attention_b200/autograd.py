@@ -1,8 +1,9 @@
 """torch.autograd glue over the library's forward and gradient kernels.
 
 Argument marshalling only: the forward runs regen_rope3d, regen_attn_fwd and
-regen_attn_fwd_kv2, the backward runs regen_attn_bwd and regen_rope3d_bwd; no
-arithmetic happens here. Tensors are bf16 [B, H, S, D] on the GPU.
+regen_attn_fwd_kv2, the backward runs regen_attn_bwd, regen_attn_bwd_kv2 and
+regen_rope3d_bwd; no arithmetic happens here. Tensors are bf16 [B, H, S, D] on
+the GPU.
 
     dit_attention(q, k, v, grid=None, theta=10000.0, scale=None) -> out
         self-attention of q over (k, v); with a latent grid (T, Hh, Ww), q and
@@ -13,9 +14,9 @@ arithmetic happens here. Tensors are bf16 [B, H, S, D] on the GPU.
         one softmax over the keys of two separately held sources (the DiT's
         reference-frame latents and conditioning tokens, ReGenVC blog page,
         "Methodology -- deep read"), in one launch over both (regen_attn_fwd_kv2).
-        Its gradient runs per source with the joint output and LSE, so that
-        each source's P is its slice of the joint softmax, and the two dq
-        shares add up.
+        Its gradient (regen_attn_bwd_kv2) takes each source's P as its slice
+        of the joint softmax, from the joint output and LSE, and accumulates
+        dq over both sources' keys.
 """
 from __future__ import annotations
 
@@ -23,7 +24,7 @@ import math
 
 import torch
 
-from . import attn_bwd, attn_fwd, attn_fwd_kv2, rope3d_, rope3d_bwd_
+from . import attn_bwd, attn_bwd_kv2, attn_fwd, attn_fwd_kv2, rope3d_, rope3d_bwd_
 
 
 def _scale(scale, q):
@@ -63,9 +64,7 @@ class _TwoSourceAttention(torch.autograd.Function):
     @staticmethod
     def backward(ctx, dout):
         q, k_a, v_a, k_b, v_b, out, lse = ctx.saved_tensors
-        dout = dout.contiguous()
-        dq, dk_a, dv_a = attn_bwd(q, k_a, v_a, out, lse, dout, ctx.scale)
-        _, dk_b, dv_b = attn_bwd(q, k_b, v_b, out, lse, dout, ctx.scale, dq=dq, accumulate_dq=True)
+        dq, dk_a, dv_a, dk_b, dv_b = attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout.contiguous(), ctx.scale)
         return dq, dk_a, dv_a, dk_b, dv_b, None
 
 

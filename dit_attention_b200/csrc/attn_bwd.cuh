@@ -172,13 +172,22 @@ __device__ __forceinline__ void probs_pair(uint32_t &s0, uint32_t &s1, uint64_t 
 // ACCUM: dK and dV are added to the bf16 values already in dk_old / dv_old
 // (the output buffers themselves: each CTA reads its own key rows before its
 // store), for gradients accumulated over several query blocks.
+// Two key sources (the joint softmax over two key buffers): the grid covers
+// the key tiles of the first source (Skv keys; tm_k, tm_v, tm_dk, tm_dv,
+// dk_old, dv_old), then those of the second (Skv2 keys; the *2 arguments).
+// Each CTA's work depends only on its own key tile and the per-row
+// statistics, so the two sources' tiles are computed as in separate calls.
+// Skv2 = 0: one source (the *2 maps are not read).
 template <int HD, bool ACCUM>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                          const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                         const float *__restrict__ ws, int Sq, int Skv, float scale, float scale_log2,
-                         uint64_t wait_limit_ns, const uint16_t *dk_old, const uint16_t *dv_old)
+                         const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_v2,
+                         const __grid_constant__ CUtensorMap tm_dk2, const __grid_constant__ CUtensorMap tm_dv2,
+                         const float *__restrict__ ws, int Sq, int Skv, int Skv2, float scale, float scale_log2,
+                         uint64_t wait_limit_ns, const uint16_t *dk_old, const uint16_t *dv_old,
+                         const uint16_t *dk_old2, const uint16_t *dv_old2)
 {
     using C = BwdCfg<HD>;
     constexpr int NQ = C::A_NQ, ND = C::A_ND;
@@ -245,9 +254,15 @@ __global__ void __launch_bounds__(384, 1)
 
     const WaitCtl wc{abort_flag, wait_limit_ns};
     const int nq = (Sq + C::BM - 1) / C::BM;
-    const int nkv = (Skv + C::BN - 1) / C::BN;
-    const int bh = static_cast<int>(blockIdx.x / nkv);
-    const int key0 = static_cast<int>(blockIdx.x % nkv) * C::BN;
+    const int nkv1 = (Skv + C::BN - 1) / C::BN;
+    const int tiles = nkv1 + (Skv2 + C::BN - 1) / C::BN;   // key tiles of one (b, h), both sources
+    const int bh = static_cast<int>(blockIdx.x / tiles);
+    const int tile = static_cast<int>(blockIdx.x % tiles);
+    const bool second = tile >= nkv1;                        // this CTA's key tile is the second source's
+    const int key0 = (second ? tile - nkv1 : tile) * C::BN;  // first key of the tile within its source
+    const int skv = second ? Skv2 : Skv;
+    const CUtensorMap *map_k = second ? &tm_k2 : &tm_k;
+    const CUtensorMap *map_v = second ? &tm_v2 : &tm_v;
 
     if (warp < 4) {
     setmaxnreg_dec<C::REGS_LOW>();
@@ -263,14 +278,14 @@ __global__ void __launch_bounds__(384, 1)
         // -------------------------------------- producer: K, V, then Q ---
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(map_k);
+            tma_prefetch_desc(map_v);
             const uint64_t keep = l2_policy_evict_last();   // Q: re-read by every key tile of the head
             const uint64_t once = l2_policy_evict_first();  // K, V: read by this CTA only
             mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
             for (int h = 0; h < C::HALVES; ++h) {
-                tma_load_3d(sbase + C::A_K_OFF + h * C::HALF_BYTES, &tm_k, bar_kv, h * 64, key0, bh, once);
-                tma_load_3d(sbase + C::A_V_OFF + h * C::HALF_BYTES, &tm_v, bar_kv, h * 64, key0, bh, once);
+                tma_load_3d(sbase + C::A_K_OFF + h * C::HALF_BYTES, map_k, bar_kv, h * 64, key0, bh, once);
+                tma_load_3d(sbase + C::A_V_OFF + h * C::HALF_BYTES, map_v, bar_kv, h * 64, key0, bh, once);
             }
             int n = 0;  // query tiles issued
             bool ok = true;
@@ -536,9 +551,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int x = 0; x < 32; ++x) add[x] = 0.f;
                 if constexpr (ACCUM) {
-                    if (key0 + krow < Skv) {
+                    if (key0 + krow < skv) {
                         const uint4 *src = reinterpret_cast<const uint4 *>(
-                            (w ? dk_old : dv_old) + (static_cast<int64_t>(bh) * Skv + key0 + krow) * HD + c * 32);
+                            (w ? (second ? dk_old2 : dk_old) : (second ? dv_old2 : dv_old)) +
+                            (static_cast<int64_t>(bh) * skv + key0 + krow) * HD + c * 32);
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
                             const uint4 u = src[g];
@@ -568,7 +584,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         named_bar_sync(1 + w, 128);
         if (ok && warp == 4 + 4 * w && lane == 0) {
-            const CUtensorMap *map = w ? &tm_dk : &tm_dv;
+            const CUtensorMap *map = w ? (second ? &tm_dk2 : &tm_dk) : (second ? &tm_dv2 : &tm_dv);
             const uint32_t src = sbase + (w ? C::A_DO_OFF : C::A_Q_OFF);
             for (int h = 0; h < C::HALVES; ++h) tma_store_3d(map, src + h * C::HALF_BYTES, h * 64, key0, bh);
             tma_store_commit();
@@ -593,12 +609,17 @@ __global__ void __launch_bounds__(384, 1)
 // thread busy for the whole tile and the elementwise warps idle ~45 % of it.)
 // K and V come from two producer warps (0 and 3).
 // ACCUM: dQ is added to the bf16 values already in dq.
+// Two key sources: the key tiles of the first (Skv keys; tm_k, tm_v), then
+// those of the second (Skv2 keys; tm_k2, tm_v2), one dQ accumulation over
+// both; each source's last tile masks its own keys past its end. Skv2 = 0:
+// one source.
 template <int HD, bool ACCUM>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_dq, const uint16_t *__restrict__ dq_old,
-                       const float *__restrict__ ws, int Sq, int Skv, float scale, float scale_log2,
+                       const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_k2,
+                       const __grid_constant__ CUtensorMap tm_v2, const uint16_t *__restrict__ dq_old,
+                       const float *__restrict__ ws, int Sq, int Skv, int Skv2, float scale, float scale_log2,
                        uint64_t wait_limit_ns)
 {
     using C = BwdCfg<HD>;
@@ -659,10 +680,19 @@ __global__ void __launch_bounds__(384, 1)
 
     const WaitCtl wc{abort_flag, wait_limit_ns};
     const int nq = (Sq + C::BM - 1) / C::BM;
-    const int nkv = (Skv + C::BN - 1) / C::BN;
+    const int nkv1 = (Skv + C::BN - 1) / C::BN;         // key tiles of the first source
+    const int nkv = nkv1 + (Skv2 + C::BN - 1) / C::BN;  // of both
     const int bh = static_cast<int>(blockIdx.x / nq);
     const int qt = static_cast<int>(blockIdx.x % nq);
     const int q0 = qt * C::BM;
+    // key tile j: its source's tensor maps, its first key row there, its valid keys
+    auto tile_k = [&](int j) { return j < nkv1 ? &tm_k : &tm_k2; };
+    auto tile_v = [&](int j) { return j < nkv1 ? &tm_v : &tm_v2; };
+    auto tile_row = [&](int j) { return (j < nkv1 ? j : j - nkv1) * C::BN; };
+    auto valid_keys = [&](int j) {
+        const int rest = (j < nkv1 ? Skv : Skv2) - tile_row(j);
+        return rest < C::BN ? rest : C::BN;
+    };
 
     if (warp < 4) {
     setmaxnreg_dec<C::REGS_LOW>();
@@ -694,6 +724,7 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
+            if (nkv > nkv1) tma_prefetch_desc(&tm_k2);
             tma_prefetch_desc(&tm_do);
             const uint64_t keep = l2_policy_evict_last();   // K: re-read by every query tile of the head
             const uint64_t once = l2_policy_evict_first();  // Q, dO: read by this CTA only
@@ -710,8 +741,8 @@ __global__ void __launch_bounds__(384, 1)
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_k_full(sk), C::TILE_BYTES);
                 for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_3d(sbase + C::B_K_OFF + sk * C::TILE_BYTES + h * C::HALF_BYTES, &tm_k, bar_k_full(sk),
-                                h * 64, j * C::BN, bh, keep);
+                    tma_load_3d(sbase + C::B_K_OFF + sk * C::TILE_BYTES + h * C::HALF_BYTES, tile_k(j), bar_k_full(sk),
+                                h * 64, tile_row(j), bh, keep);
                 ++nk;
             }
             if (!ok) {
@@ -723,6 +754,7 @@ __global__ void __launch_bounds__(384, 1)
         // ------------------------------------------------- producer: V ---
         if (lane == 0) {
             tma_prefetch_desc(&tm_v);
+            if (nkv > nkv1) tma_prefetch_desc(&tm_v2);
             const uint64_t keep = l2_policy_evict_last();   // V: re-read by every query tile of the head
             int nv = 0;
             bool ok = true;
@@ -732,8 +764,8 @@ __global__ void __launch_bounds__(384, 1)
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar_v_full(sv), C::TILE_BYTES);
                 for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_3d(sbase + C::B_V_OFF + sv * C::TILE_BYTES + h * C::HALF_BYTES, &tm_v, bar_v_full(sv),
-                                h * 64, j * C::BN, bh, keep);
+                    tma_load_3d(sbase + C::B_V_OFF + sv * C::TILE_BYTES + h * C::HALF_BYTES, tile_v(j), bar_v_full(sv),
+                                h * 64, tile_row(j), bh, keep);
                 ++nv;
             }
             if (!ok)
@@ -830,7 +862,6 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t c2 = f2_pack(scale_log2, scale_log2);
         const uint64_t nl2 = f2_pack(-lse2, -lse2);
         const uint64_t dl2 = f2_pack(delta, delta);
-        const int kv_tail = Skv - (nkv - 1) * C::BN;  // valid keys in the last tile (1..128)
         bool ok = true;
         for (int j = 0; ok && j < nkv; ++j) {
             const int b = j & 1;
@@ -848,8 +879,9 @@ __global__ void __launch_bounds__(384, 1)
             for (int hv = 0; hv < 2; ++hv)
 #pragma unroll
                 for (int c = 0; c < 16; ++c) probs_pair<C::EMU_PER8>(pr[hv][2 * c], pr[hv][2 * c + 1], c2, nl2, c);
-            if (j == nkv - 1 && kv_tail < C::BN) {
-                // keys past Skv: their logits come from zero-filled rows; P = 0
+            const int kv_tail = valid_keys(j);
+            if (kv_tail < C::BN) {
+                // keys past the source's end: their logits come from zero-filled rows; P = 0
 #pragma unroll
                 for (int x = 0; x < 64; ++x)
                     if (64 * w + x >= kv_tail) pr[x >> 5][x & 31] = 0u;

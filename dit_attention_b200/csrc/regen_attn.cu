@@ -374,11 +374,15 @@ int grid_for(int64_t work, int threads)
     return static_cast<int>(blocks < 1 ? 1 : blocks);
 }
 
+// The gradient launches: prep, dK/dV over the key tiles of both sources, dQ
+// over both. A second key source (k2, v2, dk2, dv2; Skv2 keys) shares the
+// queries, out, LSE and dO; Skv2 = 0 for one source.
 template <int HD>
 int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, const regen_bf16 *out,
                const float *lse, const regen_bf16 *dout, regen_bf16 *dq, regen_bf16 *dk, regen_bf16 *dv,
                int64_t BH, int Sq, int Skv, float scale, float *ws, bool acc_dq, bool acc_dkdv,
-               cudaStream_t stream)
+               cudaStream_t stream, const regen_bf16 *k2 = nullptr, const regen_bf16 *v2 = nullptr,
+               regen_bf16 *dk2 = nullptr, regen_bf16 *dv2 = nullptr, int Skv2 = 0)
 {
     using C = regen::BwdCfg<HD>;
     static PerContext<int> ready;
@@ -403,8 +407,13 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
         !make_bhsd_map(&tdq, dq, BH, Sq, HD) || !make_bhsd_map(&tdk, dk, BH, Skv, HD) ||
         !make_bhsd_map(&tdv, dv, BH, Skv, HD))
         return REGEN_ERR_CUDA;
+    CUtensorMap tk2 = tk, tv2 = tv, tdk2 = tdk, tdv2 = tdv;   // not read when Skv2 = 0
+    if (Skv2 > 0 &&
+        (!make_bhsd_map(&tk2, k2, BH, Skv2, HD) || !make_bhsd_map(&tv2, v2, BH, Skv2, HD) ||
+         !make_bhsd_map(&tdk2, dk2, BH, Skv2, HD) || !make_bhsd_map(&tdv2, dv2, BH, Skv2, HD)))
+        return REGEN_ERR_CUDA;
     const int nq = (Sq + C::BM - 1) / C::BM;
-    const int nkv = (Skv + C::BN - 1) / C::BN;
+    const int nkv = (Skv + C::BN - 1) / C::BN + (Skv2 + C::BN - 1) / C::BN;   // key tiles, both sources
     if (BH * nq > 0x7FFFFFFF || BH * nkv > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
     const int64_t prep_work = BH * nq * 128 * (HD / 8);
     regen::attn_bwd_prep_kernel<<<grid_for(prep_work, 256), 256, 0, stream>>>(
@@ -414,19 +423,23 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
     const uint64_t limit = g_wait_limit_ns.load();
     const uint16_t *dk_old = reinterpret_cast<const uint16_t *>(dk);
     const uint16_t *dv_old = reinterpret_cast<const uint16_t *>(dv);
+    const uint16_t *dk_old2 = reinterpret_cast<const uint16_t *>(dk2);
+    const uint16_t *dv_old2 = reinterpret_cast<const uint16_t *>(dv2);
     if (acc_dkdv)
         regen::attn_bwd_dkdv_kernel<HD, true><<<static_cast<unsigned>(BH * nkv), C::THREADS, C::A_SMEM_BYTES, stream>>>(
-            tq, tk, tv, tdo, tdk, tdv, ws, Sq, Skv, scale, scale_log2, limit, dk_old, dv_old);
+            tq, tk, tv, tdo, tdk, tdv, tk2, tv2, tdk2, tdv2, ws, Sq, Skv, Skv2, scale, scale_log2, limit, dk_old,
+            dv_old, dk_old2, dv_old2);
     else
         regen::attn_bwd_dkdv_kernel<HD, false><<<static_cast<unsigned>(BH * nkv), C::THREADS, C::A_SMEM_BYTES, stream>>>(
-            tq, tk, tv, tdo, tdk, tdv, ws, Sq, Skv, scale, scale_log2, limit, dk_old, dv_old);
+            tq, tk, tv, tdo, tdk, tdv, tk2, tv2, tdk2, tdv2, ws, Sq, Skv, Skv2, scale, scale_log2, limit, dk_old,
+            dv_old, dk_old2, dv_old2);
     if (launched() != REGEN_OK) return REGEN_ERR_CUDA;
     if (acc_dq)
         regen::attn_bwd_dq_kernel<HD, true><<<static_cast<unsigned>(BH * nq), C::THREADS, C::B_SMEM_BYTES, stream>>>(
-            tq, tk, tv, tdo, tdq, dq, ws, Sq, Skv, scale, scale_log2, limit);
+            tq, tk, tv, tdo, tdq, tk2, tv2, dq, ws, Sq, Skv, Skv2, scale, scale_log2, limit);
     else
         regen::attn_bwd_dq_kernel<HD, false><<<static_cast<unsigned>(BH * nq), C::THREADS, C::B_SMEM_BYTES, stream>>>(
-            tq, tk, tv, tdo, tdq, dq, ws, Sq, Skv, scale, scale_log2, limit);
+            tq, tk, tv, tdo, tdq, tk2, tv2, dq, ws, Sq, Skv, Skv2, scale, scale_log2, limit);
     return launched();
 }
 
@@ -839,6 +852,74 @@ REGEN_API int regen_attn_bwd(const regen_bf16 *q, const regen_bf16 *k, const reg
     if (D == 128)
         return launch_bwd<128>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, acc_dq, acc_dkdv, st);
     return launch_bwd<64>(q, k, v, out, lse, dout, dq, dk, dv, BH, Sq, Skv, scale, ws, acc_dq, acc_dkdv, st);
+}
+
+REGEN_API int regen_attn_bwd_kv2(const regen_bf16 *q, const regen_bf16 *k_a, const regen_bf16 *v_a,
+                                 const regen_bf16 *k_b, const regen_bf16 *v_b, const regen_bf16 *out,
+                                 const float *lse, const regen_bf16 *dout, regen_bf16 *dq, regen_bf16 *dk_a,
+                                 regen_bf16 *dv_a, regen_bf16 *dk_b, regen_bf16 *dv_b, int B, int H, int Sq,
+                                 int Skv_a, int Skv_b, int D, float scale, regen_stream_t stream,
+                                 void *workspace, int64_t workspace_bytes, int accumulate)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Skv_a < 0 || Skv_b < 0 || D < 0 || workspace_bytes < 0)
+        return REGEN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return REGEN_ERR_INVALID_ARG;
+    if (accumulate < 0 || accumulate > (REGEN_ACCUM_DQ | REGEN_ACCUM_DKDV)) return REGEN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return REGEN_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(Skv_a) + Skv_b > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH == 0) return REGEN_OK;
+    if (Skv_b == 0)
+        return regen_attn_bwd(q, k_a, v_a, out, lse, dout, dq, dk_a, dv_a, B, H, Sq, Skv_a, D, scale, stream,
+                              workspace, workspace_bytes, accumulate);
+    if (Skv_a == 0)
+        return regen_attn_bwd(q, k_b, v_b, out, lse, dout, dq, dk_b, dv_b, B, H, Sq, Skv_b, D, scale, stream,
+                              workspace, workspace_bytes, accumulate);
+    if (Sq == 0) {  // dk = dv = 0 for both sources (unchanged when accumulating)
+        if (!dk_a || !dv_a || !dk_b || !dv_b) return REGEN_ERR_INVALID_ARG;
+        const int64_t ba = BH * Skv_a * D * 2, bb = BH * Skv_b * D * 2;
+        if (overlaps(dk_a, ba, dk_b, bb) || overlaps(dk_a, ba, dv_b, bb) || overlaps(dv_a, ba, dk_b, bb) ||
+            overlaps(dv_a, ba, dv_b, bb))
+            return REGEN_ERR_INVALID_ARG;
+        const int st = regen_attn_bwd(q, k_a, v_a, out, lse, dout, dq, dk_a, dv_a, B, H, 0, Skv_a, D, scale,
+                                      stream, workspace, workspace_bytes, accumulate);
+        if (st != REGEN_OK) return st;
+        return regen_attn_bwd(q, k_b, v_b, out, lse, dout, dq, dk_b, dv_b, B, H, 0, Skv_b, D, scale, stream,
+                              workspace, workspace_bytes, accumulate);
+    }
+    const bool acc_dq = (accumulate & REGEN_ACCUM_DQ) != 0, acc_dkdv = (accumulate & REGEN_ACCUM_DKDV) != 0;
+    if (BH > 0x7FFFFFFF) return REGEN_ERR_UNSUPPORTED;
+    if (!q || !k_a || !v_a || !k_b || !v_b || !out || !lse || !dout || !dq || !dk_a || !dv_a || !dk_b || !dv_b ||
+        !workspace)
+        return REGEN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_a) || !aligned16(v_a) || !aligned16(k_b) || !aligned16(v_b) ||
+        !aligned16(out) || !aligned16(lse) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk_a) ||
+        !aligned16(dv_a) || !aligned16(dk_b) || !aligned16(dv_b) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return REGEN_ERR_MISALIGNED;
+    const int64_t need = bwd_workspace_bytes(BH, Sq);
+    if (workspace_bytes < need) return REGEN_ERR_INVALID_ARG;
+    const int64_t qbytes = BH * Sq * D * 2, abytes = BH * Skv_a * D * 2, bbytes = BH * Skv_b * D * 2,
+                  lbytes = BH * Sq * 4;
+    struct Span { const void *p; int64_t n; };
+    const Span ins[8] = {{q, qbytes},   {k_a, abytes}, {v_a, abytes},  {k_b, bbytes},
+                         {v_b, bbytes}, {out, qbytes}, {lse, lbytes},  {dout, qbytes}};
+    const Span outs[6] = {{dq, qbytes},   {dk_a, abytes}, {dv_a, abytes},
+                          {dk_b, bbytes}, {dv_b, bbytes}, {workspace, need}};
+    for (int a = 0; a < 6; ++a) {
+        for (const Span &in : ins)
+            if (overlaps(outs[a].p, outs[a].n, in.p, in.n)) return REGEN_ERR_INVALID_ARG;
+        for (int b = a + 1; b < 6; ++b)
+            if (overlaps(outs[a].p, outs[a].n, outs[b].p, outs[b].n)) return REGEN_ERR_INVALID_ARG;
+    }
+    float *ws = static_cast<float *>(workspace);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const DeviceScope device(dq);
+    if (device.status != REGEN_OK) return device.status;
+    if (D == 128)
+        return launch_bwd<128>(q, k_a, v_a, out, lse, dout, dq, dk_a, dv_a, BH, Sq, Skv_a, scale, ws, acc_dq,
+                               acc_dkdv, st, k_b, v_b, dk_b, dv_b, Skv_b);
+    return launch_bwd<64>(q, k_a, v_a, out, lse, dout, dq, dk_a, dv_a, BH, Sq, Skv_a, scale, ws, acc_dq, acc_dkdv,
+                          st, k_b, v_b, dk_b, dv_b, Skv_b);
 }
 
 REGEN_API int regen_lse_merge(const regen_bf16 *o_a, const float *lse_a, const regen_bf16 *o_b,

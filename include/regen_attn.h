@@ -269,6 +269,36 @@ enum { REGEN_ACCUM_DQ = 1, REGEN_ACCUM_DKDV = 2 };
 REGEN_API int64_t regen_attn_bwd_workspace_bytes(int B, int H, int Sq, int D);
 
 /*
+ * regen_attn_bwd_kv2 -- gradients of regen_attn_fwd_kv2: the cross-attention
+ * of the video tokens to the reference-frame and conditioning tokens (blog
+ * page, "Methodology -- deep read") as one softmax over the two key sets
+ * [k_a ; k_b], with that softmax's out and lse. The formulas of
+ * regen_attn_bwd over the concatenated keys; dk, dv of each key go to its
+ * source's buffer. Three launches for both sources:
+ *  - one prep;
+ *  - one dK/dV grid over the key tiles of a and then of b;
+ *  - one dQ pass over all key tiles, accumulating dq in fp32 across both
+ *    sources before its one rounding to bf16.
+ * dk and dv equal regen_attn_bwd's for each source's keys, bit for bit. dq
+ * has the same formula, rounded once instead of once per source.
+ *
+ *   q, out, dout, dq  [B, H, Sq, D] bf16;  lse [B, H, Sq] fp32
+ *   k_a, v_a, dk_a, dv_a  [B, H, Skv_a, D];  k_b, v_b, dk_b, dv_b  [B, H, Skv_b, D] bf16
+ *   D, scale, workspace (regen_attn_bwd_workspace_bytes(B, H, Sq, D) bytes) and
+ *   accumulate as regen_attn_bwd (REGEN_ACCUM_DKDV applies to both sources).
+ * The outputs must not overlap each other, an input or the workspace. One
+ * source empty: the same as regen_attn_bwd over the other (the empty
+ * source's pointers may then be NULL). Sq == 0: every dk, dv = 0 (unchanged
+ * when accumulating). B or H == 0: REGEN_OK, nothing done.
+ */
+REGEN_API int regen_attn_bwd_kv2(const regen_bf16 *q, const regen_bf16 *k_a, const regen_bf16 *v_a,
+                                 const regen_bf16 *k_b, const regen_bf16 *v_b, const regen_bf16 *out,
+                                 const float *lse, const regen_bf16 *dout, regen_bf16 *dq, regen_bf16 *dk_a,
+                                 regen_bf16 *dv_a, regen_bf16 *dk_b, regen_bf16 *dv_b, int B, int H, int Sq,
+                                 int Skv_a, int Skv_b, int D, float scale, regen_stream_t stream,
+                                 void *workspace, int64_t workspace_bytes, int accumulate);
+
+/*
  * regen_rope3d_bwd -- gradient of regen_rope3d, in place: every pair of the
  * gradients dq, dk is turned back by its angle (the transposed rotation),
  *     g'_{2j} = g_{2j} cos + g_{2j+1} sin,   g'_{2j+1} = g_{2j+1} cos - g_{2j} sin

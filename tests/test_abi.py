@@ -298,3 +298,23 @@ def test_attn_fwd_kv2_validation(lib, args, status):
     rc = lib.regen_attn_fwd_kv2(a["q"], a["k_a"], a["v_a"], a["k_b"], a["v_b"], a["out"], a["lse"], a["B"], a["H"],
                                 a["Sq"], a["Skv_a"], a["Skv_b"], a["D"], a["scale"], None)
     assert rc == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=96), -2), (dict(B=-1), -1), (dict(Skv_b=-1), -1), (dict(scale=float("inf")), -1),
+    (dict(accumulate=4), -1), (dict(B=0), 0), (dict(Skv_a=2**30, Skv_b=2**30), -2),
+    (dict(k_b=None), -1), (dict(dv_b=None), -1), (dict(ws=None), -1), (dict(dk_b=FAKE + 110 * MB + 8), -3),
+    (dict(ws=FAKE + 130 * MB + 16), -3), (dict(ws_bytes=2047), -1), (dict(dv_b=FAKE + 90 * MB), -1),
+    (dict(dq=FAKE + 10 * MB), -1), (dict(ws=FAKE + 60 * MB), -1),
+])
+def test_attn_bwd_kv2_validation(lib, args, status):
+    a = dict(q=FAKE, k_a=FAKE + 10 * MB, v_a=FAKE + 20 * MB, k_b=FAKE + 30 * MB, v_b=FAKE + 40 * MB,
+             out=FAKE + 50 * MB, lse=FAKE + 60 * MB, dout=FAKE + 70 * MB, dq=FAKE + 80 * MB, dk_a=FAKE + 90 * MB,
+             dv_a=FAKE + 100 * MB, dk_b=FAKE + 110 * MB, dv_b=FAKE + 120 * MB, ws=FAKE + 130 * MB, ws_bytes=2048,
+             B=1, H=2, Sq=100, Skv_a=60, Skv_b=40, D=128, scale=0.125, accumulate=0)
+    a.update(args)
+    rc = lib.regen_attn_bwd_kv2(a["q"], a["k_a"], a["v_a"], a["k_b"], a["v_b"], a["out"], a["lse"], a["dout"],
+                                a["dq"], a["dk_a"], a["dv_a"], a["dk_b"], a["dv_b"], a["B"], a["H"], a["Sq"],
+                                a["Skv_a"], a["Skv_b"], a["D"], a["scale"], None, a["ws"], a["ws_bytes"],
+                                a["accumulate"])
+    assert rc == status
