@@ -876,10 +876,12 @@ REGEN_API int regen_attn_bwd_kv2(const regen_bf16 *q, const regen_bf16 *k_a, con
         return regen_attn_bwd(q, k_b, v_b, out, lse, dout, dq, dk_b, dv_b, B, H, Sq, Skv_b, D, scale, stream,
                               workspace, workspace_bytes, accumulate);
     if (Sq == 0) {  // dk = dv = 0 for both sources (unchanged when accumulating)
+        // every check of both calls first, so that an error launches nothing
         if (!dk_a || !dv_a || !dk_b || !dv_b) return REGEN_ERR_INVALID_ARG;
+        if (!aligned16(dk_a) || !aligned16(dv_a) || !aligned16(dk_b) || !aligned16(dv_b)) return REGEN_ERR_MISALIGNED;
         const int64_t ba = BH * Skv_a * D * 2, bb = BH * Skv_b * D * 2;
-        if (overlaps(dk_a, ba, dk_b, bb) || overlaps(dk_a, ba, dv_b, bb) || overlaps(dv_a, ba, dk_b, bb) ||
-            overlaps(dv_a, ba, dv_b, bb))
+        if (overlaps(dk_a, ba, dv_a, ba) || overlaps(dk_b, bb, dv_b, bb) || overlaps(dk_a, ba, dk_b, bb) ||
+            overlaps(dk_a, ba, dv_b, bb) || overlaps(dv_a, ba, dk_b, bb) || overlaps(dv_a, ba, dv_b, bb))
             return REGEN_ERR_INVALID_ARG;
         const int st = regen_attn_bwd(q, k_a, v_a, out, lse, dout, dq, dk_a, dv_a, B, H, 0, Skv_a, D, scale,
                                       stream, workspace, workspace_bytes, accumulate);

@@ -306,6 +306,8 @@ def test_attn_fwd_kv2_validation(lib, args, status):
     (dict(k_b=None), -1), (dict(dv_b=None), -1), (dict(ws=None), -1), (dict(dk_b=FAKE + 110 * MB + 8), -3),
     (dict(ws=FAKE + 130 * MB + 16), -3), (dict(ws_bytes=2047), -1), (dict(dv_b=FAKE + 90 * MB), -1),
     (dict(dq=FAKE + 10 * MB), -1), (dict(ws=FAKE + 60 * MB), -1),
+    # no queries: both sources' buffers are checked before anything is launched
+    (dict(Sq=0, dv_b=FAKE + 120 * MB + 2), -3), (dict(Sq=0, dk_b=None), -1), (dict(Sq=0, dk_b=FAKE + 90 * MB), -1),
 ])
 def test_attn_bwd_kv2_validation(lib, args, status):
     a = dict(q=FAKE, k_a=FAKE + 10 * MB, v_a=FAKE + 20 * MB, k_b=FAKE + 30 * MB, v_b=FAKE + 40 * MB,
