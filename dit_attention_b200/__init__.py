@@ -449,10 +449,10 @@ def attn_bwd(q, k, v, out, lse, dout, scale=None, dq=None, dk=None, dv=None, acc
 
 
 def attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout, scale=None, dq=None, accumulate_dq=False, workspace=None,
-                 stream=None):
+                 stream=None, dkv=None, accumulate_dkdv=False):
     """Gradients of attn_fwd_kv2 -> (dq, dk_a, dv_a, dk_b, dv_b), bf16 like the
     inputs; out and lse are the two-source forward's. accumulate_dq adds into
-    the given dq."""
+    the given dq; accumulate_dkdv into the given dkv = (dk_a, dv_a, dk_b, dv_b)."""
     import torch
     B, H, Sq, D = _bhsd(q, "q")
     Skv_a, Skv_b = _bhsd(k_a, "k_a")[2], _bhsd(k_b, "k_b")[2]
@@ -460,14 +460,16 @@ def attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout, scale=None, dq=None, acc
         scale = 1.0 / math.sqrt(D)
     if accumulate_dq and dq is None:
         raise ValueError("accumulate_dq needs the dq to add into")
+    if accumulate_dkdv and dkv is None:
+        raise ValueError("accumulate_dkdv needs the dk_a, dv_a, dk_b, dv_b to add into")
     dq = torch.empty_like(q) if dq is None else dq
-    dk_a, dv_a, dk_b, dv_b = (torch.empty_like(t) for t in (k_a, v_a, k_b, v_b))
+    dk_a, dv_a, dk_b, dv_b = (torch.empty_like(t) for t in (k_a, v_a, k_b, v_b)) if dkv is None else dkv
     need = regen_attn_bwd_workspace_bytes(B, H, Sq, D)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     regen_attn_bwd_kv2(q, k_a, v_a, k_b, v_b, out, lse, dout, dq, dk_a, dv_a, dk_b, dv_b, B, H, Sq, Skv_a, Skv_b, D,
                        scale, stream, workspace, workspace.numel() * workspace.element_size(),
-                       REGEN_ACCUM_DQ if accumulate_dq else 0)
+                       (REGEN_ACCUM_DQ if accumulate_dq else 0) | (REGEN_ACCUM_DKDV if accumulate_dkdv else 0))
     return dq, dk_a, dv_a, dk_b, dv_b
 
 

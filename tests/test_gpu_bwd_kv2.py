@@ -110,6 +110,27 @@ def test_bwd_kv2_accumulates_dq():
     check_against_oracle(grads, q, ka, va, kb, vb, g, scale, "kv2 bwd accumulate", dq0=dq0)
 
 
+def test_bwd_kv2_accumulates_dk_dv_of_both_sources():
+    # query blocks (Ring attention's backward): each source's dk, dv add into the given ones
+    B, H, Sq, D = 1, 2, 300, 64
+    q, g = rand_bf16((B, H, Sq, D)), rand_bf16((B, H, Sq, D))
+    ka, va = rand_bf16((B, H, 140, D)), rand_bf16((B, H, 140, D))
+    kb, vb = rand_bf16((B, H, 200, D)), rand_bf16((B, H, 200, D))
+    olds = [rand_bf16(x.shape, 0.05) for x in (ka, va, kb, vb)]
+    scale = 1.0 / np.sqrt(D)
+    grads, _ = gpu_kv2(q, ka, va, kb, vb, g, scale, dkv=tuple(to_dev(o) for o in olds), accumulate_dkdv=True)
+    kc, vc = np.concatenate([ka, kb], axis=2), np.concatenate([va, vb], axis=2)
+    rq, rk, rv = oracle.attention_bwd(q, kc, vc, g, scale)
+    bq, bk = delta_bounds(q, kc, vc, g, scale)
+    rk = rk + np.concatenate([bits_to_f64(olds[0]), bits_to_f64(olds[2])], axis=2)
+    rv = rv + np.concatenate([bits_to_f64(olds[1]), bits_to_f64(olds[3])], axis=2)
+    check_grad(grads[0], rq, "kv2 acc dq", bq)
+    check_grad(np.concatenate([bits_to_f64(grads[1]), bits_to_f64(grads[3])], axis=2), rk, "kv2 acc dk",
+               bk + 2.0 ** -8 * np.abs(rk))
+    check_grad(np.concatenate([bits_to_f64(grads[2]), bits_to_f64(grads[4])], axis=2), rv, "kv2 acc dv",
+               2.0 ** -8 * np.abs(rv))
+
+
 def test_bwd_kv2_one_source_empty_is_the_one_source_gradient():
     B, H, Sq, D = 1, 2, 200, 64
     q, g = rand_bf16((B, H, Sq, D)), rand_bf16((B, H, Sq, D))
