@@ -53,9 +53,19 @@ struct BwdCfg {
     static constexpr int STAT_BYTES = 1024;          // lse2[128] then delta[128] of one query tile
     static constexpr int THREADS = 384;
     static constexpr uint32_t TMEM_COLS = 512;
+    // Register split after setmaxnreg: producer / MMA warpgroup at REGS_LOW,
+    // the two elementwise warpgroups at REGS_HIGH. (REGS_HIGH - R) * 256 <=
+    // (R - REGS_LOW) * 128 needs R registers per thread at launch (the build
+    // uses 168). dK/dV: 64 / 208 (R >= 160). dQ: 56 / 216 (R >= 163): its
+    // elementwise loop spilled at 208, and 216 took its cycles from 7.45 M to
+    // 7.32 M on 8 heads, where the same split made the dK/dV kernel slower
+    // (9.77 M to 9.90 M).
     static constexpr uint32_t REGS_LOW = 64;
     static constexpr uint32_t REGS_HIGH = 208;
     static constexpr int MIN_LAUNCH_REGS = 160;
+    static constexpr uint32_t B_REGS_LOW = 56;
+    static constexpr uint32_t B_REGS_HIGH = 216;
+    static constexpr int B_MIN_LAUNCH_REGS = 163;
     static constexpr int EMU_PER8 = REGEN_EXP2_EMU_PER8;
 
     // dK/dV kernel: K and V tiles resident; Q through an NQ-stage ring and dO with
@@ -695,7 +705,7 @@ __global__ void __launch_bounds__(384, 1)
     };
 
     if (warp < 4) {
-    setmaxnreg_dec<C::REGS_LOW>();
+    setmaxnreg_dec<C::B_REGS_LOW>();
     const uint64_t drain_ns = wait_limit_ns > kDrainFloorNs ? wait_limit_ns : kDrainFloorNs;
     auto drain_copies = [&](uint32_t bar, uint32_t parity) {
         const uint64_t t0 = global_timer_ns();
@@ -850,7 +860,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
     } else {
-        setmaxnreg_inc<C::REGS_HIGH>();
+        setmaxnreg_inc<C::B_REGS_HIGH>();
         // ------------------------------------------------- elementwise ---
         const int w = (warp - 4) >> 2;     // key columns [64w, 64w + 64)
         const int quad = warp & 3;

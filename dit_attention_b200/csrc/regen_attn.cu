@@ -394,10 +394,10 @@ int launch_bwd(const regen_bf16 *q, const regen_bf16 *k, const regen_bf16 *v, co
                               C::A_SMEM_BYTES, C::MIN_LAUNCH_REGS);
         if (st == REGEN_OK)
             st = kernel_setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, false>),
-                              C::B_SMEM_BYTES, C::MIN_LAUNCH_REGS);
+                              C::B_SMEM_BYTES, C::B_MIN_LAUNCH_REGS);
         if (st == REGEN_OK)
             st = kernel_setup(reinterpret_cast<const void *>(regen::attn_bwd_dq_kernel<HD, true>),
-                              C::B_SMEM_BYTES, C::MIN_LAUNCH_REGS);
+                              C::B_SMEM_BYTES, C::B_MIN_LAUNCH_REGS);
         return st;
     }, nullptr);
     if (attr_status != REGEN_OK) return attr_status;
