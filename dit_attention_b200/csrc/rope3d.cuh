@@ -67,17 +67,18 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t packed, double c, doubl
 // term covers results among the fp32 subnormals). If no bf16 rounding
 // boundary -- the midpoint between two neighbouring bf16 values -- lies
 // within that distance of the fp32 value, both round to the same bf16. The
-// test uses 2^-21 X + 2^-146 (twice the bound, which also absorbs the
-// rounding of X itself), and the midpoint of the bf16 cell that holds y,
-// whose distance to y is exact in fp32 (same sign and binade). A NaN or
-// infinite value fails the test and goes to fp64.
+// test uses fl(fl(X) * 2^-22 + 2^-146): fl(X) and the fused product each lose
+// at most a factor (1 - 2^-24), and 4 (1 - 2^-24)^2 > 3.0001 (1 + 2^-24), so
+// it is never below the bound. It measures the distance to the midpoint of the
+// bf16 cell that holds y, which is exact in fp32 (same sign and binade). A
+// NaN or infinite value fails the test and goes to fp64.
 __device__ __forceinline__ bool rotate_pair_f32(uint32_t packed, float c32, float s32, uint32_t &out)
 {
     const float x0 = __uint_as_float(packed << 16);
     const float x1 = __uint_as_float(packed & 0xFFFF0000u);
     const float y0 = __fmaf_rn(x0, c32, -__fmul_rn(x1, s32));
     const float y1 = __fmaf_rn(x0, s32, __fmul_rn(x1, c32));
-    const float bound = __fmaf_rn(__fadd_rn(fabsf(x0), fabsf(x1)), 0x1p-21f, 0x1p-146f);
+    const float bound = __fmaf_rn(__fadd_rn(fabsf(x0), fabsf(x1)), 0x1p-22f, 0x1p-146f);
     const float g0 = fabsf(__fsub_rn(y0, __uint_as_float((__float_as_uint(y0) & 0xFFFF0000u) | 0x8000u)));
     const float g1 = fabsf(__fsub_rn(y1, __uint_as_float((__float_as_uint(y1) & 0xFFFF0000u) | 0x8000u)));
     out = pack_bf16x2(y0, y1);
@@ -197,7 +198,8 @@ __global__ void rope_table_kernel(double *__restrict__ tab64, float2 *__restrict
 }
 
 // The four pairs of a 16-byte chunk: fp32 with one certificate for the whole
-// chunk; if any pair is not certified (about one chunk in 80), the chunk is
+// chunk; if any pair is not certified (rare: the check fails near a bf16
+// rounding boundary), the chunk is
 // redone in fp64 from the fp64 cosines and sines.
 __device__ __forceinline__ uint4 rotate_chunk_f32(uint4 v, const float2 (&cs)[4], const double (&c64)[4],
                                                   const double (&s64)[4])
