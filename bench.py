@@ -57,7 +57,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     p.add_argument("--configs", action="store_true",
                    help="instead of the step: CUDA-event medians of every workload's kernels (1 GPU)")
-    p.add_argument("--profile-case", choices=["attn", "fused", "kv2", "rope", "merge", "bwd", "fp8"], default=None,
+    p.add_argument("--profile-case", choices=["attn", "fused", "kv2", "rope", "merge", "bwd", "fp8", "proj", "proj_ref"],
+                   default=None,
                    help="instead of the step: a short, bounded launch sequence of one kernel for ncu (no timing)")
     p.add_argument("--heads", type=int, default=8, help="--profile-case: heads")
     p.add_argument("--seq", type=int, default=31200, help="--profile-case: query tokens (31200, 10920 or 1024)")
@@ -1023,11 +1024,34 @@ def run_profile_case(args):
     attention launches), kv2 (two-source cross-attention: 1560 reference keys
     plus the rest of --kv), rope (3D RoPE on the latent grid of --seq), merge
     (two-block LSE merge), bwd (one forward, then gradient calls: prep, dK/dV
-    and dQ launches each) or fp8 (Q, K, V quantised once, then FP8 attention
-    calls). No timing is done here."""
+    and dQ launches each), fp8 (Q, K, V quantised once, then FP8 attention
+    calls), proj (regen_qkv_proj at the model width C = 5120 with --heads
+    heads, on the latent grid of --seq) or proj_ref (a cuBLAS GEMM of the same
+    shape, the comparison point the bench times beside it). No timing is done
+    here."""
     import torch
     import dit_attention_b200 as rg
     from dit_attention_b200 import synth
+    if args.kernel_case in ("proj", "proj_ref"):
+        T, Hh, Ww = PROFILE_GRIDS[args.seq]
+        H, C, S = args.heads, C_MODEL, args.seq
+        x = torch.from_numpy(synth._normal_bf16(100, 0, (1, S, C), False).view(np.int16)).cuda().view(torch.bfloat16)
+        w = torch.from_numpy(synth.f64_to_bf16_bits(synth.normal(100, 1, 3 * H * 128 * C).reshape(3 * H * 128, C)
+                                                    / math.sqrt(C)).view(np.int16)).cuda().view(torch.bfloat16)
+        rg.load()
+        if args.kernel_case == "proj":
+            bias = torch.from_numpy((synth.normal(100, 3, 3 * H * 128) * 0.1).astype(np.float32)).cuda()
+            for _ in range(args.iters):
+                rg.qkv_proj(x, w, H, (T, Hh, Ww), bias=bias)
+        else:
+            xm, res = x.view(S, C), torch.empty((S, 3 * H * 128), dtype=torch.bfloat16, device="cuda")
+            for _ in range(args.iters):
+                torch.matmul(xm, w.t(), out=res)
+        torch.cuda.synchronize()
+        rc, site = rg.regen_last_device_error()
+        if rc != 0:
+            raise SystemExit(f"device error {rc} at wait site {site}")
+        return
     skv = args.kv or args.seq
     w = synth.Workload("profile", B=1, H=args.heads, D=args.dim, Sq=args.seq, Skv=skv, seed=7)
     q, k, v = synth.make_inputs(w)
