@@ -482,8 +482,8 @@ def run_native(args, rank, world, local_rank):
     # distillation). dO synthetic; the forward's out/lse of the snapshot step
     # (its q, k rotated once: the inputs the gradient kernels take).
     # Self: regen_attn_bwd then regen_rope3d_bwd on dq, dk (gradients w.r.t. the
-    # unrotated Q, K). Cross: one regen_attn_bwd per key block with the merged
-    # out/lse, the second accumulating dq. Each regen_attn_bwd is 3 launches.
+    # unrotated Q, K). Cross: regen_attn_bwd_kv2 over both key sources with the
+    # joint out/lse. Each gradient call is 3 launches.
     step_fused()          # cross out/lse again (the cross paths above overwrote them); same self out/lse
     bwd = run_backward(args, rg, synth, d, outs0, ws, wc, rank, dev, stream, world, barrier, to_dev)
 
